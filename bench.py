@@ -1,0 +1,371 @@
+#!/usr/bin/env python
+"""Benchmark of the GPTQ layer quantizer (sm_100a) on synthetic Llama-shaped layers.
+
+One step = the whole hot path on one layer: H = 2 X^T X over the calibration
+tokens, damping / act-order / inverse factor, the column walk with OBQ
+feedback and lazy updates, and code packing.  Inputs are resident in HBM when
+the timed region starts; each step is timed with CUDA events on the launching
+stream, with the working copy of W restored and L2 flushed between steps
+(outside the events).  Multi-GPU runs are independent replicas (one layer per
+rank, no collective on the data path): weak scaling, max over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload llama7b_q_proj]
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "GPTQ layer quantize: weights/s and ms/layer (4-bit g128); Hessian TFLOP/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="llama7b_q_proj")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return FALLBACK_PEAKS, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as exc:  # NVML missing: report that, do not guess
+            self.nv = None
+            self.error = repr(exc)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.error}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- oracle timing
+def oracle_sample(wl: workloads.Workload, seed_offset: int = 0) -> dict:
+    """Time the float64 oracle on a bounded sample of the workload and
+    extrapolate to one full layer: H over a token sample (scaled by tokens),
+    the full-size inverse and elimination, the column loop on a row sample
+    (scaled by rows; rows are independent given H^-1)."""
+    import oracle
+    n_s = min(wl.n_tokens, 2048)
+    r_s = min(wl.d_row, 32)
+    X = workloads.activations(wl, n_tokens=n_s, seed_offset=seed_offset)
+    W = workloads.gaussian_weights(r_s, wl.d_col, wl.w_std, wl.seed)
+    t0 = time.perf_counter()
+    H = oracle.hessian(X)
+    t_h = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    prep = oracle.prepare(H, W, damp=wl.damp, desc_act=wl.desc_act)
+    Minv = oracle.inverse(prep["H_damped"])
+    t_p = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.eliminate(Minv)
+    t_e = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.gptq_columns(prep["W0"], Minv, wl.bits, wl.group_size)
+    t_c = time.perf_counter() - t0
+    rows_part = max(t_c - t_e, 0.0)
+    total = t_h * wl.n_tokens / n_s + t_p + t_e + rows_part * wl.d_row / r_s
+    spent = t_h + t_p + t_e + t_c
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return dict(value=wl.d_row * wl.d_col / total, seconds_extrapolated=total, spent=spent,
+                cores=cores,
+                sample=(f"oracle (numpy + C, float64, OpenMP) on {n_s} of {wl.n_tokens} tokens for H "
+                        f"(x{wl.n_tokens / n_s:g}), full {wl.d_col}^2 inverse + elimination, column "
+                        f"loop on {r_s} of {wl.d_row} rows (x{wl.d_row / r_s:g}); "
+                        f"{spent:.1f} s of CPU work"))
+
+
+def run_reference(args, rank: int, world: int):
+    """The oracle timed as it stands (no GPU work)."""
+    if rank != 0:
+        return
+    wl = workloads.WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        oracle_sample(wl)
+    vals, spent = [], 0.0
+    last = None
+    for _ in range(args.steps):
+        last = oracle_sample(wl)
+        vals.append(last["value"])
+        spent += last["spent"]
+    value = statistics.mean(vals)
+    ms = wl.d_row * wl.d_col / value * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "weights/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": _config(wl, world),
+            "cpu_baseline": {"value": value, "unit": "weights/s", "cores": last["cores"],
+                             "kind": "oracle", "sample": last["sample"]},
+            "e2e": {"value": value, "unit": "weights/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _config(wl, world):
+    return {"workload": wl.name, "d_row": wl.d_row, "d_col": wl.d_col, "tokens": wl.n_tokens,
+            "bits": wl.bits, "group_size": wl.group_size, "desc_act": wl.desc_act,
+            "damp": wl.damp, "block": wl.block_size, "parallelism": f"replicas{world}",
+            "l2": "flushed between steps (256 MiB write); X (2 bytes x tokens x d_col) is larger "
+                  "than L2"}
+
+
+# ---------------------------------------------------------------- our path
+def run_ours(args, rank: int, world: int, dist):
+    import post_weight_quantization_gptq_b200 as g
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    wl = workloads.WORKLOADS[args.workload]
+    r, d, n = wl.d_row, wl.d_col, wl.n_tokens
+    cfg = g.GPTQConfig(bits=wl.bits, group_size=wl.group_size, desc_act=wl.desc_act, damp=wl.damp)
+
+    X = workloads.activations(wl, device=dev, seed_offset=rank)
+    W0 = workloads.weights(wl, device=dev, seed_offset=rank)
+    W = torch.empty_like(W0)
+    H = torch.empty(d, d, dtype=torch.float32, device=dev)
+    U = torch.empty(d, d, dtype=torch.float32, device=dev)
+    perm = torch.empty(d, dtype=torch.int32, device=dev)
+    dead = torch.empty(d, dtype=torch.uint8, device=dev)
+    ng = g.n_groups(d, wl.group_size)
+    codes = torch.empty(r, d, dtype=torch.uint8, device=dev)
+    scales = torch.empty(ng, r, dtype=torch.float32, device=dev)
+    zeros = torch.empty(ng, r, dtype=torch.int32, device=dev)
+    packed = torch.empty(r, g.packed_words(d, wl.bits), dtype=torch.int32, device=dev)
+    ws = torch.empty(g.gptq_workspace_size(cfg, r, d), dtype=torch.uint8, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        H.zero_()
+        g.gptq_hessian_accumulate(X, H, st)
+        if ev is not None:
+            ev[0].record(stream)
+        g.gptq_prepare_hinv(H, cfg, U, perm, dead, st, ws)
+        if ev is not None:
+            ev[1].record(stream)
+        g.gptq_quantize_layer(W, U, perm, dead, cfg, codes, scales, zeros, st, ws)
+        if ev is not None:
+            ev[2].record(stream)
+        g.gptq_pack(codes, wl.bits, packed)
+
+    def between():
+        W.copy_(W0)
+        flush.fill_(1)
+
+    for _ in range(args.warmup):
+        between()
+        step()
+    status = g.gptq_sync_status(st)
+    if status != 0:
+        raise RuntimeError(f"device status {g.STATUS.get(status, status)} during warm-up")
+
+    K = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_h0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_mid = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    clocks = ClockSampler(dev.index)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = g.gptq_launch_counter()
+    clocks.start()
+    for k in range(K):
+        between()
+        ev_s[k].record(stream)
+        H.zero_()
+        ev_h0[k].record(stream)
+        g.gptq_hessian_accumulate(X, H, st)
+        ev_mid[k][0].record(stream)
+        g.gptq_prepare_hinv(H, cfg, U, perm, dead, st, ws)
+        ev_mid[k][1].record(stream)
+        g.gptq_quantize_layer(W, U, perm, dead, cfg, codes, scales, zeros, st, ws)
+        ev_mid[k][2].record(stream)
+        g.gptq_pack(codes, wl.bits, packed)
+        ev_e[k].record(stream)
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    clocks.stop()
+    launches = (g.gptq_launch_counter() - launches0) / K
+    status = g.gptq_sync_status(st)
+    if status != 0:
+        raise RuntimeError(f"device status {g.STATUS.get(status, status)} in the timed steps")
+
+    step_ms = [ev_s[k].elapsed_time(ev_e[k]) for k in range(K)]
+    hess_ms = [ev_h0[k].elapsed_time(ev_mid[k][0]) for k in range(K)]
+    prep_ms = [ev_mid[k][0].elapsed_time(ev_mid[k][1]) for k in range(K)]
+    quant_ms = [ev_mid[k][1].elapsed_time(ev_mid[k][2]) for k in range(K)]
+    pack_ms = [ev_mid[k][2].elapsed_time(ev_e[k]) for k in range(K)]
+    ms = statistics.mean(step_ms)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    # ------------------------------------------------ end to end (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        Xh = torch.empty(X.shape, dtype=X.dtype, pin_memory=True)
+        Xh.copy_(X)
+        Wh = torch.empty(W0.shape, dtype=W0.dtype, pin_memory=True)
+        Wh.copy_(W0)
+        ph = torch.empty(packed.shape, dtype=packed.dtype, pin_memory=True)
+        sh = torch.empty(scales.shape, dtype=scales.dtype, pin_memory=True)
+        zh = torch.empty(zeros.shape, dtype=zeros.dtype, pin_memory=True)
+        Ke = max(2, min(K, 5))
+        e_s = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
+        e_e = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
+        for k in range(Ke):
+            flush.fill_(1)
+            e_s[k].record(stream)
+            X.copy_(Xh, non_blocking=True)
+            W.copy_(Wh, non_blocking=True)
+            step()
+            ph.copy_(packed, non_blocking=True)
+            sh.copy_(scales, non_blocking=True)
+            zh.copy_(zeros, non_blocking=True)
+            e_e[k].record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = statistics.mean(e_s[k].elapsed_time(e_e[k]) for k in range(Ke))
+        te = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+        if dist is not None:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * r * d / (float(te.item()) / 1e3), "unit": "weights/s",
+               "h2d_bytes_per_step": X.numel() * X.element_size() + W0.numel() * 4,
+               "d2h_bytes_per_step": packed.numel() * 4 + scales.numel() * 4 + zeros.numel() * 4,
+               "ms_per_step": float(te.item())}
+
+    if rank != 0:
+        return
+    pk, which = peaks()
+    hess_flops = n * d * (d + 1)
+    h_ms = statistics.mean(hess_ms)
+    achieved = hess_flops / (h_ms / 1e3) / 1e12
+    peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    line = {
+        "metric": METRIC, "value": world * r * d / (ms_max / 1e3), "unit": "weights/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16-in/fp32", "data": "synthetic (seeded; Student-t / half-normal activations "
+                                         "with outlier channels, Gaussian weights)",
+        "config": _config(wl, world),
+        "ms_per_layer": ms_max,
+        "hessian_tflops": achieved,
+        "stage_ms": {"hessian": h_ms, "prepare_hinv": statistics.mean(prep_ms),
+                     "quantize_layer": statistics.mean(quant_ms), "pack": statistics.mean(pack_ms)},
+        "quantize_only_weights_per_s": r * d / ((ms - h_ms) / 1e3),
+        "roofline": {"kernel": "hessian_syrk_tcgen05", "bound": "tensor", "achieved": achieved,
+                     "peak": peak, "peak_source": f"{which} bf16 dense (burst)", "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "algorithmic": f"n*d*(d+1) = {hess_flops:.4e} flop per launch"},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        cb = oracle_sample(wl)
+        line["cpu_baseline"] = {"value": cb["value"], "unit": "weights/s", "cores": cb["cores"],
+                                "kind": "oracle", "sample": cb["sample"]}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        run_ours(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,179 @@
+/*
+ * gptq.h -- C ABI of a B200 (sm_100a) GPTQ layer quantizer.
+ *
+ * The library quantizes one linear layer W (d_row x d_col, columns = the
+ * layer's inputs) with the GPTQ method as the GPTQ pages define it:
+ *
+ *   1. H = 2 X^T X over the calibration activations X (n x d_col), then
+ *      H += lambda I   ("GPTQ (GPT Quantization)", "Algorithme complet
+ *      (pseudo-code)", step 1; lambda = damp * mean(diag H), damp being the
+ *      AutoGPTQ guide's damp_percent, "Quantizar seu proprio modelo").
+ *   2. H^-1 through Cholesky (same pseudo-code, step 2), delivered as the
+ *      upper factor U with H^-1 = U^T U.
+ *   3. The columns are walked in blocks; each column is quantized with its
+ *      group's asymmetric min-max scale and zero point (AutoGPTQ guide,
+ *      "Quantizacao group-wise") and its error is fed to the later columns
+ *      with the OBQ step W_F <- W_F - e_i / (H^-1)_ii * (H^-1)_{i,F}
+ *      ("GPTQ (GPT Quantization)", "Fondation theorique : OBQ"): one column
+ *      at a time inside a block, and as one matrix product per block for the
+ *      remaining columns (the pseudo-code's "lazy update").
+ *   4. Codes are packed into uint32 words, 8 per word at 4 bits ("GPTQ"
+ *      article, "Desempenho e Precisao": 175B parameters at 4 bits, about
+ *      87.5 GB, i.e. half a byte per weight).
+ *
+ * Conventions for every entry point:
+ *   - All sizes are int64_t and all matrices row-major with the stated
+ *     leading dimension (elements, not bytes).
+ *   - Matrix arguments are DEVICE pointers to caller-owned memory; the
+ *     library never allocates or frees device memory and keeps no pointer
+ *     after a call returns.  `ws` is a caller-provided device workspace of at
+ *     least gptq_workspace_size() bytes, 256-byte aligned.
+ *   - Every call is asynchronous on `stream` (0 = legacy default stream).
+ *     Argument errors are returned synchronously before anything is launched.
+ *     Errors detected on the device (a non-positive-definite H, a bounded
+ *     wait that ran out) are written to `*dev_status` (a device int32 that
+ *     the caller zeroes once; the first error written is kept), readable with
+ *     gptq_sync_status() after the work has run.  A nonzero status means the
+ *     outputs of that call are not valid.
+ *   - Calls on the same stream are ordered; calls that share buffers on
+ *     different streams must be ordered by the caller.
+ */
+#ifndef GPTQ_B200_GPTQ_H
+#define GPTQ_B200_GPTQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gptq_status {
+    GPTQ_OK = 0,
+    GPTQ_ERR_INVALID_ARG = 1,  /* a size, pointer, stride or config is invalid   */
+    GPTQ_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. a group size)   */
+    GPTQ_ERR_NOT_PD = 3,       /* damped H is not positive definite (device)      */
+    GPTQ_ERR_TIMEOUT = 4,      /* a bounded device-side wait ran out (device)     */
+    GPTQ_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed     */
+    GPTQ_ERR_WORKSPACE = 6     /* ws is NULL, misaligned or smaller than needed   */
+} gptq_status;
+
+/* Quantizer settings (the AutoGPTQ guide's BaseQuantizeConfig, "Quantizar seu
+ * proprio modelo" and "Configuracoes de quantizacao"). */
+typedef struct gptq_config {
+    int32_t bits;        /* code width: 2, 3, 4 or 8                                  */
+    int32_t group_size;  /* weights per (scale, zero) group along d_col; -1 = one
+                            group per row.  Supported: a divisor of block_size
+                            (e.g. 32, 64, 128), a multiple of block_size (256,
+                            1024, ...), or any value >= d_col.                    */
+    int32_t block_size;  /* columns per lazy-update block; must be 128               */
+    int32_t desc_act;    /* nonzero: quantize columns by descending diag(H)          */
+    float damp;          /* lambda = damp * mean(diag H); the guide's default 0.01   */
+} gptq_config;
+
+/* Human-readable text of a status code (static storage, never NULL). */
+const char *gptq_status_string(int32_t status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int32_t gptq_version(void);
+
+/* Number of CUDA kernels this library has launched in this process since it
+ * was loaded (a host-side counter, for benchmarks and diagnostics). */
+int64_t gptq_launch_counter(void);
+
+/*
+ * Workspace bytes needed by gptq_hessian_accumulate, gptq_prepare_hinv and
+ * gptq_quantize_layer for a layer of d_row x d_col with this config (the
+ * maximum over the three, so one workspace serves all of them).
+ * Errors: GPTQ_ERR_INVALID_ARG for a NULL pointer, nonpositive sizes or an
+ * invalid config; GPTQ_ERR_UNSUPPORTED for a config outside the supported set.
+ */
+gptq_status gptq_workspace_size(const gptq_config *cfg, int64_t d_row, int64_t d_col,
+                                size_t *bytes);
+
+/*
+ * Stage 1 -- H += 2 X^T X  ("GPTQ (GPT Quantization)", pseudo-code step 1,
+ * and the OBQ section's definition H = 2 X^T X).
+ *   X     n x d bf16 (raw bit patterns), row-major, leading dimension ldx:
+ *         ldx >= d, ldx a multiple of 8 and X 16-byte aligned (the tiles are
+ *         fetched by the tensor-memory accelerator).
+ *   H     d x d fp32, leading dimension ldh >= d.  Accumulated into: the
+ *         caller zeroes H before the first chunk and may call repeatedly over
+ *         token chunks.  Only the lower triangle (row >= col) is guaranteed;
+ *         some upper-triangle entries near the diagonal are also written.
+ *   Arithmetic: products of bf16 values are exact; sums are fp32 on the
+ *   tensor cores.  Deterministic (no atomics).
+ *   n == 0 is a no-op.  ws may be NULL (this stage needs none).
+ */
+gptq_status gptq_hessian_accumulate(const uint16_t *X, int64_t n, int64_t d, int64_t ldx,
+                                    float *H, int64_t ldh, int32_t *dev_status,
+                                    void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Stages 1b-2 -- dead columns, act-order, damping, and the inverse factor
+ * ("GPTQ (GPT Quantization)", pseudo-code steps 1-2: H += lambda I,
+ * H_inv = cholesky_inverse(H)).
+ *   H     d x d fp32 (lower triangle read), leading dimension ldh.  Consumed:
+ *         overwritten with scratch.
+ *   U     d x d fp32, contiguous (leading dimension d).  Output: the upper
+ *         triangular U with U^T U = (P^T H P + lambda I)^-1 in quantization
+ *         order (P the act-order permutation); the strictly lower part is 0.
+ *         Row i of U is row i of the OBQ-eliminated inverse divided by the
+ *         square root of its pivot, so e / (H^-1)_ii * (H^-1)_{i,F} =
+ *         (e / U_ii) * U_{i,F}.
+ *   perm  int32[d] output: perm[k] = original column quantized k-th (the
+ *         identity without desc_act; otherwise a stable sort by descending
+ *         diag(H), ties by lower index).
+ *   dead  uint8[d] output: 1 where diag(H) == 0 (that column is treated as
+ *         H_ii = 1 and its weights as 0).
+ *   Device errors: GPTQ_ERR_NOT_PD if a Cholesky pivot is not positive.
+ */
+gptq_status gptq_prepare_hinv(float *H, int64_t d, int64_t ldh, const gptq_config *cfg,
+                              float *U, int32_t *perm, uint8_t *dead, int32_t *dev_status,
+                              void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Stages 3-4 -- the GPTQ column walk with OBQ error feedback.
+ *   W       d_row x d_col fp32, leading dimension ldw, in ORIGINAL column
+ *           order.  Scratch: on return column k holds the weights of original
+ *           column perm[k] as they were when quantized (after the feedback of
+ *           every earlier column).
+ *   U, perm, dead  the outputs of gptq_prepare_hinv for this layer's H (any
+ *           number of layers sharing one H may reuse them).
+ *   codes   d_row x d_col uint8, contiguous: codes[row][k] is the code of
+ *           original column perm[k].
+ *   scales  fp32 [ceil(d_col / g)][d_row] and zeros int32 (same shape),
+ *           group-major, groups in quantization order.  Dequantization:
+ *           W_hat[row][perm[k]] = scales[k/g][row] * (codes[row][k] - zeros[k/g][row]).
+ */
+gptq_status gptq_quantize_layer(float *W, int64_t d_row, int64_t d_col, int64_t ldw,
+                                const float *U, const int32_t *perm, const uint8_t *dead,
+                                const gptq_config *cfg, uint8_t *codes, float *scales,
+                                int32_t *zeros, int32_t *dev_status, void *ws,
+                                size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Stage 5 -- pack codes into each row's little-endian bit stream: code k of a
+ * row occupies bits [bits*k, bits*k + bits) of the row's uint32 words, so at
+ * 4 bits word m holds codes 8m..8m+7 (code 8m+t in bits 4t..4t+3).
+ *   codes   d_row x d_col uint8, contiguous; values must be < 2^bits.
+ *   packed  d_row x ceil(d_col * bits / 32) uint32, contiguous; a row's last
+ *           word is zero-padded past its final code.
+ */
+gptq_status gptq_pack(const uint8_t *codes, int64_t d_row, int64_t d_col, int32_t bits,
+                      uint32_t *packed, cudaStream_t stream);
+
+/*
+ * Waits for `stream`, then copies the device status word to *out.
+ * Returns GPTQ_ERR_CUDA if the wait or the copy fails, else GPTQ_OK (the
+ * device-side status itself is in *out).
+ */
+gptq_status gptq_sync_status(cudaStream_t stream, const int32_t *dev_status, int32_t *out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_B200_GPTQ_H */

@@ -1,0 +1,220 @@
+"""Python binding of the sm_100a GPTQ layer quantizer (libgptq_b200.so).
+
+Argument marshalling only: every function below forwards torch CUDA tensors
+as raw device pointers (and the current CUDA stream) to the C ABI declared in
+``include/gptq.h`` under the same name.  All arithmetic runs in the library's
+CUDA kernels; there is no CPU path.  Importing this package fails loudly when
+the library has not been built (``python
+post_weight_quantization_gptq_b200/build.py``).
+
+Stages (see the header for the exact contracts):
+
+* ``gptq_hessian_accumulate``  H += 2 X^T X            (tcgen05 bf16 GEMM)
+* ``gptq_prepare_hinv``        dead columns, act-order, damping, U = chol-inverse factor
+* ``gptq_quantize_layer``      column walk with OBQ error feedback and lazy updates
+* ``gptq_pack``                codes -> uint32 bit stream (8 codes per word at 4 bits)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "GPTQConfig", "GPTQError", "gptq_hessian_accumulate", "gptq_prepare_hinv",
+    "gptq_quantize_layer", "gptq_pack", "gptq_workspace_size", "gptq_sync_status",
+    "gptq_status_string", "gptq_version", "gptq_launch_counter", "library_path", "n_groups", "packed_words",
+    "STATUS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libgptq_b200.so")
+
+STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID_ARG", 2: "GPTQ_ERR_UNSUPPORTED",
+          3: "GPTQ_ERR_NOT_PD", 4: "GPTQ_ERR_TIMEOUT", 5: "GPTQ_ERR_CUDA",
+          6: "GPTQ_ERR_WORKSPACE"}
+
+
+class GPTQConfig(ctypes.Structure):
+    """Mirror of ``gptq_config``: bits, group_size (-1 = one group per row),
+    block_size (128), desc_act, damp (lambda = damp * mean(diag H))."""
+    _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32),
+                ("block_size", ctypes.c_int32), ("desc_act", ctypes.c_int32),
+                ("damp", ctypes.c_float)]
+
+    def __init__(self, bits=4, group_size=128, desc_act=False, damp=0.01, block_size=128):
+        super().__init__(int(bits), int(group_size), int(block_size), int(bool(desc_act)),
+                         float(damp))
+
+
+class GPTQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {STATUS.get(self.status, self.status)} "
+                         f"({gptq_status_string(self.status)})")
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"{_LIB_PATH} is missing: build the CUDA library first "
+            "(python post_weight_quantization_gptq_b200/build.py)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    cfgp = ctypes.POINTER(GPTQConfig)
+    sig = {
+        "gptq_status_string": ([i32], ctypes.c_char_p),
+        "gptq_version": ([], i32),
+        "gptq_launch_counter": ([], ctypes.c_int64),
+        "gptq_workspace_size": ([cfgp, i64, i64, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
+        "gptq_hessian_accumulate": ([P, i64, i64, i64, P, i64, P, P, ctypes.c_size_t, P],
+                                    ctypes.c_int),
+        "gptq_prepare_hinv": ([P, i64, i64, cfgp, P, P, P, P, P, ctypes.c_size_t, P],
+                              ctypes.c_int),
+        "gptq_quantize_layer": ([P, i64, i64, i64, P, P, P, cfgp, P, P, P, P, P,
+                                 ctypes.c_size_t, P], ctypes.c_int),
+        "gptq_pack": ([P, i64, i64, i32, P, P], ctypes.c_int),
+        "gptq_sync_status": ([P, P, ctypes.POINTER(i32)], ctypes.c_int),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def gptq_status_string(status: int) -> str:
+    return _lib.gptq_status_string(int(status)).decode()
+
+
+def gptq_version() -> int:
+    return int(_lib.gptq_version())
+
+
+def gptq_launch_counter() -> int:
+    """Kernels launched by the library in this process so far."""
+    return int(_lib.gptq_launch_counter())
+
+
+def n_groups(d_col: int, group_size: int) -> int:
+    g = d_col if group_size == -1 or group_size > d_col else group_size
+    return -(-d_col // g)
+
+
+def packed_words(d_col: int, bits: int) -> int:
+    return -(-(d_col * bits) // 32)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise GPTQError(status, where)
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _row_major(t: torch.Tensor, name: str) -> int:
+    """Leading dimension of a 2-D tensor with unit column stride."""
+    if t.dim() != 2 or (t.stride(1) != 1 and t.shape[1] > 1):
+        raise ValueError(f"{name} must be 2-D with contiguous rows")
+    return t.stride(0) if t.shape[0] > 1 else max(t.shape[1], t.stride(0))
+
+
+def gptq_workspace_size(cfg: GPTQConfig, d_row: int, d_col: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(_lib.gptq_workspace_size(ctypes.byref(cfg), int(d_row), int(d_col), ctypes.byref(out)),
+           "gptq_workspace_size")
+    return int(out.value)
+
+
+def gptq_hessian_accumulate(X: torch.Tensor, H: torch.Tensor, dev_status: torch.Tensor | None = None,
+                            ws: torch.Tensor | None = None, stream=None) -> None:
+    """H += 2 X^T X (X: n x d bf16, H: d x d fp32, both CUDA, row-major)."""
+    _cuda(X, "X", torch.bfloat16)
+    _cuda(H, "H", torch.float32)
+    n, d = X.shape
+    ldx = _row_major(X, "X")
+    ldh = _row_major(H, "H")
+    _check(_lib.gptq_hessian_accumulate(_ptr(X), n, d, ldx, _ptr(H), ldh, _ptr(dev_status),
+                                        _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                        _stream(stream)), "gptq_hessian_accumulate")
+
+
+def gptq_prepare_hinv(H: torch.Tensor, cfg: GPTQConfig, U: torch.Tensor, perm: torch.Tensor,
+                      dead: torch.Tensor, dev_status: torch.Tensor | None, ws: torch.Tensor,
+                      stream=None) -> None:
+    """Consumes H (lower triangle); writes U (d x d upper, quantization
+    order), perm (int32) and dead (uint8)."""
+    _cuda(H, "H", torch.float32)
+    _cuda(U, "U", torch.float32)
+    _cuda(perm, "perm", torch.int32)
+    _cuda(dead, "dead", torch.uint8)
+    d = H.shape[0]
+    if not U.is_contiguous() or tuple(U.shape) != (d, d):
+        raise ValueError("U must be a contiguous d x d tensor")
+    _check(_lib.gptq_prepare_hinv(_ptr(H), d, _row_major(H, "H"), ctypes.byref(cfg), _ptr(U),
+                                  _ptr(perm), _ptr(dead), _ptr(dev_status), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream)),
+           "gptq_prepare_hinv")
+
+
+def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, perm: torch.Tensor, dead: torch.Tensor,
+                        cfg: GPTQConfig, codes: torch.Tensor, scales: torch.Tensor,
+                        zeros: torch.Tensor, dev_status: torch.Tensor | None, ws: torch.Tensor,
+                        stream=None) -> None:
+    """W (d_row x d_col fp32, original order; overwritten) -> codes (uint8,
+    quantization order), scales (fp32 [groups][d_row]), zeros (int32)."""
+    _cuda(W, "W", torch.float32)
+    _cuda(codes, "codes", torch.uint8)
+    _cuda(scales, "scales", torch.float32)
+    _cuda(zeros, "zeros", torch.int32)
+    d_row, d_col = W.shape
+    for t, name in ((codes, "codes"), (scales, "scales"), (zeros, "zeros"), (U, "U")):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    _check(_lib.gptq_quantize_layer(_ptr(W), d_row, d_col, _row_major(W, "W"), _ptr(U), _ptr(perm),
+                                    _ptr(dead), ctypes.byref(cfg), _ptr(codes), _ptr(scales),
+                                    _ptr(zeros), _ptr(dev_status), _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream(stream)),
+           "gptq_quantize_layer")
+
+
+def gptq_pack(codes: torch.Tensor, bits: int, packed: torch.Tensor, stream=None) -> None:
+    """codes (d_row x d_col uint8) -> packed (d_row x ceil(d_col*bits/32) int32 view of uint32)."""
+    _cuda(codes, "codes", torch.uint8)
+    _cuda(packed, "packed")
+    if not codes.is_contiguous() or not packed.is_contiguous():
+        raise ValueError("codes and packed must be contiguous")
+    d_row, d_col = codes.shape
+    _check(_lib.gptq_pack(_ptr(codes), d_row, d_col, int(bits), _ptr(packed), _stream(stream)),
+           "gptq_pack")
+
+
+def gptq_sync_status(dev_status: torch.Tensor, stream=None) -> int:
+    """Wait for the stream and return the device status word."""
+    out = ctypes.c_int32(0)
+    _check(_lib.gptq_sync_status(_stream(stream), _ptr(dev_status), ctypes.byref(out)),
+           "gptq_sync_status")
+    return int(out.value)

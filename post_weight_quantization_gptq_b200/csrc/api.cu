@@ -1,0 +1,164 @@
+// C ABI of the GPTQ layer quantizer (declared in include/gptq.h): argument
+// validation, workspace carving and the launch sequence of each stage.
+// Nothing here allocates device memory.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+
+#include "kernels.h"
+
+namespace gptq {
+
+namespace {
+std::atomic<int64_t> g_launches{0};
+}
+
+void count_launches(int64_t k) { g_launches.fetch_add(k, std::memory_order_relaxed); }
+
+int64_t launches() { return g_launches.load(std::memory_order_relaxed); }
+
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+        v = 148;
+    if (dev >= 0 && dev < 64) cache[dev] = v;
+    return v;
+}
+
+}  // namespace gptq
+
+namespace {
+
+constexpr int64_t kMaxDim = (int64_t{1} << 31) - 1;
+constexpr int64_t kMaxQuantCols = 56 * 1024;  // one row of W must fit in shared memory
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+gptq_status check_config(const gptq_config* cfg, int64_t d_col) {
+    if (cfg == nullptr) return GPTQ_ERR_INVALID_ARG;
+    const int b = cfg->bits;
+    if (b != 2 && b != 3 && b != 4 && b != 8) return GPTQ_ERR_INVALID_ARG;
+    if (!(cfg->damp >= 0.f) || !std::isfinite(cfg->damp)) return GPTQ_ERR_INVALID_ARG;
+    const int g = cfg->group_size;
+    if (g == 0 || g < -1) return GPTQ_ERR_INVALID_ARG;
+    if (cfg->block_size != 128) return GPTQ_ERR_UNSUPPORTED;
+    if (g == -1 || g >= d_col) return GPTQ_OK;
+    if (g < cfg->block_size) return (cfg->block_size % g == 0) ? GPTQ_OK : GPTQ_ERR_UNSUPPORTED;
+    return (g % cfg->block_size == 0) ? GPTQ_OK : GPTQ_ERR_UNSUPPORTED;
+}
+
+gptq_status launch_status(gptq_status s) {
+    if (s != GPTQ_OK) return s;
+    return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gptq_status_string(int32_t status) {
+    switch (status) {
+        case GPTQ_OK: return "ok";
+        case GPTQ_ERR_INVALID_ARG: return "invalid argument";
+        case GPTQ_ERR_UNSUPPORTED: return "unsupported configuration";
+        case GPTQ_ERR_NOT_PD: return "damped Hessian is not positive definite";
+        case GPTQ_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+        case GPTQ_ERR_CUDA: return "CUDA runtime error";
+        case GPTQ_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        default: return "unknown status";
+    }
+}
+
+int32_t gptq_version(void) { return 100; }
+
+int64_t gptq_launch_counter(void) { return gptq::launches(); }
+
+gptq_status gptq_workspace_size(const gptq_config* cfg, int64_t d_row, int64_t d_col,
+                                size_t* bytes) {
+    if (bytes == nullptr || d_row <= 0 || d_col <= 0) return GPTQ_ERR_INVALID_ARG;
+    const gptq_status c = check_config(cfg, d_col);
+    if (c != GPTQ_OK) return c;
+    size_t need = gptq::prep_workspace_bytes(d_col);
+    const size_t q = gptq::quant_workspace_bytes(d_row, d_col, cfg->block_size);
+    const size_t ch = gptq::chol_workspace_bytes(d_col);
+    if (q > need) need = q;
+    if (ch > need) need = ch;
+    *bytes = round256(need);
+    return GPTQ_OK;
+}
+
+gptq_status gptq_hessian_accumulate(const uint16_t* X, int64_t n, int64_t d, int64_t ldx,
+                                    float* H, int64_t ldh, int32_t* dev_status, void* ws,
+                                    size_t ws_bytes, cudaStream_t stream) {
+    (void)ws;
+    (void)ws_bytes;
+    if (d <= 0 || d > kMaxDim || n < 0 || n > kMaxDim) return GPTQ_ERR_INVALID_ARG;
+    if (H == nullptr || ldh < d) return GPTQ_ERR_INVALID_ARG;
+    if (n == 0) return GPTQ_OK;
+    if (X == nullptr || ldx < d || (ldx % 8) != 0 || !aligned(X, 16)) return GPTQ_ERR_INVALID_ARG;
+    return launch_status(gptq::launch_hessian(X, n, d, ldx, H, ldh, dev_status, stream));
+}
+
+gptq_status gptq_prepare_hinv(float* H, int64_t d, int64_t ldh, const gptq_config* cfg, float* U,
+                              int32_t* perm, uint8_t* dead, int32_t* dev_status, void* ws,
+                              size_t ws_bytes, cudaStream_t stream) {
+    if (d <= 0 || d > kMaxDim || H == nullptr || ldh < d || U == nullptr || perm == nullptr ||
+        dead == nullptr)
+        return GPTQ_ERR_INVALID_ARG;
+    if (H == U) return GPTQ_ERR_INVALID_ARG;
+    const gptq_status c = check_config(cfg, d);
+    if (c != GPTQ_OK) return c;
+    if (ws == nullptr || !aligned(ws, 256) || ws_bytes < gptq::prep_workspace_bytes(d) ||
+        ws_bytes < gptq::chol_workspace_bytes(d))
+        return GPTQ_ERR_WORKSPACE;
+    gptq_status s =
+        gptq::launch_prep(H, d, ldh, cfg->damp, cfg->desc_act, U, perm, dead, ws, stream);
+    if (s != GPTQ_OK) return s;
+    s = gptq::launch_chol_inverse(U, H, ldh, d, U, dev_status, ws, stream);
+    return launch_status(s);
+}
+
+gptq_status gptq_quantize_layer(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
+                                const float* U, const int32_t* perm, const uint8_t* dead,
+                                const gptq_config* cfg, uint8_t* codes, float* scales,
+                                int32_t* zeros, int32_t* dev_status, void* ws, size_t ws_bytes,
+                                cudaStream_t stream) {
+    if (d_row <= 0 || d_row > kMaxDim || d_col <= 0 || W == nullptr || ldw < d_col ||
+        U == nullptr || perm == nullptr || dead == nullptr || codes == nullptr ||
+        scales == nullptr || zeros == nullptr)
+        return GPTQ_ERR_INVALID_ARG;
+    if (d_col > kMaxQuantCols) return GPTQ_ERR_UNSUPPORTED;
+    const gptq_status c = check_config(cfg, d_col);
+    if (c != GPTQ_OK) return c;
+    if (ws == nullptr || !aligned(ws, 256) ||
+        ws_bytes < gptq::quant_workspace_bytes(d_row, d_col, cfg->block_size))
+        return GPTQ_ERR_WORKSPACE;
+    return launch_status(gptq::launch_quantize(W, d_row, d_col, ldw, U, perm, dead, cfg->bits,
+                                               cfg->group_size, cfg->block_size, codes, scales,
+                                               zeros, dev_status, ws, stream));
+}
+
+gptq_status gptq_pack(const uint8_t* codes, int64_t d_row, int64_t d_col, int32_t bits,
+                      uint32_t* packed, cudaStream_t stream) {
+    if (codes == nullptr || packed == nullptr || d_row <= 0 || d_col <= 0 || d_row > kMaxDim ||
+        d_col > kMaxDim)
+        return GPTQ_ERR_INVALID_ARG;
+    if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return GPTQ_ERR_INVALID_ARG;
+    return launch_status(gptq::launch_pack(codes, d_row, d_col, bits, packed, stream));
+}
+
+gptq_status gptq_sync_status(cudaStream_t stream, const int32_t* dev_status, int32_t* out) {
+    if (dev_status == nullptr || out == nullptr) return GPTQ_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return GPTQ_ERR_CUDA;
+    if (cudaMemcpy(out, dev_status, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
+    return GPTQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,299 @@
+// Stage 1: H += 2 X^T X on the 5th-generation tensor cores.
+//
+// "GPTQ (GPT Quantization)", section "Fondation theorique : OBQ" defines
+// H = 2 X^T X over the calibration inputs X (n tokens x d channels), and the
+// pseudo-code ("Algorithme complet", step 1) computes it before anything
+// else.  H is symmetric, so only tiles that touch the lower triangle are
+// computed.
+//
+// Design (sm_100a):
+//  * Output tile 128 x 256 of D = X[:, m-block]^T X[:, n-block]; tcgen05.mma
+//    kind::f16 with bf16 operands and an fp32 accumulator in tensor memory.
+//  * Both operands are slices of the row-major X, so both are MN-major in
+//    shared memory: a TMA box of 64 channels (128 bytes) x 64 tokens with the
+//    128-byte swizzle is exactly one column of canonical SW128 MN-major atoms.
+//  * Each CTA owns two tiles (both accumulators live in TMEM: 2 x 256 of the
+//    512 columns) and sweeps all tokens for both, interleaving them stage by
+//    stage.  All CTAs sweep the tokens in lockstep, so each token slice of X
+//    is fetched from HBM once and served to every CTA from L2.
+//  * Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs,
+//    warps 2..5 drain the accumulators (TMEM -> registers -> H).
+//  * The epilogue stores D[m][n] into H[n][m]: for a fixed n the 32 lanes of
+//    a warp hold 32 consecutive m, so every store is one coalesced 128-byte
+//    line.  Tiles are chosen with n >= m somewhere inside them, so the
+//    written entries cover H's lower triangle.
+//  * No atomics: every H entry has exactly one owner, so the result is
+//    deterministic.  Every wait is bounded (GPTQ_ERR_TIMEOUT).
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gptq {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int kStages = 4;
+constexpr int kBox = 64;                        // channels per TMA box (128 bytes)
+constexpr int kBoxBytes = kBox * BK * 2;        // 8 KB
+constexpr int kABytes = BM * BK * 2;            // 16 KB
+constexpr int kBBytes = BN * BK * 2;            // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;  // 48 KB
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 512;
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+constexpr uint32_t kIdesc = instr_desc(/*bf16*/ 1, /*A MN*/ 1, /*B MN*/ 1, BM, BN);
+
+struct Barriers {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t acc_full;
+    uint64_t acc_empty;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// Tile t -> (m-block, n-block), n-block major: block nj needs m-blocks
+// 0 .. 2 nj + 1 (those with 128 mi <= 256 nj + 255), clipped to MT.
+__device__ __forceinline__ void tile_coords(int t, int MT, int NT, int& mi, int& nj) {
+    for (nj = 0; nj < NT; ++nj) {
+        const int cnt = min(MT, 2 * nj + 2);
+        if (t < cnt) {
+            mi = t;
+            return;
+        }
+        t -= cnt;
+    }
+    mi = 0;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    hessian_syrk_tcgen05(const __grid_constant__ CUtensorMap tmap_x, float* __restrict__ H,
+                         int64_t ldh, int d, int n, int num_tiles, int32_t* status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    Barriers* bars = reinterpret_cast<Barriers*>(smem + kStages * kStageBytes);
+    volatile int* abort = &bars->abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int MT = (d + BM - 1) / BM;
+    const int NT = (d + BN - 1) / BN;
+    const int KB = (n + BK - 1) / BK;
+    const int G = gridDim.x;
+    const int waves = (num_tiles + 2 * G - 1) / (2 * G);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], 1);
+        }
+        mbar_init(&bars->acc_full, 1);
+        mbar_init(&bars->acc_empty, 128);
+        mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmap_x);
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int w = 0; w < waves && !*abort; ++w) {
+                int tiles[2], ns = 0;
+                for (int s = 0; s < 2; ++s) {
+                    const int t = blockIdx.x + (2 * w + s) * G;
+                    if (t < num_tiles) tiles[ns++] = t;
+                }
+                int m0[2], n0[2];
+                for (int s = 0; s < ns; ++s) {
+                    int mi, nj;
+                    tile_coords(tiles[s], MT, NT, mi, nj);
+                    m0[s] = mi * BM;
+                    n0[s] = nj * BN;
+                }
+                for (int k = 0; k < KB && !*abort; ++k) {
+                    for (int s = 0; s < ns; ++s) {
+                        const uint32_t st = it % kStages;
+                        const uint32_t ph = (it / kStages) & 1u;
+                        if (!mbar_wait(&bars->empty[st], ph ^ 1u, abort)) break;
+                        uint8_t* a = smem + st * kStageBytes;
+                        uint8_t* b = a + kABytes;
+                        mbar_arrive_expect_tx(&bars->full[st], kStageBytes);
+                        const int tok = k * BK;
+#pragma unroll
+                        for (int c = 0; c < BM / kBox; ++c)
+                            tma_load_2d(a + c * kBoxBytes, &tmap_x, &bars->full[st], m0[s] + c * kBox,
+                                        tok);
+#pragma unroll
+                        for (int c = 0; c < BN / kBox; ++c)
+                            tma_load_2d(b + c * kBoxBytes, &tmap_x, &bars->full[st], n0[s] + c * kBox,
+                                        tok);
+                        ++it;
+                    }
+                }
+            }
+            // Never leave with copies in flight: wait for the last issued
+            // stages to land (bounded even when aborting).
+            const uint32_t last = it < (uint32_t)kStages ? it : (uint32_t)kStages;
+            volatile int no_abort = 0;
+            for (uint32_t j = 0; j < last; ++j) {
+                const uint32_t i2 = it - 1 - j;
+                if (!mbar_wait(&bars->full[i2 % kStages], (i2 / kStages) & 1u, &no_abort)) {
+                    *abort = 1;
+                    break;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int w = 0; w < waves && !*abort; ++w) {
+                int ns = 0;
+                for (int s = 0; s < 2; ++s)
+                    if (blockIdx.x + (2 * w + s) * G < num_tiles) ++ns;
+                if (!mbar_wait(&bars->acc_empty, (w & 1) ^ 1, abort)) break;
+                tc_fence_after();
+                bool ok = true;
+                for (int k = 0; k < KB && ok; ++k) {
+                    for (int s = 0; s < ns; ++s) {
+                        const uint32_t st = it % kStages;
+                        const uint32_t ph = (it / kStages) & 1u;
+                        if (!mbar_wait(&bars->full[st], ph, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t a = smem_u32(smem + st * kStageBytes);
+                        const uint32_t b = a + kABytes;
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            // 16 tokens = two 8-row swizzle atoms (2 x 1024 B)
+                            const uint64_t ad = smem_desc(a + kk * 2048, kBoxBytes, 1024, 2);
+                            const uint64_t bd = smem_desc(b + kk * 2048, kBoxBytes, 1024, 2);
+                            mma_f16_ss(tmem + s * BN, ad, bd, kIdesc, (k > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit(&bars->empty[st]);
+                        ++it;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&bars->acc_full);
+            }
+            // Drain: every MMA issued by this thread has finished before the
+            // tensor memory is released.
+            mma_commit(&bars->drain);
+            volatile int no_abort = 0;
+            if (!mbar_wait(&bars->drain, 0, &no_abort)) *abort = 1;
+        }
+    } else {
+        // ------------------------------------------------ epilogue warps 2..5
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        for (int w = 0; w < waves && !*abort; ++w) {
+            if (!mbar_wait(&bars->acc_full, w & 1, abort)) break;
+            tc_fence_after();
+            for (int s = 0; s < 2; ++s) {
+                const int t = blockIdx.x + (2 * w + s) * G;
+                if (t >= num_tiles) break;
+                int mi, nj;
+                tile_coords(t, MT, NT, mi, nj);
+                const int m = mi * BM + q * 32 + lane;
+                const int nb = nj * BN;
+#pragma unroll 1
+                for (int cc = 0; cc < BN / 32; ++cc) {
+                    float v[32];
+                    tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + s * BN + cc * 32, v);
+                    if (m < d) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int nn = nb + cc * 32 + j;
+                            if (nn < d) {
+                                float* p = H + static_cast<int64_t>(nn) * ldh + m;
+                                *p = *p + 2.0f * v[j];
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bars->acc_empty);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+    if (threadIdx.x == 0 && bars->abort) report(status, GPTQ_ERR_TIMEOUT);
+}
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled get_encode() {
+    static EncodeTiled fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(p);
+    }
+    return fn;
+}
+
+}  // namespace
+
+int hessian_num_tiles(int64_t d) {
+    const int MT = static_cast<int>((d + BM - 1) / BM);
+    const int NT = static_cast<int>((d + BN - 1) / BN);
+    int t = 0;
+    for (int nj = 0; nj < NT; ++nj) t += (MT < 2 * nj + 2) ? MT : 2 * nj + 2;
+    return t;
+}
+
+gptq_status launch_hessian(const uint16_t* X, int64_t n, int64_t d, int64_t ldx, float* H,
+                           int64_t ldh, int32_t* status, cudaStream_t stream) {
+    if (cudaFuncSetAttribute(hessian_syrk_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
+    EncodeTiled encode = get_encode();
+    if (encode == nullptr) return GPTQ_ERR_CUDA;
+    CUtensorMap tmap;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldx) * 2u};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBox), static_cast<cuuint32_t>(BK)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return GPTQ_ERR_INVALID_ARG;
+    const int T = hessian_num_tiles(d);
+    const int sms = num_sms();
+    int grid = (T + 1) / 2;
+    if (grid > sms) grid = sms;
+    hessian_syrk_tcgen05<<<grid, kThreads, kSmemBytes, stream>>>(
+        tmap, H, ldh, static_cast<int>(d), static_cast<int>(n), T, status);
+    count_launches(1);
+    return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
+
+}  // namespace gptq

@@ -1,0 +1,46 @@
+// Internal launchers of the GPTQ kernels (one per stage), called by the
+// C-ABI layer in api.cu after it has validated every argument.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/gptq.h"
+
+namespace gptq {
+
+// Streaming multiprocessors of the current device (cached per device).
+int num_sms();
+
+// Host-side count of kernels this library has launched (diagnostics).
+void count_launches(int64_t k);
+int64_t launches();
+
+// ---- stage 1 (hessian.cu)
+int hessian_num_tiles(int64_t d);
+gptq_status launch_hessian(const uint16_t* X, int64_t n, int64_t d, int64_t ldx, float* H,
+                           int64_t ldh, int32_t* status, cudaStream_t stream);
+
+// ---- stage 2 (prep.cu): dead columns, lambda, act-order, flipped working copy
+size_t prep_workspace_bytes(int64_t d);
+gptq_status launch_prep(const float* H, int64_t d, int64_t ldh, float damp, int desc_act,
+                        float* P, int32_t* perm, uint8_t* dead, void* ws, cudaStream_t stream);
+
+// ---- stage 2 (chol.cu): P = L L^T in place, X = L^-1, U = J X J
+size_t chol_workspace_bytes(int64_t d);
+gptq_status launch_chol_inverse(float* P, float* Xbuf, int64_t ldx, int64_t d, float* U,
+                                int32_t* status, void* ws, cudaStream_t stream);
+
+// ---- stages 3-4 (quant.cu)
+size_t quant_workspace_bytes(int64_t d_row, int64_t d_col, int block);
+gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw, const float* U,
+                            const int32_t* perm, const uint8_t* dead, int bits, int group,
+                            int block, uint8_t* codes, float* scales, int32_t* zeros,
+                            int32_t* status, void* ws, cudaStream_t stream);
+
+// ---- stage 5 (pack.cu)
+gptq_status launch_pack(const uint8_t* codes, int64_t d_row, int64_t d_col, int bits,
+                        uint32_t* packed, cudaStream_t stream);
+
+}  // namespace gptq

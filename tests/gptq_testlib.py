@@ -1,0 +1,131 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the
+C-ABI binding, run the oracle on the same inputs, and compare.
+
+Comparison rules (tolerances from the method's statement of parity and the
+fp32 arithmetic of the kernels):
+
+* H: relative Frobenius error <= 1e-3 (products of bf16 are exact; the GPU
+  sums in fp32, the oracle in fp64).
+* perm, dead, packed words: bit-exact.
+* codes / zero points: a float decides each of them, and the GPU carries its
+  weights in fp32 while the oracle carries them in fp64, so a weight that
+  sits on a rounding boundary may legitimately round either way.  Each GPU
+  code is therefore checked for validity by the oracle's column loop run in
+  teacher-forcing mode: it must be the oracle's own rounding, or the other
+  neighbour of a boundary that lies within |w_gpu - w_oracle| / s + tau of
+  the oracle's value (w_gpu is the GPU's pre-quantization weight, returned
+  in W).  At most 0.1 % of the codes may take such a tie the other way
+  (>= 99.9 % identical) and none may be invalid.
+* scales: relative error <= 1e-4 against the teacher-forced oracle.
+* proxy loss tr((W - Q) H (W - Q)^T): within 0.5 % of the free-running
+  oracle's.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+
+TAU = 1e-5  # levels: rounding of the GPU's w * (1 / s) product
+
+
+def gpu():
+    import post_weight_quantization_gptq_b200 as g
+    return g
+
+
+def gpu_hessian(X_cpu: torch.Tensor, chunks: int = 1, ldx: int | None = None) -> np.ndarray:
+    g = gpu()
+    n, d = X_cpu.shape
+    ld = ldx or d
+    Xs = torch.zeros(n, ld, dtype=torch.bfloat16)
+    Xs[:, :d] = X_cpu
+    Xd = Xs.cuda()[:, :d]
+    H = torch.zeros(d, d, dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bounds = np.linspace(0, n, chunks + 1).astype(int)
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        g.gptq_hessian_accumulate(Xd[a:b], H, st)
+    assert g.gptq_sync_status(st) == 0
+    return H.cpu().numpy()
+
+
+def lower_rel_err(Hg: np.ndarray, Ho: np.ndarray) -> float:
+    L = np.tril(np.ones_like(Ho, dtype=bool))
+    return float(np.linalg.norm((Hg - Ho)[L]) / np.linalg.norm(Ho[L]))
+
+
+def gpu_quantize(H_fp32: np.ndarray, W: torch.Tensor, bits: int, group_size: int,
+                 desc_act: bool, damp: float = 0.01) -> dict:
+    """prepare_hinv + quantize_layer + pack on the GPU from a given H."""
+    g = gpu()
+    d_row, d_col = W.shape
+    cfg = g.GPTQConfig(bits=bits, group_size=group_size, desc_act=desc_act, damp=damp)
+    ws = torch.empty(g.gptq_workspace_size(cfg, d_row, d_col), dtype=torch.uint8, device="cuda")
+    Hd = torch.from_numpy(np.ascontiguousarray(H_fp32, dtype=np.float32)).cuda()
+    U = torch.empty(d_col, d_col, dtype=torch.float32, device="cuda")
+    perm = torch.empty(d_col, dtype=torch.int32, device="cuda")
+    dead = torch.empty(d_col, dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g.gptq_prepare_hinv(Hd, cfg, U, perm, dead, st, ws)
+    Wd = W.to(torch.float32).cuda().contiguous()
+    ng = g.n_groups(d_col, group_size)
+    codes = torch.empty(d_row, d_col, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(ng, d_row, dtype=torch.float32, device="cuda")
+    zeros = torch.empty(ng, d_row, dtype=torch.int32, device="cuda")
+    g.gptq_quantize_layer(Wd, U, perm, dead, cfg, codes, scales, zeros, st, ws)
+    packed = torch.empty(d_row, g.packed_words(d_col, bits), dtype=torch.int32, device="cuda")
+    g.gptq_pack(codes, bits, packed)
+    status = g.gptq_sync_status(st)
+    return dict(status=status, U=U.cpu().numpy().astype(np.float64), perm=perm.cpu().numpy(),
+                dead=dead.cpu().numpy().astype(bool), codes=codes.cpu().numpy(),
+                scales=scales.cpu().numpy(), zeros=zeros.cpu().numpy(),
+                w_at_quant=Wd.cpu().numpy(), packed=packed.cpu().numpy().view(np.uint32))
+
+
+def compare_quantization(H64: np.ndarray, W: torch.Tensor, out: dict, bits: int,
+                         group_size: int, desc_act: bool, damp: float = 0.01,
+                         rows=None, H_loss: np.ndarray | None = None) -> dict:
+    """Check one GPU quantization against the oracle run on H64 (the exact H
+    the GPU was given, as float64).  `rows` restricts the column loop to a
+    sample of rows.  Returns the measured statistics."""
+    prep = oracle.prepare(H64, W, damp=damp, desc_act=desc_act)
+    assert out["status"] == 0, out["status"]
+    assert np.array_equal(out["perm"], prep["perm"]), "act-order permutation differs"
+    assert np.array_equal(out["dead"], prep["dead"]), "dead-column mask differs"
+    sel = np.arange(W.shape[0]) if rows is None else np.asarray(rows)
+    Minv = oracle.inverse(prep["H_damped"])
+    W0 = prep["W0"][sel]
+    codes, zeros = out["codes"][sel], out["zeros"][:, sel]
+    wq, scales = out["w_at_quant"][sel], out["scales"][:, sel]
+    forced = oracle.gptq_columns(W0, Minv, bits, group_size, forced_codes=codes,
+                                 forced_zeros=zeros, forced_w=wq, tau=TAU)
+    st = forced.stats
+    free = oracle.gptq_columns(W0, Minv, bits, group_size)
+    free_match = float(np.mean(free.codes == codes))
+    free_maxdiff = int(np.abs(free.codes.astype(int) - codes.astype(int)).max())
+    srel = float(np.max(np.abs(scales - forced.scales) / np.abs(forced.scales)))
+    Hl = prep["H_undamped"] if H_loss is None else H_loss
+    Qg = oracle.dequantize(codes, scales, zeros, group_size)
+    Qo = oracle.dequantize(free.codes, free.scales, free.zeros, group_size)
+    loss_g = oracle.proxy_loss(W0, Qg, Hl)
+    loss_o = oracle.proxy_loss(W0, Qo, Hl)
+    rc, rs, rz = oracle.rtn(W0, bits, group_size)
+    loss_rtn = oracle.proxy_loss(W0, oracle.dequantize(rc, rs, rz, group_size), Hl)
+    res = dict(code_ties=st["code_ties"], code_invalid=st["code_invalid"],
+               zero_ties=st["zero_ties"], zero_invalid=st["zero_invalid"],
+               elements=st["elements"], tie_frac=st["code_ties"] / max(1, st["elements"]),
+               max_dev=st["max_dev"], scale_rel=srel, free_match=free_match,
+               free_maxdiff=free_maxdiff, loss_gpu=loss_g, loss_oracle=loss_o,
+               loss_rtn=loss_rtn, loss_rel=abs(loss_g - loss_o) / loss_o)
+    print("parity:", {k: (round(v, 8) if isinstance(v, float) else v) for k, v in res.items()})
+    assert st["code_invalid"] == 0, res
+    assert st["zero_invalid"] == 0, res
+    assert res["tie_frac"] <= 1e-3, res
+    assert srel <= 1e-4, res
+    assert res["max_dev"] <= 0.05, res
+    assert res["loss_rel"] <= 5e-3, res
+    assert codes.max() <= (1 << bits) - 1
+    assert np.array_equal(out["packed"][sel], oracle.pack(codes, bits))
+    return res

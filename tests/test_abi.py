@@ -1,0 +1,103 @@
+"""The C-ABI library loads and exports every entry point include/gptq.h
+declares; host-side argument validation answers before anything is launched
+(no GPU needed for any call made here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gptq.h")
+
+
+@pytest.fixture(scope="module")
+def pkg():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "gptq_b200_build", os.path.join(ROOT, "post_weight_quantization_gptq_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import post_weight_quantization_gptq_b200 as p
+    return p
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gptq_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_four_stages():
+    names = _declared()
+    for n in ("gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer", "gptq_pack",
+              "gptq_workspace_size", "gptq_sync_status", "gptq_status_string", "gptq_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(pkg):
+    lib = ctypes.CDLL(pkg.library_path())
+    for name in _declared():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", pkg.library_path()],
+                         capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (gptq_[a-z_]+)\b", out))
+    assert set(_declared()) <= exported
+
+
+def test_library_is_built_for_sm_100a(pkg):
+    out = subprocess.run(["cuobjdump", "--list-elf", pkg.library_path()],
+                         capture_output=True, text=True)
+    if out.returncode != 0:
+        pytest.skip("cuobjdump unavailable")
+    assert "sm_100a" in out.stdout
+
+
+def test_status_strings_and_version(pkg):
+    assert pkg.gptq_version() >= 100
+    assert pkg.gptq_status_string(0) == "ok"
+    assert "positive definite" in pkg.gptq_status_string(3)
+    assert pkg.gptq_status_string(99) == "unknown status"
+
+
+def test_workspace_size_and_config_validation(pkg):
+    cfg = pkg.GPTQConfig(bits=4, group_size=128)
+    b = pkg.gptq_workspace_size(cfg, 4096, 4096)
+    assert b >= 4096 * 128 * 4 and b % 256 == 0
+    for bad in (dict(bits=5), dict(group_size=0), dict(group_size=-2), dict(damp=-1.0)):
+        kw = dict(bits=4, group_size=128, damp=0.01)
+        kw.update(bad)
+        with pytest.raises(pkg.GPTQError) as e:
+            pkg.gptq_workspace_size(pkg.GPTQConfig(**kw), 64, 256)
+        assert e.value.status == 1
+    for unsup in (dict(group_size=48), dict(group_size=192), dict(block_size=64)):
+        kw = dict(bits=4, group_size=128)
+        kw.update(unsup)
+        with pytest.raises(pkg.GPTQError) as e:
+            pkg.gptq_workspace_size(pkg.GPTQConfig(**kw), 64, 1024)
+        assert e.value.status == 2
+    # group sizes the column walk supports
+    for g in (1, 16, 32, 64, 128, 256, 1024, -1, 5000):
+        pkg.gptq_workspace_size(pkg.GPTQConfig(bits=4, group_size=g), 8, 4096)
+
+
+def test_invalid_arguments_are_rejected_on_the_host(pkg):
+    lib = ctypes.CDLL(pkg.library_path())
+    lib.gptq_hessian_accumulate.restype = ctypes.c_int
+    lib.gptq_pack.restype = ctypes.c_int
+    P, i64 = ctypes.c_void_p, ctypes.c_int64
+    lib.gptq_hessian_accumulate.argtypes = [P, i64, i64, i64, P, i64, P, P, ctypes.c_size_t, P]
+    lib.gptq_pack.argtypes = [P, i64, i64, ctypes.c_int32, P, P]
+    fake = ctypes.c_void_p(1 << 20)
+    # d = 0, H NULL, ldx not a multiple of 8, misaligned X: all rejected before any launch
+    assert lib.gptq_hessian_accumulate(fake, 16, 0, 16, fake, 16, None, None, 0, None) == 1
+    assert lib.gptq_hessian_accumulate(fake, 16, 16, 16, None, 16, None, None, 0, None) == 1
+    assert lib.gptq_hessian_accumulate(fake, 16, 12, 12, fake, 12, None, None, 0, None) == 1
+    assert lib.gptq_hessian_accumulate(ctypes.c_void_p((1 << 20) + 2), 16, 16, 16, fake, 16,
+                                       None, None, 0, None) == 1
+    # n == 0 is a no-op that succeeds
+    assert lib.gptq_hessian_accumulate(fake, 0, 16, 16, fake, 16, None, None, 0, None) == 0
+    assert lib.gptq_pack(fake, 4, 8, 5, fake, None) == 1
+    assert lib.gptq_pack(None, 4, 8, 4, fake, None) == 1

@@ -1,0 +1,175 @@
+"""GPU parity of every stage against the float64 oracle, through the C ABI.
+
+Sizes span several tiles and ragged tails; the tiny workload (256 x 512,
+2048 tokens) runs in full.  See gptq_testlib for the comparison rules.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from gptq_testlib import compare_quantization, gpu, gpu_hessian, gpu_quantize, lower_rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+# ------------------------------------------------------------------ stage 1
+@pytest.mark.parametrize("n,d,kind", [(2048, 512, "correlated"), (1000, 200, "student_t"),
+                                      (63, 72, "student_t"), (1, 8, "student_t"),
+                                      (4100, 520, "half_normal"), (777, 384, "student_t"),
+                                      (3000, 1040, "student_t")])
+def test_hessian_matches_oracle(n, d, kind):
+    _, X = workloads.small_layer(4, d, n, seed=n + d, kind=kind)
+    Hg = gpu_hessian(X)
+    Ho = oracle.hessian(X)
+    err = lower_rel_err(Hg, Ho)
+    print(f"H rel Frobenius error {err:.3e}")
+    assert err <= 1e-3
+    # elementwise: fp32 summation of exact products
+    L = np.tril(np.ones_like(Ho, dtype=bool))
+    scale = np.sqrt(np.outer(np.diag(Ho), np.diag(Ho)))[L] + 1e-30
+    assert np.max(np.abs(Hg - Ho)[L] / scale) <= 1e-4
+
+
+def test_hessian_tiny_workload_and_strided_x():
+    w = workloads.WORKLOADS["tiny"]
+    X = workloads.activations(w)
+    Ho = oracle.hessian(X)
+    assert lower_rel_err(gpu_hessian(X), Ho) <= 1e-5
+    assert lower_rel_err(gpu_hessian(X, ldx=520), Ho) <= 1e-5
+
+
+def test_hessian_accumulates_over_token_chunks():
+    _, X = workloads.small_layer(4, 256, 3000, seed=11)
+    one = gpu_hessian(X)
+    three = gpu_hessian(X, chunks=3)
+    L = np.tril(np.ones_like(one, dtype=bool))
+    assert np.max(np.abs(one - three)[L]) <= 1e-5 * np.max(np.abs(one))
+    assert lower_rel_err(three, oracle.hessian(X)) <= 1e-5
+
+
+# ------------------------------------------------------------------ stage 2
+@pytest.mark.parametrize("d,desc_act,n_dead", [(512, False, 0), (512, True, 0), (200, True, 3),
+                                               (130, False, 2), (1024, True, 0), (64, False, 0)])
+def test_prepare_hinv_matches_oracle_elimination(d, desc_act, n_dead):
+    rng = np.random.default_rng(d + n_dead)
+    _, X = workloads.small_layer(4, d, 4 * d, seed=d, kind="correlated")
+    Xf = X.to(torch.float32)
+    dead_idx = rng.choice(d, size=n_dead, replace=False)
+    Xf[:, dead_idx] = 0.0
+    H = oracle.hessian(Xf.to(torch.bfloat16)).astype(np.float32)
+    W = workloads.gaussian_weights(8, d, 0.02, seed=1)
+    out = gpu_quantize(H, W, 4, 128 if d % 128 == 0 else -1, desc_act)
+    assert out["status"] == 0
+    prep = oracle.prepare(H.astype(np.float64), W, damp=0.01, desc_act=desc_act)
+    assert np.array_equal(out["perm"], prep["perm"])
+    assert np.array_equal(out["dead"], prep["dead"])
+    _, Uo = oracle.eliminate(oracle.inverse(prep["H_damped"]))
+    Ug = out["U"]
+    rel = np.max(np.abs(Ug - Uo)) / np.max(np.abs(Uo))
+    cond = np.linalg.cond(prep["H_damped"])
+    print(f"d={d} cond={cond:.2e} U max rel err {rel:.3e}")
+    assert np.all(np.tril(Ug, -1) == 0.0)
+    assert rel <= 2e-3
+    # U^T U Hd = I (a property of the output at any size)
+    resid = np.max(np.abs(Ug.T @ (Ug @ prep["H_damped"]) - np.eye(d)))
+    assert resid <= 5e-2
+
+
+def test_not_positive_definite_is_reported():
+    g = gpu()
+    d = 96
+    cfg = g.GPTQConfig(bits=4, group_size=32, damp=0.0)
+    H = -torch.eye(d, dtype=torch.float32, device="cuda")
+    ws = torch.empty(g.gptq_workspace_size(cfg, 4, d), dtype=torch.uint8, device="cuda")
+    U = torch.empty(d, d, device="cuda")
+    perm = torch.empty(d, dtype=torch.int32, device="cuda")
+    dead = torch.empty(d, dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g.gptq_prepare_hinv(H, cfg, U, perm, dead, st, ws)
+    assert g.gptq_sync_status(st) == 3
+    assert torch.isfinite(U).all()
+
+
+# ------------------------------------------------------------ stages 3 + 4
+QUANT_CASES = [
+    # d_row, d_col, tokens, kind, bits, group, desc_act
+    (256, 512, 2048, "correlated", 4, 128, False),
+    (256, 512, 2048, "correlated", 4, 32, True),
+    (64, 384, 2048, "student_t", 3, 128, False),
+    (40, 256, 1024, "half_normal", 2, 64, True),
+    (33, 512, 2048, "student_t", 4, -1, False),
+    (16, 512, 2048, "student_t", 4, 256, True),
+    (7, 200, 800, "student_t", 4, 8, False),
+    (5, 130, 700, "correlated", 8, 128, True),
+    (1, 64, 256, "student_t", 4, 32, False),
+    (300, 1024, 4096, "student_t", 4, 128, True),
+]
+
+
+@pytest.mark.parametrize("d_row,d_col,n,kind,bits,g,desc_act", QUANT_CASES)
+def test_quantize_layer_matches_oracle(d_row, d_col, n, kind, bits, g, desc_act):
+    W, X = workloads.small_layer(d_row, d_col, n, seed=d_row * 7 + d_col, kind=kind)
+    H = oracle.hessian(X).astype(np.float32)
+    out = gpu_quantize(H, W, bits, g, desc_act)
+    compare_quantization(H.astype(np.float64), W, out, bits, g, desc_act)
+
+
+def test_dead_columns_are_zero_weight():
+    W, X = workloads.small_layer(24, 256, 1024, seed=5)
+    Xf = X.to(torch.float32)
+    Xf[:, [3, 100, 255]] = 0.0
+    H = oracle.hessian(Xf.to(torch.bfloat16)).astype(np.float32)
+    out = gpu_quantize(H, W, 4, 128, True)
+    compare_quantization(H.astype(np.float64), W, out, 4, 128, True)
+    pos = np.nonzero(np.isin(out["perm"], [3, 100, 255]))[0]
+    Q = oracle.dequantize(out["codes"], out["scales"], out["zeros"], 128)
+    assert np.all(Q[:, pos] == 0.0)
+
+
+def test_identity_hessian_gives_round_to_nearest():
+    d = 256
+    W = workloads.gaussian_weights(32, d, 0.03, seed=2)
+    H = (5.0 * np.eye(d)).astype(np.float32)
+    out = gpu_quantize(H, W, 4, 64, False)
+    rc, rs, rz = oracle.rtn(W.numpy().astype(np.float64), 4, 64)
+    assert np.array_equal(out["codes"], rc)
+    assert np.array_equal(out["zeros"], rz)
+    assert np.max(np.abs(out["scales"] - rs) / rs) <= 1e-6
+
+
+def test_end_to_end_tiny_workload_from_activations():
+    """X -> H (GPU) -> U -> codes -> packed, checked against the oracle run
+    from the same X (its own float64 H)."""
+    w = workloads.WORKLOADS["tiny"]
+    W, X = workloads.weights(w), workloads.activations(w)
+    g = gpu()
+    cfg = g.GPTQConfig(bits=w.bits, group_size=w.group_size, desc_act=w.desc_act, damp=w.damp)
+    Hg = gpu_hessian(X)
+    Ho = oracle.hessian(X)
+    assert lower_rel_err(Hg, Ho) <= 1e-3
+    out = gpu_quantize(np.tril(Hg), W, w.bits, w.group_size, w.desc_act, w.damp)
+    res = compare_quantization(Ho, W, out, w.bits, w.group_size, w.desc_act, w.damp)
+    assert res["loss_gpu"] < res["loss_rtn"]
+    del cfg
+
+
+# ------------------------------------------------------------------ stage 5
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("d", [8, 64, 100, 4096])
+def test_pack_is_bit_exact(bits, d):
+    g = gpu()
+    rng = np.random.default_rng(bits * d)
+    c = rng.integers(0, 1 << bits, size=(37, d), dtype=np.uint8)
+    cd = torch.from_numpy(c).cuda()
+    packed = torch.empty(37, g.packed_words(d, bits), dtype=torch.int32, device="cuda")
+    g.gptq_pack(cd, bits, packed)
+    torch.cuda.synchronize()
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), oracle.pack(c, bits))
