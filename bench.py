@@ -17,6 +17,7 @@ Prints one JSON line (rank 0).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -44,6 +45,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="llama7b_q_proj")
+    p.add_argument("--tokens", type=int, default=None,
+                   help="override the calibration token count (profiling of a smaller case)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args()
@@ -189,6 +192,8 @@ def run_ours(args, rank: int, world: int, dist):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     wl = workloads.WORKLOADS[args.workload]
+    if args.tokens:
+        wl = dataclasses.replace(wl, n_tokens=args.tokens)
     r, d, n = wl.d_row, wl.d_col, wl.n_tokens
     cfg = g.GPTQConfig(bits=wl.bits, group_size=wl.group_size, desc_act=wl.desc_act, damp=wl.damp)
 

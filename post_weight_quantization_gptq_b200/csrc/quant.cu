@@ -89,6 +89,14 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
 
     float s = 1.f, inv_s = 1.f, zf = 0.f;
+    if (live && (c0 % g) != 0) {
+        // this block continues a group opened by an earlier block (group
+        // size > block): take that group's scale and zero point
+        const int64_t grp = c0 / g;
+        s = scales[grp * r + row];
+        zf = static_cast<float>(zeros[grp * r + row]);
+        inv_s = 1.f / s;
+    }
 #pragma unroll
     for (int j = 0; j < kBlock; ++j) {
         if (j < bw) {
