@@ -155,6 +155,36 @@ gptq_status gptq_quantize_layer(float *W, int64_t d_row, int64_t d_col, int64_t 
                                 size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * gptq_quantize_layer without a workspace argument.  The GPTQ pages have no
+ * counterpart to this entry point: it is a packaging variant of stages 3-4
+ * for callers that cannot allocate device memory -- a plugin or operator
+ * interface whose enqueue call may not allocate, a process whose memory pool
+ * has already reserved nearly all of HBM, or a latency-critical path that
+ * cannot afford cudaMalloc / cudaFree (both can synchronize the device).
+ *   Arguments and results: exactly those of gptq_quantize_layer, minus ws /
+ *   ws_bytes.  The scratch is one fixed device array inside this library of
+ *   gptq_noalloc_scratch_bytes() bytes (16 MiB) per device, held by every GPU
+ *   that loads the library until the process exits; no allocation is made.
+ *   Limit: a layer whose gptq_quantize_layer workspace would exceed that
+ *   array (currently d_row * 512 bytes, i.e. d_row <= 32768) is rejected with
+ *   GPTQ_ERR_WORKSPACE before anything is launched.
+ *   Set-up: the first call on each device (with that device current) looks
+ *   up the array's device address and caches it; make that first call before
+ *   any stream capture on the device.
+ *   Sharing: every call uses the same array, which keeps the last call's
+ *   contents; nothing in it needs to start at zero.  Calls whose work overlaps
+ *   on the GPU (e.g. on two unordered streams) race on the array: order them.
+ */
+gptq_status gptq_quantize_layer_noalloc(float *W, int64_t d_row, int64_t d_col, int64_t ldw,
+                                        const float *U, const int32_t *perm,
+                                        const uint8_t *dead, const gptq_config *cfg,
+                                        uint8_t *codes, float *scales, int32_t *zeros,
+                                        int32_t *dev_status, cudaStream_t stream);
+
+/* Bytes of the fixed scratch array used by gptq_quantize_layer_noalloc. */
+size_t gptq_noalloc_scratch_bytes(void);
+
+/*
  * Stage 5 -- pack codes into each row's little-endian bit stream: code k of a
  * row occupies bits [bits*k, bits*k + bits) of the row's uint32 words, so at
  * 4 bits word m holds codes 8m..8m+7 (code 8m+t in bits 4t..4t+3).

@@ -23,7 +23,7 @@ import torch
 
 __all__ = [
     "GPTQConfig", "GPTQError", "gptq_hessian_accumulate", "gptq_prepare_hinv",
-    "gptq_quantize_layer", "gptq_pack", "gptq_workspace_size", "gptq_sync_status",
+    "gptq_quantize_layer", "gptq_quantize_layer_noalloc", "gptq_noalloc_scratch_bytes", "gptq_pack", "gptq_workspace_size", "gptq_sync_status",
     "gptq_status_string", "gptq_version", "gptq_launch_counter", "library_path", "n_groups", "packed_words",
     "STATUS",
 ]
@@ -75,6 +75,9 @@ def _load():
         "gptq_quantize_layer": ([P, i64, i64, i64, P, P, P, cfgp, P, P, P, P, P,
                                  ctypes.c_size_t, P], ctypes.c_int),
         "gptq_pack": ([P, i64, i64, i32, P, P], ctypes.c_int),
+        "gptq_quantize_layer_noalloc": ([P, i64, i64, i64, P, P, P, cfgp, P, P, P, P, P],
+                                        ctypes.c_int),
+        "gptq_noalloc_scratch_bytes": ([], ctypes.c_size_t),
         "gptq_sync_status": ([P, P, ctypes.POINTER(i32)], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
@@ -199,6 +202,35 @@ def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, perm: torch.Tensor, de
                                     _ptr(zeros), _ptr(dev_status), _ptr(ws),
                                     ws.numel() * ws.element_size(), _stream(stream)),
            "gptq_quantize_layer")
+
+
+def gptq_quantize_layer_noalloc(W: torch.Tensor, U: torch.Tensor, perm: torch.Tensor,
+                                dead: torch.Tensor, cfg: GPTQConfig, codes: torch.Tensor,
+                                scales: torch.Tensor, zeros: torch.Tensor,
+                                dev_status: torch.Tensor | None, stream=None) -> None:
+    """gptq_quantize_layer without a workspace, for callers that cannot
+    allocate device memory (an enqueue call that may not allocate, a memory
+    pool that already holds nearly all of HBM, a path that cannot afford the
+    device synchronization of cudaMalloc / cudaFree).  The scratch is a fixed
+    array inside the library (gptq_noalloc_scratch_bytes() per device), shared
+    by every call: calls that overlap on the GPU race on it."""
+    _cuda(W, "W", torch.float32)
+    _cuda(codes, "codes", torch.uint8)
+    _cuda(scales, "scales", torch.float32)
+    _cuda(zeros, "zeros", torch.int32)
+    d_row, d_col = W.shape
+    for t, name in ((codes, "codes"), (scales, "scales"), (zeros, "zeros"), (U, "U")):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    _check(_lib.gptq_quantize_layer_noalloc(_ptr(W), d_row, d_col, _row_major(W, "W"), _ptr(U),
+                                            _ptr(perm), _ptr(dead), ctypes.byref(cfg),
+                                            _ptr(codes), _ptr(scales), _ptr(zeros),
+                                            _ptr(dev_status), _stream(stream)),
+           "gptq_quantize_layer_noalloc")
+
+
+def gptq_noalloc_scratch_bytes() -> int:
+    return int(_lib.gptq_noalloc_scratch_bytes())
 
 
 def gptq_pack(codes: torch.Tensor, bits: int, packed: torch.Tensor, stream=None) -> None:
