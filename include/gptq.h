@@ -116,7 +116,9 @@ gptq_status gptq_hessian_accumulate(const uint16_t *X, int64_t n, int64_t d, int
  * ("GPTQ (GPT Quantization)", pseudo-code steps 1-2: H += lambda I,
  * H_inv = cholesky_inverse(H)).
  *   H     d x d fp32 (lower triangle read), leading dimension ldh.  Consumed:
- *         overwritten with scratch.
+ *         overwritten with scratch.  d and ldh must be multiples of 4 and H
+ *         and U 16-byte aligned (tiles move by the tensor-memory accelerator);
+ *         otherwise GPTQ_ERR_UNSUPPORTED.
  *   U     d x d fp32, contiguous (leading dimension d).  Output: the upper
  *         triangular U with U^T U = (P^T H P + lambda I)^-1 in quantization
  *         order (P the act-order permutation); the strictly lower part is 0.
@@ -141,7 +143,8 @@ gptq_status gptq_prepare_hinv(float *H, int64_t d, int64_t ldh, const gptq_confi
  *           column perm[k] as they were when quantized (after the feedback of
  *           every earlier column).
  *   U, perm, dead  the outputs of gptq_prepare_hinv for this layer's H (any
- *           number of layers sharing one H may reuse them).
+ *           number of layers sharing one H may reuse them).  d_col must be a
+ *           multiple of 4 (GPTQ_ERR_UNSUPPORTED otherwise) and at most 57344.
  *   codes   d_row x d_col uint8, contiguous: codes[row][k] is the code of
  *           original column perm[k].
  *   scales  fp32 [ceil(d_col / g)][d_row] and zeros int32 (same shape),

@@ -112,6 +112,8 @@ gptq_status gptq_prepare_hinv(float* H, int64_t d, int64_t ldh, const gptq_confi
         dead == nullptr)
         return GPTQ_ERR_INVALID_ARG;
     if (H == U) return GPTQ_ERR_INVALID_ARG;
+    if ((d % 4) != 0 || (ldh % 4) != 0 || !aligned(H, 16) || !aligned(U, 16))
+        return GPTQ_ERR_UNSUPPORTED;  // tensor-memory-accelerator tiles need 16-byte rows
     const gptq_status c = check_config(cfg, d);
     if (c != GPTQ_OK) return c;
     if (ws == nullptr || !aligned(ws, 256) || ws_bytes < gptq::prep_workspace_bytes(d) ||
@@ -133,7 +135,7 @@ gptq_status gptq_quantize_layer(float* W, int64_t d_row, int64_t d_col, int64_t 
         U == nullptr || perm == nullptr || dead == nullptr || codes == nullptr ||
         scales == nullptr || zeros == nullptr)
         return GPTQ_ERR_INVALID_ARG;
-    if (d_col > kMaxQuantCols) return GPTQ_ERR_UNSUPPORTED;
+    if (d_col > kMaxQuantCols || (d_col % 4) != 0 || !aligned(U, 16)) return GPTQ_ERR_UNSUPPORTED;
     const gptq_status c = check_config(cfg, d_col);
     if (c != GPTQ_OK) return c;
     if (ws == nullptr || !aligned(ws, 256) ||

@@ -1,0 +1,241 @@
+// fp32-accurate GEMM tiles on the tcgen05 tensor cores ("3xTF32").
+//
+// D[128 x 128] = sum_k A[m][k] B[n][k] with fp32 operands: each operand is
+// split in shared memory into hi = tf32(x) (round to nearest) and
+// lo = x - hi, and three kind::tf32 MMAs accumulate hi*hi + hi*lo + lo*hi
+// into one fp32 TMEM accumulator.  The dropped lo*lo term and the tf32
+// truncation of lo leave an error of about 2^-21 of |a||b| per product, close
+// to fp32 FFMA, at tensor-core speed.
+//
+// One output tile per CTA.  Operands arrive through TMA, K-major (a row's K
+// values contiguous: box of 32 K x 128 rows, 128-byte swizzle) or MN-major
+// (a K row's M/N values contiguous: four boxes of 32 x 32, 128-byte swizzle
+// with 32-byte chunks).  Warp roles:
+//   warp 0      TMA producer
+//   warp 1      TMEM owner and MMA issuer
+//   warps 2..5  split each stage into hi / lo, then drain the accumulator
+//               through the scheduler's store() (tcgen05.ld, one row per
+//               thread, 32 columns at a time).
+// Every wait is bounded; on expiry GPTQ_ERR_TIMEOUT is recorded and the CTA
+// winds down after its copies and MMAs have landed.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace gptq {
+namespace g3 {
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int BK = 32;                        // K per stage: 128 bytes of fp32
+constexpr int kStages = 3;
+constexpr int kTileBytes = 128 * BK * 4;      // 16 KB
+constexpr int kStageBytes = 4 * kTileBytes;   // A (hi in place), A lo, B (hi in place), B lo
+constexpr int kThreads = 192;
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+constexpr uint32_t kTmemCols = 128;
+
+// One output tile: rows m0.. of A, rows n0.. of B, K from ka0 (A) / kb0 (B),
+// nk stages of 32.  nk <= 0 skips the tile.
+struct Job {
+    int m0, n0, ka0, kb0, nk;
+};
+
+struct Bars {
+    uint64_t full[kStages];
+    uint64_t conv[kStages];
+    uint64_t empty[kStages];
+    uint64_t acc_full;
+    uint64_t drain;
+    uint32_t tmem;
+    int abort;
+};
+
+__device__ __forceinline__ float tf32_hi(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <bool MN>
+__device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
+                                             int row0, int k) {
+    if (MN) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tma_load_2d(dst + c * 4096, map, bar, row0 + 32 * c, k);
+    } else {
+        tma_load_2d(dst, map, bar, k, row0);
+    }
+}
+
+// Descriptor of K-step kk (8 tf32 values of K) inside a 32-wide stage.
+//  K-major: 128-byte swizzle, 8-row atoms (SBO 1024), 32 bytes of K per step.
+//  MN-major: 32-bit MN-major operands use the 128-byte swizzle with 32-byte
+//  chunks (layout type 1): 4-row atoms of 512 bytes (SBO), 32-element MN
+//  chunks 4 KB apart (LBO), 8 K-rows = 1024 bytes per step.
+template <bool MN>
+__device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk) {
+    if (MN) return smem_desc(base + kk * 1024, 4096, 512, 1);
+    return smem_desc(base + kk * 32, 16, 1024, 2);
+}
+
+template <class Sched, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
+                       const Sched sched, int32_t* status) {
+    const Job job = sched.job(blockIdx.x);
+    if (job.nk <= 0) return;
+    constexpr uint32_t kIdesc = instr_desc(/*tf32*/ 2, A_MN ? 1 : 0, B_MN ? 1 : 0, BM, BN);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    Bars* bars = reinterpret_cast<Bars*>(smem + kStages * kStageBytes);
+    volatile int* abort = &bars->abort;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->conv[s], 128);
+            mbar_init(&bars->empty[s], 1);
+        }
+        mbar_init(&bars->acc_full, 1);
+        mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tma);
+        tma_prefetch_desc(&tmb);
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars->tmem, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int issued = 0;
+            for (int s = 0; s < job.nk && !*abort; ++s) {
+                const int st = s % kStages;
+                const uint32_t ph = (s / kStages) & 1;
+                if (!mbar_wait(&bars->empty[st], ph ^ 1u, abort)) break;
+                uint8_t* a = smem + st * kStageBytes;
+                mbar_arrive_expect_tx(&bars->full[st], 2 * kTileBytes);
+                load_operand<A_MN>(a, &tma, &bars->full[st], job.m0, job.ka0 + s * BK);
+                load_operand<B_MN>(a + 2 * kTileBytes, &tmb, &bars->full[st], job.n0, job.kb0 + s * BK);
+                ++issued;
+            }
+            volatile int no_abort = 0;
+            const int last = issued < kStages ? issued : kStages;
+            for (int j = 0; j < last; ++j) {
+                const int i2 = issued - 1 - j;
+                if (!mbar_wait(&bars->full[i2 % kStages], (i2 / kStages) & 1, &no_abort)) {
+                    *abort = 1;
+                    break;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            bool ok = true;
+            for (int s = 0; s < job.nk; ++s) {
+                const int st = s % kStages;
+                const uint32_t ph = (s / kStages) & 1;
+                if (!mbar_wait(&bars->conv[st], ph, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a = smem_u32(smem + st * kStageBytes);
+                const uint32_t alo = a + kTileBytes, b = a + 2 * kTileBytes, blo = a + 3 * kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < BK / 8; ++kk) {
+                    const uint64_t ah = operand_desc<A_MN>(a, kk), al = operand_desc<A_MN>(alo, kk);
+                    const uint64_t bh = operand_desc<B_MN>(b, kk), bl = operand_desc<B_MN>(blo, kk);
+                    mma_tf32_ss(tmem, ah, bh, kIdesc, (s > 0 || kk > 0) ? 1u : 0u);
+                    mma_tf32_ss(tmem, ah, bl, kIdesc, 1u);
+                    mma_tf32_ss(tmem, al, bh, kIdesc, 1u);
+                }
+                mma_commit(&bars->empty[st]);
+            }
+            if (ok) mma_commit(&bars->acc_full);
+            mma_commit(&bars->drain);
+            volatile int no_abort = 0;
+            if (!mbar_wait(&bars->drain, 0, &no_abort)) *abort = 1;
+        }
+    } else {
+        // ---- split each stage into hi (in place) and lo
+        const int t = threadIdx.x - 64;
+        bool ok = true;
+        for (int s = 0; s < job.nk; ++s) {
+            const int st = s % kStages;
+            const uint32_t ph = (s / kStages) & 1;
+            if (!mbar_wait(&bars->full[st], ph, abort)) {
+                ok = false;
+                break;
+            }
+            float4* a = reinterpret_cast<float4*>(smem + st * kStageBytes);
+            float4* alo = a + kTileBytes / 16;
+            float4* b = a + 2 * (kTileBytes / 16);
+            float4* blo = a + 3 * (kTileBytes / 16);
+#pragma unroll 4
+            for (int i = t; i < kTileBytes / 16; i += 128) {
+                float4 x = a[i], h, l;
+                h.x = tf32_hi(x.x); h.y = tf32_hi(x.y); h.z = tf32_hi(x.z); h.w = tf32_hi(x.w);
+                l.x = x.x - h.x; l.y = x.y - h.y; l.z = x.z - h.z; l.w = x.w - h.w;
+                a[i] = h;
+                alo[i] = l;
+                x = b[i];
+                h.x = tf32_hi(x.x); h.y = tf32_hi(x.y); h.z = tf32_hi(x.z); h.w = tf32_hi(x.w);
+                l.x = x.x - h.x; l.y = x.y - h.y; l.z = x.z - h.z; l.w = x.w - h.w;
+                b[i] = h;
+                blo[i] = l;
+            }
+            fence_async_smem();
+            mbar_arrive(&bars->conv[st]);
+        }
+        // ---- epilogue: TMEM -> registers -> scheduler
+        if (ok && mbar_wait(&bars->acc_full, 0, abort)) {
+            tc_fence_after();
+            const int q = warp & 3;
+            const int row = q * 32 + lane;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                float v[32];
+                tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c * 32, v);
+                sched.store(job, row, c * 32, v);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+    if (threadIdx.x == 0 && bars->abort) report(status, GPTQ_ERR_TIMEOUT);
+}
+
+template <class Sched, bool A_MN, bool B_MN>
+inline cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const Sched& sched,
+                          int tiles, int32_t* status, cudaStream_t stream) {
+    auto kern = gemm_tf32x3_kernel<Sched, A_MN, B_MN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (tiles <= 0) return cudaSuccess;
+    kern<<<tiles, kThreads, kSmemBytes, stream>>>(ta, tb, sched, status);
+    return cudaGetLastError();
+}
+
+}  // namespace g3
+}  // namespace gptq

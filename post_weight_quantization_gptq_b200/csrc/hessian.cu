@@ -241,24 +241,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0 && bars->abort) report(status, GPTQ_ERR_TIMEOUT);
 }
 
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled get_encode() {
-    static EncodeTiled fn = nullptr;
-    if (fn == nullptr) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiled>(p);
-    }
-    return fn;
-}
-
 }  // namespace
 
 int hessian_num_tiles(int64_t d) {
@@ -274,17 +256,9 @@ gptq_status launch_hessian(const uint16_t* X, int64_t n, int64_t d, int64_t ldx,
     if (cudaFuncSetAttribute(hessian_syrk_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSmemBytes) != cudaSuccess)
         return GPTQ_ERR_CUDA;
-    EncodeTiled encode = get_encode();
-    if (encode == nullptr) return GPTQ_ERR_CUDA;
     CUtensorMap tmap;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldx) * 2u};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBox), static_cast<cuuint32_t>(BK)};
-    const cuuint32_t estr[2] = {1, 1};
-    if (encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides,
-               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    if (!make_tmap_2d(&tmap, /*bf16=*/true, X, static_cast<uint64_t>(d), static_cast<uint64_t>(n),
+                      static_cast<uint64_t>(ldx), kBox, BK, Swz::k128))
         return GPTQ_ERR_INVALID_ARG;
     const int T = hessian_num_tiles(d);
     const int sms = num_sms();

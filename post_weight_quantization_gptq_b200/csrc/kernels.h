@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/gptq.h"
@@ -16,6 +17,16 @@ int num_sms();
 // Host-side count of kernels this library has launched (diagnostics).
 void count_launches(int64_t k);
 int64_t launches();
+
+// Shared-memory swizzle of a TMA box: none, 128-byte (16-byte chunks), or
+// 128-byte with 32-byte chunks (the layout 32-bit MN-major MMA operands use).
+enum class Swz { kNone, k128, k128Atom32 };
+
+// 2-D TMA tensor map over a row-major matrix of `outer` rows x `inner`
+// columns (leading dimension ld_elems), boxes of box_outer x box_inner
+// elements, fp32 or bf16 (tmap.cu).
+bool make_tmap_2d(CUtensorMap* map, bool bf16, const void* base, uint64_t inner, uint64_t outer,
+                  uint64_t ld_elems, uint32_t box_inner, uint32_t box_outer, Swz swizzle);
 
 // ---- stage 1 (hessian.cu)
 int hessian_num_tiles(int64_t d);

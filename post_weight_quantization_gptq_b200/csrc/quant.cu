@@ -16,10 +16,12 @@
 //  block_quant_kernel   one 128-column block: row-parallel, 8 lanes per row,
 //                       the block's U in shared memory, the column loop
 //                       sequential with one shuffle per column
-//  lazy_update_kernel   W[:, c1:] -= Err * U[c0:c1, c1:]
+//  lazy update          W[:, c1:] -= Err * U[c0:c1, c1:] on the tensor cores
+//                       (3xTF32 tcgen05 GEMM, fp32-accurate)
 #include <cmath>
 
 #include "common.cuh"
+#include "gemm_tf32x3.cuh"
 #include "kernels.h"
 
 namespace gptq {
@@ -54,20 +56,35 @@ __global__ void permute_rows_kernel(float* __restrict__ W, int64_t r, int64_t d,
 __device__ __forceinline__ int col_of(int t, int l) { return 32 * (t >> 2) + 4 * l + (t & 3); }
 
 __global__ void __launch_bounds__(kWarps * 32)
-    block_quant_kernel(float* __restrict__ W, int64_t r, int64_t d, int64_t ldw,
-                       const float* __restrict__ U, int64_t c0, int bw, int bits, int g,
+    block_quant_kernel(const __grid_constant__ CUtensorMap tmu, float* __restrict__ W, int64_t r,
+                       int64_t d, int64_t ldw, int64_t c0, int bw, int bits, int g,
                        uint8_t* __restrict__ codes, float* __restrict__ scales,
-                       int32_t* __restrict__ zeros, float* __restrict__ err_out) {
-    extern __shared__ __align__(16) float smem[];
-    float* Us = smem;                    // [kBlock][kBlock], strict upper part of U's block
+                       int32_t* __restrict__ zeros, float* __restrict__ err_out,
+                       int32_t* status) {
+    extern __shared__ uint8_t smem_raw[];
+    float* smem = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+    float* Us = smem;                      // [kBlock][kBlock]: U's diagonal block, strict upper part kept
     float* dinv = smem + kBlock * kBlock;  // 1 / U_jj
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int ok;
     const int tid = threadIdx.x;
-    for (int e = tid; e < kBlock * kBlock; e += blockDim.x) {
-        const int j = e / kBlock, f = e % kBlock;
-        Us[e] = (j < bw && f < bw && f > j) ? U[(c0 + j) * d + c0 + f] : 0.f;
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+        mbar_arrive_expect_tx(&bar, kBlock * kBlock * 4);
+        tma_load_2d(Us, &tmu, &bar, static_cast<int>(c0), static_cast<int>(c0));
+        volatile int no_abort = 0;
+        ok = mbar_wait(&bar, 0, &no_abort) ? 1 : 0;
+        if (!ok) report(status, GPTQ_ERR_TIMEOUT);
     }
+    __syncthreads();
+    if (!ok) return;
     for (int j = tid; j < kBlock; j += blockDim.x)
-        dinv[j] = (j < bw) ? 1.f / U[(c0 + j) * d + c0 + j] : 0.f;
+        dinv[j] = (j < bw) ? 1.f / Us[j * kBlock + j] : 0.f;
+    __syncthreads();
+    for (int e = tid; e < kBlock * kBlock; e += blockDim.x)
+        if ((e & (kBlock - 1)) <= (e >> 7)) Us[e] = 0.f;  // diagonal and below
     __syncthreads();
 
     const int lane = tid & 31;
@@ -80,10 +97,22 @@ __global__ void __launch_bounds__(kWarps * 32)
 
     float w[16], ev[16];
     uint32_t qv[16];
+    const bool vec = (ldw & 3) == 0 && bw == kBlock;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        if (live && vec) {
+            const float4 v = *reinterpret_cast<const float4*>(W + row * ldw + c0 + 32 * m + 4 * l);
+            w[4 * m] = v.x; w[4 * m + 1] = v.y; w[4 * m + 2] = v.z; w[4 * m + 3] = v.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int c = 32 * m + 4 * l + i;
+                w[4 * m + i] = (live && c < bw) ? W[row * ldw + c0 + c] : 0.f;
+            }
+        }
+    }
 #pragma unroll
     for (int t = 0; t < 16; ++t) {
-        const int c = col_of(t, l);
-        w[t] = (live && c < bw) ? W[row * ldw + c0 + c] : 0.f;
         ev[t] = 0.f;
         qv[t] = 0;
     }
@@ -166,64 +195,60 @@ __global__ void __launch_bounds__(kWarps * 32)
 
     if (!live) return;
 #pragma unroll
-    for (int t = 0; t < 16; ++t) {
-        const int c = col_of(t, l);
-        if (c < bw) {
-            W[row * ldw + c0 + c] = w[t];
-            err_out[row * kBlock + c] = ev[t];
-            codes[row * d + c0 + c] = static_cast<uint8_t>(qv[t]);
+    for (int m = 0; m < 4; ++m) {
+        const int cb = 32 * m + 4 * l;
+        *reinterpret_cast<float4*>(err_out + row * kBlock + cb) =
+            make_float4(ev[4 * m], ev[4 * m + 1], ev[4 * m + 2], ev[4 * m + 3]);
+        if (vec) {
+            *reinterpret_cast<float4*>(W + row * ldw + c0 + cb) =
+                make_float4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]);
+        }
+        if (vec && (d & 3) == 0) {
+            *reinterpret_cast<uint32_t*>(codes + row * d + c0 + cb) =
+                qv[4 * m] | (qv[4 * m + 1] << 8) | (qv[4 * m + 2] << 16) | (qv[4 * m + 3] << 24);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int c = cb + i;
+            if (c < bw) {
+                if (!vec) W[row * ldw + c0 + c] = w[4 * m + i];
+                if (!(vec && (d & 3) == 0)) codes[row * d + c0 + c] = static_cast<uint8_t>(qv[4 * m + i]);
+            }
         }
     }
 }
 
 // ------------------------------------------------------------------------
-// W[:, c1:d] -= Err[:, 0:bw] * U[c0:c0+bw, c1:d]  (fp32 FFMA, 64 x 64 tiles)
-constexpr int TS = 64;
-__global__ void __launch_bounds__(256)
-    lazy_update_kernel(float* __restrict__ W, int64_t r, int64_t d, int64_t ldw,
-                       const float* __restrict__ U, int64_t c0, int bw,
-                       const float* __restrict__ err) {
-    __shared__ float As[TS][TS + 1];  // Err tile: rows, k
-    __shared__ float Bs[TS][TS + 1];  // U^T tile: cols, k
-    const int tid = threadIdx.x;
-    const int64_t c1 = c0 + bw;
-    const int64_t col0 = c1 + static_cast<int64_t>(blockIdx.x) * TS;
-    const int64_t row0 = static_cast<int64_t>(blockIdx.y) * TS;
-    const int tx = tid & 15, ty = tid >> 4;
-    float acc[4][4] = {};
-    for (int k0 = 0; k0 < bw; k0 += TS) {
-        for (int e = tid; e < TS * TS; e += 256) {
-            const int i = e / TS, k = e % TS;
-            As[i][k] = (row0 + i < r && k0 + k < bw) ? err[(row0 + i) * kBlock + k0 + k] : 0.f;
-            const int kk = e / TS, cc = e % TS;
-            Bs[cc][kk] = (k0 + kk < bw && col0 + cc < d) ? U[(c0 + k0 + kk) * d + col0 + cc] : 0.f;
-        }
-        __syncthreads();
-#pragma unroll 4
-        for (int k = 0; k < TS; ++k) {
-            float a[4], b[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = As[ty + 16 * i][k];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) b[i] = Bs[tx + 16 * i][k];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) acc[i][q] = fmaf(a[i], b[q], acc[i][q]);
-        }
-        __syncthreads();
+// Lazy update W[:, c1:d] -= Err[:, 0:128] U[c0:c0+128, c1:d] as 128 x 128
+// output tiles of the 3xTF32 GEMM: A = Err (K-major), B = U's rows (MN-major).
+struct LazySched {
+    float* W;
+    int64_t ldw;
+    int r, d, c0, c1, mt;
+    __device__ g3::Job job(int t) const {
+        const int mi = t % mt, ni = t / mt;
+        return {128 * mi, c1 + 128 * ni, 0, c0, kBlock / 32};
     }
+    __device__ void store(const g3::Job& jb, int row, int col0, const float (&v)[32]) const {
+        const int rr = jb.m0 + row;
+        if (rr >= r) return;
+        float* dst = W + static_cast<int64_t>(rr) * ldw + jb.n0 + col0;
+        const int c = jb.n0 + col0;
+        if (c + 32 <= d && (ldw & 3) == 0) {
+            float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int64_t rr = row0 + ty + 16 * i;
-        if (rr >= r) continue;
+            for (int q = 0; q < 8; ++q) {
+                float4 x = d4[q];
+                x.x -= v[4 * q]; x.y -= v[4 * q + 1]; x.z -= v[4 * q + 2]; x.w -= v[4 * q + 3];
+                d4[q] = x;
+            }
+        } else {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int64_t cc = col0 + tx + 16 * q;
-            if (cc < d) W[rr * ldw + cc] -= acc[i][q];
+            for (int j = 0; j < 32; ++j)
+                if (c + j < d) dst[j] -= v[j];
         }
     }
-}
+};
 
 }  // namespace
 
@@ -235,7 +260,6 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
                             const int32_t* perm, const uint8_t* dead, int bits, int group,
                             int block, uint8_t* codes, float* scales, int32_t* zeros,
                             int32_t* status, void* ws, cudaStream_t stream) {
-    (void)status;
     if (block != kBlock) return GPTQ_ERR_UNSUPPORTED;
     const int g = (group == -1 || group > d_col) ? static_cast<int>(d_col) : group;
     float* err = static_cast<float*>(ws);
@@ -246,26 +270,36 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
         return GPTQ_ERR_CUDA;
     const int prow_grid = static_cast<int>(d_row < 4 * num_sms() ? d_row : 4 * num_sms());
     permute_rows_kernel<<<prow_grid, 256, row_smem, stream>>>(W, d_row, d_col, ldw, perm, dead);
-    count_launches(1);
 
-    const size_t q_smem = (kBlock * kBlock + kBlock) * sizeof(float);
+    CUtensorMap tU, tUmn, tErr;
+    if (!make_tmap_2d(&tU, false, U, d_col, d_col, d_col, kBlock, kBlock, Swz::kNone) ||
+        !make_tmap_2d(&tUmn, false, U, d_col, d_col, d_col, 32, 32, Swz::k128Atom32) ||
+        !make_tmap_2d(&tErr, false, err, kBlock, d_row, kBlock, 32, 128, Swz::k128))
+        return GPTQ_ERR_INVALID_ARG;
+    const size_t q_smem = (kBlock * kBlock + kBlock) * sizeof(float) + 1024;
     if (cudaFuncSetAttribute(block_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(q_smem)) != cudaSuccess)
         return GPTQ_ERR_CUDA;
     const unsigned qgrid = static_cast<unsigned>((d_row + kRowsPerCta - 1) / kRowsPerCta);
+    const int mt = static_cast<int>((d_row + 127) / 128);
+    int64_t launches = 1;
     for (int64_t c0 = 0; c0 < d_col; c0 += kBlock) {
         const int bw = static_cast<int>((d_col - c0 < kBlock) ? d_col - c0 : kBlock);
         block_quant_kernel<<<qgrid, kWarps * 32, q_smem, stream>>>(
-            W, d_row, d_col, ldw, U, c0, bw, bits, g, codes, scales, zeros, err);
-        count_launches(1);
+            tU, W, d_row, d_col, ldw, c0, bw, bits, g, codes, scales, zeros, err, status);
+        ++launches;
         const int64_t rest = d_col - c0 - bw;
         if (rest > 0) {
-            dim3 grid(static_cast<unsigned>((rest + TS - 1) / TS),
-                      static_cast<unsigned>((d_row + TS - 1) / TS));
-            lazy_update_kernel<<<grid, 256, 0, stream>>>(W, d_row, d_col, ldw, U, c0, bw, err);
-            count_launches(1);
+            const int nt = static_cast<int>((rest + 127) / 128);
+            LazySched ls{W, ldw, static_cast<int>(d_row), static_cast<int>(d_col),
+                         static_cast<int>(c0), static_cast<int>(c0 + bw), mt};
+            if (g3::launch<LazySched, false, true>(tErr, tUmn, ls, mt * nt, status, stream) !=
+                cudaSuccess)
+                return GPTQ_ERR_CUDA;
+            ++launches;
         }
     }
+    count_launches(launches);
     return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
 }
 

@@ -57,7 +57,7 @@ def test_hessian_accumulates_over_token_chunks():
 
 # ------------------------------------------------------------------ stage 2
 @pytest.mark.parametrize("d,desc_act,n_dead", [(512, False, 0), (512, True, 0), (200, True, 3),
-                                               (130, False, 2), (1024, True, 0), (64, False, 0)])
+                                               (132, False, 2), (1024, True, 0), (64, False, 0)])
 def test_prepare_hinv_matches_oracle_elimination(d, desc_act, n_dead):
     rng = np.random.default_rng(d + n_dead)
     _, X = workloads.small_layer(4, d, 4 * d, seed=d, kind="correlated")
@@ -108,7 +108,7 @@ QUANT_CASES = [
     (33, 512, 2048, "student_t", 4, -1, False),
     (16, 512, 2048, "student_t", 4, 256, True),
     (7, 200, 800, "student_t", 4, 8, False),
-    (5, 130, 700, "correlated", 8, 128, True),
+    (5, 132, 700, "correlated", 8, 128, True),
     (1, 64, 256, "student_t", 4, 32, False),
     (300, 1024, 4096, "student_t", 4, 128, True),
 ]
