@@ -35,14 +35,21 @@ constexpr int NB = 128;      // panel width
 constexpr int LDA = NB + 1;  // shared-memory row pitch of the diagonal block
 constexpr int kDiagThreads = 256;
 constexpr int kDiagSmem = (2 * NB * LDA + 64 * 65 + NB) * 4;
-constexpr unsigned kFull = 0xffffffffu;
 
 // ------------------------------------------------------------------------
 // Diagonal block: L = chol(A) and X = L^-1 for a kw x kw (kw <= 128) block,
-// padded with the identity.  Four 32-wide strips: one warp factors and
-// inverts the strip's 32 x 32 diagonal block in registers, then the CTA
-// solves the strip below and updates the trailing part; finally the four
-// 32 x 32 inverses are joined by two levels of recursive doubling.
+// padded with the identity.  Four 32-wide strips; for each, one warp factors
+// the strip's 32 x 32 diagonal block, then four warps run one forward
+// substitution on 128 right-hand sides (the identity -> the strip's inverse,
+// and the rows below -> the strip of L), then the CTA updates the trailing
+// part; finally the four 32 x 32 inverses are joined by two levels of
+// recursive doubling.
+//
+// The warp keeps its rows in registers and rotates them after every column
+// step, so the pivot column is always register 0: the step loop stays rolled
+// (small code, the kernel runs once per panel on a cold SM) while all
+// register indices are compile-time constants and each step is 31
+// independent shuffle + FMA pairs.
 __global__ void __launch_bounds__(kDiagThreads, 1)
     potrf_inv_128_kernel(float* __restrict__ P, int64_t ldp, int64_t kb, int kw,
                          float* __restrict__ X, int64_t ldx, int32_t* status) {
@@ -52,88 +59,92 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
     float* T = Xs + NB * LDA;   // [64][65] doubling temporary
     float* dinv = T + 64 * 65;  // [128] 1 / L_ii
     __shared__ int bad;
+    __shared__ float colbuf[32];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) bad = 0;
-    for (int e = tid; e < NB * NB; e += kDiagThreads) {
-        const int i = e >> 7, j = e & (NB - 1);
-        float v = (i == j) ? 1.f : 0.f;
-        if (i < kw && j <= i) v = P[(kb + i) * ldp + kb + j];
-        A[i * LDA + j] = v;
-        Xs[i * LDA + j] = 0.f;
+    {
+        // rows of the block: 16 float4 loads per thread, all in flight
+        // (ldp, kb and kw are multiples of 4, so a float4 never crosses kw)
+        float4 v[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const int e = tid + q * kDiagThreads;
+            const int i = e >> 5, j = (e & 31) * 4;
+            v[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < kw && j <= i) v[q] = *reinterpret_cast<const float4*>(P + (kb + i) * ldp + kb + j);
+        }
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const int e = tid + q * kDiagThreads;
+            const int i = e >> 5, j = (e & 31) * 4;
+            const float vv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const int jj = j + t;
+                A[i * LDA + jj] = (jj <= i && i < kw) ? vv[t] : (i == jj ? 1.f : 0.f);
+                Xs[i * LDA + jj] = 0.f;
+            }
+        }
     }
     __syncthreads();
 
     for (int b = 0; b < 4; ++b) {
         const int o = 32 * b;
         if (warp == 0) {
-            // -- 32 x 32 Cholesky in registers: lane i holds row o + i
+            // -- 32 x 32 Cholesky: lane i holds row o + i, register r = column c + r
             float a[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) a[j] = (j <= lane) ? A[(o + lane) * LDA + o + j] : 0.f;
-#pragma unroll
+            for (int r = 0; r < 32; ++r) a[r] = (r <= lane) ? A[(o + lane) * LDA + o + r] : 0.f;
+#pragma unroll 1
             for (int c = 0; c < 32; ++c) {
-                float piv = __shfl_sync(kFull, a[c], c);
+                float piv = __shfl_sync(0xffffffffu, a[0], c);
                 if (!(piv > 0.f)) {  // not positive definite (or NaN): flag, stay finite
                     bad = 1;
                     piv = 1.f;
                 }
-                const float lcc = sqrtf(piv);
-                const float inv = 1.f / lcc;
-                if (lane == c) a[c] = lcc;
-                else if (lane > c) a[c] *= inv;
+                const float inv = rsqrtf(piv);
+                const float lcc = piv * inv;
+                const float a0 = (lane == c) ? lcc : ((lane > c) ? a[0] * inv : a[0]);
+                colbuf[lane] = a0;
+                if (lane >= c) A[(o + lane) * LDA + o + c] = a0;
+                if (lane == c) dinv[o + c] = inv;
+                __syncwarp();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    if (j > c) {
-                        const float ljc = __shfl_sync(kFull, a[c], j);
-                        if (lane >= j) a[j] = fmaf(-a[c], ljc, a[j]);
-                    }
-                }
+                for (int r = 1; r < 32; ++r)
+                    a[r - 1] = fmaf(-a0, colbuf[(c + r) & 31], a[r]);  // update and rotate
+                a[31] = 0.f;
+                __syncwarp();
             }
-            float dl = 1.f;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                if (j <= lane) A[(o + lane) * LDA + o + j] = a[j];
-                if (j == lane) dl = a[j];
-            }
-            dinv[o + lane] = 1.f / dl;
-            __syncwarp();
-            // -- its inverse: lane j owns column j
-            float x[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                float acc = 0.f;
-#pragma unroll
-                for (int k = 0; k < 32; ++k)
-                    if (k < i) acc = fmaf(A[(o + i) * LDA + o + k], x[k], acc);
-                const float di = dinv[o + i];
-                x[i] = (i == lane) ? di : ((i > lane) ? -acc * di : 0.f);
-            }
-#pragma unroll
-            for (int i = 0; i < 32; ++i) Xs[(o + i) * LDA + o + lane] = x[i];
         }
         __syncthreads();
         const int r0 = o + 32;
-        if (r0 < NB) {
-            // -- strip solve: L[i][o+j] = sum_{k<=j} A[i][o+k] Xs[o+j][o+k], i >= r0
-            const int j = lane;
-            float out[12];
+        if (warp < 4) {
+            // -- forward substitution with L_bb on 128 right-hand sides at once:
+            //    lanes 0..31 the identity (-> the strip's inverse, a column per
+            //    lane), lanes 32..127 the rows below (-> the strip of L)
+            const int hs = tid;
+            const int i = r0 + hs - 32;  // row for hs >= 32
+            const bool act = hs < 32 || i < NB;
+            float x[32];
 #pragma unroll
-            for (int q = 0; q < 12; ++q) {
-                const int i = r0 + warp + 8 * q;
-                float acc = 0.f;
-                if (i < NB) {
-                    for (int k = 0; k <= j; ++k)
-                        acc = fmaf(A[i * LDA + o + k], Xs[(o + j) * LDA + o + k], acc);
+            for (int r = 0; r < 32; ++r)
+                x[r] = (hs < 32) ? ((r == hs) ? 1.f : 0.f) : (act ? A[i * LDA + o + r] : 0.f);
+#pragma unroll 1
+            for (int c = 0; c < 32; ++c) {
+                const float xc = x[0] * dinv[o + c];
+                if (hs < 32) Xs[(o + c) * LDA + o + hs] = xc;
+                else if (act) A[i * LDA + o + c] = xc;
+                const float* lcol = A + (o + c) * LDA + o + c;  // L[o+c+r][o+c] at lcol[r * LDA]
+#pragma unroll
+                for (int r = 1; r < 32; ++r) {
+                    const float l = (c + r < 32) ? lcol[r * LDA] : 0.f;
+                    x[r - 1] = fmaf(-l, xc, x[r]);
                 }
-                out[q] = acc;
+                x[31] = 0.f;
             }
-            __syncthreads();
-#pragma unroll
-            for (int q = 0; q < 12; ++q) {
-                const int i = r0 + warp + 8 * q;
-                if (i < NB) A[i * LDA + o + j] = out[q];
-            }
-            __syncthreads();
+        }
+        __syncthreads();
+        if (r0 < NB) {
             // -- trailing update of the lower part, 4 x 4 register blocks
             const int mb = (NB - r0) / 4;
             const int units = mb * (mb + 1) / 2;
@@ -143,7 +154,7 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
                 while ((bi + 1) * (bi + 2) / 2 <= u) ++bi;
                 const int bj = u - bi * (bi + 1) / 2;
                 const int i0 = r0 + 4 * bi, j0 = r0 + 4 * bj;
-                float acc[4][4] = {};
+                float acc2[4][4] = {};
 #pragma unroll 4
                 for (int k = 0; k < 32; ++k) {
                     float li[4], lj[4];
@@ -155,51 +166,92 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
 #pragma unroll
                     for (int t = 0; t < 4; ++t)
 #pragma unroll
-                        for (int w = 0; w < 4; ++w) acc[t][w] = fmaf(li[t], lj[w], acc[t][w]);
+                        for (int w = 0; w < 4; ++w) acc2[t][w] = fmaf(li[t], lj[w], acc2[t][w]);
                 }
 #pragma unroll
                 for (int t = 0; t < 4; ++t)
 #pragma unroll
                     for (int w = 0; w < 4; ++w)
-                        if (j0 + w <= i0 + t) A[(i0 + t) * LDA + j0 + w] -= acc[t][w];
+                        if (j0 + w <= i0 + t) A[(i0 + t) * LDA + j0 + w] -= acc2[t][w];
             }
         }
         __syncthreads();
     }
 
-    // -- join the 32 x 32 inverses: X_CA = -X_CC (L_CA X_AA); T[p*s + c][a]
+    // -- join the 32 x 32 inverses: X_CA = -X_CC (L_CA X_AA), 4 x 4 register
+    //    blocks (rows c, columns a); T[p*s + c][a] holds L_CA X_AA
     for (int s = 32; s < NB; s *= 2) {
         const int pairs = NB / (2 * s);
-        const int outs = pairs * s * s;
-        for (int e = tid; e < outs; e += kDiagThreads) {
-            const int p = e / (s * s), c = (e / s) % s, a = e % s;
+        const int nb4 = s / 4;
+        const int blocks = pairs * nb4 * nb4;
+        for (int e = tid; e < blocks; e += kDiagThreads) {
+            const int p = e / (nb4 * nb4), c0 = ((e / nb4) % nb4) * 4, a0 = (e % nb4) * 4;
             const int A0 = 2 * s * p, C0 = A0 + s;
-            float acc = 0.f;
-            for (int k = a; k < s; ++k)
-                acc = fmaf(A[(C0 + c) * LDA + A0 + k], Xs[(A0 + k) * LDA + A0 + a], acc);
-            T[(p * s + c) * 65 + a] = acc;
+            float acc[4][4] = {};
+#pragma unroll 8
+            for (int k = 0; k < s; ++k) {  // X_AA is zero above its diagonal
+                float l[4], xx[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    l[t] = A[(C0 + c0 + t) * LDA + A0 + k];
+                    xx[t] = Xs[(A0 + k) * LDA + A0 + a0 + t];
+                }
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) acc[t][w] = fmaf(l[t], xx[w], acc[t][w]);
+            }
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+#pragma unroll
+                for (int w = 0; w < 4; ++w) T[(p * s + c0 + t) * 65 + a0 + w] = acc[t][w];
         }
         __syncthreads();
-        for (int e = tid; e < outs; e += kDiagThreads) {
-            const int p = e / (s * s), c = (e / s) % s, a = e % s;
+        for (int e = tid; e < blocks; e += kDiagThreads) {
+            const int p = e / (nb4 * nb4), c0 = ((e / nb4) % nb4) * 4, a0 = (e % nb4) * 4;
             const int A0 = 2 * s * p, C0 = A0 + s;
-            float acc = 0.f;
-            for (int k = 0; k <= c; ++k)
-                acc = fmaf(Xs[(C0 + c) * LDA + C0 + k], T[(p * s + k) * 65 + a], acc);
-            Xs[(C0 + c) * LDA + A0 + a] = -acc;
+            float acc[4][4] = {};
+#pragma unroll 8
+            for (int k = 0; k < s; ++k) {  // X_CC is zero above its diagonal
+                float xc[4], tt[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    xc[t] = Xs[(C0 + c0 + t) * LDA + C0 + k];
+                    tt[t] = T[(p * s + k) * 65 + a0 + t];
+                }
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) acc[t][w] = fmaf(xc[t], tt[w], acc[t][w]);
+            }
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+#pragma unroll
+                for (int w = 0; w < 4; ++w) Xs[(C0 + c0 + t) * LDA + A0 + a0 + w] = -acc[t][w];
         }
         __syncthreads();
     }
 
-    for (int e = tid; e < kw * kw; e += kDiagThreads) {
-        const int i = e / kw, j = e % kw;
-        if (j <= i) P[(kb + i) * ldp + kb + j] = A[i * LDA + j];
-    }
-    // X's diagonal block, zeros above the diagonal included (the tensor-core
-    // GEMMs read it as a full tile)
-    for (int e = tid; e < kw * kw; e += kDiagThreads) {
-        const int i = e / kw, j = e % kw;
-        X[(kb + i) * ldx + kb + j] = (j <= i) ? Xs[i * LDA + j] : 0.f;
+    // -- write L (lower part) and X (zeros above the diagonal included: the
+    //    tensor-core GEMMs read it as a full tile), float4 per access
+#pragma unroll 4
+    for (int e = tid; e < NB * NB / 4; e += kDiagThreads) {
+        const int i = e >> 5, j = (e & 31) * 4;
+        if (i >= kw || j >= kw) continue;
+        float l4[4], x4[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            l4[t] = A[i * LDA + j + t];
+            x4[t] = (j + t <= i) ? Xs[i * LDA + j + t] : 0.f;
+        }
+        *reinterpret_cast<float4*>(X + (kb + i) * ldx + kb + j) = make_float4(x4[0], x4[1], x4[2], x4[3]);
+        if (j + 3 <= i) {
+            *reinterpret_cast<float4*>(P + (kb + i) * ldp + kb + j) = make_float4(l4[0], l4[1], l4[2], l4[3]);
+        } else if (j <= i) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+                if (j + t <= i) P[(kb + i) * ldp + kb + j + t] = l4[t];
+        }
     }
     if (tid == 0 && bad) report(status, GPTQ_ERR_NOT_PD);
 }
@@ -213,6 +265,24 @@ __device__ __forceinline__ void tri_coords(int t, int& I, int& J) {
     J = t - i * (i + 1) / 2;
 }
 
+// 32 consecutive floats: dst[j] = sign * v[j] (or dst[j] -= v[j] with sub),
+// as float4 accesses (callers guarantee 16-byte alignment and bounds).
+template <bool kSub>
+__device__ __forceinline__ void put32(float* dst, const float (&v)[32], float sign) {
+    float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        if (kSub) {
+            float4 x = d4[q];
+            x.x -= v[4 * q]; x.y -= v[4 * q + 1]; x.z -= v[4 * q + 2]; x.w -= v[4 * q + 3];
+            d4[q] = x;
+        } else {
+            d4[q] = make_float4(sign * v[4 * q], sign * v[4 * q + 1], sign * v[4 * q + 2],
+                                sign * v[4 * q + 3]);
+        }
+    }
+}
+
 // ---------------------------------------------------------------- schedulers
 // Panel solve: L[m0.., kb..kb+kw) = A[m0.., kb..) (L_kk^-1)^T   (in place)
 struct TrsmSched {
@@ -224,9 +294,13 @@ struct TrsmSched {
         const int r = jb.m0 + row;
         if (r >= d) return;
         float* dst = P + static_cast<int64_t>(r) * ldp + kb + col0;
+        if (col0 + 32 <= kw) {
+            put32<false>(dst, v, 1.f);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-            if (col0 + j < kw) dst[j] = v[j];
+            for (int j = 0; j < 32; ++j)
+                if (col0 + j < kw) dst[j] = v[j];
+        }
     }
 };
 
@@ -244,10 +318,13 @@ struct SyrkSched {
         const int r = jb.m0 + row;
         if (r >= d) return;
         float* dst = P + static_cast<int64_t>(r) * ldp + jb.n0 + col0;
+        const int c = jb.n0 + col0;
+        if (c + 31 <= r && c + 32 <= d) {
+            put32<true>(dst, v, 1.f);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const int c = jb.n0 + col0 + j;
-            if (c < d && c <= r) dst[j] -= v[j];
+            for (int j = 0; j < 32; ++j)
+                if (c + j < d && c + j <= r) dst[j] -= v[j];
         }
     }
 };
@@ -268,9 +345,13 @@ struct Trinv1Sched {
     }
     __device__ void store(const g3::Job& jb, int row, int col0, const float (&v)[32]) const {
         float* dst = P + static_cast<int64_t>(jb.m0 + row) * ldp + jb.n0 + col0;
+        if (jb.n0 + col0 + 32 <= d) {
+            put32<false>(dst, v, 1.f);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-            if (jb.n0 + col0 + j < d) dst[j] = v[j];
+            for (int j = 0; j < 32; ++j)
+                if (jb.n0 + col0 + j < d) dst[j] = v[j];
+        }
     }
 };
 
@@ -291,9 +372,7 @@ struct Trinv2Sched {
     __device__ void store(const g3::Job& jb, int row, int col0, const float (&v)[32]) const {
         const int r = jb.m0 + row;
         if (r >= d) return;
-        float* dst = X + static_cast<int64_t>(r) * ldx + jb.n0 + col0;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) dst[j] = -v[j];
+        put32<false>(X + static_cast<int64_t>(r) * ldx + jb.n0 + col0, v, -1.f);
     }
 };
 
@@ -331,10 +410,10 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
         if (m > 0) {
             const int mt = static_cast<int>((m + NB - 1) / NB);
             TrsmSched ts{P, ldp, di, static_cast<int>(kb), kw};
-            if (g3::launch<TrsmSched, false, false>(tP, tX, ts, mt, status, stream) != cudaSuccess)
+            if (g3::launch<TrsmSched, false, false>(tP, tX, ts, mt, status, stream, num_sms()) != cudaSuccess)
                 return GPTQ_ERR_CUDA;
             SyrkSched ss{P, ldp, di, static_cast<int>(kb), kw, static_cast<int>(kb + kw)};
-            if (g3::launch<SyrkSched, false, false>(tP, tP, ss, mt * (mt + 1) / 2, status, stream) !=
+            if (g3::launch<SyrkSched, false, false>(tP, tP, ss, mt * (mt + 1) / 2, status, stream, num_sms()) !=
                 cudaSuccess)
                 return GPTQ_ERR_CUDA;
             launches += 2;
@@ -346,8 +425,8 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
         const int grid = static_cast<int>(pairs * tiles * tiles);
         Trinv1Sched t1{P, ldp, di, static_cast<int>(s), tiles};
         Trinv2Sched t2{X, ldx, di, static_cast<int>(s), tiles};
-        if (g3::launch<Trinv1Sched, true, false>(tXmn, tP, t1, grid, status, stream) != cudaSuccess ||
-            g3::launch<Trinv2Sched, false, false>(tX, tP, t2, grid, status, stream) != cudaSuccess)
+        if (g3::launch<Trinv1Sched, true, false>(tXmn, tP, t1, grid, status, stream, num_sms()) != cudaSuccess ||
+            g3::launch<Trinv2Sched, false, false>(tX, tP, t2, grid, status, stream, num_sms()) != cudaSuccess)
             return GPTQ_ERR_CUDA;
         launches += 2;
     }

@@ -7,15 +7,18 @@
 // truncation of lo leave an error of about 2^-21 of |a||b| per product, close
 // to fp32 FFMA, at tensor-core speed.
 //
-// One output tile per CTA.  Operands arrive through TMA, K-major (a row's K
+// Persistent: each CTA walks a static list of output tiles (tile, tile +
+// grid, ...), the stage ring runs on across tiles and two TMEM accumulators
+// let the epilogue of one tile overlap the loads and MMAs of the next.
+// Operands arrive through TMA, K-major (a row's K
 // values contiguous: box of 32 K x 128 rows, 128-byte swizzle) or MN-major
 // (a K row's M/N values contiguous: four boxes of 32 x 32, 128-byte swizzle
 // with 32-byte chunks).  Warp roles:
 //   warp 0      TMA producer
 //   warp 1      TMEM owner and MMA issuer
-//   warps 2..5  split each stage into hi / lo, then drain the accumulator
-//               through the scheduler's store() (tcgen05.ld, one row per
-//               thread, 32 columns at a time).
+//   warps 2..5  split each stage into hi / lo
+//   warps 6..9  drain the accumulator through the scheduler's store()
+//               (tcgen05.ld, one row per thread, 32 columns at a time).
 // Every wait is bounded; on expiry GPTQ_ERR_TIMEOUT is recorded and the CTA
 // winds down after its copies and MMAs have landed.
 #pragma once
@@ -33,9 +36,9 @@ constexpr int BK = 32;                        // K per stage: 128 bytes of fp32
 constexpr int kStages = 3;
 constexpr int kTileBytes = 128 * BK * 4;      // 16 KB
 constexpr int kStageBytes = 4 * kTileBytes;   // A (hi in place), A lo, B (hi in place), B lo
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;                 // TMA, MMA, 4 split warps, 4 epilogue warps
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
-constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t kTmemCols = 256;           // two 128-column accumulators
 
 // One output tile: rows m0.. of A, rows n0.. of B, K from ka0 (A) / kb0 (B),
 // nk stages of 32.  nk <= 0 skips the tile.
@@ -47,7 +50,8 @@ struct Bars {
     uint64_t full[kStages];
     uint64_t conv[kStages];
     uint64_t empty[kStages];
-    uint64_t acc_full;
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
     uint64_t drain;
     uint32_t tmem;
     int abort;
@@ -88,9 +92,7 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk) {
 template <class Sched, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
-                       const Sched sched, int32_t* status) {
-    const Job job = sched.job(blockIdx.x);
-    if (job.nk <= 0) return;
+                       const Sched sched, int tiles, int32_t* status) {
     constexpr uint32_t kIdesc = instr_desc(/*tf32*/ 2, A_MN ? 1 : 0, B_MN ? 1 : 0, BM, BN);
 
     extern __shared__ uint8_t smem_raw[];
@@ -107,7 +109,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->conv[s], 128);
             mbar_init(&bars->empty[s], 1);
         }
-        mbar_init(&bars->acc_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars->acc_full[s], 1);
+            mbar_init(&bars->acc_empty[s], 128);
+        }
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
         fence_barrier_init();
@@ -124,22 +129,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = bars->tmem;
 
     if (warp == 0) {
+        // ---------------------------------------------------- TMA producer
         if (lane == 0) {
-            int issued = 0;
-            for (int s = 0; s < job.nk && !*abort; ++s) {
-                const int st = s % kStages;
-                const uint32_t ph = (s / kStages) & 1;
-                if (!mbar_wait(&bars->empty[st], ph ^ 1u, abort)) break;
-                uint8_t* a = smem + st * kStageBytes;
-                mbar_arrive_expect_tx(&bars->full[st], 2 * kTileBytes);
-                load_operand<A_MN>(a, &tma, &bars->full[st], job.m0, job.ka0 + s * BK);
-                load_operand<B_MN>(a + 2 * kTileBytes, &tmb, &bars->full[st], job.n0, job.kb0 + s * BK);
-                ++issued;
+            int it = 0;
+            for (int t = blockIdx.x; t < tiles && !*abort; t += gridDim.x) {
+                const Job job = sched.job(t);
+                for (int s = 0; s < job.nk && !*abort; ++s, ++it) {
+                    const int st = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1;
+                    if (!mbar_wait(&bars->empty[st], ph ^ 1u, abort)) break;
+                    uint8_t* a = smem + st * kStageBytes;
+                    mbar_arrive_expect_tx(&bars->full[st], 2 * kTileBytes);
+                    load_operand<A_MN>(a, &tma, &bars->full[st], job.m0, job.ka0 + s * BK);
+                    load_operand<B_MN>(a + 2 * kTileBytes, &tmb, &bars->full[st], job.n0,
+                                       job.kb0 + s * BK);
+                }
             }
+            // never leave with copies in flight (bounded even when aborting)
             volatile int no_abort = 0;
-            const int last = issued < kStages ? issued : kStages;
+            const int last = it < kStages ? it : kStages;
             for (int j = 0; j < last; ++j) {
-                const int i2 = issued - 1 - j;
+                const int i2 = it - 1 - j;
                 if (!mbar_wait(&bars->full[i2 % kStages], (i2 / kStages) & 1, &no_abort)) {
                     *abort = 1;
                     break;
@@ -147,75 +157,105 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == 1) {
+        // ---------------------------------------------------- MMA issuer
         if (lane == 0) {
+            int it = 0, lt = 0;
             bool ok = true;
-            for (int s = 0; s < job.nk; ++s) {
-                const int st = s % kStages;
-                const uint32_t ph = (s / kStages) & 1;
-                if (!mbar_wait(&bars->conv[st], ph, abort)) {
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                const Job job = sched.job(t);
+                if (job.nk <= 0) continue;
+                const int slot = lt & 1;
+                const uint32_t use = static_cast<uint32_t>(lt >> 1);
+                if (!mbar_wait(&bars->acc_empty[slot], (use & 1u) ^ 1u, abort)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a = smem_u32(smem + st * kStageBytes);
-                const uint32_t alo = a + kTileBytes, b = a + 2 * kTileBytes, blo = a + 3 * kTileBytes;
+                const uint32_t acc = tmem + slot * BN;
+                for (int s = 0; s < job.nk; ++s, ++it) {
+                    const int st = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1;
+                    if (!mbar_wait(&bars->conv[st], ph, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a = smem_u32(smem + st * kStageBytes);
+                    const uint32_t alo = a + kTileBytes, b = a + 2 * kTileBytes, blo = a + 3 * kTileBytes;
 #pragma unroll
-                for (int kk = 0; kk < BK / 8; ++kk) {
-                    const uint64_t ah = operand_desc<A_MN>(a, kk), al = operand_desc<A_MN>(alo, kk);
-                    const uint64_t bh = operand_desc<B_MN>(b, kk), bl = operand_desc<B_MN>(blo, kk);
-                    mma_tf32_ss(tmem, ah, bh, kIdesc, (s > 0 || kk > 0) ? 1u : 0u);
-                    mma_tf32_ss(tmem, ah, bl, kIdesc, 1u);
-                    mma_tf32_ss(tmem, al, bh, kIdesc, 1u);
+                    for (int kk = 0; kk < BK / 8; ++kk) {
+                        const uint64_t ah = operand_desc<A_MN>(a, kk), al = operand_desc<A_MN>(alo, kk);
+                        const uint64_t bh = operand_desc<B_MN>(b, kk), bl = operand_desc<B_MN>(blo, kk);
+                        mma_tf32_ss(acc, ah, bh, kIdesc, (s > 0 || kk > 0) ? 1u : 0u);
+                        mma_tf32_ss(acc, ah, bl, kIdesc, 1u);
+                        mma_tf32_ss(acc, al, bh, kIdesc, 1u);
+                    }
+                    mma_commit(&bars->empty[st]);
                 }
-                mma_commit(&bars->empty[st]);
+                if (!ok) break;
+                mma_commit(&bars->acc_full[slot]);
+                ++lt;
             }
-            if (ok) mma_commit(&bars->acc_full);
             mma_commit(&bars->drain);
             volatile int no_abort = 0;
             if (!mbar_wait(&bars->drain, 0, &no_abort)) *abort = 1;
         }
-    } else {
-        // ---- split each stage into hi (in place) and lo
-        const int t = threadIdx.x - 64;
+    } else if (warp < 6) {
+        // ---------------------------------------------------- split into hi / lo
+        const int t0 = threadIdx.x - 64;
+        int it = 0;
         bool ok = true;
-        for (int s = 0; s < job.nk; ++s) {
-            const int st = s % kStages;
-            const uint32_t ph = (s / kStages) & 1;
-            if (!mbar_wait(&bars->full[st], ph, abort)) {
-                ok = false;
-                break;
-            }
-            float4* a = reinterpret_cast<float4*>(smem + st * kStageBytes);
-            float4* alo = a + kTileBytes / 16;
-            float4* b = a + 2 * (kTileBytes / 16);
-            float4* blo = a + 3 * (kTileBytes / 16);
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            const Job job = sched.job(t);
+            for (int s = 0; s < job.nk; ++s, ++it) {
+                const int st = it % kStages;
+                const uint32_t ph = (it / kStages) & 1;
+                if (!mbar_wait(&bars->full[st], ph, abort)) {
+                    ok = false;
+                    break;
+                }
+                float4* a = reinterpret_cast<float4*>(smem + st * kStageBytes);
+                float4* alo = a + kTileBytes / 16;
+                float4* b = a + 2 * (kTileBytes / 16);
+                float4* blo = a + 3 * (kTileBytes / 16);
 #pragma unroll 4
-            for (int i = t; i < kTileBytes / 16; i += 128) {
-                float4 x = a[i], h, l;
-                h.x = tf32_hi(x.x); h.y = tf32_hi(x.y); h.z = tf32_hi(x.z); h.w = tf32_hi(x.w);
-                l.x = x.x - h.x; l.y = x.y - h.y; l.z = x.z - h.z; l.w = x.w - h.w;
-                a[i] = h;
-                alo[i] = l;
-                x = b[i];
-                h.x = tf32_hi(x.x); h.y = tf32_hi(x.y); h.z = tf32_hi(x.z); h.w = tf32_hi(x.w);
-                l.x = x.x - h.x; l.y = x.y - h.y; l.z = x.z - h.z; l.w = x.w - h.w;
-                b[i] = h;
-                blo[i] = l;
+                for (int i = t0; i < kTileBytes / 16; i += 128) {
+                    float4 x = a[i], h, l;
+                    h.x = tf32_hi(x.x); h.y = tf32_hi(x.y); h.z = tf32_hi(x.z); h.w = tf32_hi(x.w);
+                    l.x = x.x - h.x; l.y = x.y - h.y; l.z = x.z - h.z; l.w = x.w - h.w;
+                    a[i] = h;
+                    alo[i] = l;
+                    x = b[i];
+                    h.x = tf32_hi(x.x); h.y = tf32_hi(x.y); h.z = tf32_hi(x.z); h.w = tf32_hi(x.w);
+                    l.x = x.x - h.x; l.y = x.y - h.y; l.z = x.z - h.z; l.w = x.w - h.w;
+                    b[i] = h;
+                    blo[i] = l;
+                }
+                fence_async_smem();
+                mbar_arrive(&bars->conv[st]);
             }
-            fence_async_smem();
-            mbar_arrive(&bars->conv[st]);
         }
-        // ---- epilogue: TMEM -> registers -> scheduler
-        if (ok && mbar_wait(&bars->acc_full, 0, abort)) {
+    } else {
+        // ---------------------------------------------------- epilogue
+        const int q = warp & 3;  // TMEM lane quarter of this warp
+        const int row = q * 32 + lane;
+        int lt = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+            const Job job = sched.job(t);
+            if (job.nk <= 0) continue;
+            const int slot = lt & 1;
+            const uint32_t use = static_cast<uint32_t>(lt >> 1);
+            if (!mbar_wait(&bars->acc_full[slot], use & 1u, abort)) break;
             tc_fence_after();
-            const int q = warp & 3;
-            const int row = q * 32 + lane;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 float v[32];
-                tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c * 32, v);
+                tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + slot * BN + c * 32, v);
                 sched.store(job, row, c * 32, v);
             }
+            tc_fence_before();
+            mbar_arrive(&bars->acc_empty[slot]);
+            ++lt;
         }
     }
 
@@ -228,12 +268,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <class Sched, bool A_MN, bool B_MN>
 inline cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const Sched& sched,
-                          int tiles, int32_t* status, cudaStream_t stream) {
+                          int tiles, int32_t* status, cudaStream_t stream, int sms) {
     auto kern = gemm_tf32x3_kernel<Sched, A_MN, B_MN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     if (tiles <= 0) return cudaSuccess;
-    kern<<<tiles, kThreads, kSmemBytes, stream>>>(ta, tb, sched, status);
+    const int grid = tiles < sms ? tiles : sms;
+    kern<<<grid, kThreads, kSmemBytes, stream>>>(ta, tb, sched, tiles, status);
     return cudaGetLastError();
 }
 

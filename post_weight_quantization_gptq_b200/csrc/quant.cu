@@ -49,12 +49,74 @@ __global__ void permute_rows_kernel(float* __restrict__ W, int64_t r, int64_t d,
     }
 }
 
-// Column j of the block lives in lane ((j % 32) / 4) of its row group, in
-// register 4 * (j / 32) + (j % 4): each lane owns four runs of 4 columns, 32
-// apart, so the 8 lanes of a row read one 128-byte row segment of the U
-// block per vector load without bank conflicts.
-__device__ __forceinline__ int col_of(int t, int l) { return 32 * (t >> 2) + 4 * l + (t & 3); }
+// Register layout: the block's 128 columns form four 32-column chunks; in
+// every chunk lane l of a row's 8-lane group owns columns 4l .. 4l+3, so the
+// 8 lanes of a row read one 128-byte row segment of the U block per vector
+// load without bank conflicts.  A lane keeps the chunk being quantized in
+// cur[4] and the later chunks in nxt[12]; after each chunk the window
+// rotates, so every register index below is a compile-time constant while the
+// chunk loop stays rolled (the code fits the instruction cache).
+struct GroupParams {
+    float s, inv_s, zf;
+};
 
+// Scale / zero point of the group [c0 + j, c0 + j + g) of this row from its
+// current weights: the group's columns in this block (cur: chunk m, nxt:
+// chunks m+1..3) plus, for groups wider than the block, the later columns in
+// W (which already hold every earlier block's feedback).  Range widened to
+// contain 0; an all-zero group gets the range [-1, 1] (zero point exactly
+// 2^(bits-1)).
+__device__ __forceinline__ GroupParams group_params(const float (&cur)[4], const float (&nxt)[12],
+                                                    int m, int jj, int l, int g, int bw,
+                                                    const float* __restrict__ wrow, int64_t c0,
+                                                    int64_t d, bool live, int bits) {
+    const int j = 32 * m + jj;
+    float lo = 0.f, hi = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int c = 32 * m + 4 * l + i;
+        if (c >= j && c < j + g && c < bw) {
+            lo = fminf(lo, cur[i]);
+            hi = fmaxf(hi, cur[i]);
+        }
+    }
+#pragma unroll
+    for (int s = 0; s < 3; ++s)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int c = 32 * (m + 1 + s) + 4 * l + i;
+            if (m + 1 + s < 4 && c < j + g && c < bw) {
+                lo = fminf(lo, nxt[4 * s + i]);
+                hi = fmaxf(hi, nxt[4 * s + i]);
+            }
+        }
+    const int64_t gend = (c0 + j + g < d) ? c0 + j + g : d;
+    if (live && gend > c0 + bw) {
+        for (int64_t c = c0 + bw + l; c < gend; c += 8) {
+            const float v = wrow[c];
+            lo = fminf(lo, v);
+            hi = fmaxf(hi, v);
+        }
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    const float maxq = static_cast<float>((1 << bits) - 1);
+    GroupParams p;
+    if (hi == lo) {
+        p.s = 2.f / maxq;
+        p.zf = static_cast<float>(1 << (bits - 1));
+    } else {
+        p.s = (hi - lo) / maxq;
+        p.zf = rintf(-lo / p.s);
+    }
+    p.inv_s = 1.f / p.s;
+    return p;
+}
+
+template <bool kSmallGroup>  // group_size < 32: groups start inside a chunk
 __global__ void __launch_bounds__(kWarps * 32)
     block_quant_kernel(const __grid_constant__ CUtensorMap tmu, float* __restrict__ W, int64_t r,
                        int64_t d, int64_t ldw, int64_t c0, int bw, int bits, int g,
@@ -94,126 +156,120 @@ __global__ void __launch_bounds__(kWarps * 32)
                         (lane >> 3);
     const bool live = row < r;
     const float maxq = static_cast<float>((1 << bits) - 1);
-
-    float w[16], ev[16];
-    uint32_t qv[16];
+    float* wrow = W + (live ? row : 0) * ldw;
     const bool vec = (ldw & 3) == 0 && bw == kBlock;
+
+    float cur[4], nxt[12];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
+        float v[4];
         if (live && vec) {
-            const float4 v = *reinterpret_cast<const float4*>(W + row * ldw + c0 + 32 * m + 4 * l);
-            w[4 * m] = v.x; w[4 * m + 1] = v.y; w[4 * m + 2] = v.z; w[4 * m + 3] = v.w;
+            const float4 t = *reinterpret_cast<const float4*>(wrow + c0 + 32 * m + 4 * l);
+            v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
         } else {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int c = 32 * m + 4 * l + i;
-                w[4 * m + i] = (live && c < bw) ? W[row * ldw + c0 + c] : 0.f;
+                v[i] = (live && c < bw) ? wrow[c0 + c] : 0.f;
             }
         }
-    }
 #pragma unroll
-    for (int t = 0; t < 16; ++t) {
-        ev[t] = 0.f;
-        qv[t] = 0;
+        for (int i = 0; i < 4; ++i) {
+            if (m == 0) cur[i] = v[i];
+            else nxt[4 * (m - 1) + i] = v[i];
+        }
     }
 
-    float s = 1.f, inv_s = 1.f, zf = 0.f;
+    GroupParams gp{1.f, 1.f, 0.f};
     if (live && (c0 % g) != 0) {
         // this block continues a group opened by an earlier block (group
         // size > block): take that group's scale and zero point
         const int64_t grp = c0 / g;
-        s = scales[grp * r + row];
-        zf = static_cast<float>(zeros[grp * r + row]);
-        inv_s = 1.f / s;
-    }
-#pragma unroll
-    for (int j = 0; j < kBlock; ++j) {
-        if (j < bw) {
-        if (((c0 + j) % g) == 0) {
-            // group [c0 + j, c0 + j + g): current weights, range widened to 0
-            float lo = 0.f, hi = 0.f;
-#pragma unroll
-            for (int t = 0; t < 16; ++t) {
-                const int c = col_of(t, l);
-                if (c >= j && c < j + g && c < bw) {
-                    lo = fminf(lo, w[t]);
-                    hi = fmaxf(hi, w[t]);
-                }
-            }
-            const int64_t gend = (c0 + j + g < d) ? c0 + j + g : d;
-            if (live && gend > c0 + bw) {
-                // group continues past this block (group_size > block): those
-                // columns already hold every earlier block's feedback
-                for (int64_t c = c0 + bw + l; c < gend; c += 8) {
-                    const float v = W[row * ldw + c];
-                    lo = fminf(lo, v);
-                    hi = fmaxf(hi, v);
-                }
-            }
-#pragma unroll
-            for (int o = 1; o < 8; o <<= 1) {
-                lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-                hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-            }
-            if (hi == lo) {
-                // all-zero group: range [-1, 1], zero point exactly 2^(bits-1)
-                s = 2.f / maxq;
-                zf = static_cast<float>(1 << (bits - 1));
-            } else {
-                s = (hi - lo) / maxq;
-                zf = rintf(-lo / s);
-            }
-            inv_s = 1.f / s;
-            if (live && l == 0) {
-                const int64_t grp = (c0 + j) / g;
-                scales[grp * r + row] = s;
-                zeros[grp * r + row] = static_cast<int32_t>(zf);
-            }
-        }
-        const int owner = (j & 31) >> 2;
-        const int tj = 4 * (j >> 5) + (j & 3);
-        const float wj = __shfl_sync(0xffffffffu, w[tj], gbase + owner);
-        const float qf = fminf(fmaxf(rintf(wj * inv_s) + zf, 0.f), maxq);
-        const float e = (wj - s * (qf - zf)) * dinv[j];
-        if (l == owner) {
-            qv[tj] = static_cast<uint32_t>(qf);
-            ev[tj] = e;
-        }
-        // feedback into this block's later columns (U row j is zero at and
-        // left of the diagonal, so earlier columns are untouched)
-        const float4* urow = reinterpret_cast<const float4*>(Us + j * kBlock);
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const float4 u = urow[8 * m + l];
-            w[4 * m + 0] = fmaf(-e, u.x, w[4 * m + 0]);
-            w[4 * m + 1] = fmaf(-e, u.y, w[4 * m + 1]);
-            w[4 * m + 2] = fmaf(-e, u.z, w[4 * m + 2]);
-            w[4 * m + 3] = fmaf(-e, u.w, w[4 * m + 3]);
-        }
-        }
+        gp.s = scales[grp * r + row];
+        gp.zf = static_cast<float>(zeros[grp * r + row]);
+        gp.inv_s = 1.f / gp.s;
     }
 
-    if (!live) return;
-#pragma unroll
+#pragma unroll 1
     for (int m = 0; m < 4; ++m) {
-        const int cb = 32 * m + 4 * l;
-        *reinterpret_cast<float4*>(err_out + row * kBlock + cb) =
-            make_float4(ev[4 * m], ev[4 * m + 1], ev[4 * m + 2], ev[4 * m + 3]);
-        if (vec) {
-            *reinterpret_cast<float4*>(W + row * ldw + c0 + cb) =
-                make_float4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]);
+        if (32 * m >= bw) break;
+        if (!kSmallGroup && ((c0 + 32 * m) % g) == 0) {
+            gp = group_params(cur, nxt, m, 0, l, g, bw, wrow, c0, d, live, bits);
+            if (live && l == 0) {
+                const int64_t grp = (c0 + 32 * m) / g;
+                scales[grp * r + row] = gp.s;
+                zeros[grp * r + row] = static_cast<int32_t>(gp.zf);
+            }
         }
-        if (vec && (d & 3) == 0) {
-            *reinterpret_cast<uint32_t*>(codes + row * d + c0 + cb) =
-                qv[4 * m] | (qv[4 * m + 1] << 8) | (qv[4 * m + 2] << 16) | (qv[4 * m + 3] << 24);
+        float ev[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t qv[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+            const int j = 32 * m + jj;
+            if (j < bw) {
+                if (kSmallGroup && ((c0 + j) % g) == 0) {
+                    gp = group_params(cur, nxt, m, jj, l, g, bw, wrow, c0, d, live, bits);
+                    if (live && l == 0) {
+                        const int64_t grp = (c0 + j) / g;
+                        scales[grp * r + row] = gp.s;
+                        zeros[grp * r + row] = static_cast<int32_t>(gp.zf);
+                    }
+                }
+                const float wj = __shfl_sync(0xffffffffu, cur[jj & 3], gbase + (jj >> 2));
+                const float qf = fminf(fmaxf(rintf(wj * gp.inv_s) + gp.zf, 0.f), maxq);
+                const float e = (wj - gp.s * (qf - gp.zf)) * dinv[j];
+                if (l == (jj >> 2)) {
+                    qv[jj & 3] = static_cast<uint32_t>(qf);
+                    ev[jj & 3] = e;
+                }
+                // feedback into this block's later columns (U row j is zero
+                // at and left of the diagonal, so earlier columns are untouched)
+                const float4* urow = reinterpret_cast<const float4*>(Us + j * kBlock);
+                float4 u = urow[8 * m + l];
+                cur[0] = fmaf(-e, u.x, cur[0]);
+                cur[1] = fmaf(-e, u.y, cur[1]);
+                cur[2] = fmaf(-e, u.z, cur[2]);
+                cur[3] = fmaf(-e, u.w, cur[3]);
+#pragma unroll
+                for (int s = 0; s < 3; ++s) {
+                    if (m + 1 + s < 4) {
+                        u = urow[8 * (m + 1 + s) + l];
+                        nxt[4 * s + 0] = fmaf(-e, u.x, nxt[4 * s + 0]);
+                        nxt[4 * s + 1] = fmaf(-e, u.y, nxt[4 * s + 1]);
+                        nxt[4 * s + 2] = fmaf(-e, u.z, nxt[4 * s + 2]);
+                        nxt[4 * s + 3] = fmaf(-e, u.w, nxt[4 * s + 3]);
+                    }
+                }
+            }
         }
+        // chunk m done: pre-quantization weights, scaled errors, codes
+        if (live) {
+            const int cb = 32 * m + 4 * l;
+            *reinterpret_cast<float4*>(err_out + row * kBlock + cb) =
+                make_float4(ev[0], ev[1], ev[2], ev[3]);
+            if (vec) {
+                *reinterpret_cast<float4*>(wrow + c0 + cb) = make_float4(cur[0], cur[1], cur[2], cur[3]);
+            }
+            if (vec && (d & 3) == 0) {
+                *reinterpret_cast<uint32_t*>(codes + row * d + c0 + cb) =
+                    qv[0] | (qv[1] << 8) | (qv[2] << 16) | (qv[3] << 24);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int c = cb + i;
+                if (c < bw) {
+                    if (!vec) wrow[c0 + c] = cur[i];
+                    if (!(vec && (d & 3) == 0)) codes[row * d + c0 + c] = static_cast<uint8_t>(qv[i]);
+                }
+            }
+        }
+        // rotate the window
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int c = cb + i;
-            if (c < bw) {
-                if (!vec) W[row * ldw + c0 + c] = w[4 * m + i];
-                if (!(vec && (d & 3) == 0)) codes[row * d + c0 + c] = static_cast<uint8_t>(qv[4 * m + i]);
-            }
+            cur[i] = nxt[i];
+            nxt[i] = nxt[4 + i];
+            nxt[4 + i] = nxt[8 + i];
+            nxt[8 + i] = 0.f;
         }
     }
 }
@@ -277,7 +333,9 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
         !make_tmap_2d(&tErr, false, err, kBlock, d_row, kBlock, 32, 128, Swz::k128))
         return GPTQ_ERR_INVALID_ARG;
     const size_t q_smem = (kBlock * kBlock + kBlock) * sizeof(float) + 1024;
-    if (cudaFuncSetAttribute(block_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const bool small_group = g < 32;
+    auto qkern = small_group ? block_quant_kernel<true> : block_quant_kernel<false>;
+    if (cudaFuncSetAttribute(qkern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(q_smem)) != cudaSuccess)
         return GPTQ_ERR_CUDA;
     const unsigned qgrid = static_cast<unsigned>((d_row + kRowsPerCta - 1) / kRowsPerCta);
@@ -285,7 +343,7 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
     int64_t launches = 1;
     for (int64_t c0 = 0; c0 < d_col; c0 += kBlock) {
         const int bw = static_cast<int>((d_col - c0 < kBlock) ? d_col - c0 : kBlock);
-        block_quant_kernel<<<qgrid, kWarps * 32, q_smem, stream>>>(
+        qkern<<<qgrid, kWarps * 32, q_smem, stream>>>(
             tU, W, d_row, d_col, ldw, c0, bw, bits, g, codes, scales, zeros, err, status);
         ++launches;
         const int64_t rest = d_col - c0 - bw;
@@ -293,7 +351,7 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
             const int nt = static_cast<int>((rest + 127) / 128);
             LazySched ls{W, ldw, static_cast<int>(d_row), static_cast<int>(d_col),
                          static_cast<int>(c0), static_cast<int>(c0 + bw), mt};
-            if (g3::launch<LazySched, false, true>(tErr, tUmn, ls, mt * nt, status, stream) !=
+            if (g3::launch<LazySched, false, true>(tErr, tUmn, ls, mt * nt, status, stream, num_sms()) !=
                 cudaSuccess)
                 return GPTQ_ERR_CUDA;
             ++launches;
