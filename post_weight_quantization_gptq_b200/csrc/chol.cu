@@ -21,8 +21,11 @@
 //   potrf_inv_128_kernel  L_kk = chol(A_kk) and L_kk^-1 (one CTA)
 //   panel solve           L_ik = A_ik L_kk^-T          (3xTF32 tcgen05 GEMM)
 //   trailing update       A_ij -= L_ik L_jk^T, i >= j  (3xTF32 tcgen05 GEMM)
-// then L^-1 by recursive doubling (X_CA = -X_CC (L_CA X_AA)) on the same GEMM.
+// and L^-1 built block row by block row on the same GEMM,
+//   X[k, :k] = -X_kk (L[k, :k] X[:k, :k]),
+// in the shadow of the panel chain (see launch_chol_inverse).
 #include <cmath>
+#include <mutex>
 
 #include "common.cuh"
 #include "gemm_tf32x3.cuh"
@@ -305,13 +308,24 @@ struct TrsmSched {
 };
 
 // Trailing update: P[I, J] -= L[I, panel] L[J, panel]^T on lower tiles.
+// part 0: every lower tile; 1: the first tile column (the next panel);
+// 2: the tiles right of it.
 struct SyrkSched {
     float* P;
     int64_t ldp;
-    int d, kb, kw, s0;
+    int d, kb, kw, s0, part;
     __device__ g3::Job job(int t) const {
         int I, J;
-        tri_coords(t, I, J);
+        if (part == 1) {
+            I = t;
+            J = 0;
+        } else {
+            tri_coords(t, I, J);
+            if (part == 2) {
+                ++I;
+                ++J;
+            }
+        }
         return {s0 + NB * I, s0 + NB * J, kb, kb, (kw + 31) / 32};
     }
     __device__ void store(const g3::Job& jb, int row, int col0, const float (&v)[32]) const {
@@ -329,50 +343,39 @@ struct SyrkSched {
     }
 };
 
-// Recursive doubling, step 1: T^T[a][c] = sum_k X[k][a] L[c][k] into P[a][c].
-struct Trinv1Sched {
+// Block row kb of L^-1, left of the diagonal, once L_kk^-1 is known:
+//   X[kb.., :kb] = -X_kk (L[kb.., :kb] X[:kb, :kb]).
+// Step 1: T^T[a][m] = sum_{a <= j < kb} X[j][a] L[kb+m][j], stored in the
+// free upper triangle at P[a][kb+m] (a < kb).
+struct XRow1Sched {
     float* P;
     int64_t ldp;
-    int d, s, tiles;  // tiles = s / NB per side
+    int d, kb, kw;
     __device__ g3::Job job(int t) const {
-        const int per = tiles * tiles;
-        const int pair = t / per, rem = t % per;
-        const int ct = rem / tiles, at = rem % tiles;
-        const int A0 = 2 * s * pair, C0 = A0 + s;
-        const int c0 = C0 + NB * ct, a0 = A0 + NB * at;
-        if (c0 >= d) return {0, 0, 0, 0, 0};
-        return {a0, c0, a0, a0, (C0 - a0) / 32};
+        const int a0 = NB * t;
+        return {a0, kb, a0, a0, (kb - a0) / 32};
     }
     __device__ void store(const g3::Job& jb, int row, int col0, const float (&v)[32]) const {
-        float* dst = P + static_cast<int64_t>(jb.m0 + row) * ldp + jb.n0 + col0;
-        if (jb.n0 + col0 + 32 <= d) {
+        float* dst = P + static_cast<int64_t>(jb.m0 + row) * ldp + kb + col0;
+        if (col0 + 32 <= kw) {
             put32<false>(dst, v, 1.f);
         } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-                if (jb.n0 + col0 + j < d) dst[j] = v[j];
+                if (col0 + j < kw) dst[j] = v[j];
         }
     }
 };
 
-// Step 2: X[c][a] = -sum_{C0 <= k <= c} X[c][k] T[k][a], T[k][a] = P[a][k].
-struct Trinv2Sched {
+// Step 2: X[kb+m][a] = -sum_j X[kb+m][kb+j] T[j][a], T[j][a] = P[a][kb+j].
+struct XRow2Sched {
     float* X;
     int64_t ldx;
-    int d, s, tiles;
-    __device__ g3::Job job(int t) const {
-        const int per = tiles * tiles;
-        const int pair = t / per, rem = t % per;
-        const int ct = rem / tiles, at = rem % tiles;
-        const int A0 = 2 * s * pair, C0 = A0 + s;
-        const int c0 = C0 + NB * ct, a0 = A0 + NB * at;
-        if (c0 >= d) return {0, 0, 0, 0, 0};
-        return {c0, a0, C0, C0, (c0 + NB - C0) / 32};
-    }
+    int d, kb, kw;
+    __device__ g3::Job job(int t) const { return {kb, NB * t, kb, kb, (kw + 31) / 32}; }
     __device__ void store(const g3::Job& jb, int row, int col0, const float (&v)[32]) const {
-        const int r = jb.m0 + row;
-        if (r >= d) return;
-        put32<false>(X + static_cast<int64_t>(r) * ldx + jb.n0 + col0, v, -1.f);
+        if (row >= kw) return;
+        put32<false>(X + static_cast<int64_t>(kb + row) * ldx + jb.n0 + col0, v, -1.f);
     }
 };
 
@@ -389,6 +392,38 @@ __global__ void flip_kernel(const float* __restrict__ X, int64_t ldx, float* __r
 
 size_t chol_workspace_bytes(int64_t) { return 0; }
 
+// Side stream and events of the lookahead schedule (created once per device;
+// streams and events, no device memory).
+namespace {
+struct Lookahead {
+    cudaStream_t side = nullptr;
+    cudaEvent_t ev[8] = {};  // [0..3] panel column ready, [4..7] trailing update done
+    bool ok = false;
+};
+std::mutex g_la_mutex;
+Lookahead g_la[64];
+
+// Caller holds g_la_mutex.
+Lookahead* lookahead_resources() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    Lookahead& la = g_la[dev];
+    if (!la.ok) {
+        if (cudaStreamCreateWithFlags(&la.side, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+        for (auto& e : la.ev)
+            if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+        la.ok = true;
+    }
+    return &la;
+}
+}  // namespace
+
+// Lookahead schedule.  The caller's stream runs the panel chain
+//   potrf(k) -> panel solve(k) -> update of panel k+1's column -> potrf(k+1)
+// while a side stream runs the rest of each trailing update and block row k
+// of L^-1 in its shadow.  Ordering: the update of panel k+1's column waits
+// for the previous panel's rest-of-update (both touch that column); potrf and
+// the panel solve of k+1 then see every update they need.
 gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, float* U,
                                 int32_t* status, void*, cudaStream_t stream) {
     const int64_t ldp = d;
@@ -401,34 +436,67 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
     if (cudaFuncSetAttribute(potrf_inv_128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kDiagSmem) != cudaSuccess)
         return GPTQ_ERR_CUDA;
+    // one enqueue sequence at a time per process: the side stream and the
+    // event ring are shared by every call on a device
+    std::lock_guard<std::mutex> lock(g_la_mutex);
+    Lookahead* la = lookahead_resources();
+    if (la == nullptr) return GPTQ_ERR_CUDA;
+    const int sms = num_sms();
+    const int side_sms = sms > 32 ? sms - 16 : sms;  // leave SMs for the panel chain
+    cudaStream_t side = la->side;
+    const int npan = static_cast<int>((d + NB - 1) / NB);
     int64_t launches = 0;
-    for (int64_t kb = 0; kb < d; kb += NB) {
+    bool side_used = false;
+    // the side stream starts after everything the caller queued before us
+    if (cudaEventRecord(la->ev[0], stream) != cudaSuccess ||
+        cudaStreamWaitEvent(side, la->ev[0], 0) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
+    for (int k = 0; k < npan; ++k) {
+        const int64_t kb = static_cast<int64_t>(k) * NB;
         const int kw = static_cast<int>((d - kb < NB) ? d - kb : NB);
         potrf_inv_128_kernel<<<1, kDiagThreads, kDiagSmem, stream>>>(P, ldp, kb, kw, X, ldx, status);
         ++launches;
         const int64_t m = d - kb - kw;
+        const int mt = static_cast<int>((m + NB - 1) / NB);
+        cudaEvent_t ready = la->ev[k & 3], done = la->ev[4 + (k & 3)];
         if (m > 0) {
-            const int mt = static_cast<int>((m + NB - 1) / NB);
             TrsmSched ts{P, ldp, di, static_cast<int>(kb), kw};
-            if (g3::launch<TrsmSched, false, false>(tP, tX, ts, mt, status, stream, num_sms()) != cudaSuccess)
+            if (g3::launch<TrsmSched, false, false>(tP, tX, ts, mt, status, stream, sms) != cudaSuccess)
                 return GPTQ_ERR_CUDA;
-            SyrkSched ss{P, ldp, di, static_cast<int>(kb), kw, static_cast<int>(kb + kw)};
-            if (g3::launch<SyrkSched, false, false>(tP, tP, ss, mt * (mt + 1) / 2, status, stream, num_sms()) !=
-                cudaSuccess)
+            if (k > 0 && cudaStreamWaitEvent(stream, la->ev[4 + ((k - 1) & 3)], 0) != cudaSuccess)
+                return GPTQ_ERR_CUDA;
+            SyrkSched nx{P, ldp, di, static_cast<int>(kb), kw, static_cast<int>(kb + kw), 1};
+            if (g3::launch<SyrkSched, false, false>(tP, tP, nx, mt, status, stream, sms) != cudaSuccess)
                 return GPTQ_ERR_CUDA;
             launches += 2;
         }
-    }
-    for (int64_t s = NB; s < d; s *= 2) {
-        const int64_t pairs = (d + 2 * s - 1) / (2 * s);
-        const int tiles = static_cast<int>(s / NB);
-        const int grid = static_cast<int>(pairs * tiles * tiles);
-        Trinv1Sched t1{P, ldp, di, static_cast<int>(s), tiles};
-        Trinv2Sched t2{X, ldx, di, static_cast<int>(s), tiles};
-        if (g3::launch<Trinv1Sched, true, false>(tXmn, tP, t1, grid, status, stream, num_sms()) != cudaSuccess ||
-            g3::launch<Trinv2Sched, false, false>(tX, tP, t2, grid, status, stream, num_sms()) != cudaSuccess)
+        if (cudaEventRecord(ready, stream) != cudaSuccess ||
+            cudaStreamWaitEvent(side, ready, 0) != cudaSuccess)
             return GPTQ_ERR_CUDA;
-        launches += 2;
+        if (mt > 1) {
+            SyrkSched rs{P, ldp, di, static_cast<int>(kb), kw, static_cast<int>(kb + kw), 2};
+            if (g3::launch<SyrkSched, false, false>(tP, tP, rs, mt * (mt + 1) / 2 - mt, status, side,
+                                                    side_sms) != cudaSuccess)
+                return GPTQ_ERR_CUDA;
+            ++launches;
+        }
+        if (cudaEventRecord(done, side) != cudaSuccess) return GPTQ_ERR_CUDA;
+        if (k > 0) {
+            XRow1Sched x1{P, ldp, di, static_cast<int>(kb), kw};
+            XRow2Sched x2{X, ldx, di, static_cast<int>(kb), kw};
+            if (g3::launch<XRow1Sched, true, false>(tXmn, tP, x1, k, status, side, side_sms) !=
+                    cudaSuccess ||
+                g3::launch<XRow2Sched, false, false>(tX, tP, x2, k, status, side, side_sms) !=
+                    cudaSuccess)
+                return GPTQ_ERR_CUDA;
+            launches += 2;
+        }
+        side_used = true;
+    }
+    if (side_used) {
+        if (cudaEventRecord(la->ev[4], side) != cudaSuccess ||
+            cudaStreamWaitEvent(stream, la->ev[4], 0) != cudaSuccess)
+            return GPTQ_ERR_CUDA;
     }
     dim3 grid(static_cast<unsigned>((d + 255) / 256 < 8 ? (d + 255) / 256 : 8),
               static_cast<unsigned>(d));
