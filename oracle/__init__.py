@@ -23,6 +23,7 @@ from .gptq import (  # noqa: F401
     eliminate,
     gptq_blocked,
     gptq_columns,
+    gptq_columns_u,
     hessian,
     hessian_rows,
     inverse,
@@ -35,4 +36,5 @@ from .gptq import (  # noqa: F401
     quantize_layer,
     rtn,
     unpack,
+    upper_factor,
 )

@@ -58,8 +58,11 @@ def _lib():
         lib.orc_quantize.argtypes = [ctypes.c_double, ctypes.c_double, ctypes.c_int32, ctypes.c_int]
         lib.orc_quantize.restype = ctypes.c_int32
         lib.orc_gptq_columns.argtypes = [P, i64, i64, P, ctypes.c_int, i64, P, P, P, P,
-                                         P, P, P, ctypes.c_double, P, P]
+                                         P, P, P, P, ctypes.c_double, P, P]
         lib.orc_gptq_columns.restype = ctypes.c_int
+        lib.orc_gptq_columns_u.argtypes = [P, i64, i64, P, ctypes.c_int, i64, P, P, P,
+                                           P, P, P, P, ctypes.c_double, P, P]
+        lib.orc_gptq_columns_u.restype = ctypes.c_int
         lib.orc_eliminate.argtypes = [P, i64, i64, P]
         lib.orc_eliminate.restype = ctypes.c_int
         lib.orc_gptq_blocked.argtypes = [P, i64, i64, P, ctypes.c_int, i64, i64, P, P, P]
@@ -262,7 +265,7 @@ class GPTQResult:
 
 
 def gptq_columns(W0, Hinv, bits: int, group_size: int, want_U: bool = False,
-                 forced_codes=None, forced_zeros=None, forced_w=None,
+                 forced_codes=None, forced_zeros=None, forced_w=None, forced_scales=None,
                  tau: float = 0.0) -> GPTQResult:
     """The OBQ/GPTQ loop one column at a time with explicit elimination of
     H^-1 after every column [OBQ].
@@ -272,7 +275,9 @@ def gptq_columns(W0, Hinv, bits: int, group_size: int, want_U: bool = False,
     adopted, so one tie decided the other way does not desynchronise the rest
     of its row: a code is valid when it is the oracle's own rounding or a
     neighbouring level whose rounding boundary lies within
-    tau + |forced_w - w| / s of the oracle's real level w / s + z."""
+    tau + |forced_w - w| / s + |y - z| |forced_s - s| / s of the oracle's real
+    level y = w / s + z (the other side's own deviation in the decision's
+    inputs)."""
     W = _f64(W0).copy()
     r, d = W.shape
     g = _g(d, group_size)
@@ -285,10 +290,11 @@ def gptq_columns(W0, Hinv, bits: int, group_size: int, want_U: bool = False,
     fc = None if forced_codes is None else np.ascontiguousarray(forced_codes, dtype=np.uint8)
     fz = None if forced_zeros is None else np.ascontiguousarray(forced_zeros, dtype=np.int32)
     fw = None if forced_w is None else _f64(forced_w)
+    fs = None if forced_scales is None else _f64(forced_scales)
     stats = np.zeros(6, dtype=np.int64)
     max_dev = ctypes.c_double(0.0)
     rc = _lib().orc_gptq_columns(_ptr(W), r, d, _ptr(M), bits, g, _ptr(codes), _ptr(scales),
-                                 _ptr(zeros), _ptr(U), _ptr(fc), _ptr(fz), _ptr(fw),
+                                 _ptr(zeros), _ptr(U), _ptr(fc), _ptr(fz), _ptr(fw), _ptr(fs),
                                  float(tau), _ptr(stats), ctypes.byref(max_dev))
     if rc != 0:
         raise np.linalg.LinAlgError(f"oracle column loop failed ({rc})")
@@ -296,6 +302,44 @@ def gptq_columns(W0, Hinv, bits: int, group_size: int, want_U: bool = False,
               zero_ties=int(stats[2]), zero_invalid=int(stats[3]),
               elements=int(stats[4]), groups=int(stats[5]), max_dev=max_dev.value)
     return GPTQResult(codes, scales, zeros, W, U, st)
+
+
+def upper_factor(Hd) -> np.ndarray:
+    """U upper with U^T U = inverse(Hd), from library routines (a Cholesky of
+    the library inverse).  The elimination rows of `eliminate` are this same
+    matrix; the pins check the two against each other.  Used where the
+    explicit elimination is too slow (d > 4096)."""
+    return np.ascontiguousarray(np.linalg.cholesky(inverse(Hd)).T)
+
+
+def gptq_columns_u(W0, U, bits: int, group_size: int, forced_codes=None, forced_zeros=None,
+                   forced_w=None, forced_scales=None, tau: float = 0.0) -> GPTQResult:
+    """The OBQ column loop driven by U's rows: W_F <- W_F - (e / U_ii) U_{i,F}
+    [OBQ] with row i of the reduced inverse equal to U_ii U[i, i:].  Same
+    teacher-forcing options as gptq_columns."""
+    W = _f64(W0).copy()
+    r, d = W.shape
+    g = _g(d, group_size)
+    ng = n_groups(d, group_size)
+    Uc = np.ascontiguousarray(U, dtype=np.float64)
+    codes = np.zeros((r, d), dtype=np.uint8)
+    scales = np.zeros((ng, r), dtype=np.float64)
+    zeros = np.zeros((ng, r), dtype=np.int32)
+    fc = None if forced_codes is None else np.ascontiguousarray(forced_codes, dtype=np.uint8)
+    fz = None if forced_zeros is None else np.ascontiguousarray(forced_zeros, dtype=np.int32)
+    fw = None if forced_w is None else _f64(forced_w)
+    fs = None if forced_scales is None else _f64(forced_scales)
+    stats = np.zeros(6, dtype=np.int64)
+    max_dev = ctypes.c_double(0.0)
+    rc = _lib().orc_gptq_columns_u(_ptr(W), r, d, _ptr(Uc), bits, g, _ptr(codes), _ptr(scales),
+                                   _ptr(zeros), _ptr(fc), _ptr(fz), _ptr(fw), _ptr(fs),
+                                   float(tau), _ptr(stats), ctypes.byref(max_dev))
+    if rc != 0:
+        raise np.linalg.LinAlgError(f"oracle U-row loop failed ({rc})")
+    st = dict(code_ties=int(stats[0]), code_invalid=int(stats[1]),
+              zero_ties=int(stats[2]), zero_invalid=int(stats[3]),
+              elements=int(stats[4]), groups=int(stats[5]), max_dev=max_dev.value)
+    return GPTQResult(codes, scales, zeros, W, None, st)
 
 
 def gptq_blocked(W0, U, bits: int, group_size: int, block: int):
@@ -348,7 +392,7 @@ def unpack(packed, d: int, bits: int) -> np.ndarray:
 # --------------------------------------------------------------------------
 def quantize_layer(H, W, bits: int = 4, group_size: int = 128, desc_act: bool = False,
                    damp: float = 0.01, want_U: bool = False, rows=None,
-                   forced_codes=None, forced_zeros=None, forced_w=None,
+                   forced_codes=None, forced_zeros=None, forced_w=None, forced_scales=None,
                    tau: float = 0.0) -> dict:
     """H (d x d, original column order) and W (r x d) -> GPTQ result.
 
@@ -361,7 +405,7 @@ def quantize_layer(H, W, bits: int = 4, group_size: int = 128, desc_act: bool = 
     Minv = inverse(prep["H_damped"])
     res = gptq_columns(W0, Minv, bits, group_size, want_U=want_U,
                        forced_codes=forced_codes, forced_zeros=forced_zeros,
-                       forced_w=forced_w, tau=tau)
+                       forced_w=forced_w, forced_scales=forced_scales, tau=tau)
     Q = dequantize(res.codes, res.scales, res.zeros, group_size)
     rc, rs, rz = rtn(W0, bits, group_size)
     Qr = dequantize(rc, rs, rz, group_size)

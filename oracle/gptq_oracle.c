@@ -98,11 +98,14 @@ static int code_is_valid(int32_t c, int32_t q, double y, double tol, int bits)
  *   codes   r x d uint8; scales / zeros  [ceil(d/g)][r].
  *   U       optional d x d row-major (NULL to skip): row i receives the
  *           eliminated row of M scaled by 1/sqrt(M_ii), for columns >= i.
- *   fcodes, fzeros, fwpre  optional (NULL): another implementation's codes,
- *           zero points and pre-quantization weights.  When given, the loop
- *           checks each of them for validity and then continues with them
- *           (teacher forcing), so a legitimate tie decided the other way does
- *           not desynchronise the rest of the row.
+ *   fcodes, fzeros, fwpre, fscales  optional (NULL): another
+ *           implementation's codes, zero points, pre-quantization weights and
+ *           scales.  When given, the loop checks each code and zero point for
+ *           validity and then continues with them (teacher forcing), so a
+ *           legitimate tie decided the other way does not desynchronise the
+ *           rest of the row.  The validity window of a code widens by the
+ *           other side's own deviation in the decision's inputs:
+ *           |w' - w| / s + |y - z| |s' - s| / s levels.
  *   tau     slack (in quantization levels) added to every validity window.
  *   stats   out [6]: code ties taken the other way, invalid codes, zero-point
  *           ties taken the other way, invalid zero points, elements compared,
@@ -112,7 +115,7 @@ static int code_is_valid(int32_t c, int32_t q, double y, double tol, int bits)
 int orc_gptq_columns(double *W, int64_t r, int64_t d, double *M, int bits,
                      int64_t g, uint8_t *codes, double *scales, int32_t *zeros,
                      double *U, const uint8_t *fcodes, const int32_t *fzeros,
-                     const double *fwpre, double tau, int64_t *stats,
+                     const double *fwpre, const double *fscales, double tau, int64_t *stats,
                      double *max_dev)
 {
     int64_t s_code_tie = 0, s_code_bad = 0, s_zero_tie = 0, s_zero_bad = 0;
@@ -121,14 +124,21 @@ int orc_gptq_columns(double *W, int64_t r, int64_t d, double *M, int bits,
     double *cur_s = (double *)malloc(sizeof(double) * (size_t)r);
     int32_t *cur_z = (int32_t *)malloc(sizeof(int32_t) * (size_t)r);
     double *coef = (double *)malloc(sizeof(double) * (size_t)r);
-    if (!cur_s || !cur_z || !coef) { free(cur_s); free(cur_z); free(coef); return -1; }
+    /* a zero point that differs from the oracle's is judged at the end of its
+     * group, against the drift the other side showed on that group's weights */
+    double *zwin = (double *)calloc((size_t)r, sizeof(double));
+    double *gdev = (double *)calloc((size_t)r, sizeof(double));
+    if (!cur_s || !cur_z || !coef || !zwin || !gdev) {
+        free(cur_s); free(cur_z); free(coef); free(zwin); free(gdev);
+        return -1;
+    }
 
     for (int64_t i = 0; i < d; ++i) {
         const double piv = M[i * d + i];
-        if (!(piv > 0.0)) { free(cur_s); free(cur_z); free(coef); return -2; }
+        if (!(piv > 0.0)) { free(cur_s); free(cur_z); free(coef); free(zwin); free(gdev); return -2; }
         const int64_t grp = i / g;
         const int new_group = (i % g) == 0;
-        const int64_t gend = (i + g < d) ? i + g : d;
+        const int64_t gend = (grp * g + g < d) ? grp * g + g : d; /* end of i's group */
 
 #pragma omp parallel for reduction(+:s_code_tie,s_code_bad,s_zero_tie,s_zero_bad,s_elems,s_groups) reduction(max:dev) schedule(static)
         for (int64_t row = 0; row < r; ++row) {
@@ -141,10 +151,11 @@ int orc_gptq_columns(double *W, int64_t r, int64_t d, double *M, int bits,
                 orc_quant_params(w + i, gend - i, bits, &s, &zr, &z);
                 if (fzeros) {
                     int32_t zf = fzeros[grp * r + row];
-                    if (zf != z) {
-                        if (fabs((double)zf - zr) <= 0.5 + tau) ++s_zero_tie;
-                        else ++s_zero_bad;
-                    }
+                    /* distance past the rounding window, judged at group end */
+                    zwin[row] = (zf != z) ? fabs((double)zf - zr) - 0.5 - tau : -1.0;
+                    if (zf != z && fscales)
+                        zwin[row] -= fabs(zr) * fabs(fscales[grp * r + row] - s) / s;
+                    gdev[row] = 0.0;
                     z = zf;
                     ++s_groups;
                 }
@@ -163,8 +174,10 @@ int orc_gptq_columns(double *W, int64_t r, int64_t d, double *M, int bits,
                 if (fwpre) {
                     double dv = fabs(fwpre[row * d + i] - wi) / s;
                     if (dv > dev) dev = dv;
+                    if (dv > gdev[row]) gdev[row] = dv;
                     tol += dv;
                 }
+                if (fscales) tol += fabs(y - (double)z) * fabs(fscales[grp * r + row] - s) / s;
                 int32_t c = (int32_t)fcodes[row * d + i];
                 if (c != q) {
                     if (code_is_valid(c, q, y, tol, bits)) ++s_code_tie;
@@ -174,6 +187,10 @@ int orc_gptq_columns(double *W, int64_t r, int64_t d, double *M, int bits,
                 ++s_elems;
             }
             codes[row * d + i] = (uint8_t)q;
+            if (fzeros && (i + 1 == gend) && zwin[row] >= 0.0) {
+                if (zwin[row] <= gdev[row]) ++s_zero_tie;
+                else ++s_zero_bad;
+            }
             const double what = s * (double)(q - z);
             /* OBQ step: W_F <- W_F - e / M_ii * M_{i,F} */
             coef[row] = (wi - what) / piv;
@@ -212,8 +229,91 @@ int orc_gptq_columns(double *W, int64_t r, int64_t d, double *M, int bits,
         stats[4] = s_elems; stats[5] = s_groups;
     }
     if (max_dev) *max_dev = dev;
-    free(cur_s); free(cur_z); free(coef);
+    free(cur_s); free(cur_z); free(coef); free(zwin); free(gdev);
     return 0;
+}
+
+/*
+ * The same column loop driven by the rows of U instead of an elimination of
+ * M: with U upper and U^T U = H^-1, row i of the reduced inverse is
+ * U_ii * U[i, i:], so the OBQ step is W_F <- W_F - (e / U_ii) U_{i,F}
+ * (identical to orc_gptq_columns up to rounding; pinned against it).  For
+ * large d, where the explicit elimination is too slow, U comes from a
+ * library Cholesky factor of the library inverse.  Arguments as in
+ * orc_gptq_columns, with U (d x d, row-major, upper) in place of M.
+ */
+int orc_gptq_columns_u(double *W, int64_t r, int64_t d, const double *U, int bits, int64_t g,
+                       uint8_t *codes, double *scales, int32_t *zeros,
+                       const uint8_t *fcodes, const int32_t *fzeros, const double *fwpre,
+                       const double *fscales, double tau, int64_t *stats, double *max_dev)
+{
+    int64_t s_code_tie = 0, s_code_bad = 0, s_zero_tie = 0, s_zero_bad = 0;
+    int64_t s_elems = 0, s_groups = 0;
+    double dev = 0.0;
+    int rc = 0;
+#pragma omp parallel for reduction(+:s_code_tie,s_code_bad,s_zero_tie,s_zero_bad,s_elems,s_groups) reduction(max:dev) schedule(dynamic, 1)
+    for (int64_t row = 0; row < r; ++row) {
+        double *w = W + row * d;
+        double s = 1.0;
+        int32_t z = 0;
+        double zwin = -1.0, gdv = 0.0; /* pending zero-point check, group drift */
+        for (int64_t i = 0; i < d; ++i) {
+            const double uii = U[i * d + i];
+            if (!(uii > 0.0)) { rc = -2; break; }
+            if (i % g == 0) {
+                const int64_t gend = (i + g < d) ? i + g : d;
+                double zr;
+                orc_quant_params(w + i, gend - i, bits, &s, &zr, &z);
+                if (fzeros) {
+                    int32_t zf = fzeros[(i / g) * r + row];
+                    zwin = (zf != z) ? fabs((double)zf - zr) - 0.5 - tau : -1.0;
+                    if (zf != z && fscales)
+                        zwin -= fabs(zr) * fabs(fscales[(i / g) * r + row] - s) / s;
+                    gdv = 0.0;
+                    z = zf;
+                    ++s_groups;
+                }
+                scales[(i / g) * r + row] = s;
+                zeros[(i / g) * r + row] = z;
+            }
+            const double wi = w[i];
+            int32_t q = orc_quantize(wi, s, z, bits);
+            if (fcodes) {
+                const double y = wi / s + (double)z;
+                double tol = tau;
+                if (fwpre) {
+                    double dv = fabs(fwpre[row * d + i] - wi) / s;
+                    if (dv > dev) dev = dv;
+                    if (dv > gdv) gdv = dv;
+                    tol += dv;
+                }
+                if (fscales) tol += fabs(y - (double)z) * fabs(fscales[(i / g) * r + row] - s) / s;
+                int32_t c = (int32_t)fcodes[row * d + i];
+                if (c != q) {
+                    if (code_is_valid(c, q, y, tol, bits)) ++s_code_tie;
+                    else ++s_code_bad;
+                }
+                q = c;
+                ++s_elems;
+            }
+            codes[row * d + i] = (uint8_t)q;
+            if (fzeros && ((i + 1) % g == 0 || i + 1 == d) && zwin >= 0.0) {
+                if (zwin <= gdv) ++s_zero_tie;
+                else ++s_zero_bad;
+                zwin = -1.0;
+            }
+            const double e = (wi - s * (double)(q - z)) / uii;
+            const double *ui = U + i * d;
+            for (int64_t f = i + 1; f < d; ++f) w[f] -= e * ui[f];
+        }
+    }
+    if (stats) {
+        stats[0] = s_code_tie; stats[1] = s_code_bad;
+        stats[2] = s_zero_tie; stats[3] = s_zero_bad;
+        stats[4] = s_elems; stats[5] = s_groups;
+    }
+    if (max_dev) *max_dev = dev;
+    return rc;
 }
 
 /*

@@ -12,9 +12,10 @@ fp32 arithmetic of the kernels):
   sits on a rounding boundary may legitimately round either way.  Each GPU
   code is therefore checked for validity by the oracle's column loop run in
   teacher-forcing mode: it must be the oracle's own rounding, or the other
-  neighbour of a boundary that lies within |w_gpu - w_oracle| / s + tau of
-  the oracle's value (w_gpu is the GPU's pre-quantization weight, returned
-  in W).  At most 0.1 % of the codes may take such a tie the other way
+  neighbour of a boundary that lies within |w_gpu - w_oracle| / s +
+  |y - z| |s_gpu - s_oracle| / s + tau of the oracle's value y = w / s + z
+  (w_gpu is the GPU's pre-quantization weight, returned in W): a decision is
+  valid when the GPU's own inputs to it justify it.  At most 0.1 % of the codes may take such a tie the other way
   (>= 99.9 % identical) and none may be invalid.
 * scales: relative error <= 1e-4 against the teacher-forced oracle.
 * proxy loss tr((W - Q) H (W - Q)^T): within 0.5 % of the free-running
@@ -95,14 +96,26 @@ def compare_quantization(H64: np.ndarray, W: torch.Tensor, out: dict, bits: int,
     assert np.array_equal(out["perm"], prep["perm"]), "act-order permutation differs"
     assert np.array_equal(out["dead"], prep["dead"]), "dead-column mask differs"
     sel = np.arange(W.shape[0]) if rows is None else np.asarray(rows)
-    Minv = oracle.inverse(prep["H_damped"])
     W0 = prep["W0"][sel]
     codes, zeros = out["codes"][sel], out["zeros"][:, sel]
     wq, scales = out["w_at_quant"][sel], out["scales"][:, sel]
-    forced = oracle.gptq_columns(W0, Minv, bits, group_size, forced_codes=codes,
-                                 forced_zeros=zeros, forced_w=wq, tau=TAU)
+    d = W0.shape[1]
+    if d <= 4096:
+        # the definition: explicit per-column elimination of H^-1
+        Minv = oracle.inverse(prep["H_damped"])
+        forced = oracle.gptq_columns(W0, Minv, bits, group_size, forced_codes=codes,
+                                     forced_zeros=zeros, forced_w=wq, forced_scales=scales,
+                                     tau=TAU)
+        free = oracle.gptq_columns(W0, Minv, bits, group_size)
+    else:
+        # too slow to eliminate on the host: the same loop driven by U's rows
+        # (U from a library Cholesky of the library inverse; pinned equal)
+        U = oracle.upper_factor(prep["H_damped"])
+        forced = oracle.gptq_columns_u(W0, U, bits, group_size, forced_codes=codes,
+                                       forced_zeros=zeros, forced_w=wq, forced_scales=scales,
+                                       tau=TAU)
+        free = oracle.gptq_columns_u(W0, U, bits, group_size)
     st = forced.stats
-    free = oracle.gptq_columns(W0, Minv, bits, group_size)
     free_match = float(np.mean(free.codes == codes))
     free_maxdiff = int(np.abs(free.codes.astype(int) - codes.astype(int)).max())
     srel = float(np.max(np.abs(scales - forced.scales) / np.abs(forced.scales)))

@@ -329,3 +329,24 @@ def test_teacher_forcing_accepts_itself_and_flags_a_planted_error():
     bad[row, col] = q - 1 if y >= q else q + 1   # one level away from y's side
     planted = oracle.gptq_columns(W0, Minv, 4, 16, forced_codes=bad, forced_zeros=ref.zeros)
     assert planted.stats["code_invalid"] >= 1
+
+
+@pytest.mark.parametrize("d,g", [(64, 16), (200, 32), (256, -1)])
+def test_u_row_loop_equals_the_eliminated_loop(d, g):
+    """Driving the column loop by the rows of U (from a library Cholesky of
+    the library inverse) gives the eliminated loop's codes, scales and
+    weights, and the library U equals the elimination rows."""
+    rng = np.random.default_rng(d)
+    H = _spd(d, 5 * d, cond_spread=0.6)
+    W0 = rng.standard_normal((9, d)) * 0.02
+    res = oracle.gptq_columns(W0, oracle.inverse(H), 4, g, want_U=True)
+    U = oracle.upper_factor(H)
+    assert np.abs(U - res.U).max() <= 1e-10 * np.abs(U).max()
+    ru = oracle.gptq_columns_u(W0, U, 4, g)
+    assert np.array_equal(ru.codes, res.codes)
+    assert np.array_equal(ru.zeros, res.zeros)
+    assert np.allclose(ru.scales, res.scales, rtol=1e-12, atol=0)
+    assert np.abs(ru.w_at_quant - res.w_at_quant).max() <= 1e-10 * np.abs(W0).max()
+    forced = oracle.gptq_columns_u(W0, U, 4, g, forced_codes=res.codes, forced_zeros=res.zeros,
+                                   forced_w=res.w_at_quant)
+    assert forced.stats["code_invalid"] == 0 and forced.stats["code_ties"] == 0
