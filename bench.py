@@ -61,6 +61,31 @@ def peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
+# ---------------------------------------------------------------- replicas
+# The layers of a model are independent quantization problems, so N GPUs run
+# N replicas: rank k quantizes its own layer (seed offset k) with no
+# collective on the data path.  The step time is the slowest rank's; the
+# job's throughput counts every rank's weights.
+def replica_seed_offset(rank: int) -> int:
+    return int(rank)
+
+
+def max_over_ranks(value: float, dist=None, device=None) -> float:
+    """The largest per-rank value (a device-timed step: the job waits for the
+    slowest rank).  All ranks call it; all get the maximum."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_weights_per_s(world: int, d_row: int, d_col: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank quantizes one d_row x d_col layer per
+    step, and a step lasts as long as the slowest rank's."""
+    return world * d_row * d_col / (ms_max / 1e3)
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML while running."""
@@ -197,8 +222,8 @@ def run_ours(args, rank: int, world: int, dist):
     r, d, n = wl.d_row, wl.d_col, wl.n_tokens
     cfg = g.GPTQConfig(bits=wl.bits, group_size=wl.group_size, desc_act=wl.desc_act, damp=wl.damp)
 
-    X = workloads.activations(wl, device=dev, seed_offset=rank)
-    W0 = workloads.weights(wl, device=dev, seed_offset=rank)
+    X = workloads.activations(wl, device=dev, seed_offset=replica_seed_offset(rank))
+    W0 = workloads.weights(wl, device=dev, seed_offset=replica_seed_offset(rank))
     W = torch.empty_like(W0)
     H = torch.empty(d, d, dtype=torch.float32, device=dev)
     U = torch.empty(d, d, dtype=torch.float32, device=dev)
@@ -277,10 +302,7 @@ def run_ours(args, rank: int, world: int, dist):
     quant_ms = [ev_mid[k][1].elapsed_time(ev_mid[k][2]) for k in range(K)]
     pack_ms = [ev_mid[k][2].elapsed_time(ev_e[k]) for k in range(K)]
     ms = statistics.mean(step_ms)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dist, dev)
 
     # ------------------------------------------------ end to end (host buffers)
     e2e = None
@@ -306,24 +328,26 @@ def run_ours(args, rank: int, world: int, dist):
             zh.copy_(zeros, non_blocking=True)
             e_e[k].record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = statistics.mean(e_s[k].elapsed_time(e_e[k]) for k in range(Ke))
-        te = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-        if dist is not None:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * r * d / (float(te.item()) / 1e3), "unit": "weights/s",
+        e_ms = max_over_ranks(statistics.mean(e_s[k].elapsed_time(e_e[k]) for k in range(Ke)),
+                              dist, dev)
+        e2e = {"value": job_weights_per_s(world, r, d, e_ms), "unit": "weights/s",
                "h2d_bytes_per_step": X.numel() * X.element_size() + W0.numel() * 4,
                "d2h_bytes_per_step": packed.numel() * 4 + scales.numel() * 4 + zeros.numel() * 4,
-               "ms_per_step": float(te.item())}
+               "ms_per_step": e_ms}
 
     if rank != 0:
         return
     pk, which = peaks()
     hess_flops = n * d * (d + 1)
+    # DRAM traffic of one Hessian launch from ncu (profiles/
+    # hessian_syrk_tcgen05_llama7b_q_proj_65k_tokens.md): 790.2 MB at 65,536 tokens,
+    # d = 4,096; X reads and the per-16k-token drains both grow with the tokens.
+    traffic = 790.2e6 * n / 65536 if (d == 4096 and n % 16384 == 0) else None
     h_ms = statistics.mean(hess_ms)
     achieved = hess_flops / (h_ms / 1e3) / 1e12
     peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     line = {
-        "metric": METRIC, "value": world * r * d / (ms_max / 1e3), "unit": "weights/s",
+        "metric": METRIC, "value": job_weights_per_s(world, r, d, ms_max), "unit": "weights/s",
         "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_max,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16-in/fp32", "data": "synthetic (seeded; Student-t / half-normal activations "
@@ -336,7 +360,7 @@ def run_ours(args, rank: int, world: int, dist):
         "quantize_only_weights_per_s": r * d / ((ms - h_ms) / 1e3),
         "roofline": {"kernel": "hessian_syrk_tcgen05", "bound": "tensor", "achieved": achieved,
                      "peak": peak, "peak_source": f"{which} bf16 dense (burst)", "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": traffic,
                      "algorithmic": f"n*d*(d+1) = {hess_flops:.4e} flop per launch"},
         "gpu_launches": launches,
         "clocks": clocks.summary(),
