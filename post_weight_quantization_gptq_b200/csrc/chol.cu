@@ -12,8 +12,7 @@
 // the gather that builds P (prep.cu) and into the final store here.
 //
 //   P buffer (d x d, ld d, the caller's U): lower triangle = P on entry, L
-//            after the factorization; its strict upper triangle holds the
-//            recursive-inverse temporaries; finally U.
+//            after the factorization; finally U.
 //   X buffer (the caller's consumed H, ld ldx): lower triangle = L^-1, with
 //            every 128 x 128 diagonal block's strict upper part zeroed.
 //
@@ -21,8 +20,11 @@
 //   potrf_inv_128_kernel  L_kk = chol(A_kk) and L_kk^-1 (one CTA)
 //   panel solve           L_ik = A_ik L_kk^-T          (3xTF32 tcgen05 GEMM)
 //   trailing update       A_ij -= L_ik L_jk^T, i >= j  (3xTF32 tcgen05 GEMM)
-// and L^-1 built block row by block row on the same GEMM,
-//   X[k, :k] = -X_kk (L[k, :k] X[:k, :k]),
+// and L^-1 by right-looking forward substitution on the identity, on the
+// same GEMM: with B the strictly lower block part of X (zero at the start),
+// after panel k
+//   X[k, :k] = L_kk^-1 B[k, :k]                (row k of L^-1 is then final)
+//   B[i, :k+1] -= L[i, k] X[k, :k+1],  i > k   (its share of the later rows)
 // in the shadow of the panel chain (see launch_chol_inverse).
 #include <cmath>
 #include <mutex>
@@ -35,9 +37,13 @@ namespace gptq {
 namespace {
 
 constexpr int NB = 128;      // panel width
-constexpr int LDA = NB + 1;  // shared-memory row pitch of the diagonal block
+constexpr int LDA = NB + 4;  // shared-memory row pitch: float4-aligned rows, rows 4 banks apart
+constexpr int TP = 68;       // pitch of the doubling temporary
 constexpr int kDiagThreads = 256;
-constexpr int kDiagSmem = (2 * NB * LDA + 64 * 65 + NB) * 4;
+constexpr int kDiagSmem = (2 * NB * LDA + 64 * TP + 32 * 32 + 32 * LDA + NB) * 4;
+
+__device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void sts4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 
 // ------------------------------------------------------------------------
 // Diagonal block: L = chol(A) and X = L^-1 for a kw x kw (kw <= 128) block,
@@ -48,21 +54,25 @@ constexpr int kDiagSmem = (2 * NB * LDA + 64 * 65 + NB) * 4;
 // part; finally the four 32 x 32 inverses are joined by two levels of
 // recursive doubling.
 //
-// The warp keeps its rows in registers and rotates them after every column
-// step, so the pivot column is always register 0: the step loop stays rolled
-// (small code, the kernel runs once per panel on a cold SM) while all
-// register indices are compile-time constants and each step is 31
-// independent shuffle + FMA pairs.
+// Column c of the strip's L below the diagonal is also kept as a row of Lc
+// (Lc[c][m] = L[o+c+1+m][o+c], zero past the strip), so each elimination
+// step reads it with eight broadcast float4 loads; the strip's rows below
+// the diagonal block are kept transposed in Ls for the trailing update.  The factor warp keeps its
+// rows in registers and rotates them after every column step, so the pivot
+// column is always register 0: the step loop stays rolled (small code, the
+// kernel runs once per panel on a cold SM) while every register index is a
+// compile-time constant.
 __global__ void __launch_bounds__(kDiagThreads, 1)
     potrf_inv_128_kernel(float* __restrict__ P, int64_t ldp, int64_t kb, int kw,
                          float* __restrict__ X, int64_t ldx, int32_t* status) {
-    extern __shared__ float sm[];
-    float* A = sm;              // [128][129] the block, L in its lower part
-    float* Xs = A + NB * LDA;   // [128][129] L^-1
-    float* T = Xs + NB * LDA;   // [64][65] doubling temporary
-    float* dinv = T + 64 * 65;  // [128] 1 / L_ii
+    extern __shared__ __align__(16) float sm[];
+    float* A = sm;              // [128][LDA] the block, L in its lower part
+    float* Xs = A + NB * LDA;   // [128][LDA] L^-1
+    float* T = Xs + NB * LDA;   // [64][TP] doubling temporary
+    float* Lc = T + 64 * TP;    // [32][32] the current strip's columns of L, shifted
+    float* Ls = Lc + 32 * 32;   // [32][LDA] the current strip of L below it, transposed
+    float* dinv = Ls + 32 * LDA; // [128] 1 / L_ii
     __shared__ int bad;
-    __shared__ float colbuf[32];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) bad = 0;
     {
@@ -80,13 +90,12 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
         for (int q = 0; q < 16; ++q) {
             const int e = tid + q * kDiagThreads;
             const int i = e >> 5, j = (e & 31) * 4;
-            const float vv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+            float vv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const int jj = j + t;
-                A[i * LDA + jj] = (jj <= i && i < kw) ? vv[t] : (i == jj ? 1.f : 0.f);
-                Xs[i * LDA + jj] = 0.f;
-            }
+            for (int t = 0; t < 4; ++t)
+                vv[t] = (j + t <= i && i < kw) ? vv[t] : (i == j + t ? 1.f : 0.f);
+            sts4(A + i * LDA + j, make_float4(vv[0], vv[1], vv[2], vv[3]));
+            sts4(Xs + i * LDA + j, make_float4(0.f, 0.f, 0.f, 0.f));
         }
     }
     __syncthreads();
@@ -97,7 +106,12 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
             // -- 32 x 32 Cholesky: lane i holds row o + i, register r = column c + r
             float a[32];
 #pragma unroll
-            for (int r = 0; r < 32; ++r) a[r] = (r <= lane) ? A[(o + lane) * LDA + o + r] : 0.f;
+            for (int q = 0; q < 8; ++q) {
+                const float4 t = lds4(A + (o + lane) * LDA + o + 4 * q);
+                a[4 * q] = t.x; a[4 * q + 1] = t.y; a[4 * q + 2] = t.z; a[4 * q + 3] = t.w;
+            }
+#pragma unroll
+            for (int r = 0; r < 32; ++r) a[r] = (r <= lane) ? a[r] : 0.f;
 #pragma unroll 1
             for (int c = 0; c < 32; ++c) {
                 float piv = __shfl_sync(0xffffffffu, a[0], c);
@@ -106,49 +120,68 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
                     piv = 1.f;
                 }
                 const float inv = rsqrtf(piv);
-                const float lcc = piv * inv;
-                const float a0 = (lane == c) ? lcc : ((lane > c) ? a[0] * inv : a[0]);
-                colbuf[lane] = a0;
+                const float a0 = (lane == c) ? piv * inv : ((lane > c) ? a[0] * inv : 0.f);
                 if (lane >= c) A[(o + lane) * LDA + o + c] = a0;
                 if (lane == c) dinv[o + c] = inv;
+                // lane i > c holds L[o+i][o+c] -> Lc[c][i-c-1]; lanes <= c fill the tail with 0
+                Lc[c * 32 + ((lane - c - 1) & 31)] = a0 * (lane > c ? 1.f : 0.f);
                 __syncwarp();
 #pragma unroll
-                for (int r = 1; r < 32; ++r)
-                    a[r - 1] = fmaf(-a0, colbuf[(c + r) & 31], a[r]);  // update and rotate
-                a[31] = 0.f;
-                __syncwarp();
+                for (int q = 0; q < 8; ++q) {  // update and rotate
+                    const float4 l = lds4(Lc + c * 32 + 4 * q);
+                    a[4 * q] = fmaf(-a0, l.x, a[4 * q + 1]);
+                    a[4 * q + 1] = fmaf(-a0, l.y, a[4 * q + 2]);
+                    a[4 * q + 2] = fmaf(-a0, l.z, a[4 * q + 3]);
+                    a[4 * q + 3] = (q < 7) ? fmaf(-a0, l.w, a[4 * q + 4]) : 0.f;
+                }
             }
         }
         __syncthreads();
         const int r0 = o + 32;
         if (warp < 4) {
             // -- forward substitution with L_bb on 128 right-hand sides at once:
-            //    lanes 0..31 the identity (-> the strip's inverse, a column per
-            //    lane), lanes 32..127 the rows below (-> the strip of L)
+            //    threads 0..31 the identity (-> the strip's inverse, a column per
+            //    thread), threads 32..127 the rows below (-> the strip of L)
             const int hs = tid;
             const int i = r0 + hs - 32;  // row for hs >= 32
             const bool act = hs < 32 || i < NB;
             float x[32];
+            if (hs >= 32 && act) {
 #pragma unroll
-            for (int r = 0; r < 32; ++r)
-                x[r] = (hs < 32) ? ((r == hs) ? 1.f : 0.f) : (act ? A[i * LDA + o + r] : 0.f);
+                for (int q = 0; q < 8; ++q) {
+                    const float4 t = lds4(A + i * LDA + o + 4 * q);
+                    x[4 * q] = t.x; x[4 * q + 1] = t.y; x[4 * q + 2] = t.z; x[4 * q + 3] = t.w;
+                }
+            } else {
+#pragma unroll
+                for (int r = 0; r < 32; ++r) x[r] = (r == hs) ? 1.f : 0.f;
+            }
 #pragma unroll 1
             for (int c = 0; c < 32; ++c) {
-                const float xc = x[0] * dinv[o + c];
-                if (hs < 32) Xs[(o + c) * LDA + o + hs] = xc;
-                else if (act) A[i * LDA + o + c] = xc;
-                const float* lcol = A + (o + c) * LDA + o + c;  // L[o+c+r][o+c] at lcol[r * LDA]
+                // the step's column of L first: its loads do not wait behind the stores
+                float4 l[8];
 #pragma unroll
-                for (int r = 1; r < 32; ++r) {
-                    const float l = (c + r < 32) ? lcol[r * LDA] : 0.f;
-                    x[r - 1] = fmaf(-l, xc, x[r]);
+                for (int q = 0; q < 8; ++q) l[q] = lds4(Lc + c * 32 + 4 * q);
+                const float xc = x[0] * dinv[o + c];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    x[4 * q] = fmaf(-l[q].x, xc, x[4 * q + 1]);
+                    x[4 * q + 1] = fmaf(-l[q].y, xc, x[4 * q + 2]);
+                    x[4 * q + 2] = fmaf(-l[q].z, xc, x[4 * q + 3]);
+                    x[4 * q + 3] = (q < 7) ? fmaf(-l[q].w, xc, x[4 * q + 4]) : 0.f;
                 }
-                x[31] = 0.f;
+                if (hs < 32) {
+                    Xs[(o + c) * LDA + o + hs] = xc;
+                } else if (act) {
+                    A[i * LDA + o + c] = xc;
+                    Ls[c * LDA + i] = xc;
+                }
             }
         }
         __syncthreads();
         if (r0 < NB) {
-            // -- trailing update of the lower part, 4 x 4 register blocks
+            // -- trailing update of the lower part, 4 x 4 register blocks read from
+            //    the transposed strip (consecutive blocks -> consecutive float4)
             const int mb = (NB - r0) / 4;
             const int units = mb * (mb + 1) / 2;
             for (int u = tid; u < units; u += kDiagThreads) {
@@ -158,31 +191,36 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
                 const int bj = u - bi * (bi + 1) / 2;
                 const int i0 = r0 + 4 * bi, j0 = r0 + 4 * bj;
                 float acc2[4][4] = {};
-#pragma unroll 4
+#pragma unroll 8
                 for (int k = 0; k < 32; ++k) {
-                    float li[4], lj[4];
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        li[t] = A[(i0 + t) * LDA + o + k];
-                        lj[t] = A[(j0 + t) * LDA + o + k];
-                    }
+                    const float4 li = lds4(Ls + k * LDA + i0), lj = lds4(Ls + k * LDA + j0);
+                    const float a4[4] = {li.x, li.y, li.z, li.w}, b4[4] = {lj.x, lj.y, lj.z, lj.w};
 #pragma unroll
                     for (int t = 0; t < 4; ++t)
 #pragma unroll
-                        for (int w = 0; w < 4; ++w) acc2[t][w] = fmaf(li[t], lj[w], acc2[t][w]);
+                        for (int w = 0; w < 4; ++w) acc2[t][w] = fmaf(a4[t], b4[w], acc2[t][w]);
                 }
 #pragma unroll
-                for (int t = 0; t < 4; ++t)
+                for (int t = 0; t < 4; ++t) {
+                    float* dst = A + (i0 + t) * LDA + j0;
+                    if (j0 + 3 <= i0 + t) {
+                        float4 d4 = lds4(dst);
+                        d4.x -= acc2[t][0]; d4.y -= acc2[t][1]; d4.z -= acc2[t][2]; d4.w -= acc2[t][3];
+                        sts4(dst, d4);
+                    } else {
 #pragma unroll
-                    for (int w = 0; w < 4; ++w)
-                        if (j0 + w <= i0 + t) A[(i0 + t) * LDA + j0 + w] -= acc2[t][w];
+                        for (int w = 0; w < 4; ++w)
+                            if (j0 + w <= i0 + t) dst[w] -= acc2[t][w];
+                    }
+                }
             }
         }
         __syncthreads();
     }
 
     // -- join the 32 x 32 inverses: X_CA = -X_CC (L_CA X_AA), 4 x 4 register
-    //    blocks (rows c, columns a); T[p*s + c][a] holds L_CA X_AA
+    //    blocks (rows c, columns a); T[p*s + c][a] holds L_CA X_AA.  X_AA and
+    //    X_CC are lower triangular, so the sums skip their zero parts.
     for (int s = 32; s < NB; s *= 2) {
         const int pairs = NB / (2 * s);
         const int nb4 = s / 4;
@@ -191,46 +229,59 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
             const int p = e / (nb4 * nb4), c0 = ((e / nb4) % nb4) * 4, a0 = (e % nb4) * 4;
             const int A0 = 2 * s * p, C0 = A0 + s;
             float acc[4][4] = {};
-#pragma unroll 8
-            for (int k = 0; k < s; ++k) {  // X_AA is zero above its diagonal
-                float l[4], xx[4];
+#pragma unroll 2
+            for (int k = a0; k < s; k += 4) {  // X_AA[k][a] = 0 for k < a
+                float4 l[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) l[t] = lds4(A + (C0 + c0 + t) * LDA + A0 + k);
+                float4 xx[4];
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) xx[kk] = lds4(Xs + (A0 + k + kk) * LDA + A0 + a0);
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
-                    l[t] = A[(C0 + c0 + t) * LDA + A0 + k];
-                    xx[t] = Xs[(A0 + k) * LDA + A0 + a0 + t];
+                    const float lt[4] = {l[t].x, l[t].y, l[t].z, l[t].w};
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        acc[t][0] = fmaf(lt[kk], xx[kk].x, acc[t][0]);
+                        acc[t][1] = fmaf(lt[kk], xx[kk].y, acc[t][1]);
+                        acc[t][2] = fmaf(lt[kk], xx[kk].z, acc[t][2]);
+                        acc[t][3] = fmaf(lt[kk], xx[kk].w, acc[t][3]);
+                    }
                 }
-#pragma unroll
-                for (int t = 0; t < 4; ++t)
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) acc[t][w] = fmaf(l[t], xx[w], acc[t][w]);
             }
 #pragma unroll
             for (int t = 0; t < 4; ++t)
-#pragma unroll
-                for (int w = 0; w < 4; ++w) T[(p * s + c0 + t) * 65 + a0 + w] = acc[t][w];
+                sts4(T + (p * s + c0 + t) * TP + a0, make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]));
         }
         __syncthreads();
         for (int e = tid; e < blocks; e += kDiagThreads) {
             const int p = e / (nb4 * nb4), c0 = ((e / nb4) % nb4) * 4, a0 = (e % nb4) * 4;
             const int A0 = 2 * s * p, C0 = A0 + s;
             float acc[4][4] = {};
-#pragma unroll 8
-            for (int k = 0; k < s; ++k) {  // X_CC is zero above its diagonal
-                float xc[4], tt[4];
+#pragma unroll 2
+            for (int k = 0; k <= c0; k += 4) {  // X_CC[c][k] = 0 for k > c
+                float4 xc[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) xc[t] = lds4(Xs + (C0 + c0 + t) * LDA + C0 + k);
+                float4 tt[4];
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) tt[kk] = lds4(T + (p * s + k + kk) * TP + a0);
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
-                    xc[t] = Xs[(C0 + c0 + t) * LDA + C0 + k];
-                    tt[t] = T[(p * s + k) * 65 + a0 + t];
+                    const float xt[4] = {xc[t].x, xc[t].y, xc[t].z, xc[t].w};
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        acc[t][0] = fmaf(xt[kk], tt[kk].x, acc[t][0]);
+                        acc[t][1] = fmaf(xt[kk], tt[kk].y, acc[t][1]);
+                        acc[t][2] = fmaf(xt[kk], tt[kk].z, acc[t][2]);
+                        acc[t][3] = fmaf(xt[kk], tt[kk].w, acc[t][3]);
+                    }
                 }
-#pragma unroll
-                for (int t = 0; t < 4; ++t)
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) acc[t][w] = fmaf(xc[t], tt[w], acc[t][w]);
             }
 #pragma unroll
             for (int t = 0; t < 4; ++t)
-#pragma unroll
-                for (int w = 0; w < 4; ++w) Xs[(C0 + c0 + t) * LDA + A0 + a0 + w] = -acc[t][w];
+                sts4(Xs + (C0 + c0 + t) * LDA + A0 + a0,
+                     make_float4(-acc[t][0], -acc[t][1], -acc[t][2], -acc[t][3]));
         }
         __syncthreads();
     }
@@ -241,19 +292,20 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
     for (int e = tid; e < NB * NB / 4; e += kDiagThreads) {
         const int i = e >> 5, j = (e & 31) * 4;
         if (i >= kw || j >= kw) continue;
-        float l4[4], x4[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            l4[t] = A[i * LDA + j + t];
-            x4[t] = (j + t <= i) ? Xs[i * LDA + j + t] : 0.f;
-        }
-        *reinterpret_cast<float4*>(X + (kb + i) * ldx + kb + j) = make_float4(x4[0], x4[1], x4[2], x4[3]);
+        const float4 l4 = lds4(A + i * LDA + j);
+        float4 x4 = lds4(Xs + i * LDA + j);
+        if (j + 1 > i) x4.y = 0.f;
+        if (j + 2 > i) x4.z = 0.f;
+        if (j + 3 > i) x4.w = 0.f;
+        if (j > i) x4.x = 0.f;
+        *reinterpret_cast<float4*>(X + (kb + i) * ldx + kb + j) = x4;
         if (j + 3 <= i) {
-            *reinterpret_cast<float4*>(P + (kb + i) * ldp + kb + j) = make_float4(l4[0], l4[1], l4[2], l4[3]);
+            *reinterpret_cast<float4*>(P + (kb + i) * ldp + kb + j) = l4;
         } else if (j <= i) {
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
             for (int t = 0; t < 4; ++t)
-                if (j + t <= i) P[(kb + i) * ldp + kb + j + t] = l4[t];
+                if (j + t <= i) P[(kb + i) * ldp + kb + j + t] = lv[t];
         }
     }
     if (tid == 0 && bad) report(status, GPTQ_ERR_NOT_PD);
@@ -268,27 +320,20 @@ __device__ __forceinline__ void tri_coords(int t, int& I, int& J) {
     J = t - i * (i + 1) / 2;
 }
 
-// 32 consecutive floats: dst[j] = sign * v[j] (or dst[j] -= v[j] with sub),
-// as float4 accesses (callers guarantee 16-byte alignment and bounds).
-template <bool kSub>
+// 32 consecutive floats: dst[j] = sign * v[j], as float4 stores (callers
+// guarantee 16-byte alignment and bounds).
 __device__ __forceinline__ void put32(float* dst, const float (&v)[32], float sign) {
     float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        if (kSub) {
-            float4 x = d4[q];
-            x.x -= v[4 * q]; x.y -= v[4 * q + 1]; x.z -= v[4 * q + 2]; x.w -= v[4 * q + 3];
-            d4[q] = x;
-        } else {
-            d4[q] = make_float4(sign * v[4 * q], sign * v[4 * q + 1], sign * v[4 * q + 2],
-                                sign * v[4 * q + 3]);
-        }
-    }
+    for (int q = 0; q < 8; ++q)
+        d4[q] = make_float4(sign * v[4 * q], sign * v[4 * q + 1], sign * v[4 * q + 2],
+                            sign * v[4 * q + 3]);
 }
 
 // ---------------------------------------------------------------- schedulers
 // Panel solve: L[m0.., kb..kb+kw) = A[m0.., kb..) (L_kk^-1)^T   (in place)
 struct TrsmSched {
+    static constexpr bool kRmw = false;
     float* P;
     int64_t ldp;
     int d, kb, kw;
@@ -298,7 +343,7 @@ struct TrsmSched {
         if (r >= d) return;
         float* dst = P + static_cast<int64_t>(r) * ldp + kb + col0;
         if (col0 + 32 <= kw) {
-            put32<false>(dst, v, 1.f);
+            put32(dst, v, 1.f);
         } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
@@ -328,56 +373,64 @@ struct SyrkSched {
         }
         return {s0 + NB * I, s0 + NB * J, kb, kb, (kw + 31) / 32};
     }
-    __device__ void store(const g3::Job& jb, int row, int col0, const float (&v)[32]) const {
+    static constexpr bool kRmw = true;
+    __device__ float* dst(const g3::Job& jb, int row) const {
         const int r = jb.m0 + row;
-        if (r >= d) return;
-        float* dst = P + static_cast<int64_t>(r) * ldp + jb.n0 + col0;
-        const int c = jb.n0 + col0;
-        if (c + 31 <= r && c + 32 <= d) {
-            put32<true>(dst, v, 1.f);
-        } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                if (c + j < d && c + j <= r) dst[j] -= v[j];
-        }
+        return r < d ? P + static_cast<int64_t>(r) * ldp + jb.n0 : nullptr;
     }
+    // lower triangle only: columns n0 .. min(r, d - 1) are written; the rest of
+    // the row segment inside the matrix may be read
+    __device__ int ncols(const g3::Job& jb, int row) const {
+        const int lim = min(jb.m0 + row + 1, d) - jb.n0;
+        return lim < g3::BN ? lim : g3::BN;
+    }
+    __device__ int nreadable(const g3::Job& jb) const { return min(d - jb.n0, g3::BN); }
 };
 
-// Block row kb of L^-1, left of the diagonal, once L_kk^-1 is known:
-//   X[kb.., :kb] = -X_kk (L[kb.., :kb] X[:kb, :kb]).
-// Step 1: T^T[a][m] = sum_{a <= j < kb} X[j][a] L[kb+m][j], stored in the
-// free upper triangle at P[a][kb+m] (a < kb).
-struct XRow1Sched {
-    float* P;
-    int64_t ldp;
-    int d, kb, kw;
-    __device__ g3::Job job(int t) const {
-        const int a0 = NB * t;
-        return {a0, kb, a0, a0, (kb - a0) / 32};
-    }
-    __device__ void store(const g3::Job& jb, int row, int col0, const float (&v)[32]) const {
-        float* dst = P + static_cast<int64_t>(jb.m0 + row) * ldp + kb + col0;
-        if (col0 + 32 <= kw) {
-            put32<false>(dst, v, 1.f);
-        } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                if (col0 + j < kw) dst[j] = v[j];
-        }
-    }
-};
-
-// Step 2: X[kb+m][a] = -sum_j X[kb+m][kb+j] T[j][a], T[j][a] = P[a][kb+j].
-struct XRow2Sched {
+// Row k of L^-1 left of the diagonal block, in place:
+//   X[kb+m][n] = sum_j X_kk[m][j] B[kb+j][n],  n < kb
+// (A = X_kk, K-major; B = the block row of B, MN-major).  A CTA reads its
+// whole B tile before its epilogue overwrites that tile.
+struct XFinSched {
+    static constexpr bool kRmw = false;
     float* X;
     int64_t ldx;
-    int d, kb, kw;
+    int kb, kw;
     __device__ g3::Job job(int t) const { return {kb, NB * t, kb, kb, (kw + 31) / 32}; }
     __device__ void store(const g3::Job& jb, int row, int col0, const float (&v)[32]) const {
         if (row >= kw) return;
-        put32<false>(X + static_cast<int64_t>(kb + row) * ldx + jb.n0 + col0, v, -1.f);
+        put32(X + static_cast<int64_t>(kb + row) * ldx + jb.n0 + col0, v, 1.f);
     }
 };
+
+// Panel k's share of the later block rows of L^-1:
+//   B[i][n] -= sum_j L[i][kb+j] X[kb+j][n],  i >= kb + 128, n < kb + 128
+// (A = the panel of L, K-major; B = block row k of X, MN-major).
+struct BUpdSched {
+    static constexpr bool kRmw = true;
+    float* X;
+    int64_t ldx;
+    int d, kb, mt;
+    __device__ g3::Job job(int t) const {
+        return {kb + NB + NB * (t % mt), NB * (t / mt), kb, kb, NB / 32};
+    }
+    __device__ float* dst(const g3::Job& jb, int row) const {
+        const int r = jb.m0 + row;
+        return r < d ? X + static_cast<int64_t>(r) * ldx + jb.n0 : nullptr;
+    }
+    __device__ int ncols(const g3::Job&, int) const { return g3::BN; }
+    __device__ int nreadable(const g3::Job&) const { return g3::BN; }
+};
+
+// B = 0 on the strictly lower 128 x 128 blocks of X (the diagonal blocks are
+// written by potrf_inv_128_kernel).
+__global__ void zero_lower_blocks_kernel(float* __restrict__ X, int64_t ldx, int64_t d) {
+    const int64_t i = blockIdx.y;
+    const int64_t jend = (i / NB) * NB;  // columns left of row i's diagonal block
+    for (int64_t j = 4 * (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x); j < jend;
+         j += 4 * static_cast<int64_t>(gridDim.x) * blockDim.x)
+        *reinterpret_cast<float4*>(X + i * ldx + j) = make_float4(0.f, 0.f, 0.f, 0.f);
+}
 
 // U[i][j] = X[d-1-i][d-1-j] for j >= i, 0 below the diagonal.
 __global__ void flip_kernel(const float* __restrict__ X, int64_t ldx, float* __restrict__ U,
@@ -392,12 +445,17 @@ __global__ void flip_kernel(const float* __restrict__ X, int64_t ldx, float* __r
 
 size_t chol_workspace_bytes(int64_t) { return 0; }
 
-// Side stream and events of the lookahead schedule (created once per device;
-// streams and events, no device memory).
+// Side streams and events of the lookahead schedule (created once per
+// device; streams and events, no device memory).
 namespace {
 struct Lookahead {
-    cudaStream_t side = nullptr;
-    cudaEvent_t ev[8] = {};  // [0..3] panel column ready, [4..7] trailing update done
+    cudaStream_t side = nullptr;   // rest of each trailing update
+    cudaStream_t inv = nullptr;    // L^-1
+    cudaEvent_t start = nullptr;
+    cudaEvent_t solved[4] = {};    // panel k's L_kk^-1 and L[:, k] are final
+    cudaEvent_t ready[4] = {};     // panel k+1's column updated
+    cudaEvent_t done[4] = {};      // rest of panel k's trailing update done
+    cudaEvent_t side_end = nullptr, inv_end = nullptr;
     bool ok = false;
 };
 std::mutex g_la_mutex;
@@ -409,9 +467,17 @@ Lookahead* lookahead_resources() {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
     Lookahead& la = g_la[dev];
     if (!la.ok) {
-        if (cudaStreamCreateWithFlags(&la.side, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
-        for (auto& e : la.ev)
-            if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+        if (cudaStreamCreateWithFlags(&la.side, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&la.inv, cudaStreamNonBlocking) != cudaSuccess)
+            return nullptr;
+        cudaEvent_t* all[] = {&la.start, &la.side_end, &la.inv_end};
+        for (auto* e : all)
+            if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+        for (int i = 0; i < 4; ++i)
+            if (cudaEventCreateWithFlags(&la.solved[i], cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&la.ready[i], cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&la.done[i], cudaEventDisableTiming) != cudaSuccess)
+                return nullptr;
         la.ok = true;
     }
     return &la;
@@ -419,11 +485,14 @@ Lookahead* lookahead_resources() {
 }  // namespace
 
 // Lookahead schedule.  The caller's stream runs the panel chain
-//   potrf(k) -> panel solve(k) -> update of panel k+1's column -> potrf(k+1)
-// while a side stream runs the rest of each trailing update and block row k
-// of L^-1 in its shadow.  Ordering: the update of panel k+1's column waits
-// for the previous panel's rest-of-update (both touch that column); potrf and
-// the panel solve of k+1 then see every update they need.
+//   potrf(k) -> panel solve(k) -> update of panel k+1's column -> potrf(k+1);
+// the side stream runs the rest of each trailing update and the inverse
+// stream builds L^-1, both in the shadow of the chain.  Ordering: the update
+// of panel k+1's column waits for the previous panel's rest-of-update (both
+// touch that column), so potrf and the panel solve of k+1 see every update
+// they need; the inverse stream waits for each panel's solve and is in order
+// with itself; nothing on the chain waits for it.  The SMs are shared out so
+// that the chain's one-wave launches always find free SMs.
 gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, float* U,
                                 int32_t* status, void*, cudaStream_t stream) {
     const int64_t ldp = d;
@@ -436,21 +505,27 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
     if (cudaFuncSetAttribute(potrf_inv_128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kDiagSmem) != cudaSuccess)
         return GPTQ_ERR_CUDA;
-    // one enqueue sequence at a time per process: the side stream and the
-    // event ring are shared by every call on a device
+    // one enqueue sequence at a time per process: the side streams and the
+    // events are shared by every call on a device
     std::lock_guard<std::mutex> lock(g_la_mutex);
     Lookahead* la = lookahead_resources();
     if (la == nullptr) return GPTQ_ERR_CUDA;
     const int sms = num_sms();
-    const int side_sms = sms > 32 ? sms - 16 : sms;  // leave SMs for the panel chain
-    cudaStream_t side = la->side;
+    const int inv_sms = sms >= 128 ? 32 : (sms + 3) / 4;
+    const int side_sms = sms >= 128 ? sms - 32 - inv_sms : (sms + 1) / 2;
     const int npan = static_cast<int>((d + NB - 1) / NB);
     int64_t launches = 0;
-    bool side_used = false;
-    // the side stream starts after everything the caller queued before us
-    if (cudaEventRecord(la->ev[0], stream) != cudaSuccess ||
-        cudaStreamWaitEvent(side, la->ev[0], 0) != cudaSuccess)
+    // the side streams start after everything the caller queued before us
+    if (cudaEventRecord(la->start, stream) != cudaSuccess ||
+        cudaStreamWaitEvent(la->side, la->start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(la->inv, la->start, 0) != cudaSuccess)
         return GPTQ_ERR_CUDA;
+    if (npan > 1) {
+        const dim3 zgrid(static_cast<unsigned>((d / 4 + 255) / 256 < 4 ? (d / 4 + 255) / 256 : 4),
+                         static_cast<unsigned>(d));
+        zero_lower_blocks_kernel<<<zgrid, 256, 0, la->inv>>>(X, ldx, d);
+        ++launches;
+    }
     for (int k = 0; k < npan; ++k) {
         const int64_t kb = static_cast<int64_t>(k) * NB;
         const int kw = static_cast<int>((d - kb < NB) ? d - kb : NB);
@@ -458,46 +533,55 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
         ++launches;
         const int64_t m = d - kb - kw;
         const int mt = static_cast<int>((m + NB - 1) / NB);
-        cudaEvent_t ready = la->ev[k & 3], done = la->ev[4 + (k & 3)];
         if (m > 0) {
             TrsmSched ts{P, ldp, di, static_cast<int>(kb), kw};
             if (g3::launch<TrsmSched, false, false>(tP, tX, ts, mt, status, stream, sms) != cudaSuccess)
                 return GPTQ_ERR_CUDA;
-            if (k > 0 && cudaStreamWaitEvent(stream, la->ev[4 + ((k - 1) & 3)], 0) != cudaSuccess)
+            ++launches;
+        }
+        if (cudaEventRecord(la->solved[k & 3], stream) != cudaSuccess ||
+            cudaStreamWaitEvent(la->inv, la->solved[k & 3], 0) != cudaSuccess)
+            return GPTQ_ERR_CUDA;
+        if (m > 0) {
+            if (k > 0 && cudaStreamWaitEvent(stream, la->done[(k - 1) & 3], 0) != cudaSuccess)
                 return GPTQ_ERR_CUDA;
             SyrkSched nx{P, ldp, di, static_cast<int>(kb), kw, static_cast<int>(kb + kw), 1};
             if (g3::launch<SyrkSched, false, false>(tP, tP, nx, mt, status, stream, sms) != cudaSuccess)
                 return GPTQ_ERR_CUDA;
-            launches += 2;
+            ++launches;
         }
-        if (cudaEventRecord(ready, stream) != cudaSuccess ||
-            cudaStreamWaitEvent(side, ready, 0) != cudaSuccess)
+        if (cudaEventRecord(la->ready[k & 3], stream) != cudaSuccess ||
+            cudaStreamWaitEvent(la->side, la->ready[k & 3], 0) != cudaSuccess)
             return GPTQ_ERR_CUDA;
         if (mt > 1) {
             SyrkSched rs{P, ldp, di, static_cast<int>(kb), kw, static_cast<int>(kb + kw), 2};
-            if (g3::launch<SyrkSched, false, false>(tP, tP, rs, mt * (mt + 1) / 2 - mt, status, side,
-                                                    side_sms) != cudaSuccess)
+            if (g3::launch<SyrkSched, false, false>(tP, tP, rs, mt * (mt + 1) / 2 - mt, status,
+                                                    la->side, side_sms) != cudaSuccess)
                 return GPTQ_ERR_CUDA;
             ++launches;
         }
-        if (cudaEventRecord(done, side) != cudaSuccess) return GPTQ_ERR_CUDA;
+        if (cudaEventRecord(la->done[k & 3], la->side) != cudaSuccess) return GPTQ_ERR_CUDA;
+        // inverse stream: finish row k of L^-1, then pass panel k on to the rows below
         if (k > 0) {
-            XRow1Sched x1{P, ldp, di, static_cast<int>(kb), kw};
-            XRow2Sched x2{X, ldx, di, static_cast<int>(kb), kw};
-            if (g3::launch<XRow1Sched, true, false>(tXmn, tP, x1, k, status, side, side_sms) !=
-                    cudaSuccess ||
-                g3::launch<XRow2Sched, false, false>(tX, tP, x2, k, status, side, side_sms) !=
-                    cudaSuccess)
+            XFinSched xf{X, ldx, static_cast<int>(kb), kw};
+            if (g3::launch<XFinSched, false, true>(tX, tXmn, xf, k, status, la->inv, inv_sms) !=
+                cudaSuccess)
                 return GPTQ_ERR_CUDA;
-            launches += 2;
+            ++launches;
         }
-        side_used = true;
+        if (m > 0) {
+            BUpdSched bu{X, ldx, di, static_cast<int>(kb), mt};
+            if (g3::launch<BUpdSched, false, true>(tP, tXmn, bu, mt * (k + 1), status, la->inv,
+                                                   inv_sms) != cudaSuccess)
+                return GPTQ_ERR_CUDA;
+            ++launches;
+        }
     }
-    if (side_used) {
-        if (cudaEventRecord(la->ev[4], side) != cudaSuccess ||
-            cudaStreamWaitEvent(stream, la->ev[4], 0) != cudaSuccess)
-            return GPTQ_ERR_CUDA;
-    }
+    if (cudaEventRecord(la->side_end, la->side) != cudaSuccess ||
+        cudaEventRecord(la->inv_end, la->inv) != cudaSuccess ||
+        cudaStreamWaitEvent(stream, la->side_end, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(stream, la->inv_end, 0) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
     dim3 grid(static_cast<unsigned>((d + 255) / 256 < 8 ? (d + 255) / 256 : 8),
               static_cast<unsigned>(d));
     flip_kernel<<<grid, 256, 0, stream>>>(X, ldx, U, d);

@@ -1,11 +1,13 @@
 // fp32-accurate GEMM tiles on the tcgen05 tensor cores ("3xTF32").
 //
-// D[128 x 128] = sum_k A[m][k] B[n][k] with fp32 operands: each operand is
-// split in shared memory into hi = tf32(x) (round to nearest) and
-// lo = x - hi, and three kind::tf32 MMAs accumulate hi*hi + hi*lo + lo*hi
-// into one fp32 TMEM accumulator.  The dropped lo*lo term and the tf32
-// truncation of lo leave an error of about 2^-21 of |a||b| per product, close
-// to fp32 FFMA, at tensor-core speed.
+// D[128 x 128] = sum_k A[m][k] B[n][k] with fp32 operands split as
+// x = hi + lo, and three kind::tf32 MMAs accumulate hi*hi + hi*lo + lo*hi
+// into one fp32 TMEM accumulator.  kind::tf32 reads a 32-bit operand and
+// ignores its 13 low mantissa bits (truncation, measured on sm_100a), so hi
+// is the fp32 value as TMA delivered it and only lo = x - trunc13(x) (exact
+// in fp32) is written, into a second buffer.  The tensor core truncates lo in
+// turn; that and the dropped lo*lo term leave an error of about 2^-20 of
+// |a||b| per product, close to fp32 FFMA, at tensor-core speed.
 //
 // Persistent: each CTA walks a static list of output tiles (tile, tile +
 // grid, ...), the stage ring runs on across tiles and two TMEM accumulators
@@ -16,9 +18,13 @@
 // with 32-byte chunks).  Warp roles:
 //   warp 0      TMA producer
 //   warp 1      TMEM owner and MMA issuer
-//   warps 2..5  split each stage into hi / lo
-//   warps 6..9  drain the accumulator through the scheduler's store()
-//               (tcgen05.ld, one row per thread, 32 columns at a time).
+//   warps 2..5  write each stage's lo parts
+//   warps 6..9  drain the accumulator (tcgen05.ld, one row per thread, 32
+//               columns at a time) through the scheduler: store() for
+//               plain outputs; for read-modify-write outputs (kRmw, D -= AB^T)
+//               the warp loads its whole destination row segment into
+//               registers before the tile's MMAs finish, so the epilogue
+//               costs one store pass instead of a load round trip per chunk.
 // Every wait is bounded; on expiry GPTQ_ERR_TIMEOUT is recorded and the CTA
 // winds down after its copies and MMAs have landed.
 #pragma once
@@ -35,7 +41,7 @@ constexpr int BN = 128;
 constexpr int BK = 32;                        // K per stage: 128 bytes of fp32
 constexpr int kStages = 3;
 constexpr int kTileBytes = 128 * BK * 4;      // 16 KB
-constexpr int kStageBytes = 4 * kTileBytes;   // A (hi in place), A lo, B (hi in place), B lo
+constexpr int kStageBytes = 4 * kTileBytes;   // A (as loaded), A lo, B (as loaded), B lo
 constexpr int kThreads = 320;                 // TMA, MMA, 4 split warps, 4 epilogue warps
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
 constexpr uint32_t kTmemCols = 256;           // two 128-column accumulators
@@ -57,10 +63,9 @@ struct Bars {
     int abort;
 };
 
-__device__ __forceinline__ float tf32_hi(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
+// x minus the part of it a kind::tf32 MMA sees (exact: both share x's exponent)
+__device__ __forceinline__ float tf32_rest(float x) {
+    return x - __uint_as_float(__float_as_uint(x) & 0xffffe000u);
 }
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -214,22 +219,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                float4* a = reinterpret_cast<float4*>(smem + st * kStageBytes);
-                float4* alo = a + kTileBytes / 16;
-                float4* b = a + 2 * (kTileBytes / 16);
-                float4* blo = a + 3 * (kTileBytes / 16);
+                const float4* a = reinterpret_cast<const float4*>(smem + st * kStageBytes);
+                float4* alo = const_cast<float4*>(a) + kTileBytes / 16;
+                const float4* b = a + 2 * (kTileBytes / 16);
+                float4* blo = const_cast<float4*>(a) + 3 * (kTileBytes / 16);
 #pragma unroll 4
                 for (int i = t0; i < kTileBytes / 16; i += 128) {
-                    float4 x = a[i], h, l;
-                    h.x = tf32_hi(x.x); h.y = tf32_hi(x.y); h.z = tf32_hi(x.z); h.w = tf32_hi(x.w);
-                    l.x = x.x - h.x; l.y = x.y - h.y; l.z = x.z - h.z; l.w = x.w - h.w;
-                    a[i] = h;
-                    alo[i] = l;
-                    x = b[i];
-                    h.x = tf32_hi(x.x); h.y = tf32_hi(x.y); h.z = tf32_hi(x.z); h.w = tf32_hi(x.w);
-                    l.x = x.x - h.x; l.y = x.y - h.y; l.z = x.z - h.z; l.w = x.w - h.w;
-                    b[i] = h;
-                    blo[i] = l;
+                    const float4 x = a[i], y = b[i];
+                    alo[i] = make_float4(tf32_rest(x.x), tf32_rest(x.y), tf32_rest(x.z), tf32_rest(x.w));
+                    blo[i] = make_float4(tf32_rest(y.x), tf32_rest(y.y), tf32_rest(y.z), tf32_rest(y.w));
                 }
                 fence_async_smem();
                 mbar_arrive(&bars->conv[st]);
@@ -245,13 +243,59 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (job.nk <= 0) continue;
             const int slot = lt & 1;
             const uint32_t use = static_cast<uint32_t>(lt >> 1);
-            if (!mbar_wait(&bars->acc_full[slot], use & 1u, abort)) break;
-            tc_fence_after();
+            if constexpr (Sched::kRmw) {
+                // destination row segment: the first nc of its BN columns are updated;
+                // when all BN columns may be read (aligned), the segment is loaded
+                // before the accumulator is ready
+                float* dst = sched.dst(job, row);
+                const int nc = dst != nullptr ? sched.ncols(job, row) : 0;
+                const bool pre = dst != nullptr && sched.nreadable(job) == BN &&
+                                 (reinterpret_cast<uintptr_t>(dst) & 15) == 0;
+                const bool full = pre && nc == BN;
+                float4 old[BN / 4];
+                if (pre) {
+#pragma unroll
+                    for (int i = 0; i < BN / 4; ++i) old[i] = reinterpret_cast<const float4*>(dst)[i];
+                }
+                if (!mbar_wait(&bars->acc_full[slot], use & 1u, abort)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < BN / 16; ++c) {  // 16 columns at a time: the
+                    float v[16];                      // prefetched row holds the registers
+                    tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + slot * BN + c * 16, v);
+                    if (full) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float4 o = old[4 * c + i];
+                            reinterpret_cast<float4*>(dst)[4 * c + i] =
+                                make_float4(o.x - v[4 * i], o.y - v[4 * i + 1], o.z - v[4 * i + 2],
+                                            o.w - v[4 * i + 3]);
+                        }
+                    } else if (pre) {  // partly written row (a diagonal tile)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float4 o = old[4 * c + i];
+                            const int j = 16 * c + 4 * i;
+                            if (j + 0 < nc) dst[j + 0] = o.x - v[4 * i + 0];
+                            if (j + 1 < nc) dst[j + 1] = o.y - v[4 * i + 1];
+                            if (j + 2 < nc) dst[j + 2] = o.z - v[4 * i + 2];
+                            if (j + 3 < nc) dst[j + 3] = o.w - v[4 * i + 3];
+                        }
+                    } else {  // row at the matrix edge: element-wise
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (16 * c + j < nc) dst[16 * c + j] -= v[j];
+                    }
+                }
+            } else {
+                if (!mbar_wait(&bars->acc_full[slot], use & 1u, abort)) break;
+                tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                float v[32];
-                tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + slot * BN + c * 32, v);
-                sched.store(job, row, c * 32, v);
+                for (int c = 0; c < BN / 32; ++c) {
+                    float v[32];
+                    tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + slot * BN + c * 32, v);
+                    sched.store(job, row, c * 32, v);
+                }
             }
             tc_fence_before();
             mbar_arrive(&bars->acc_empty[slot]);

@@ -285,25 +285,15 @@ struct LazySched {
         const int mi = t % mt, ni = t / mt;
         return {128 * mi, c1 + 128 * ni, 0, c0, kBlock / 32};
     }
-    __device__ void store(const g3::Job& jb, int row, int col0, const float (&v)[32]) const {
+    static constexpr bool kRmw = true;
+    __device__ float* dst(const g3::Job& jb, int row) const {
         const int rr = jb.m0 + row;
-        if (rr >= r) return;
-        float* dst = W + static_cast<int64_t>(rr) * ldw + jb.n0 + col0;
-        const int c = jb.n0 + col0;
-        if (c + 32 <= d && (ldw & 3) == 0) {
-            float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                float4 x = d4[q];
-                x.x -= v[4 * q]; x.y -= v[4 * q + 1]; x.z -= v[4 * q + 2]; x.w -= v[4 * q + 3];
-                d4[q] = x;
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                if (c + j < d) dst[j] -= v[j];
-        }
+        return rr < r ? W + static_cast<int64_t>(rr) * ldw + jb.n0 : nullptr;
     }
+    __device__ int ncols(const g3::Job& jb, int) const {
+        return d - jb.n0 < g3::BN ? d - jb.n0 : g3::BN;
+    }
+    __device__ int nreadable(const g3::Job& jb) const { return ncols(jb, 0); }
 };
 
 }  // namespace
