@@ -56,8 +56,14 @@ __global__ void permute_rows_kernel(float* __restrict__ W, int64_t r, int64_t d,
 // cur[4] and the later chunks in nxt[12]; after each chunk the window
 // rotates, so every register index below is a compile-time constant while the
 // chunk loop stays rolled (the code fits the instruction cache).
+//
+// The column being quantized is held by every lane of the group (wcur): a
+// lane derives columns j+1 and j+2 from values shuffled from their owners two
+// steps earlier, applying the same FMAs the owners apply (so the copies are
+// bit-identical to the owners' registers).  The shuffle then has a whole step
+// to land, and the column-to-column chain is FMA -> quantize -> FMA.
 struct GroupParams {
-    float s, inv_s, zf;
+    float s, inv_s, zf, hi;  // scale, 1/scale, zero point, maxq - zero point
 };
 
 // Scale / zero point of the group [c0 + j, c0 + j + g) of this row from its
@@ -113,11 +119,29 @@ __device__ __forceinline__ GroupParams group_params(const float (&cur)[4], const
         p.zf = rintf(-lo / p.s);
     }
     p.inv_s = 1.f / p.s;
+    p.hi = maxq - p.zf;
     return p;
 }
 
-template <bool kSmallGroup>  // group_size < 32: groups start inside a chunk
-__global__ void __launch_bounds__(kWarps * 32)
+// Value of column 32 m + k (3 <= k < 35, k = 4 jq + i4 + 3) of this row, as
+// held by its owner lane: the current chunk for k < 32, the next one after.
+__device__ __forceinline__ float owner_value(int k, int i4, const float (&cur)[4],
+                                             const float (&nxt)[12], int gbase) {
+    // k & 3 == (i4 + 3) & 3 with i4 a compile-time constant
+    const float v = (k < 32) ? cur[(i4 + 3) & 3] : nxt[(i4 + 3) & 3];
+    return __shfl_sync(0xffffffffu, v, gbase + ((k & 31) >> 2));
+}
+
+// Round half to even of |x| <= 2^22 by adding and removing 1.5 * 2^23 (its
+// ulp is 1, so the first add rounds x to an integer under the IEEE
+// round-to-nearest-even mode; both adds are explicit _rn, never contracted).
+__device__ __forceinline__ float round_even(float x) {
+    return __fadd_rn(__fadd_rn(x, 12582912.f), -12582912.f);
+}
+
+template <bool kSmallGroup,  // group_size < 32: groups start inside a chunk
+          bool kFull>        // a full 128-column block (no column guard)
+__global__ void __launch_bounds__(kWarps * 32, 4)
     block_quant_kernel(const __grid_constant__ CUtensorMap tmu, float* __restrict__ W, int64_t r,
                        int64_t d, int64_t ldw, int64_t c0, int bw, int bits, int g,
                        uint8_t* __restrict__ codes, float* __restrict__ scales,
@@ -136,18 +160,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         fence_barrier_init();
         mbar_arrive_expect_tx(&bar, kBlock * kBlock * 4);
         tma_load_2d(Us, &tmu, &bar, static_cast<int>(c0), static_cast<int>(c0));
-        volatile int no_abort = 0;
-        ok = mbar_wait(&bar, 0, &no_abort) ? 1 : 0;
-        if (!ok) report(status, GPTQ_ERR_TIMEOUT);
     }
-    __syncthreads();
-    if (!ok) return;
-    for (int j = tid; j < kBlock; j += blockDim.x)
-        dinv[j] = (j < bw) ? 1.f / Us[j * kBlock + j] : 0.f;
-    __syncthreads();
-    for (int e = tid; e < kBlock * kBlock; e += blockDim.x)
-        if ((e & (kBlock - 1)) <= (e >> 7)) Us[e] = 0.f;  // diagonal and below
-    __syncthreads();
 
     const int lane = tid & 31;
     const int l = lane & 7;
@@ -155,10 +168,10 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + (tid >> 5) * kRowsPerWarp +
                         (lane >> 3);
     const bool live = row < r;
-    const float maxq = static_cast<float>((1 << bits) - 1);
     float* wrow = W + (live ? row : 0) * ldw;
     const bool vec = (ldw & 3) == 0 && bw == kBlock;
 
+    // the row's slice of the block (in flight while the U block arrives)
     float cur[4], nxt[12];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
@@ -179,8 +192,7 @@ __global__ void __launch_bounds__(kWarps * 32)
             else nxt[4 * (m - 1) + i] = v[i];
         }
     }
-
-    GroupParams gp{1.f, 1.f, 0.f};
+    GroupParams gp{1.f, 1.f, 0.f, 0.f};
     if (live && (c0 % g) != 0) {
         // this block continues a group opened by an earlier block (group
         // size > block): take that group's scale and zero point
@@ -188,7 +200,33 @@ __global__ void __launch_bounds__(kWarps * 32)
         gp.s = scales[grp * r + row];
         gp.zf = static_cast<float>(zeros[grp * r + row]);
         gp.inv_s = 1.f / gp.s;
+        gp.hi = static_cast<float>((1 << bits) - 1) - gp.zf;
     }
+
+    if (tid == 0) {
+        volatile int no_abort = 0;
+        ok = mbar_wait(&bar, 0, &no_abort) ? 1 : 0;
+        if (!ok) report(status, GPTQ_ERR_TIMEOUT);
+    }
+    __syncthreads();
+    if (!ok) return;
+    // 1 / U_jj, then row j of the block is cleared at and left of its diagonal
+    // (a thread owns whole rows, so no barrier between the two)
+    for (int j = tid; j < kBlock; j += blockDim.x) {
+        float* ur = Us + j * kBlock;
+        dinv[j] = (j < bw) ? 1.f / ur[j] : 0.f;
+        int c = 0;
+        for (; c + 3 <= j; c += 4) *reinterpret_cast<float4*>(ur + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (; c <= j; ++c) ur[c] = 0.f;
+    }
+    __syncthreads();
+
+    // columns 0, 1, 2 for every lane of the group; afterwards, at the start of
+    // step j: wcur = column j (final), t1 = column j+1 after the feedback of
+    // columns < j, t2 = column j+2 after the feedback of columns < j
+    float wcur = __shfl_sync(0xffffffffu, cur[0], gbase);
+    float t1 = __shfl_sync(0xffffffffu, cur[1], gbase);
+    float t2 = __shfl_sync(0xffffffffu, cur[2], gbase);
 
 #pragma unroll 1
     for (int m = 0; m < 4; ++m) {
@@ -203,10 +241,15 @@ __global__ void __launch_bounds__(kWarps * 32)
         }
         float ev[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t qv[4] = {0u, 0u, 0u, 0u};
+        // 8 rolled steps of 4 unrolled columns: register indices stay
+        // compile-time while the loop body stays small
+#pragma unroll 1
+        for (int jq = 0; jq < 8; ++jq) {
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
+        for (int i4 = 0; i4 < 4; ++i4) {
+            const int jj = 4 * jq + i4;
             const int j = 32 * m + jj;
-            if (j < bw) {
+            if (kFull || j < bw) {
                 if (kSmallGroup && ((c0 + j) % g) == 0) {
                     gp = group_params(cur, nxt, m, jj, l, g, bw, wrow, c0, d, live, bits);
                     if (live && l == 0) {
@@ -215,17 +258,24 @@ __global__ void __launch_bounds__(kWarps * 32)
                         zeros[grp * r + row] = static_cast<int32_t>(gp.zf);
                     }
                 }
-                const float wj = __shfl_sync(0xffffffffu, cur[jj & 3], gbase + (jj >> 2));
-                const float qf = fminf(fmaxf(rintf(wj * gp.inv_s) + gp.zf, 0.f), maxq);
-                const float e = (wj - gp.s * (qf - gp.zf)) * dinv[j];
-                if (l == (jj >> 2)) {
-                    qv[jj & 3] = static_cast<uint32_t>(qf);
-                    ev[jj & 3] = e;
-                }
+                const float* urow = Us + j * kBlock;
+                const float dj = dinv[j];
+                const float u1 = urow[(j + 1) & (kBlock - 1)];
+                const float u2 = urow[(j + 2) & (kBlock - 1)];
+                // q = clamp(rint(w / s) + z, 0, maxq) = rint(clamp(w / s, -z, maxq - z)) + z
+                // (z and maxq are integers); e = (w - s (q - z)) / U_jj
+                const float cq = round_even(fminf(fmaxf(wcur * gp.inv_s, -gp.zf), gp.hi));
+                const float e = fmaf(-(gp.s * dj), cq, wcur * dj);
+                const bool mine = l == jq;
+                qv[i4] = mine ? static_cast<uint32_t>(cq + gp.zf) : qv[i4];
+                ev[i4] = mine ? e : ev[i4];
+                // columns j+1 and j+2 for every lane: the owners' own updates, replicated
+                wcur = fmaf(-e, u1, t1);
+                t1 = fmaf(-e, u2, t2);
                 // feedback into this block's later columns (U row j is zero
                 // at and left of the diagonal, so earlier columns are untouched)
-                const float4* urow = reinterpret_cast<const float4*>(Us + j * kBlock);
-                float4 u = urow[8 * m + l];
+                const float4* urow4 = reinterpret_cast<const float4*>(urow);
+                float4 u = urow4[8 * m + l];
                 cur[0] = fmaf(-e, u.x, cur[0]);
                 cur[1] = fmaf(-e, u.y, cur[1]);
                 cur[2] = fmaf(-e, u.z, cur[2]);
@@ -233,14 +283,17 @@ __global__ void __launch_bounds__(kWarps * 32)
 #pragma unroll
                 for (int s = 0; s < 3; ++s) {
                     if (m + 1 + s < 4) {
-                        u = urow[8 * (m + 1 + s) + l];
+                        u = urow4[8 * (m + 1 + s) + l];
                         nxt[4 * s + 0] = fmaf(-e, u.x, nxt[4 * s + 0]);
                         nxt[4 * s + 1] = fmaf(-e, u.y, nxt[4 * s + 1]);
                         nxt[4 * s + 2] = fmaf(-e, u.z, nxt[4 * s + 2]);
                         nxt[4 * s + 3] = fmaf(-e, u.w, nxt[4 * s + 3]);
                     }
                 }
+                // column j+3 as of this step (used one step later)
+                t2 = owner_value(jj + 3, i4, cur, nxt, gbase);
             }
+        }
         }
         // chunk m done: pre-quantization weights, scaled errors, codes
         if (live) {
@@ -324,8 +377,11 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
         return GPTQ_ERR_INVALID_ARG;
     const size_t q_smem = (kBlock * kBlock + kBlock) * sizeof(float) + 1024;
     const bool small_group = g < 32;
-    auto qkern = small_group ? block_quant_kernel<true> : block_quant_kernel<false>;
-    if (cudaFuncSetAttribute(qkern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto qfull = small_group ? block_quant_kernel<true, true> : block_quant_kernel<false, true>;
+    auto qpart = small_group ? block_quant_kernel<true, false> : block_quant_kernel<false, false>;
+    if (cudaFuncSetAttribute(qfull, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(q_smem)) != cudaSuccess ||
+        cudaFuncSetAttribute(qpart, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(q_smem)) != cudaSuccess)
         return GPTQ_ERR_CUDA;
     const unsigned qgrid = static_cast<unsigned>((d_row + kRowsPerCta - 1) / kRowsPerCta);
@@ -333,7 +389,7 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
     int64_t launches = 1;
     for (int64_t c0 = 0; c0 < d_col; c0 += kBlock) {
         const int bw = static_cast<int>((d_col - c0 < kBlock) ? d_col - c0 : kBlock);
-        qkern<<<qgrid, kWarps * 32, q_smem, stream>>>(
+        (bw == kBlock ? qfull : qpart)<<<qgrid, kWarps * 32, q_smem, stream>>>(
             tU, W, d_row, d_col, ldw, c0, bw, bits, g, codes, scales, zeros, err, status);
         ++launches;
         const int64_t rest = d_col - c0 - bw;
