@@ -139,11 +139,11 @@ gptq_status gptq_quantize_layer(float* W, int64_t d_row, int64_t d_col, int64_t 
     const gptq_status c = check_config(cfg, d_col);
     if (c != GPTQ_OK) return c;
     if (ws == nullptr || !aligned(ws, 256) ||
-        ws_bytes < gptq::quant_workspace_bytes(d_row, d_col, cfg->block_size))
+        ws_bytes < gptq::quant_min_workspace_bytes(d_row, cfg->block_size))
         return GPTQ_ERR_WORKSPACE;
     return launch_status(gptq::launch_quantize(W, d_row, d_col, ldw, U, perm, dead, cfg->bits,
                                                cfg->group_size, cfg->block_size, codes, scales,
-                                               zeros, dev_status, ws, stream));
+                                               zeros, dev_status, ws, ws_bytes, stream));
 }
 
 gptq_status gptq_pack(const uint8_t* codes, int64_t d_row, int64_t d_col, int32_t bits,

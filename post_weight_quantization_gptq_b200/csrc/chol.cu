@@ -75,6 +75,8 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
     __shared__ int bad;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) bad = 0;
+    pdl_trigger();
+    pdl_wait();
     {
         // rows of the block: 16 float4 loads per thread, all in flight
         // (ldp, kb and kw are multiples of 4, so a float4 never crosses kw)
@@ -529,13 +531,17 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
     for (int k = 0; k < npan; ++k) {
         const int64_t kb = static_cast<int64_t>(k) * NB;
         const int kw = static_cast<int>((d - kb < NB) ? d - kb : NB);
-        potrf_inv_128_kernel<<<1, kDiagThreads, kDiagSmem, stream>>>(P, ldp, kb, kw, X, ldx, status);
+        // (after the previous panel's column update, or the gather for k = 0)
+        if (launch_kernel(true, potrf_inv_128_kernel, dim3(1), dim3(kDiagThreads), kDiagSmem, stream,
+                          P, ldp, kb, kw, X, ldx, status) != cudaSuccess)
+            return GPTQ_ERR_CUDA;
         ++launches;
         const int64_t m = d - kb - kw;
         const int mt = static_cast<int>((m + NB - 1) / NB);
         if (m > 0) {
             TrsmSched ts{P, ldp, di, static_cast<int>(kb), kw};
-            if (g3::launch<TrsmSched, false, false>(tP, tX, ts, mt, status, stream, sms) != cudaSuccess)
+            if (g3::launch<TrsmSched, false, false>(tP, tX, ts, mt, status, stream, sms, true) !=
+                cudaSuccess)
                 return GPTQ_ERR_CUDA;
             ++launches;
         }
@@ -572,7 +578,7 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
         if (m > 0) {
             BUpdSched bu{X, ldx, di, static_cast<int>(kb), mt};
             if (g3::launch<BUpdSched, false, true>(tP, tXmn, bu, mt * (k + 1), status, la->inv,
-                                                   inv_sms) != cudaSuccess)
+                                                   inv_sms, k > 0) != cudaSuccess)
                 return GPTQ_ERR_CUDA;
             ++launches;
         }

@@ -38,6 +38,15 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
 }
 
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// serialization attribute may start while the kernel before it in the stream
+// is still running; it touches no global memory before pdl_wait(), which
+// returns once every earlier kernel in the stream has completed and its
+// writes are visible.  pdl_trigger() lets this kernel's own dependent start
+// its set-up early.  Both are no-ops for ordinary launches.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_barrier_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }

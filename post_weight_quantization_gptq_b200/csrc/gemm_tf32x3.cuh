@@ -32,6 +32,7 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "kernels.h"
 
 namespace gptq {
 namespace g3 {
@@ -107,6 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort = &bars->abort;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    pdl_trigger();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -132,6 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem;
+    pdl_wait();  // set-up above touched no global memory
 
     if (warp == 0) {
         // ---------------------------------------------------- TMA producer
@@ -310,16 +313,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0 && bars->abort) report(status, GPTQ_ERR_TIMEOUT);
 }
 
+// pdl: launched with programmatic serialization (see launch_kernel).
 template <class Sched, bool A_MN, bool B_MN>
 inline cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const Sched& sched,
-                          int tiles, int32_t* status, cudaStream_t stream, int sms) {
+                          int tiles, int32_t* status, cudaStream_t stream, int sms,
+                          bool pdl = false) {
     auto kern = gemm_tf32x3_kernel<Sched, A_MN, B_MN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     if (tiles <= 0) return cudaSuccess;
     const int grid = tiles < sms ? tiles : sms;
-    kern<<<grid, kThreads, kSmemBytes, stream>>>(ta, tb, sched, tiles, status);
-    return cudaGetLastError();
+    return launch_kernel(pdl, kern, dim3(grid), dim3(kThreads), kSmemBytes, stream, ta, tb, sched,
+                         tiles, status);
 }
 
 }  // namespace g3

@@ -18,6 +18,26 @@ int num_sms();
 void count_launches(int64_t k);
 int64_t launches();
 
+// Launch with the programmatic-serialization attribute when pdl is set (the
+// kernel must call pdl_wait() before its first global memory access); an
+// ordinary launch otherwise.  Kernels that follow a cudaStreamWaitEvent are
+// launched without it.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block,
+                                 size_t smem, cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Shared-memory swizzle of a TMA box: none, 128-byte (16-byte chunks), or
 // 128-byte with 32-byte chunks (the layout 32-bit MN-major MMA operands use).
 enum class Swz { kNone, k128, k128Atom32 };
@@ -44,11 +64,14 @@ gptq_status launch_chol_inverse(float* P, float* Xbuf, int64_t ldx, int64_t d, f
                                 int32_t* status, void* ws, cudaStream_t stream);
 
 // ---- stages 3-4 (quant.cu)
+// Workspace of the fastest schedule, and the least the column walk accepts
+// (a smaller workspace shortens the deferred runs of the lazy update).
 size_t quant_workspace_bytes(int64_t d_row, int64_t d_col, int block);
+size_t quant_min_workspace_bytes(int64_t d_row, int block);
 gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw, const float* U,
                             const int32_t* perm, const uint8_t* dead, int bits, int group,
                             int block, uint8_t* codes, float* scales, int32_t* zeros,
-                            int32_t* status, void* ws, cudaStream_t stream);
+                            int32_t* status, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 // ---- stage 5 (pack.cu)
 gptq_status launch_pack(const uint8_t* codes, int64_t d_row, int64_t d_col, int bits,

@@ -62,7 +62,7 @@ extern "C" gptq_status gptq_quantize_layer_noalloc(float* W, int64_t d_row, int6
     size_t need = 0;
     const gptq_status s = gptq_workspace_size(cfg, d_row, d_col, &need);
     if (s != GPTQ_OK) return s;
-    if (gptq::quant_workspace_bytes(d_row, d_col, cfg->block_size) > kNoAllocScratchBytes)
+    if (gptq::quant_min_workspace_bytes(d_row, cfg->block_size) > kNoAllocScratchBytes)
         return GPTQ_ERR_WORKSPACE;  // the layer needs more scratch than the fixed array holds
     void* ws = scratch_on_current_device();
     if (ws == nullptr) return GPTQ_ERR_CUDA;

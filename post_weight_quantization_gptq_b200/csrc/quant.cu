@@ -19,6 +19,8 @@
 //  lazy update          W[:, c1:] -= Err * U[c0:c1, c1:] on the tensor cores
 //                       (3xTF32 tcgen05 GEMM, fp32-accurate)
 #include <cmath>
+#include <tuple>
+#include <vector>
 
 #include "common.cuh"
 #include "gemm_tf32x3.cuh"
@@ -37,6 +39,7 @@ __global__ void permute_rows_kernel(float* __restrict__ W, int64_t r, int64_t d,
                                     const int32_t* __restrict__ perm,
                                     const uint8_t* __restrict__ dead) {
     extern __shared__ float rowbuf[];
+    pdl_trigger();
     for (int64_t row = blockIdx.x; row < r; row += gridDim.x) {
         float* w = W + row * ldw;
         for (int64_t k = threadIdx.x; k < d; k += blockDim.x) rowbuf[k] = w[k];
@@ -146,7 +149,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
                        int64_t d, int64_t ldw, int64_t c0, int bw, int bits, int g,
                        uint8_t* __restrict__ codes, float* __restrict__ scales,
                        int32_t* __restrict__ zeros, float* __restrict__ err_out,
-                       int32_t* status) {
+                       int64_t err_ld, int32_t* status) {
     extern __shared__ uint8_t smem_raw[];
     float* smem = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -155,9 +158,13 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
     __shared__ __align__(8) uint64_t bar;
     __shared__ int ok;
     const int tid = threadIdx.x;
+    pdl_trigger();
     if (tid == 0) {
         mbar_init(&bar, 1);
         fence_barrier_init();
+    }
+    pdl_wait();
+    if (tid == 0) {
         mbar_arrive_expect_tx(&bar, kBlock * kBlock * 4);
         tma_load_2d(Us, &tmu, &bar, static_cast<int>(c0), static_cast<int>(c0));
     }
@@ -298,7 +305,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
         // chunk m done: pre-quantization weights, scaled errors, codes
         if (live) {
             const int cb = 32 * m + 4 * l;
-            *reinterpret_cast<float4*>(err_out + row * kBlock + cb) =
+            *reinterpret_cast<float4*>(err_out + row * err_ld + cb) =
                 make_float4(ev[0], ev[1], ev[2], ev[3]);
             if (vec) {
                 *reinterpret_cast<float4*>(wrow + c0 + cb) = make_float4(cur[0], cur[1], cur[2], cur[3]);
@@ -328,17 +335,18 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
 }
 
 // ------------------------------------------------------------------------
-// Lazy update W[:, c1:d] -= Err[:, 0:128] U[c0:c0+128, c1:d] as 128 x 128
-// output tiles of the 3xTF32 GEMM: A = Err (K-major), B = U's rows (MN-major).
+// Lazy update of the columns [c1, c1 + n) from the errors of the columns
+// [k0, k0 + klen):  W[:, c1:] -= Err[:, k0:k0+klen] U[k0:k0+klen, c1:]
+// as 128 x 128 output tiles of the 3xTF32 GEMM: A = Err (K-major, held in the
+// error buffer from column ke), B = U's rows (MN-major).
 struct LazySched {
+    static constexpr bool kRmw = true;
     float* W;
     int64_t ldw;
-    int r, d, c0, c1, mt;
+    int r, d, c1, mt, ke, k0, nk;
     __device__ g3::Job job(int t) const {
-        const int mi = t % mt, ni = t / mt;
-        return {128 * mi, c1 + 128 * ni, 0, c0, kBlock / 32};
+        return {128 * (t % mt), c1 + 128 * (t / mt), ke, k0, nk};
     }
-    static constexpr bool kRmw = true;
     __device__ float* dst(const g3::Job& jb, int row) const {
         const int rr = jb.m0 + row;
         return rr < r ? W + static_cast<int64_t>(rr) * ldw + jb.n0 : nullptr;
@@ -351,17 +359,94 @@ struct LazySched {
 
 }  // namespace
 
-size_t quant_workspace_bytes(int64_t d_row, int64_t, int block) {
+namespace {
+
+constexpr int kMaxDefer = 8;  // blocks whose errors the lazy update may defer
+
+int64_t num_blocks(int64_t d_col) { return (d_col + kBlock - 1) / kBlock; }
+
+// Host model of the deferred schedule (see launch_quantize): applied[b] =
+// the number of leading blocks whose feedback block b has received.  Checks
+// that every block, and every later block its group reads when the group
+// starts there, is complete when it is quantized.
+bool schedule_valid(int nb, int defer, int g_blocks) {
+    std::vector<int> applied(nb, 0);
+    bool ok = true;
+    auto gemm = [&](int a, int c, int e) {
+        for (int b = c; b < e; ++b) {
+            ok = ok && applied[b] == a;
+            applied[b] = c;
+        }
+    };
+    auto quant = [&](int b) {
+        ok = ok && applied[b] == b;
+        if (g_blocks > 1 && b % g_blocks == 0)
+            for (int x = b + 1; x < nb && x < b + g_blocks; ++x) ok = ok && applied[x] == b;
+    };
+    // recursion on [lo, hi): quantize [lo, mid), update [mid, hi), quantize [mid, hi)
+    for (int s0 = 0; s0 < nb; s0 += defer) {
+        const int s1 = s0 + defer < nb ? s0 + defer : nb;
+        std::vector<std::tuple<int, int, int>> stack{{s0, s1, 0}};
+        while (!stack.empty()) {
+            auto [lo, hi, state] = stack.back();
+            stack.pop_back();
+            if (hi - lo == 1) {
+                quant(lo);
+                continue;
+            }
+            int half = 1;
+            while (2 * half < hi - lo) half *= 2;
+            const int mid = lo + half;
+            if (state == 0) {
+                stack.push_back({lo, hi, 1});
+                stack.push_back({lo, mid, 0});
+            } else {
+                gemm(lo, mid, hi);
+                stack.push_back({mid, hi, 0});
+            }
+        }
+        if (s1 < nb) gemm(s0, s1, nb);
+    }
+    return ok;
+}
+
+}  // namespace
+
+size_t quant_workspace_bytes(int64_t d_row, int64_t d_col, int block) {
+    const int64_t nb = num_blocks(d_col);
+    const int64_t defer = nb < kMaxDefer ? nb : kMaxDefer;
+    return ((static_cast<size_t>(d_row) * block * defer * sizeof(float) + 255) / 256) * 256;
+}
+
+size_t quant_min_workspace_bytes(int64_t d_row, int block) {
     return ((static_cast<size_t>(d_row) * block * sizeof(float) + 255) / 256) * 256;
 }
 
+// The column walk.  Blocks of 128 columns are quantized in order; the lazy
+// update of the pages' batched form is deferred and regrouped so that most of
+// its arithmetic runs as long-K products: within a run of up to kMaxDefer
+// blocks (as many as the workspace holds), blocks [lo, hi) are handled as
+// [lo, mid) -> W[:, mid:hi] -= Err[:, lo:mid] U[lo:mid, mid:hi] -> [mid, hi),
+// recursively; after the run, one product applies its errors to every later
+// column.  Every block still receives the feedback of every earlier block
+// before it is quantized (the same sums, in another order).  Groups wider than
+// a block must find their later columns complete when the group starts; the
+// host checks the schedule and shortens the runs (down to the per-block
+// form) when a group size does not fit it.
 gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw, const float* U,
                             const int32_t* perm, const uint8_t* dead, int bits, int group,
                             int block, uint8_t* codes, float* scales, int32_t* zeros,
-                            int32_t* status, void* ws, cudaStream_t stream) {
+                            int32_t* status, void* ws, size_t ws_bytes, cudaStream_t stream) {
     if (block != kBlock) return GPTQ_ERR_UNSUPPORTED;
     const int g = (group == -1 || group > d_col) ? static_cast<int>(d_col) : group;
+    const int nb = static_cast<int>(num_blocks(d_col));
+    int defer = nb < kMaxDefer ? nb : kMaxDefer;
+    while (defer > 1 && static_cast<size_t>(d_row) * kBlock * defer * sizeof(float) > ws_bytes)
+        defer /= 2;
+    const int g_blocks = g > kBlock ? (g + kBlock - 1) / kBlock : 1;
+    while (defer > 1 && !schedule_valid(nb, defer, g_blocks)) defer /= 2;
     float* err = static_cast<float*>(ws);
+    const int64_t err_ld = static_cast<int64_t>(defer) * kBlock;
 
     const size_t row_smem = static_cast<size_t>(d_col) * sizeof(float);
     if (cudaFuncSetAttribute(permute_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -373,7 +458,7 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
     CUtensorMap tU, tUmn, tErr;
     if (!make_tmap_2d(&tU, false, U, d_col, d_col, d_col, kBlock, kBlock, Swz::kNone) ||
         !make_tmap_2d(&tUmn, false, U, d_col, d_col, d_col, 32, 32, Swz::k128Atom32) ||
-        !make_tmap_2d(&tErr, false, err, kBlock, d_row, kBlock, 32, 128, Swz::k128))
+        !make_tmap_2d(&tErr, false, err, err_ld, d_row, err_ld, 32, 128, Swz::k128))
         return GPTQ_ERR_INVALID_ARG;
     const size_t q_smem = (kBlock * kBlock + kBlock) * sizeof(float) + 1024;
     const bool small_group = g < 32;
@@ -386,22 +471,55 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
         return GPTQ_ERR_CUDA;
     const unsigned qgrid = static_cast<unsigned>((d_row + kRowsPerCta - 1) / kRowsPerCta);
     const int mt = static_cast<int>((d_row + 127) / 128);
+    const int sms = num_sms();
     int64_t launches = 1;
-    for (int64_t c0 = 0; c0 < d_col; c0 += kBlock) {
+    int run0 = 0;  // first block of the current run (its errors sit at column 0 of err)
+
+    auto quantize_block = [&](int b) -> bool {
+        const int64_t c0 = static_cast<int64_t>(b) * kBlock;
         const int bw = static_cast<int>((d_col - c0 < kBlock) ? d_col - c0 : kBlock);
-        (bw == kBlock ? qfull : qpart)<<<qgrid, kWarps * 32, q_smem, stream>>>(
-            tU, W, d_row, d_col, ldw, c0, bw, bits, g, codes, scales, zeros, err, status);
         ++launches;
-        const int64_t rest = d_col - c0 - bw;
-        if (rest > 0) {
-            const int nt = static_cast<int>((rest + 127) / 128);
-            LazySched ls{W, ldw, static_cast<int>(d_row), static_cast<int>(d_col),
-                         static_cast<int>(c0), static_cast<int>(c0 + bw), mt};
-            if (g3::launch<LazySched, false, true>(tErr, tUmn, ls, mt * nt, status, stream, num_sms()) !=
-                cudaSuccess)
-                return GPTQ_ERR_CUDA;
-            ++launches;
+        return launch_kernel(true, bw == kBlock ? qfull : qpart, dim3(qgrid), dim3(kWarps * 32),
+                             q_smem, stream, tU, W, d_row, d_col, ldw, c0, bw, bits, g, codes,
+                             scales, zeros, err + static_cast<int64_t>(b - run0) * kBlock, err_ld,
+                             status) == cudaSuccess;
+    };
+    // W[:, blocks [c, e)) -= Err[:, blocks [a, c)) U[blocks [a, c), blocks [c, e))
+    auto update = [&](int a, int c, int e) -> bool {
+        const int64_t c1 = static_cast<int64_t>(c) * kBlock;
+        const int64_t cend = static_cast<int64_t>(e) * kBlock < d_col ? static_cast<int64_t>(e) * kBlock
+                                                                    : d_col;
+        const int nt = static_cast<int>((cend - c1 + 127) / 128);
+        LazySched ls{W, ldw, static_cast<int>(d_row), static_cast<int>(cend), static_cast<int>(c1), mt,
+                     (a - run0) * kBlock, a * kBlock, (c - a) * (kBlock / 32)};
+        ++launches;
+        return g3::launch<LazySched, false, true>(tErr, tUmn, ls, mt * nt, status, stream, sms, true) ==
+               cudaSuccess;
+    };
+    // blocks [lo, hi) of the current run, complete w.r.t. every block < lo
+    std::vector<std::tuple<int, int, int>> stack;
+    for (run0 = 0; run0 < nb; run0 += defer) {
+        const int run1 = run0 + defer < nb ? run0 + defer : nb;
+        stack.assign(1, {run0, run1, 0});
+        while (!stack.empty()) {
+            auto [lo, hi, state] = stack.back();
+            stack.pop_back();
+            if (hi - lo == 1) {
+                if (!quantize_block(lo)) return GPTQ_ERR_CUDA;
+                continue;
+            }
+            int half = 1;
+            while (2 * half < hi - lo) half *= 2;
+            const int mid = lo + half;
+            if (state == 0) {
+                stack.push_back({lo, hi, 1});
+                stack.push_back({lo, mid, 0});
+            } else {
+                if (!update(lo, mid, hi)) return GPTQ_ERR_CUDA;
+                stack.push_back({mid, hi, 0});
+            }
         }
+        if (run1 < nb && !update(run0, run1, nb)) return GPTQ_ERR_CUDA;
     }
     count_launches(launches);
     return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
