@@ -12,7 +12,7 @@
 // the gather that builds P (prep.cu) and into the final store here.
 //
 //   P buffer (d x d, ld d, the caller's U): lower triangle = P on entry, L
-//            after the factorization; finally U.
+//            below the diagonal blocks after the factorization; finally U.
 //   X buffer (the caller's consumed H, ld ldx): lower triangle = L^-1, with
 //            every 128 x 128 diagonal block's strict upper part zeroed.
 //
@@ -79,14 +79,17 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
     pdl_wait();
     {
         // rows of the block: 16 float4 loads per thread, all in flight
-        // (ldp, kb and kw are multiples of 4, so a float4 never crosses kw)
+        // (ldp, kb and kw are multiples of 4, so a float4 never crosses kw).
+        // Coherent (L2) loads: with a programmatic launch the kernel before
+        // this one in the stream may still have been writing P when this one
+        // started, so the read-only (non-coherent) path must not be used.
         float4 v[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
             const int e = tid + q * kDiagThreads;
             const int i = e >> 5, j = (e & 31) * 4;
             v[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (i < kw && j <= i) v[q] = *reinterpret_cast<const float4*>(P + (kb + i) * ldp + kb + j);
+            if (i < kw && j <= i) v[q] = __ldcg(reinterpret_cast<const float4*>(P + (kb + i) * ldp + kb + j));
         }
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
@@ -102,43 +105,81 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
     }
     __syncthreads();
 
-    for (int b = 0; b < 4; ++b) {
-        const int o = 32 * b;
-        if (warp == 0) {
-            // -- 32 x 32 Cholesky: lane i holds row o + i, register r = column c + r
-            float a[32];
+    // -- 32 x 32 Cholesky of the diagonal block at o, by warp 0: lane i holds
+    //    row o + i, register r = column c + r
+    auto chol32 = [&](int o) {
+        float a[32];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float4 t = lds4(A + (o + lane) * LDA + o + 4 * q);
-                a[4 * q] = t.x; a[4 * q + 1] = t.y; a[4 * q + 2] = t.z; a[4 * q + 3] = t.w;
+        for (int q = 0; q < 8; ++q) {
+            const float4 t = lds4(A + (o + lane) * LDA + o + 4 * q);
+            a[4 * q] = t.x; a[4 * q + 1] = t.y; a[4 * q + 2] = t.z; a[4 * q + 3] = t.w;
+        }
+#pragma unroll
+        for (int r = 0; r < 32; ++r) a[r] = (r <= lane) ? a[r] : 0.f;
+#pragma unroll 1
+        for (int c = 0; c < 32; ++c) {
+            float piv = __shfl_sync(0xffffffffu, a[0], c);
+            if (!(piv > 0.f)) {  // not positive definite (or NaN): flag, stay finite
+                bad = 1;
+                piv = 1.f;
+            }
+            const float inv = rsqrtf(piv);
+            const float a0 = (lane == c) ? piv * inv : ((lane > c) ? a[0] * inv : 0.f);
+            if (lane >= c) A[(o + lane) * LDA + o + c] = a0;
+            if (lane == c) dinv[o + c] = inv;
+            // lane i > c holds L[o+i][o+c] -> Lc[c][i-c-1]; lanes <= c fill the tail with 0
+            Lc[c * 32 + ((lane - c - 1) & 31)] = a0 * (lane > c ? 1.f : 0.f);
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {  // update and rotate
+                const float4 l = lds4(Lc + c * 32 + 4 * q);
+                a[4 * q] = fmaf(-a0, l.x, a[4 * q + 1]);
+                a[4 * q + 1] = fmaf(-a0, l.y, a[4 * q + 2]);
+                a[4 * q + 2] = fmaf(-a0, l.z, a[4 * q + 3]);
+                a[4 * q + 3] = (q < 7) ? fmaf(-a0, l.w, a[4 * q + 4]) : 0.f;
+            }
+        }
+    };
+    // -- trailing update of the lower part below strip o, 4 x 4 register blocks
+    //    u in [u0, u1) (triangular numbering from row r0), read from the
+    //    transposed strip (consecutive blocks -> consecutive float4)
+    auto trail = [&](int r0, int u0, int u1, int t, int stride) {
+        for (int u = u0 + t; u < u1; u += stride) {
+            int bi = static_cast<int>((sqrtf(8.f * u + 1.f) - 1.f) * 0.5f);
+            while (bi * (bi + 1) / 2 > u) --bi;
+            while ((bi + 1) * (bi + 2) / 2 <= u) ++bi;
+            const int bj = u - bi * (bi + 1) / 2;
+            const int i0 = r0 + 4 * bi, j0 = r0 + 4 * bj;
+            float acc2[4][4] = {};
+#pragma unroll 8
+            for (int k = 0; k < 32; ++k) {
+                const float4 li = lds4(Ls + k * LDA + i0), lj = lds4(Ls + k * LDA + j0);
+                const float a4[4] = {li.x, li.y, li.z, li.w}, b4[4] = {lj.x, lj.y, lj.z, lj.w};
+#pragma unroll
+                for (int t4 = 0; t4 < 4; ++t4)
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) acc2[t4][w] = fmaf(a4[t4], b4[w], acc2[t4][w]);
             }
 #pragma unroll
-            for (int r = 0; r < 32; ++r) a[r] = (r <= lane) ? a[r] : 0.f;
-#pragma unroll 1
-            for (int c = 0; c < 32; ++c) {
-                float piv = __shfl_sync(0xffffffffu, a[0], c);
-                if (!(piv > 0.f)) {  // not positive definite (or NaN): flag, stay finite
-                    bad = 1;
-                    piv = 1.f;
-                }
-                const float inv = rsqrtf(piv);
-                const float a0 = (lane == c) ? piv * inv : ((lane > c) ? a[0] * inv : 0.f);
-                if (lane >= c) A[(o + lane) * LDA + o + c] = a0;
-                if (lane == c) dinv[o + c] = inv;
-                // lane i > c holds L[o+i][o+c] -> Lc[c][i-c-1]; lanes <= c fill the tail with 0
-                Lc[c * 32 + ((lane - c - 1) & 31)] = a0 * (lane > c ? 1.f : 0.f);
-                __syncwarp();
+            for (int t4 = 0; t4 < 4; ++t4) {
+                float* dst = A + (i0 + t4) * LDA + j0;
+                if (j0 + 3 <= i0 + t4) {
+                    float4 d4 = lds4(dst);
+                    d4.x -= acc2[t4][0]; d4.y -= acc2[t4][1]; d4.z -= acc2[t4][2]; d4.w -= acc2[t4][3];
+                    sts4(dst, d4);
+                } else {
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {  // update and rotate
-                    const float4 l = lds4(Lc + c * 32 + 4 * q);
-                    a[4 * q] = fmaf(-a0, l.x, a[4 * q + 1]);
-                    a[4 * q + 1] = fmaf(-a0, l.y, a[4 * q + 2]);
-                    a[4 * q + 2] = fmaf(-a0, l.z, a[4 * q + 3]);
-                    a[4 * q + 3] = (q < 7) ? fmaf(-a0, l.w, a[4 * q + 4]) : 0.f;
+                    for (int w = 0; w < 4; ++w)
+                        if (j0 + w <= i0 + t4) dst[w] -= acc2[t4][w];
                 }
             }
         }
-        __syncthreads();
+    };
+
+    if (warp == 0) chol32(0);
+    __syncthreads();
+    for (int b = 0; b < 4; ++b) {
+        const int o = 32 * b;
         const int r0 = o + 32;
         if (warp < 4) {
             // -- forward substitution with L_bb on 128 right-hand sides at once:
@@ -182,42 +223,16 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
         }
         __syncthreads();
         if (r0 < NB) {
-            // -- trailing update of the lower part, 4 x 4 register blocks read from
-            //    the transposed strip (consecutive blocks -> consecutive float4)
+            // the next strip's 32 x 32 diagonal block first (units 0..35), then
+            // warp 0 factors it while warps 1..7 finish the trailing update
             const int mb = (NB - r0) / 4;
             const int units = mb * (mb + 1) / 2;
-            for (int u = tid; u < units; u += kDiagThreads) {
-                int bi = static_cast<int>((sqrtf(8.f * u + 1.f) - 1.f) * 0.5f);
-                while (bi * (bi + 1) / 2 > u) --bi;
-                while ((bi + 1) * (bi + 2) / 2 <= u) ++bi;
-                const int bj = u - bi * (bi + 1) / 2;
-                const int i0 = r0 + 4 * bi, j0 = r0 + 4 * bj;
-                float acc2[4][4] = {};
-#pragma unroll 8
-                for (int k = 0; k < 32; ++k) {
-                    const float4 li = lds4(Ls + k * LDA + i0), lj = lds4(Ls + k * LDA + j0);
-                    const float a4[4] = {li.x, li.y, li.z, li.w}, b4[4] = {lj.x, lj.y, lj.z, lj.w};
-#pragma unroll
-                    for (int t = 0; t < 4; ++t)
-#pragma unroll
-                        for (int w = 0; w < 4; ++w) acc2[t][w] = fmaf(a4[t], b4[w], acc2[t][w]);
-                }
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    float* dst = A + (i0 + t) * LDA + j0;
-                    if (j0 + 3 <= i0 + t) {
-                        float4 d4 = lds4(dst);
-                        d4.x -= acc2[t][0]; d4.y -= acc2[t][1]; d4.z -= acc2[t][2]; d4.w -= acc2[t][3];
-                        sts4(dst, d4);
-                    } else {
-#pragma unroll
-                        for (int w = 0; w < 4; ++w)
-                            if (j0 + w <= i0 + t) dst[w] -= acc2[t][w];
-                    }
-                }
-            }
+            trail(r0, 0, 36, tid, kDiagThreads);
+            __syncthreads();
+            if (warp == 0) chol32(r0);
+            else trail(r0, 36, units, tid - 32, kDiagThreads - 32);
+            __syncthreads();
         }
-        __syncthreads();
     }
 
     // -- join the 32 x 32 inverses: X_CA = -X_CC (L_CA X_AA), 4 x 4 register
@@ -288,27 +303,19 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
         __syncthreads();
     }
 
-    // -- write L (lower part) and X (zeros above the diagonal included: the
-    //    tensor-core GEMMs read it as a full tile), float4 per access
+    // -- write X (zeros above the diagonal included: the tensor-core GEMMs read
+    //    it as a full tile), float4 per access.  L's diagonal block is not
+    //    written back: nothing reads it after this kernel.
 #pragma unroll 4
     for (int e = tid; e < NB * NB / 4; e += kDiagThreads) {
         const int i = e >> 5, j = (e & 31) * 4;
         if (i >= kw || j >= kw) continue;
-        const float4 l4 = lds4(A + i * LDA + j);
         float4 x4 = lds4(Xs + i * LDA + j);
         if (j + 1 > i) x4.y = 0.f;
         if (j + 2 > i) x4.z = 0.f;
         if (j + 3 > i) x4.w = 0.f;
         if (j > i) x4.x = 0.f;
         *reinterpret_cast<float4*>(X + (kb + i) * ldx + kb + j) = x4;
-        if (j + 3 <= i) {
-            *reinterpret_cast<float4*>(P + (kb + i) * ldp + kb + j) = l4;
-        } else if (j <= i) {
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-            for (int t = 0; t < 4; ++t)
-                if (j + t <= i) P[(kb + i) * ldp + kb + j + t] = lv[t];
-        }
     }
     if (tid == 0 && bad) report(status, GPTQ_ERR_NOT_PD);
 }
@@ -455,7 +462,6 @@ struct Lookahead {
     cudaStream_t inv = nullptr;    // L^-1
     cudaEvent_t start = nullptr;
     cudaEvent_t solved[4] = {};    // panel k's L_kk^-1 and L[:, k] are final
-    cudaEvent_t ready[4] = {};     // panel k+1's column updated
     cudaEvent_t done[4] = {};      // rest of panel k's trailing update done
     cudaEvent_t side_end = nullptr, inv_end = nullptr;
     bool ok = false;
@@ -477,7 +483,6 @@ Lookahead* lookahead_resources() {
             if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
         for (int i = 0; i < 4; ++i)
             if (cudaEventCreateWithFlags(&la.solved[i], cudaEventDisableTiming) != cudaSuccess ||
-                cudaEventCreateWithFlags(&la.ready[i], cudaEventDisableTiming) != cudaSuccess ||
                 cudaEventCreateWithFlags(&la.done[i], cudaEventDisableTiming) != cudaSuccess)
                 return nullptr;
         la.ok = true;
@@ -489,12 +494,14 @@ Lookahead* lookahead_resources() {
 // Lookahead schedule.  The caller's stream runs the panel chain
 //   potrf(k) -> panel solve(k) -> update of panel k+1's column -> potrf(k+1);
 // the side stream runs the rest of each trailing update and the inverse
-// stream builds L^-1, both in the shadow of the chain.  Ordering: the update
-// of panel k+1's column waits for the previous panel's rest-of-update (both
-// touch that column), so potrf and the panel solve of k+1 see every update
-// they need; the inverse stream waits for each panel's solve and is in order
-// with itself; nothing on the chain waits for it.  The SMs are shared out so
-// that the chain's one-wave launches always find free SMs.
+// stream builds L^-1, both in the shadow of the chain.  Ordering: both side
+// streams start on panel k once its solve is done; the update of panel k+1's
+// column waits for the previous panel's rest-of-update (both touch that
+// column), so potrf and the panel solve of k+1 see every update they need;
+// the inverse stream is in order with itself; nothing on the chain waits for
+// it.  A programmatic (early) launch is used only for a kernel whose
+// predecessor in its stream is a kernel.  The SMs are shared out so that the
+// chain's one-wave launches find free SMs.
 gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, float* U,
                                 int32_t* status, void*, cudaStream_t stream) {
     const int64_t ldp = d;
@@ -531,8 +538,9 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
     for (int k = 0; k < npan; ++k) {
         const int64_t kb = static_cast<int64_t>(k) * NB;
         const int kw = static_cast<int>((d - kb < NB) ? d - kb : NB);
-        // (after the previous panel's column update, or the gather for k = 0)
-        if (launch_kernel(true, potrf_inv_128_kernel, dim3(1), dim3(kDiagThreads), kDiagSmem, stream,
+        // directly after the previous panel's column update (programmatic
+        // launch); panel 0 follows an event record and is launched plainly
+        if (launch_kernel(k > 0, potrf_inv_128_kernel, dim3(1), dim3(kDiagThreads), kDiagSmem, stream,
                           P, ldp, kb, kw, X, ldx, status) != cudaSuccess)
             return GPTQ_ERR_CUDA;
         ++launches;
@@ -545,8 +553,11 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
                 return GPTQ_ERR_CUDA;
             ++launches;
         }
+        // panel k is final: the inverse stream and the rest of the trailing
+        // update (whose tiles the next column's update does not touch) may go
         if (cudaEventRecord(la->solved[k & 3], stream) != cudaSuccess ||
-            cudaStreamWaitEvent(la->inv, la->solved[k & 3], 0) != cudaSuccess)
+            cudaStreamWaitEvent(la->inv, la->solved[k & 3], 0) != cudaSuccess ||
+            cudaStreamWaitEvent(la->side, la->solved[k & 3], 0) != cudaSuccess)
             return GPTQ_ERR_CUDA;
         if (m > 0) {
             if (k > 0 && cudaStreamWaitEvent(stream, la->done[(k - 1) & 3], 0) != cudaSuccess)
@@ -556,9 +567,6 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
                 return GPTQ_ERR_CUDA;
             ++launches;
         }
-        if (cudaEventRecord(la->ready[k & 3], stream) != cudaSuccess ||
-            cudaStreamWaitEvent(la->side, la->ready[k & 3], 0) != cudaSuccess)
-            return GPTQ_ERR_CUDA;
         if (mt > 1) {
             SyrkSched rs{P, ldp, di, static_cast<int>(kb), kw, static_cast<int>(kb + kw), 2};
             if (g3::launch<SyrkSched, false, false>(tP, tP, rs, mt * (mt + 1) / 2 - mt, status,

@@ -42,8 +42,10 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 // serialization attribute may start while the kernel before it in the stream
 // is still running; it touches no global memory before pdl_wait(), which
 // returns once every earlier kernel in the stream has completed and its
-// writes are visible.  pdl_trigger() lets this kernel's own dependent start
-// its set-up early.  Both are no-ops for ordinary launches.
+// writes are visible to coherent loads (not to the read-only non-coherent
+// path, which such a kernel must avoid for data written before it).
+// pdl_trigger() lets this kernel's own dependent start its set-up early.
+// Both are no-ops for ordinary launches.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 

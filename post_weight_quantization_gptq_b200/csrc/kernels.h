@@ -18,10 +18,14 @@ int num_sms();
 void count_launches(int64_t k);
 int64_t launches();
 
-// Launch with the programmatic-serialization attribute when pdl is set (the
-// kernel must call pdl_wait() before its first global memory access); an
-// ordinary launch otherwise.  Kernels that follow a cudaStreamWaitEvent are
-// launched without it.
+// Launch with the programmatic-serialization attribute when pdl is set; an
+// ordinary launch otherwise.  Such a kernel calls pdl_wait() before its first
+// global memory access, and reads data an earlier kernel wrote only through
+// coherent paths (TMA, or plain / L2 loads -- never the read-only
+// non-coherent path, which a const __restrict__ pointer the kernel never
+// writes may compile to): the earlier kernel may still have been running
+// when this one started.  Used only where the predecessor in the stream is
+// a kernel (not an event record or wait).
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_kernel(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block,
                                  size_t smem, cudaStream_t stream, Args&&... args) {

@@ -83,6 +83,33 @@ def test_prepare_hinv_matches_oracle_elimination(d, desc_act, n_dead):
     assert resid <= 5e-2
 
 
+@pytest.mark.parametrize("fill", [float("nan"), 123.0])
+def test_prepare_hinv_ignores_prior_output_contents(fill):
+    """12 panels (side streams, lookahead and early-started launches all in
+    play) with U pre-filled: nothing the caller left in U may leak into it,
+    and every panel must see every update before it is factored."""
+    g = gpu()
+    d = 1536
+    _, X = workloads.small_layer(4, d, 3 * d, seed=77, kind="student_t")
+    H = oracle.hessian(X)
+    cfg = g.GPTQConfig(bits=4, group_size=128)
+    ws = torch.empty(g.gptq_workspace_size(cfg, 8, d), dtype=torch.uint8, device="cuda")
+    prep = oracle.prepare(H, torch.zeros(1, d), damp=0.01, desc_act=False)
+    Uo = oracle.upper_factor(prep["H_damped"])
+    for _ in range(3):
+        U = torch.full((d, d), fill, device="cuda")
+        perm = torch.empty(d, dtype=torch.int32, device="cuda")
+        dead = torch.empty(d, dtype=torch.uint8, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        g.gptq_prepare_hinv(torch.from_numpy(H.astype(np.float32)).cuda(), cfg, U, perm, dead, st, ws)
+        assert g.gptq_sync_status(st) == 0
+        Ug = U.cpu().numpy().astype(np.float64)
+        assert np.isfinite(Ug).all()
+        rel = np.max(np.abs(Ug - Uo)) / np.max(np.abs(Uo))
+        print(f"fill={fill} U max rel err {rel:.3e}")
+        assert rel <= 1e-4
+
+
 def test_not_positive_definite_is_reported():
     g = gpu()
     d = 96
