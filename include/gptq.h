@@ -112,6 +112,42 @@ gptq_status gptq_hessian_accumulate(const uint16_t *X, int64_t n, int64_t d, int
                                     void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * Stage 1 with X in HOST memory -- H += 2 X^T X over the calibration tokens
+ * ("GPTQ (GPT Quantization)", "Fondation theorique : OBQ": H = 2 X^T X, a sum
+ * over tokens, so it may be accumulated chunk by chunk as the data arrives).
+ *   X_host  n x d bf16 (raw bit patterns) in host memory, row-major with
+ *           leading dimension ldx >= d, any alignment.  Pinned (page-locked)
+ *           memory lets the copies overlap the GEMM; pageable memory is
+ *           accepted but its copies are staged synchronously by the driver.
+ *           The caller keeps X_host unchanged until the stream reaches the
+ *           end of this call's work.
+ *   H, ldh  as gptq_hessian_accumulate (accumulated into; lower triangle).
+ *   staging caller-owned DEVICE buffer, 256-byte aligned, of at least
+ *           gptq_hessian_staging_size(d, 64) bytes; split into two slots of
+ *           `chunk` token rows each (chunk = the largest multiple of 16384
+ *           tokens that fits, else of 64).  The copy engine fills one slot
+ *           while the tensor cores read the other.  Its contents are
+ *           scratch.
+ *   Copies run on a stream the library owns (one per device) and are ordered
+ *   after everything queued on `stream` before the call; every GEMM runs on
+ *   `stream`, so work queued on `stream` afterwards sees the finished H.
+ *   When chunk is a multiple of 16384 the result is bitwise identical to
+ *   gptq_hessian_accumulate on the same X in device memory.
+ *   Errors: GPTQ_ERR_INVALID_ARG (sizes, NULL X_host / H, ldx < d, ldh < d),
+ *   GPTQ_ERR_WORKSPACE (staging NULL, misaligned or too small for 64 tokens).
+ *   n == 0 is a no-op.
+ */
+gptq_status gptq_hessian_accumulate_host(const uint16_t *X_host, int64_t n, int64_t d,
+                                         int64_t ldx, float *H, int64_t ldh, int32_t *dev_status,
+                                         void *staging, size_t staging_bytes,
+                                         cudaStream_t stream);
+
+/* Staging bytes gptq_hessian_accumulate_host needs for chunks of
+ * chunk_tokens tokens (rounded up to a multiple of 64) of a d-wide X; 0 for
+ * invalid sizes. */
+size_t gptq_hessian_staging_size(int64_t d, int64_t chunk_tokens);
+
+/*
  * Stages 1b-2 -- dead columns, act-order, damping, and the inverse factor
  * ("GPTQ (GPT Quantization)", pseudo-code steps 1-2: H += lambda I,
  * H_inv = cholesky_inverse(H)).

@@ -10,6 +10,8 @@ post_weight_quantization_gptq_b200/build.py``).
 Stages (see the header for the exact contracts):
 
 * ``gptq_hessian_accumulate``  H += 2 X^T X            (tcgen05 bf16 GEMM)
+* ``gptq_hessian_accumulate_host``  the same with X in host memory, copies
+  overlapped with the GEMM through a two-slot device staging buffer
 * ``gptq_prepare_hinv``        dead columns, act-order, damping, U = chol-inverse factor
 * ``gptq_quantize_layer``      column walk with OBQ error feedback and lazy updates
 * ``gptq_pack``                codes -> uint32 bit stream (8 codes per word at 4 bits)
@@ -22,7 +24,8 @@ import os
 import torch
 
 __all__ = [
-    "GPTQConfig", "GPTQError", "gptq_hessian_accumulate", "gptq_prepare_hinv",
+    "GPTQConfig", "GPTQError", "gptq_hessian_accumulate", "gptq_hessian_accumulate_host",
+    "gptq_hessian_staging_size", "gptq_prepare_hinv",
     "gptq_quantize_layer", "gptq_quantize_layer_noalloc", "gptq_noalloc_scratch_bytes", "gptq_pack", "gptq_workspace_size", "gptq_sync_status",
     "gptq_status_string", "gptq_version", "gptq_launch_counter", "library_path", "n_groups", "packed_words",
     "STATUS",
@@ -70,6 +73,9 @@ def _load():
         "gptq_workspace_size": ([cfgp, i64, i64, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
         "gptq_hessian_accumulate": ([P, i64, i64, i64, P, i64, P, P, ctypes.c_size_t, P],
                                     ctypes.c_int),
+        "gptq_hessian_accumulate_host": ([P, i64, i64, i64, P, i64, P, P, ctypes.c_size_t, P],
+                                         ctypes.c_int),
+        "gptq_hessian_staging_size": ([i64, i64], ctypes.c_size_t),
         "gptq_prepare_hinv": ([P, i64, i64, cfgp, P, P, P, P, P, ctypes.c_size_t, P],
                               ctypes.c_int),
         "gptq_quantize_layer": ([P, i64, i64, i64, P, P, P, cfgp, P, P, P, P, P,
@@ -163,6 +169,28 @@ def gptq_hessian_accumulate(X: torch.Tensor, H: torch.Tensor, dev_status: torch.
     _check(_lib.gptq_hessian_accumulate(_ptr(X), n, d, ldx, _ptr(H), ldh, _ptr(dev_status),
                                         _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                         _stream(stream)), "gptq_hessian_accumulate")
+
+
+def gptq_hessian_accumulate_host(X: torch.Tensor, H: torch.Tensor, staging: torch.Tensor,
+                                 dev_status: torch.Tensor | None = None, stream=None) -> None:
+    """H += 2 X^T X with X (n x d bf16) in HOST memory, streamed through the
+    device buffer ``staging`` (two slots; copies overlap the GEMM when X is
+    pinned).  X must stay unchanged until the stream has run the call."""
+    if not isinstance(X, torch.Tensor) or X.is_cuda or X.dtype != torch.bfloat16:
+        raise TypeError("X must be a host bf16 tensor")
+    _cuda(H, "H", torch.float32)
+    _cuda(staging, "staging")
+    n, d = X.shape
+    ldx = _row_major(X, "X")
+    _check(_lib.gptq_hessian_accumulate_host(_ptr(X), n, d, ldx, _ptr(H), _row_major(H, "H"),
+                                             _ptr(dev_status), _ptr(staging),
+                                             staging.numel() * staging.element_size(),
+                                             _stream(stream)), "gptq_hessian_accumulate_host")
+
+
+def gptq_hessian_staging_size(d: int, chunk_tokens: int) -> int:
+    """Bytes of staging gptq_hessian_accumulate_host needs for chunk_tokens-token chunks."""
+    return int(_lib.gptq_hessian_staging_size(int(d), int(chunk_tokens)))
 
 
 def gptq_prepare_hinv(H: torch.Tensor, cfg: GPTQConfig, U: torch.Tensor, perm: torch.Tensor,

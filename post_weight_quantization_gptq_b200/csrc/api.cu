@@ -105,6 +105,27 @@ gptq_status gptq_hessian_accumulate(const uint16_t* X, int64_t n, int64_t d, int
     return launch_status(gptq::launch_hessian(X, n, d, ldx, H, ldh, dev_status, stream));
 }
 
+gptq_status gptq_hessian_accumulate_host(const uint16_t* X_host, int64_t n, int64_t d,
+                                         int64_t ldx, float* H, int64_t ldh, int32_t* dev_status,
+                                         void* staging, size_t staging_bytes,
+                                         cudaStream_t stream) {
+    if (d <= 0 || d > kMaxDim || n < 0 || n > kMaxDim) return GPTQ_ERR_INVALID_ARG;
+    if (H == nullptr || ldh < d) return GPTQ_ERR_INVALID_ARG;
+    if (n == 0) return GPTQ_OK;
+    if (X_host == nullptr || ldx < d) return GPTQ_ERR_INVALID_ARG;
+    if (staging == nullptr || !aligned(staging, 256) ||
+        gptq::hessian_stream_chunk_tokens(d, staging_bytes) <= 0)
+        return GPTQ_ERR_WORKSPACE;
+    return launch_status(gptq::launch_hessian_from_host(X_host, n, d, ldx, H, ldh, dev_status,
+                                                        staging, staging_bytes, stream));
+}
+
+size_t gptq_hessian_staging_size(int64_t d, int64_t chunk_tokens) {
+    if (d <= 0 || d > kMaxDim || chunk_tokens <= 0) return 0;
+    const int64_t c = (chunk_tokens + 63) / 64 * 64;
+    return static_cast<size_t>(2 * c * gptq::hessian_stream_row_pitch(d) * 2);
+}
+
 gptq_status gptq_prepare_hinv(float* H, int64_t d, int64_t ldh, const gptq_config* cfg, float* U,
                               int32_t* perm, uint8_t* dead, int32_t* dev_status, void* ws,
                               size_t ws_bytes, cudaStream_t stream) {

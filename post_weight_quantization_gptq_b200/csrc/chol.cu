@@ -38,43 +38,91 @@ namespace {
 
 constexpr int NB = 128;      // panel width
 constexpr int LDA = NB + 4;  // shared-memory row pitch: float4-aligned rows, rows 4 banks apart
-constexpr int TP = 68;       // pitch of the doubling temporary
 constexpr int kDiagThreads = 256;
-constexpr int kDiagSmem = (2 * NB * LDA + 64 * TP + 32 * 32 + 32 * LDA + NB) * 4;
+// A, X, the strip's column of L, two strips of L below the diagonal, 1 / L_ii
+constexpr int kDiagSmem = (2 * NB * LDA + 32 * 32 + 2 * 32 * LDA + NB) * 4;
+// Bound of the substitution warps' wait for a published factor step (polls
+// of a shared-memory word; the factor warp never waits, so this is a guard).
+constexpr int kStepSpinLimit = 1 << 22;
 
 __device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 __device__ __forceinline__ void sts4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 
+// 4 x 4 block of  D[i0.., j0..] -= sum_c Ls[c][i0..] * R[c][j0..]  (32 terms;
+// R rows ldr apart), float4 loads and read-modify-write stores.
+__device__ __forceinline__ void rank32_update4(float* D, const float* Ls, const float* R, int ldr,
+                                               int i0, int j0) {
+    float acc[4][4] = {};
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) {
+        const float4 li = lds4(Ls + k * LDA + i0), rj = lds4(R + k * ldr + j0);
+        const float a4[4] = {li.x, li.y, li.z, li.w}, b4[4] = {rj.x, rj.y, rj.z, rj.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) acc[t][w] = fmaf(a4[t], b4[w], acc[t][w]);
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        float* dst = D + (i0 + t) * LDA + j0;
+        float4 d4 = lds4(dst);
+        d4.x -= acc[t][0]; d4.y -= acc[t][1]; d4.z -= acc[t][2]; d4.w -= acc[t][3];
+        sts4(dst, d4);
+    }
+}
+
+// Triangular index u -> (bi, bj), bi >= bj.
+__device__ __forceinline__ void tri_index(int u, int& bi, int& bj) {
+    int i = static_cast<int>((sqrtf(8.f * u + 1.f) - 1.f) * 0.5f);
+    while (i * (i + 1) / 2 > u) --i;
+    while ((i + 1) * (i + 2) / 2 <= u) ++i;
+    bi = i;
+    bj = u - i * (i + 1) / 2;
+}
+
 // ------------------------------------------------------------------------
-// Diagonal block: L = chol(A) and X = L^-1 for a kw x kw (kw <= 128) block,
-// padded with the identity.  Four 32-wide strips; for each, one warp factors
-// the strip's 32 x 32 diagonal block, then four warps run one forward
-// substitution on 128 right-hand sides (the identity -> the strip's inverse,
-// and the rows below -> the strip of L), then the CTA updates the trailing
-// part; finally the four 32 x 32 inverses are joined by two levels of
-// recursive doubling.
+// Diagonal block: X = L^-1 with L = chol(A), for a kw x kw (kw <= 128) block
+// padded with the identity.  (L itself is not needed outside: the panel
+// solve and the inverse stream use only L^-1.)
 //
-// Column c of the strip's L below the diagonal is also kept as a row of Lc
-// (Lc[c][m] = L[o+c+1+m][o+c], zero past the strip), so each elimination
-// step reads it with eight broadcast float4 loads; the strip's rows below
-// the diagonal block are kept transposed in Ls for the trailing update.  The factor warp keeps its
-// rows in registers and rotates them after every column step, so the pivot
-// column is always register 0: the step loop stays rolled (small code, the
-// kernel runs once per panel on a cold SM) while every register index is a
-// compile-time constant.
+// Right-looking over four 32-wide strips, with X built in place of a
+// right-hand side B (the identity at the start): for strip b at o = 32 b,
+//   factor     L_bb = chol(A_bb)                                  (warp 0)
+//   substitute X[o.., :o+32] = L_bb^-1 B[o.., :o+32]  and
+//              L[i, o..] = A[i, o..] L_bb^-T for the rows i below  (warps 4-7)
+//   update     A[i, j] -= L[i, o..] L[j, o..]^T,  B[i, :o+32] -= L[i, o..] X[o.., :o+32]
+//              for the rows i below the strip.
+// The substitution has exactly 128 right-hand sides at every strip (o + 32
+// columns of B, 96 - o rows below), one per thread of warps 4-7, and runs one
+// column step behind the factor: warp 0 publishes each step's column of L in
+// shared memory with a step counter, and the substitution warps wait for it
+// (bounded).  The update is split so that only what the next strip reads
+// first (its diagonal block, its columns below it, its rows of B) sits
+// between two strips; the rest runs on warps 1-3 beside the next strip's
+// factor, and those warps also store each finished strip of X.
+//
+// The factor warp keeps its rows in registers and rotates them after every
+// column step, so the pivot column is always register 0: the step loop stays
+// rolled while every register index is a compile-time constant.  Column c of
+// L below the diagonal is published as a row of Lc (Lc[c][m] = L[o+c+1+m][o+c],
+// zero past the strip), read back with eight broadcast float4 loads.
 __global__ void __launch_bounds__(kDiagThreads, 1)
     potrf_inv_128_kernel(float* __restrict__ P, int64_t ldp, int64_t kb, int kw,
                          float* __restrict__ X, int64_t ldx, int32_t* status) {
     extern __shared__ __align__(16) float sm[];
-    float* A = sm;              // [128][LDA] the block, L in its lower part
-    float* Xs = A + NB * LDA;   // [128][LDA] L^-1
-    float* T = Xs + NB * LDA;   // [64][TP] doubling temporary
-    float* Lc = T + 64 * TP;    // [32][32] the current strip's columns of L, shifted
-    float* Ls = Lc + 32 * 32;   // [32][LDA] the current strip of L below it, transposed
-    float* dinv = Ls + 32 * LDA; // [128] 1 / L_ii
-    __shared__ int bad;
+    float* A = sm;                // [128][LDA] the block (lower part updated)
+    float* Xs = A + NB * LDA;     // [128][LDA] B, becoming L^-1 strip by strip
+    float* Lc = Xs + NB * LDA;    // [32][32] the current strip's columns of L, shifted
+    float* Lsb = Lc + 32 * 32;    // [2][32][LDA] strips of L below them, transposed
+    float* dinv = Lsb + 2 * 32 * LDA;  // [128] 1 / L_ii
+    __shared__ int bad, stalled;
+    __shared__ int progress;      // factor steps published so far (32 b + c + 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (tid == 0) bad = 0;
+    if (tid == 0) {
+        bad = 0;
+        stalled = 0;
+        progress = 0;
+    }
     pdl_trigger();
     pdl_wait();
     {
@@ -96,18 +144,20 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
             const int e = tid + q * kDiagThreads;
             const int i = e >> 5, j = (e & 31) * 4;
             float vv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+            float id[4];
 #pragma unroll
-            for (int t = 0; t < 4; ++t)
-                vv[t] = (j + t <= i && i < kw) ? vv[t] : (i == j + t ? 1.f : 0.f);
+            for (int t = 0; t < 4; ++t) {
+                id[t] = (i == j + t) ? 1.f : 0.f;
+                vv[t] = (j + t <= i && i < kw) ? vv[t] : id[t];
+            }
             sts4(A + i * LDA + j, make_float4(vv[0], vv[1], vv[2], vv[3]));
-            sts4(Xs + i * LDA + j, make_float4(0.f, 0.f, 0.f, 0.f));
+            sts4(Xs + i * LDA + j, make_float4(id[0], id[1], id[2], id[3]));
         }
     }
     __syncthreads();
 
-    // -- 32 x 32 Cholesky of the diagonal block at o, by warp 0: lane i holds
-    //    row o + i, register r = column c + r
-    auto chol32 = [&](int o) {
+    // -- strip factor (warp 0): lane i holds row o + i, register r = column c + r
+    auto factor = [&](int o, int b) {
         float a[32];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -124,12 +174,13 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
                 piv = 1.f;
             }
             const float inv = rsqrtf(piv);
-            const float a0 = (lane == c) ? piv * inv : ((lane > c) ? a[0] * inv : 0.f);
-            if (lane >= c) A[(o + lane) * LDA + o + c] = a0;
+            const float a0 = (lane > c) ? a[0] * inv : 0.f;
             if (lane == c) dinv[o + c] = inv;
             // lane i > c holds L[o+i][o+c] -> Lc[c][i-c-1]; lanes <= c fill the tail with 0
-            Lc[c * 32 + ((lane - c - 1) & 31)] = a0 * (lane > c ? 1.f : 0.f);
+            Lc[c * 32 + ((lane - c - 1) & 31)] = a0;
+            __threadfence_block();
             __syncwarp();
+            if (lane == 0) *reinterpret_cast<volatile int*>(&progress) = 32 * b + c + 1;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {  // update and rotate
                 const float4 l = lds4(Lc + c * 32 + 4 * q);
@@ -140,184 +191,124 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
             }
         }
     };
-    // -- trailing update of the lower part below strip o, 4 x 4 register blocks
-    //    u in [u0, u1) (triangular numbering from row r0), read from the
-    //    transposed strip (consecutive blocks -> consecutive float4)
-    auto trail = [&](int r0, int u0, int u1, int t, int stride) {
-        for (int u = u0 + t; u < u1; u += stride) {
-            int bi = static_cast<int>((sqrtf(8.f * u + 1.f) - 1.f) * 0.5f);
-            while (bi * (bi + 1) / 2 > u) --bi;
-            while ((bi + 1) * (bi + 2) / 2 <= u) ++bi;
-            const int bj = u - bi * (bi + 1) / 2;
-            const int i0 = r0 + 4 * bi, j0 = r0 + 4 * bj;
-            float acc2[4][4] = {};
-#pragma unroll 8
-            for (int k = 0; k < 32; ++k) {
-                const float4 li = lds4(Ls + k * LDA + i0), lj = lds4(Ls + k * LDA + j0);
-                const float a4[4] = {li.x, li.y, li.z, li.w}, b4[4] = {lj.x, lj.y, lj.z, lj.w};
+
+    // -- substitution (warps 4-7), one step behind the factor: thread t
+    //    solves for column t of B (t < o + 32) or for row t of L below the strip
+    auto substitute = [&](int o, int b) {
+        const int t = tid - 128;
+        const bool rhs = t < o + 32;
+        float* Ls = Lsb + (b & 1) * 32 * LDA;
+        float x[32];
+        if (rhs) {
 #pragma unroll
-                for (int t4 = 0; t4 < 4; ++t4)
+            for (int r = 0; r < 32; ++r) x[r] = Xs[(o + r) * LDA + t];
+        } else {
 #pragma unroll
-                    for (int w = 0; w < 4; ++w) acc2[t4][w] = fmaf(a4[t4], b4[w], acc2[t4][w]);
+            for (int q = 0; q < 8; ++q) {
+                const float4 v4 = lds4(A + t * LDA + o + 4 * q);
+                x[4 * q] = v4.x; x[4 * q + 1] = v4.y; x[4 * q + 2] = v4.z; x[4 * q + 3] = v4.w;
             }
+        }
+        int spins = 0;
+#pragma unroll 1
+        for (int c = 0; c < 32; ++c) {
+            const int need = 32 * b + c + 1;
+            while (*reinterpret_cast<volatile int*>(&progress) < need) {
+                if (++spins > kStepSpinLimit) {
+                    stalled = 1;
+                    break;
+                }
+            }
+            __threadfence_block();
+            float4 l[8];
 #pragma unroll
-            for (int t4 = 0; t4 < 4; ++t4) {
-                float* dst = A + (i0 + t4) * LDA + j0;
-                if (j0 + 3 <= i0 + t4) {
-                    float4 d4 = lds4(dst);
-                    d4.x -= acc2[t4][0]; d4.y -= acc2[t4][1]; d4.z -= acc2[t4][2]; d4.w -= acc2[t4][3];
-                    sts4(dst, d4);
+            for (int q = 0; q < 8; ++q) l[q] = lds4(Lc + c * 32 + 4 * q);
+            const float xc = x[0] * dinv[o + c];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                x[4 * q] = fmaf(-l[q].x, xc, x[4 * q + 1]);
+                x[4 * q + 1] = fmaf(-l[q].y, xc, x[4 * q + 2]);
+                x[4 * q + 2] = fmaf(-l[q].z, xc, x[4 * q + 3]);
+                x[4 * q + 3] = (q < 7) ? fmaf(-l[q].w, xc, x[4 * q + 4]) : 0.f;
+            }
+            if (rhs) Xs[(o + c) * LDA + t] = xc;
+            else Ls[c * LDA + t] = xc;
+        }
+    };
+
+    // -- strip b's update of what lies below it.  Units of 4 x 4: the next
+    //    strip's diagonal block (36), its columns below it, its rows of B
+    //    ("first"), or everything further below ("rest").
+    auto update = [&](int b, bool first, int u0, int stride) {
+        const int o = 32 * b, o1 = o + 32;  // o1: the next strip
+        const float* Ls = Lsb + (b & 1) * 32 * LDA;
+        const float* Xr = Xs + o * LDA;     // strip b's rows of X
+        const int nb4 = o1 / 4;             // 4-column blocks of B's live columns
+        const int below = (NB - o1 - 32) / 4;  // 4-row blocks below the next strip
+        if (first) {
+            const int n_diag = 36, n_panel = below * 8, n_b = 8 * nb4;
+            for (int u = u0; u < n_diag + n_panel + n_b; u += stride) {
+                if (u < n_diag) {
+                    int bi, bj;
+                    tri_index(u, bi, bj);
+                    rank32_update4(A, Ls, Ls, LDA, o1 + 4 * bi, o1 + 4 * bj);
+                } else if (u < n_diag + n_panel) {
+                    const int v = u - n_diag;
+                    rank32_update4(A, Ls, Ls, LDA, o1 + 32 + 4 * (v >> 3), o1 + 4 * (v & 7));
                 } else {
-#pragma unroll
-                    for (int w = 0; w < 4; ++w)
-                        if (j0 + w <= i0 + t4) dst[w] -= acc2[t4][w];
+                    const int v = u - n_diag - n_panel;
+                    rank32_update4(Xs, Ls, Xr, LDA, o1 + 4 * (v / nb4), 4 * (v % nb4));
+                }
+            }
+        } else {
+            const int n_a = below * (below + 1) / 2, n_b = below * nb4;
+            for (int u = u0; u < n_a + n_b; u += stride) {
+                if (u < n_a) {
+                    int bi, bj;
+                    tri_index(u, bi, bj);
+                    rank32_update4(A, Ls, Ls, LDA, o1 + 32 + 4 * bi, o1 + 32 + 4 * bj);
+                } else {
+                    const int v = u - n_a;
+                    rank32_update4(Xs, Ls, Xr, LDA, o1 + 32 + 4 * (v / nb4), 4 * (v % nb4));
                 }
             }
         }
     };
 
-    if (warp == 0) chol32(0);
-    __syncthreads();
+    // -- rows [r0, r0 + nr) of X to global memory (zeros above the diagonal
+    //    included: the tensor-core GEMMs read it as a full tile)
+    auto store_rows = [&](int r0, int nr, int t0, int stride) {
+        for (int e = t0; e < nr * (NB / 4); e += stride) {
+            const int i = r0 + e / (NB / 4), j = (e % (NB / 4)) * 4;
+            if (i >= kw || j >= kw) continue;
+            float4 x4 = lds4(Xs + i * LDA + j);
+            if (j + 1 > i) x4.y = 0.f;
+            if (j + 2 > i) x4.z = 0.f;
+            if (j + 3 > i) x4.w = 0.f;
+            if (j > i) x4.x = 0.f;
+            *reinterpret_cast<float4*>(X + (kb + i) * ldx + kb + j) = x4;
+        }
+    };
+
     for (int b = 0; b < 4; ++b) {
         const int o = 32 * b;
-        const int r0 = o + 32;
-        if (warp < 4) {
-            // -- forward substitution with L_bb on 128 right-hand sides at once:
-            //    threads 0..31 the identity (-> the strip's inverse, a column per
-            //    thread), threads 32..127 the rows below (-> the strip of L)
-            const int hs = tid;
-            const int i = r0 + hs - 32;  // row for hs >= 32
-            const bool act = hs < 32 || i < NB;
-            float x[32];
-            if (hs >= 32 && act) {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 t = lds4(A + i * LDA + o + 4 * q);
-                    x[4 * q] = t.x; x[4 * q + 1] = t.y; x[4 * q + 2] = t.z; x[4 * q + 3] = t.w;
-                }
-            } else {
-#pragma unroll
-                for (int r = 0; r < 32; ++r) x[r] = (r == hs) ? 1.f : 0.f;
-            }
-#pragma unroll 1
-            for (int c = 0; c < 32; ++c) {
-                // the step's column of L first: its loads do not wait behind the stores
-                float4 l[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) l[q] = lds4(Lc + c * 32 + 4 * q);
-                const float xc = x[0] * dinv[o + c];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    x[4 * q] = fmaf(-l[q].x, xc, x[4 * q + 1]);
-                    x[4 * q + 1] = fmaf(-l[q].y, xc, x[4 * q + 2]);
-                    x[4 * q + 2] = fmaf(-l[q].z, xc, x[4 * q + 3]);
-                    x[4 * q + 3] = (q < 7) ? fmaf(-l[q].w, xc, x[4 * q + 4]) : 0.f;
-                }
-                if (hs < 32) {
-                    Xs[(o + c) * LDA + o + hs] = xc;
-                } else if (act) {
-                    A[i * LDA + o + c] = xc;
-                    Ls[c * LDA + i] = xc;
-                }
-            }
+        if (warp == 0) {
+            factor(o, b);
+        } else if (warp >= 4) {
+            substitute(o, b);
+        } else if (b > 0) {
+            update(b - 1, false, tid - 32, 96);  // the previous strip's rest
+            store_rows(o - 32, 32, tid - 32, 96);  // the previous strip of X is final
         }
         __syncthreads();
-        if (r0 < NB) {
-            // the next strip's 32 x 32 diagonal block first (units 0..35), then
-            // warp 0 factors it while warps 1..7 finish the trailing update
-            const int mb = (NB - r0) / 4;
-            const int units = mb * (mb + 1) / 2;
-            trail(r0, 0, 36, tid, kDiagThreads);
-            __syncthreads();
-            if (warp == 0) chol32(r0);
-            else trail(r0, 36, units, tid - 32, kDiagThreads - 32);
+        if (b < 3) {
+            update(b, true, tid, kDiagThreads);
             __syncthreads();
         }
     }
-
-    // -- join the 32 x 32 inverses: X_CA = -X_CC (L_CA X_AA), 4 x 4 register
-    //    blocks (rows c, columns a); T[p*s + c][a] holds L_CA X_AA.  X_AA and
-    //    X_CC are lower triangular, so the sums skip their zero parts.
-    for (int s = 32; s < NB; s *= 2) {
-        const int pairs = NB / (2 * s);
-        const int nb4 = s / 4;
-        const int blocks = pairs * nb4 * nb4;
-        for (int e = tid; e < blocks; e += kDiagThreads) {
-            const int p = e / (nb4 * nb4), c0 = ((e / nb4) % nb4) * 4, a0 = (e % nb4) * 4;
-            const int A0 = 2 * s * p, C0 = A0 + s;
-            float acc[4][4] = {};
-#pragma unroll 2
-            for (int k = a0; k < s; k += 4) {  // X_AA[k][a] = 0 for k < a
-                float4 l[4];
-#pragma unroll
-                for (int t = 0; t < 4; ++t) l[t] = lds4(A + (C0 + c0 + t) * LDA + A0 + k);
-                float4 xx[4];
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) xx[kk] = lds4(Xs + (A0 + k + kk) * LDA + A0 + a0);
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const float lt[4] = {l[t].x, l[t].y, l[t].z, l[t].w};
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        acc[t][0] = fmaf(lt[kk], xx[kk].x, acc[t][0]);
-                        acc[t][1] = fmaf(lt[kk], xx[kk].y, acc[t][1]);
-                        acc[t][2] = fmaf(lt[kk], xx[kk].z, acc[t][2]);
-                        acc[t][3] = fmaf(lt[kk], xx[kk].w, acc[t][3]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int t = 0; t < 4; ++t)
-                sts4(T + (p * s + c0 + t) * TP + a0, make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]));
-        }
-        __syncthreads();
-        for (int e = tid; e < blocks; e += kDiagThreads) {
-            const int p = e / (nb4 * nb4), c0 = ((e / nb4) % nb4) * 4, a0 = (e % nb4) * 4;
-            const int A0 = 2 * s * p, C0 = A0 + s;
-            float acc[4][4] = {};
-#pragma unroll 2
-            for (int k = 0; k <= c0; k += 4) {  // X_CC[c][k] = 0 for k > c
-                float4 xc[4];
-#pragma unroll
-                for (int t = 0; t < 4; ++t) xc[t] = lds4(Xs + (C0 + c0 + t) * LDA + C0 + k);
-                float4 tt[4];
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) tt[kk] = lds4(T + (p * s + k + kk) * TP + a0);
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const float xt[4] = {xc[t].x, xc[t].y, xc[t].z, xc[t].w};
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        acc[t][0] = fmaf(xt[kk], tt[kk].x, acc[t][0]);
-                        acc[t][1] = fmaf(xt[kk], tt[kk].y, acc[t][1]);
-                        acc[t][2] = fmaf(xt[kk], tt[kk].z, acc[t][2]);
-                        acc[t][3] = fmaf(xt[kk], tt[kk].w, acc[t][3]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int t = 0; t < 4; ++t)
-                sts4(Xs + (C0 + c0 + t) * LDA + A0 + a0,
-                     make_float4(-acc[t][0], -acc[t][1], -acc[t][2], -acc[t][3]));
-        }
-        __syncthreads();
-    }
-
-    // -- write X (zeros above the diagonal included: the tensor-core GEMMs read
-    //    it as a full tile), float4 per access.  L's diagonal block is not
-    //    written back: nothing reads it after this kernel.
-#pragma unroll 4
-    for (int e = tid; e < NB * NB / 4; e += kDiagThreads) {
-        const int i = e >> 5, j = (e & 31) * 4;
-        if (i >= kw || j >= kw) continue;
-        float4 x4 = lds4(Xs + i * LDA + j);
-        if (j + 1 > i) x4.y = 0.f;
-        if (j + 2 > i) x4.z = 0.f;
-        if (j + 3 > i) x4.w = 0.f;
-        if (j > i) x4.x = 0.f;
-        *reinterpret_cast<float4*>(X + (kb + i) * ldx + kb + j) = x4;
-    }
+    store_rows(96, 32, tid, kDiagThreads);
     if (tid == 0 && bad) report(status, GPTQ_ERR_NOT_PD);
+    if (tid == 0 && stalled) report(status, GPTQ_ERR_TIMEOUT);
 }
 
 // Lower-triangular tile index t -> (I, J), I >= J.

@@ -57,6 +57,14 @@ int hessian_num_tiles(int64_t d);
 gptq_status launch_hessian(const uint16_t* X, int64_t n, int64_t d, int64_t ldx, float* H,
                            int64_t ldh, int32_t* status, cudaStream_t stream);
 
+// ---- stage 1 from host memory (hessian_host.cu): copy / GEMM pipeline over
+// a two-slot device staging buffer
+int64_t hessian_stream_row_pitch(int64_t d);
+int64_t hessian_stream_chunk_tokens(int64_t d, size_t staging_bytes);
+gptq_status launch_hessian_from_host(const uint16_t* Xh, int64_t n, int64_t d, int64_t ldx,
+                                     float* H, int64_t ldh, int32_t* status, void* staging,
+                                     size_t staging_bytes, cudaStream_t stream);
+
 // ---- stage 2 (prep.cu): dead columns, lambda, act-order, flipped working copy
 size_t prep_workspace_bytes(int64_t d);
 gptq_status launch_prep(const float* H, int64_t d, int64_t ldh, float damp, int desc_act,

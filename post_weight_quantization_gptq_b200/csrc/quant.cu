@@ -33,6 +33,7 @@ constexpr int kBlock = 128;       // columns per block (the only supported block
 constexpr int kRowsPerWarp = 4;   // 8 lanes per row
 constexpr int kWarps = 4;
 constexpr int kRowsPerCta = kRowsPerWarp * kWarps;
+static_assert(kWarps * 32 == kBlock, "block_quant_kernel: one thread per column of the U block");
 
 // ------------------------------------------------------------------------
 __global__ void permute_rows_kernel(float* __restrict__ W, int64_t r, int64_t d, int64_t ldw,
@@ -159,15 +160,36 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
     __shared__ int ok;
     const int tid = threadIdx.x;
     pdl_trigger();
+    // U is an input of the whole call that none of its kernels writes, so
+    // its diagonal block is fetched and prepared before waiting for the
+    // previous kernel (which may still be updating W)
     if (tid == 0) {
         mbar_init(&bar, 1);
         fence_barrier_init();
-    }
-    pdl_wait();
-    if (tid == 0) {
         mbar_arrive_expect_tx(&bar, kBlock * kBlock * 4);
         tma_load_2d(Us, &tmu, &bar, static_cast<int>(c0), static_cast<int>(c0));
+        volatile int no_abort = 0;
+        ok = mbar_wait(&bar, 0, &no_abort) ? 1 : 0;
+        if (!ok) report(status, GPTQ_ERR_TIMEOUT);
     }
+    __syncthreads();
+    if (!ok) return;
+    // 1 / U_jj (thread j), then the block is cleared at and below its
+    // diagonal, float4 by float4 spread over all threads
+    const float ujj = Us[tid * kBlock + tid];
+    __syncthreads();
+    for (int q = tid; q < kBlock * kBlock / 4; q += kWarps * 32) {
+        const int i = q >> 5, c = (q & 31) * 4;
+        if (c > i) continue;
+        float* u4 = Us + i * kBlock + c;
+        if (c + 3 <= i) {
+            *reinterpret_cast<float4*>(u4) = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+            for (int t = 0; c + t <= i; ++t) u4[t] = 0.f;
+        }
+    }
+    dinv[tid] = (tid < bw) ? 1.f / ujj : 0.f;
+    pdl_wait();
 
     const int lane = tid & 31;
     const int l = lane & 7;
@@ -210,23 +232,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
         gp.hi = static_cast<float>((1 << bits) - 1) - gp.zf;
     }
 
-    if (tid == 0) {
-        volatile int no_abort = 0;
-        ok = mbar_wait(&bar, 0, &no_abort) ? 1 : 0;
-        if (!ok) report(status, GPTQ_ERR_TIMEOUT);
-    }
-    __syncthreads();
-    if (!ok) return;
-    // 1 / U_jj, then row j of the block is cleared at and left of its diagonal
-    // (a thread owns whole rows, so no barrier between the two)
-    for (int j = tid; j < kBlock; j += blockDim.x) {
-        float* ur = Us + j * kBlock;
-        dinv[j] = (j < bw) ? 1.f / ur[j] : 0.f;
-        int c = 0;
-        for (; c + 3 <= j; c += 4) *reinterpret_cast<float4*>(ur + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (; c <= j; ++c) ur[c] = 0.f;
-    }
-    __syncthreads();
+    __syncthreads();  // the prepared U block and 1 / U_jj
 
     // columns 0, 1, 2 for every lane of the group; afterwards, at the start of
     // step j: wcur = column j (final), t1 = column j+1 after the feedback of

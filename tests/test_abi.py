@@ -101,3 +101,28 @@ def test_invalid_arguments_are_rejected_on_the_host(pkg):
     assert lib.gptq_hessian_accumulate(fake, 0, 16, 16, fake, 16, None, None, 0, None) == 0
     assert lib.gptq_pack(fake, 4, 8, 5, fake, None) == 1
     assert lib.gptq_pack(None, 4, 8, 4, fake, None) == 1
+
+
+def test_host_streaming_hessian_validation(pkg):
+    lib = ctypes.CDLL(pkg.library_path())
+    P, i64 = ctypes.c_void_p, ctypes.c_int64
+    f = lib.gptq_hessian_accumulate_host
+    f.restype = ctypes.c_int
+    f.argtypes = [P, i64, i64, i64, P, i64, P, P, ctypes.c_size_t, P]
+    lib.gptq_hessian_staging_size.restype = ctypes.c_size_t
+    lib.gptq_hessian_staging_size.argtypes = [i64, i64]
+    fake = ctypes.c_void_p(1 << 20)
+    # two slots of 64-token rows, rows padded to a multiple of 8 channels
+    assert lib.gptq_hessian_staging_size(4096, 16384) == 2 * 16384 * 4096 * 2
+    assert lib.gptq_hessian_staging_size(12, 1) == 2 * 64 * 16 * 2
+    assert lib.gptq_hessian_staging_size(0, 64) == 0
+    need = lib.gptq_hessian_staging_size(16, 64)
+    # bad sizes / pointers -> invalid argument; missing, misaligned or small staging -> workspace
+    assert f(fake, 16, 0, 16, fake, 16, None, fake, need, None) == 1
+    assert f(None, 16, 16, 16, fake, 16, None, fake, need, None) == 1
+    assert f(fake, 16, 16, 8, fake, 16, None, fake, need, None) == 1
+    assert f(fake, 16, 16, 16, None, 16, None, fake, need, None) == 1
+    assert f(fake, 16, 16, 16, fake, 16, None, None, need, None) == 6
+    assert f(fake, 16, 16, 16, fake, 16, None, ctypes.c_void_p((1 << 20) + 16), need, None) == 6
+    assert f(fake, 16, 16, 16, fake, 16, None, fake, need - 1, None) == 6
+    assert f(fake, 0, 16, 16, fake, 16, None, fake, need, None) == 0
