@@ -392,7 +392,7 @@ def run_ours(args, rank: int, world: int, dist):
     if world == 1 and not args.no_cpu_baseline:
         # a larger sample than the per-step one of --impl reference: about
         # 10-30 s of host work in one measurement
-        cb = oracle_sample(wl, n_tokens=32768, n_rows=1024)
+        cb = oracle_sample(wl, n_tokens=131072, n_rows=4096)
         line["cpu_baseline"] = {"value": cb["value"], "unit": "weights/s", "cores": cb["cores"],
                                 "kind": "oracle", "sample": cb["sample"]}
     print(json.dumps(line), flush=True)
