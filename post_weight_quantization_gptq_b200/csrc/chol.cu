@@ -71,6 +71,12 @@ __device__ __forceinline__ void rank32_update4(float* D, const float* Ls, const 
     }
 }
 
+// Barrier among the `count` threads (whole warps) that execute it with this
+// id (ids other than 0, which __syncthreads uses).
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Triangular index u -> (bi, bj), bi >= bj.
 __device__ __forceinline__ void tri_index(int u, int& bi, int& bj) {
     int i = static_cast<int>((sqrtf(8.f * u + 1.f) - 1.f) * 0.5f);
@@ -239,24 +245,27 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
     // -- strip b's update of what lies below it.  Units of 4 x 4: the next
     //    strip's diagonal block (36), its columns below it, its rows of B
     //    ("first"), or everything further below ("rest").
-    auto update = [&](int b, bool first, int u0, int stride) {
+    //    part 0: the next strip's diagonal block; part 1: its columns below
+    //    it and its rows of B; part 2: everything further below
+    auto update = [&](int b, int part, int u0, int stride) {
         const int o = 32 * b, o1 = o + 32;  // o1: the next strip
         const float* Ls = Lsb + (b & 1) * 32 * LDA;
         const float* Xr = Xs + o * LDA;     // strip b's rows of X
         const int nb4 = o1 / 4;             // 4-column blocks of B's live columns
         const int below = (NB - o1 - 32) / 4;  // 4-row blocks below the next strip
-        if (first) {
-            const int n_diag = 36, n_panel = below * 8, n_b = 8 * nb4;
-            for (int u = u0; u < n_diag + n_panel + n_b; u += stride) {
-                if (u < n_diag) {
-                    int bi, bj;
-                    tri_index(u, bi, bj);
-                    rank32_update4(A, Ls, Ls, LDA, o1 + 4 * bi, o1 + 4 * bj);
-                } else if (u < n_diag + n_panel) {
-                    const int v = u - n_diag;
-                    rank32_update4(A, Ls, Ls, LDA, o1 + 32 + 4 * (v >> 3), o1 + 4 * (v & 7));
+        if (part == 0) {
+            for (int u = u0; u < 36; u += stride) {
+                int bi, bj;
+                tri_index(u, bi, bj);
+                rank32_update4(A, Ls, Ls, LDA, o1 + 4 * bi, o1 + 4 * bj);
+            }
+        } else if (part == 1) {
+            const int n_panel = below * 8, n_b = 8 * nb4;
+            for (int u = u0; u < n_panel + n_b; u += stride) {
+                if (u < n_panel) {
+                    rank32_update4(A, Ls, Ls, LDA, o1 + 32 + 4 * (u >> 3), o1 + 4 * (u & 7));
                 } else {
-                    const int v = u - n_diag - n_panel;
+                    const int v = u - n_panel;
                     rank32_update4(Xs, Ls, Xr, LDA, o1 + 4 * (v / nb4), 4 * (v % nb4));
                 }
             }
@@ -297,15 +306,25 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
         } else if (warp >= 4) {
             substitute(o, b);
         } else if (b > 0) {
-            update(b - 1, false, tid - 32, 96);  // the previous strip's rest
+            update(b - 1, 2, tid - 32, 96);  // the previous strip's rest
             store_rows(o - 32, 32, tid - 32, 96);  // the previous strip of X is final
         }
         __syncthreads();
         if (b < 3) {
-            update(b, true, tid, kDiagThreads);
-            __syncthreads();
+            // what the next strip reads first: warps 0-1 update its diagonal
+            // block (then warp 0 factors it), warps 2-7 its columns below it
+            // and its rows of B (then warps 4-7 substitute); each group goes on
+            // as soon as its own part is done
+            if (warp < 2) {
+                update(b, 0, tid, 64);
+                named_barrier_sync(1, 64);
+            } else {
+                update(b, 1, tid - 64, 192);
+                named_barrier_sync(2, 192);
+            }
         }
     }
+    __syncthreads();
     store_rows(96, 32, tid, kDiagThreads);
     if (tid == 0 && bad) report(status, GPTQ_ERR_NOT_PD);
     if (tid == 0 && stalled) report(status, GPTQ_ERR_TIMEOUT);
@@ -511,8 +530,14 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
     Lookahead* la = lookahead_resources();
     if (la == nullptr) return GPTQ_ERR_CUDA;
     const int sms = num_sms();
-    const int inv_sms = sms >= 128 ? 32 : (sms + 3) / 4;
-    const int side_sms = sms >= 128 ? sms - 32 - inv_sms : (sms + 1) / 2;
+    // SMs shared by the two side streams (the panel chain keeps the rest:
+    // its launches are one wave of at most 31 tiles).  Each panel's rest of
+    // the trailing update gets enough of them to finish in about five waves
+    // (it must be done before the column update two launches later on the
+    // chain); the inverse stream, whose work grows as the trailing updates
+    // shrink, gets the others.
+    const int pool = sms >= 128 ? sms - 32 : (3 * sms) / 4;
+    const int pool_min = pool / 8 > 1 ? pool / 8 : 1;
     const int npan = static_cast<int>((d + NB - 1) / NB);
     int64_t launches = 0;
     // the side streams start after everything the caller queued before us
@@ -558,6 +583,10 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
                 return GPTQ_ERR_CUDA;
             ++launches;
         }
+        const int side_tiles = mt * (mt + 1) / 2 - mt;
+        int side_sms = (side_tiles + 4) / 5;
+        side_sms = side_sms < pool_min ? pool_min : (side_sms > pool - pool_min ? pool - pool_min : side_sms);
+        const int inv_sms = pool - side_sms;
         if (mt > 1) {
             SyrkSched rs{P, ldp, di, static_cast<int>(kb), kw, static_cast<int>(kb + kw), 2};
             if (g3::launch<SyrkSched, false, false>(tP, tP, rs, mt * (mt + 1) / 2 - mt, status,
