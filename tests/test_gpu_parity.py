@@ -182,6 +182,20 @@ def test_quantize_layer_matches_oracle(d_row, d_col, n, kind, bits, g, desc_act)
     compare_quantization(H.astype(np.float64), W, out, bits, g, desc_act)
 
 
+@pytest.mark.parametrize("d_row,d_col,g,damp,desc_act", [(24, 2048, 1024, 0.01, False),
+                                                         (24, 2048, 1024, 0.005, True),
+                                                         (48, 768, 32, 0.005, True)])
+def test_quantize_layer_wide_groups_and_light_damping(d_row, d_col, g, damp, desc_act):
+    """The guide's other knobs: groups of 1024 columns (eight blocks share one
+    scale and zero point, the deferred lazy-update schedule shortens its runs
+    so the group's later columns are complete when it opens) and its
+    high-accuracy damping of 0.005."""
+    W, X = workloads.small_layer(d_row, d_col, 3 * d_col, seed=d_col + g, kind="student_t")
+    H = oracle.hessian(X).astype(np.float32)
+    out = gpu_quantize(H, W, 4, g, desc_act, damp)
+    compare_quantization(H.astype(np.float64), W, out, 4, g, desc_act, damp)
+
+
 def test_dead_columns_are_zero_weight():
     W, X = workloads.small_layer(24, 256, 1024, seed=5)
     Xf = X.to(torch.float32)
