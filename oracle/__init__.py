@@ -19,6 +19,7 @@ from .gptq import (  # noqa: F401
     act_order,
     damp_lambda,
     dead_columns,
+    dequant_matmul,
     dequantize,
     eliminate,
     gptq_blocked,

@@ -388,6 +388,23 @@ def unpack(packed, d: int, bits: int) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# Using the quantized layer  "GPTQ (GPT Quantization)", "Limitations" (items
+# 1-2): weight-only quantization, the activations stay at 16 bits and the
+# integer weights are dequantized before each product
+# --------------------------------------------------------------------------
+def dequant_matmul(X, packed, scales, zeros, perm, bits: int, group_size: int,
+                   d_col: int) -> np.ndarray:
+    """Y = X W_hat^T for a layer quantized by this library: X is tokens x d_col
+    in the layer's original column order, the packed codes are in quantization
+    order, and W_hat[:, perm[k]] = scale[k // g] * (code[:, k] - zero[k // g]).
+    perm None is the identity.  float64 throughout."""
+    Xf = _f64(X)
+    Xq = Xf if perm is None else Xf[:, np.asarray(perm)]
+    Q = dequantize(unpack(packed, d_col, bits), scales, zeros, group_size)
+    return Xq @ Q.T
+
+
+# --------------------------------------------------------------------------
 # The whole layer
 # --------------------------------------------------------------------------
 def quantize_layer(H, W, bits: int = 4, group_size: int = 128, desc_act: bool = False,

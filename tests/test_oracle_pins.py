@@ -350,3 +350,34 @@ def test_u_row_loop_equals_the_eliminated_loop(d, g):
     forced = oracle.gptq_columns_u(W0, U, 4, g, forced_codes=res.codes, forced_zeros=res.zeros,
                                    forced_w=res.w_at_quant)
     assert forced.stats["code_invalid"] == 0 and forced.stats["code_ties"] == 0
+
+
+def _golden_kv(name):
+    out = {}
+    for line in open(os.path.join(GOLDEN, name)):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        k, v = (t.strip() for t in line.split("|", 1))
+        out[k] = v.split()
+    return out
+
+
+def test_dequant_matmul_hand_example():
+    """Product with a quantized layer: hand-computed example (golden file),
+    act-order permutation and two groups included."""
+    g = _golden_kv("dequant_matmul_worked_example.txt")
+    bits, gs = int(g["bits"][0]), int(g["group"][0])
+    perm = np.array([int(v) for v in g["perm"]])
+    X = np.array([[float(v) for v in g["x"]]])
+    packed = np.array([[int(w, 16)] for w in g["packed"]], dtype=np.uint32)
+    sc = np.array([float(v) for v in g["scales"]]).reshape(2, 2)
+    ze = np.array([int(v) for v in g["zeros"]], dtype=np.int32).reshape(2, 2)
+    Y = oracle.dequant_matmul(X, packed, sc, ze, perm, bits, gs, len(perm))
+    assert np.array_equal(Y, np.array([[float(v) for v in g["y"]]]))
+    # the packed words are the pages' layout of these codes
+    codes = np.array([[1, 2, 3, 4, 5, 6, 7, 8], [15, 0, 15, 0, 3, 3, 3, 3]], dtype=np.uint8)
+    assert np.array_equal(oracle.pack(codes, 4), packed)
+    # without the permutation the same codes meet the activations unreversed
+    Y_id = oracle.dequant_matmul(X, packed, sc, ze, None, bits, gs, len(perm))
+    assert Y_id[0, 1] == 1 * 16 + 2 * -14 + 3 * 16 + 4 * -14
