@@ -49,6 +49,9 @@ def parse():
                    help="override the calibration token count (profiling of a smaller case)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--dequant-matmul", type=int, default=0, metavar="TOKENS",
+                   help="instead of the quantizer step, time the product of TOKENS tokens with a "
+                        "quantized Llama-70B down_proj (gptq_dequant_matmul)")
     return p.parse_args()
 
 
@@ -398,6 +401,78 @@ def run_ours(args, rank: int, world: int, dist):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- the product
+def run_dequant_matmul(args, rank: int, world: int, dist):
+    """Y = X W_hat^T for a quantized 8192 x 28672 layer (4-bit, g128, act-order),
+    decode form; HBM-bound on the packed words for one token."""
+    import post_weight_quantization_gptq_b200 as g
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    n_tok, d_row, d_col, bits, gs = args.dequant_matmul, 8192, 28672, 4, 128
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4321 + rank)
+    ng = d_col // gs
+    packed = torch.randint(-(1 << 31), 1 << 31, (d_row, d_col * bits // 32), dtype=torch.int64,
+                           device=dev, generator=gen).to(torch.int32)
+    scales = torch.rand(ng, d_row, device=dev, generator=gen) * 0.02 + 1e-3
+    zeros = torch.randint(0, 1 << bits, (ng, d_row), dtype=torch.int32, device=dev, generator=gen)
+    perm = torch.randperm(d_col, device=dev, generator=gen).to(torch.int32)
+    X = torch.randn(n_tok, d_col, device=dev, generator=gen).to(torch.bfloat16)
+    Y = torch.empty(n_tok, d_row, dtype=torch.float32, device=dev)
+    ws = torch.empty(g.gptq_dequant_matmul_workspace_size(n_tok, d_col), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        g.gptq_dequant_matmul(X, packed, scales, zeros, perm, bits, gs, Y, ws)
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    clocks = ClockSampler(dev.index)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = g.gptq_launch_counter()
+    clocks.start()
+    for k in range(K):
+        flush.fill_(1)
+        ev[k][0].record(stream)
+        g.gptq_dequant_matmul(X, packed, scales, zeros, perm, bits, gs, Y, ws)
+        ev[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    clocks.stop()
+    launches = (g.gptq_launch_counter() - launches0) / K
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    ms_max = max_over_ranks(ms, dist, dev)
+    if rank != 0:
+        return
+    pk, which = peaks()
+    nbytes = (d_row * d_col * bits // 8 + 8 * ng * d_row + 2 * n_tok * d_col + 4 * d_col
+              + 4 * n_tok * d_row)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    peak = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    line = {
+        "metric": f"dequantized product with a quantized layer ({n_tok} token(s)): weights/s",
+        "value": world * d_row * d_col / (ms_max / 1e3), "unit": "weights/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16-in/fp32",
+        "data": "synthetic (seeded random codes, scales, zeros, act-order permutation)",
+        "config": {"workload": "llama70b_down_proj_dequant_matmul", "d_row": d_row, "d_col": d_col,
+                   "tokens": n_tok, "bits": bits, "group_size": gs, "desc_act": True,
+                   "l2": "flushed between steps (256 MiB write)"},
+        "roofline": {"kernel": "dequant_matmul_kernel", "bound": "hbm", "achieved": gbs,
+                     "peak": peak, "peak_source": f"{which} HBM copy", "unit": "GB/s",
+                     "frac": gbs / peak, "traffic": None,
+                     "algorithmic": f"packed codes + scales + zeros + X + perm + Y = {nbytes} bytes"},
+        "gpu_launches": launches, "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -414,7 +489,10 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = tdist
     try:
-        run_ours(args, rank, world, dist)
+        if args.dequant_matmul > 0:
+            run_dequant_matmul(args, rank, world, dist)
+        else:
+            run_ours(args, rank, world, dist)
     finally:
         if dist is not None:
             dist.destroy_process_group()

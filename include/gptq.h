@@ -235,6 +235,46 @@ gptq_status gptq_pack(const uint8_t *codes, int64_t d_row, int64_t d_col, int32_
                       uint32_t *packed, cudaStream_t stream);
 
 /*
+ * Using the quantized layer -- Y = X W_hat^T with the weights dequantized on
+ * the fly ("GPTQ (GPT Quantization)", "Limitations", items 1-2: the
+ * quantization is weight-only, the activations stay at 16 bits and the integer
+ * weights are dequantized before each product).  Decode form: tokens are taken
+ * 8 per launch and each launch streams the packed layer once, so it is meant
+ * for a few tokens at a time.
+ *   X       n_tok x d_col bf16 (raw bit patterns), row-major, leading
+ *           dimension ldx >= d_col, in the layer's ORIGINAL column order.
+ *   packed  d_row x (d_col * bits / 32) uint32, contiguous: gptq_pack output
+ *           (codes in quantization order).
+ *   scales, zeros  fp32 / int32 [ceil(d_col / g)][d_row], as
+ *           gptq_quantize_layer writes them.
+ *   perm    int32[d_col] from gptq_prepare_hinv (quantization position k holds
+ *           original column perm[k]); NULL means the identity.
+ *   Y       n_tok x d_row fp32, leading dimension ldy >= d_row (overwritten):
+ *           Y[t][n] = sum_k X[t][perm[k]] * scales[k/g][n] * (code[n][k] - zeros[k/g][n]).
+ *   Arithmetic: fp32 (per word, the dot of the token values with the codes
+ *   and their plain sum; the group's scale and zero point enter once per word).
+ *   ws      caller-owned device workspace, 256-byte aligned, of at least
+ *           gptq_dequant_matmul_workspace_size(n_tok, d_col) bytes: the
+ *           tokens gathered into quantization order (fp32), up to 8 at a time.
+ *   Supported: bits 2, 4 or 8 (a word holds whole codes), d_col a multiple of
+ *   32 / bits, group size -1, >= d_col or a multiple of 32 / bits (a word
+ *   never spans two groups); otherwise GPTQ_ERR_UNSUPPORTED (3-bit codes
+ *   straddle words).  Device pointers; n_tok == 0 is a no-op.
+ *   Errors: GPTQ_ERR_INVALID_ARG for NULL pointers, bad sizes or strides,
+ *   misaligned pointers or an invalid bits / group size; GPTQ_ERR_WORKSPACE
+ *   for a missing, misaligned or small workspace.
+ */
+gptq_status gptq_dequant_matmul(const uint16_t *X, int64_t n_tok, int64_t d_col, int64_t ldx,
+                                const uint32_t *packed, const float *scales, const int32_t *zeros,
+                                const int32_t *perm, int64_t d_row, int32_t bits,
+                                int32_t group_size, float *Y, int64_t ldy, void *ws,
+                                size_t ws_bytes, cudaStream_t stream);
+
+/* Workspace bytes gptq_dequant_matmul needs for n_tok tokens of a d_col-wide
+ * layer; 0 for invalid sizes. */
+size_t gptq_dequant_matmul_workspace_size(int64_t n_tok, int64_t d_col);
+
+/*
  * Waits for `stream`, then copies the device status word to *out.
  * Returns GPTQ_ERR_CUDA if the wait or the copy fails, else GPTQ_OK (the
  * device-side status itself is in *out).

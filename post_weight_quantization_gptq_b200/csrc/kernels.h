@@ -85,6 +85,15 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
                             int block, uint8_t* codes, float* scales, int32_t* zeros,
                             int32_t* status, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+// ---- using the quantized layer (dequant_matmul.cu): Y = X W_hat^T, decode form
+int dequant_matmul_tokens_per_launch(int bits);
+size_t dequant_matmul_workspace_bytes(int64_t n_tok, int64_t d_col);
+gptq_status launch_dequant_matmul(const uint16_t* X, int64_t n_tok, int64_t d_col, int64_t ldx,
+                                  const uint32_t* packed, const float* scales,
+                                  const int32_t* zeros, const int32_t* perm, int64_t d_row,
+                                  int bits, int group, float* Y, int64_t ldy, void* ws,
+                                  cudaStream_t stream);
+
 // ---- stage 5 (pack.cu)
 gptq_status launch_pack(const uint8_t* codes, int64_t d_row, int64_t d_col, int bits,
                         uint32_t* packed, cudaStream_t stream);

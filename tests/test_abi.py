@@ -126,3 +126,36 @@ def test_host_streaming_hessian_validation(pkg):
     assert f(fake, 16, 16, 16, fake, 16, None, ctypes.c_void_p((1 << 20) + 16), need, None) == 6
     assert f(fake, 16, 16, 16, fake, 16, None, fake, need - 1, None) == 6
     assert f(fake, 0, 16, 16, fake, 16, None, fake, need, None) == 0
+
+
+def test_dequant_matmul_validation(pkg):
+    lib = ctypes.CDLL(pkg.library_path())
+    P, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    f = lib.gptq_dequant_matmul
+    f.restype = ctypes.c_int
+    f.argtypes = [P, i64, i64, i64, P, P, P, P, i64, i32, i32, P, i64, P, ctypes.c_size_t, P]
+    lib.gptq_dequant_matmul_workspace_size.restype = ctypes.c_size_t
+    lib.gptq_dequant_matmul_workspace_size.argtypes = [i64, i64]
+    assert lib.gptq_dequant_matmul_workspace_size(1, 256) == 1024
+    assert lib.gptq_dequant_matmul_workspace_size(20, 256) == 8 * 256 * 4  # 8 tokens per launch
+    assert lib.gptq_dequant_matmul_workspace_size(0, 256) == 0
+    a = ctypes.c_void_p(1 << 20)
+    ok = dict(X=a, n=1, k=256, ldx=256, pk=a, sc=a, ze=a, perm=None, n_out=64, bits=4, g=128,
+              Y=a, ldy=64, ws=a, wsb=1024)
+
+    def call(**kw):
+        v = dict(ok)
+        v.update(kw)
+        return f(v["X"], v["n"], v["k"], v["ldx"], v["pk"], v["sc"], v["ze"], v["perm"],
+                 v["n_out"], v["bits"], v["g"], v["Y"], v["ldy"], v["ws"], v["wsb"], None)
+
+    assert call(n=0) == 0                                   # no tokens: nothing to do
+    assert call(X=None) == 1 and call(Y=None) == 1 and call(pk=None) == 1
+    assert call(k=0) == 1 and call(n_out=0) == 1 and call(ldx=100) == 1 and call(ldy=10) == 1
+    assert call(bits=5) == 1 and call(g=0) == 1 and call(g=-3) == 1
+    assert call(pk=ctypes.c_void_p((1 << 20) + 2)) == 1     # misaligned words
+    assert call(bits=3) == 2                                # 3-bit codes straddle words
+    assert call(k=252) == 2                                 # not whole 4-bit words
+    assert call(g=12) == 2                                  # a word would span two groups
+    assert call(ws=None) == 6 and call(wsb=1023) == 6       # workspace missing / too small
+    assert call(ws=ctypes.c_void_p((1 << 20) + 16)) == 6    # workspace misaligned
