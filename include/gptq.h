@@ -179,7 +179,8 @@ gptq_status gptq_prepare_hinv(float *H, int64_t d, int64_t ldh, const gptq_confi
  *           column perm[k] as they were when quantized (after the feedback of
  *           every earlier column).
  *   U, perm, dead  the outputs of gptq_prepare_hinv for this layer's H (any
- *           number of layers sharing one H may reuse them).  d_col must be a
+ *           number of layers sharing one H may reuse them), with the same
+ *           desc_act: without act-order perm is the identity and is not read.  d_col must be a
  *           multiple of 4 (GPTQ_ERR_UNSUPPORTED otherwise) and at most 57344.
  *   codes   d_row x d_col uint8, contiguous: codes[row][k] is the code of
  *           original column perm[k].

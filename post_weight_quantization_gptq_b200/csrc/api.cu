@@ -162,7 +162,7 @@ gptq_status gptq_quantize_layer(float* W, int64_t d_row, int64_t d_col, int64_t 
     if (ws == nullptr || !aligned(ws, 256) ||
         ws_bytes < gptq::quant_min_workspace_bytes(d_row, cfg->block_size))
         return GPTQ_ERR_WORKSPACE;
-    return launch_status(gptq::launch_quantize(W, d_row, d_col, ldw, U, perm, dead, cfg->bits,
+    return launch_status(gptq::launch_quantize(W, d_row, d_col, ldw, U, perm, dead, cfg->desc_act, cfg->bits,
                                                cfg->group_size, cfg->block_size, codes, scales,
                                                zeros, dev_status, ws, ws_bytes, stream));
 }

@@ -451,13 +451,23 @@ __global__ void zero_lower_blocks_kernel(float* __restrict__ X, int64_t ldx, int
         *reinterpret_cast<float4*>(X + i * ldx + j) = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// U[i][j] = X[d-1-i][d-1-j] for j >= i, 0 below the diagonal.
+// U[i][j] = X[d-1-i][d-1-j] for j >= i, 0 below the diagonal; four columns
+// per thread (d and ldx are multiples of 4, so the reversed float4 of X that
+// holds them is aligned).
 __global__ void flip_kernel(const float* __restrict__ X, int64_t ldx, float* __restrict__ U,
                             int64_t d) {
     const int64_t i = blockIdx.y;
-    for (int64_t j = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; j < d;
-         j += static_cast<int64_t>(gridDim.x) * blockDim.x)
-        U[i * d + j] = (j >= i) ? X[(d - 1 - i) * ldx + (d - 1 - j)] : 0.f;
+    const float* xr = X + (d - 1 - i) * ldx;
+    for (int64_t j = 4 * (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x); j < d;
+         j += 4 * static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float4 x = *reinterpret_cast<const float4*>(xr + (d - 4 - j));  // columns d-4-j .. d-1-j
+        float4 u = make_float4(x.w, x.z, x.y, x.x);                           // columns j .. j+3 of U
+        if (j < i) u.x = 0.f;
+        if (j + 1 < i) u.y = 0.f;
+        if (j + 2 < i) u.z = 0.f;
+        if (j + 3 < i) u.w = 0.f;
+        *reinterpret_cast<float4*>(U + i * d + j) = u;
+    }
 }
 
 }  // namespace
@@ -616,7 +626,7 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
         cudaStreamWaitEvent(stream, la->side_end, 0) != cudaSuccess ||
         cudaStreamWaitEvent(stream, la->inv_end, 0) != cudaSuccess)
         return GPTQ_ERR_CUDA;
-    dim3 grid(static_cast<unsigned>((d + 255) / 256 < 8 ? (d + 255) / 256 : 8),
+    dim3 grid(static_cast<unsigned>((d / 4 + 255) / 256 < 4 ? (d / 4 + 255) / 256 : 4),
               static_cast<unsigned>(d));
     flip_kernel<<<grid, 256, 0, stream>>>(X, ldx, U, d);
     count_launches(launches + 1);

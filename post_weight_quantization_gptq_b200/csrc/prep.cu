@@ -77,8 +77,8 @@ __global__ void iota_kernel(int32_t* __restrict__ perm, int64_t d) {
 
 // P[a][b] for the lower triangle, 32 x 32 tiles through shared memory so that
 // both the reads of H's lower triangle and the writes of P are coalesced
-// when the permutation is the identity.
-__global__ void __launch_bounds__(1024)
+// when the permutation is the identity; 32 x 8 threads, four rows each.
+__global__ void __launch_bounds__(256)
     gather_kernel(const float* __restrict__ H, int64_t d, int64_t ldh,
                   const int32_t* __restrict__ perm, const float* __restrict__ keys,
                   const PrepScratch* __restrict__ scratch, float* __restrict__ P) {
@@ -88,12 +88,15 @@ __global__ void __launch_bounds__(1024)
     if (b0 > a0 + 31) return;  // strictly upper tile
     const int tx = threadIdx.x, ty = threadIdx.y;
     const float lam = static_cast<float>(scratch->lambda);
-    // load: element (a = a0 + tx, b = b0 + ty)
-    {
-        const int64_t a = a0 + tx, b = b0 + ty;
+    // load: element (a = a0 + tx, b = b0 + y)
+    const int64_t a = a0 + tx;
+    const int64_t qa = a < d ? perm[d - 1 - a] : 0;
+#pragma unroll
+    for (int y = ty; y < 32; y += 8) {
+        const int64_t b = b0 + y;
         float v = 0.f;
         if (a < d && b < d) {
-            const int64_t qa = perm[d - 1 - a], qb = perm[d - 1 - b];
+            const int64_t qb = perm[d - 1 - b];
             if (qa == qb) {
                 v = keys[qa] + lam;
             } else {
@@ -101,12 +104,15 @@ __global__ void __launch_bounds__(1024)
                 v = H[r * ldh + c];
             }
         }
-        tile[ty][tx] = v;
+        tile[y][tx] = v;
     }
     __syncthreads();
-    // store: P[a0 + ty][b0 + tx] = element (a0 + ty, b0 + tx) = tile[tx][ty]
-    const int64_t a = a0 + ty, b = b0 + tx;
-    if (a < d && b < d && b <= a) P[a * d + b] = tile[tx][ty];
+    // store: P[a0 + y][b0 + tx] = element (a0 + y, b0 + tx) = tile[tx][y]
+#pragma unroll
+    for (int y = ty; y < 32; y += 8) {
+        const int64_t ar = a0 + y, b = b0 + tx;
+        if (ar < d && b < d && b <= ar) P[ar * d + b] = tile[tx][y];
+    }
 }
 
 }  // namespace
@@ -127,7 +133,7 @@ gptq_status launch_prep(const float* H, int64_t d, int64_t ldh, float damp, int 
         iota_kernel<<<static_cast<unsigned>((d + 255) / 256), 256, 0, stream>>>(perm, d);
     }
     const unsigned nt = static_cast<unsigned>((d + 31) / 32);
-    gather_kernel<<<dim3(nt, nt), dim3(32, 32), 0, stream>>>(H, d, ldh, perm, keys, scratch, P);
+    gather_kernel<<<dim3(nt, nt), dim3(32, 8), 0, stream>>>(H, d, ldh, perm, keys, scratch, P);
     count_launches(3);
     return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
 }

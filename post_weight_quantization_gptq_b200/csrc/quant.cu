@@ -79,7 +79,8 @@ struct GroupParams {
 __device__ __forceinline__ GroupParams group_params(const float (&cur)[4], const float (&nxt)[12],
                                                     int m, int jj, int l, int g, int bw,
                                                     const float* __restrict__ wrow, int64_t c0,
-                                                    int64_t d, bool live, int bits) {
+                                                    int64_t d, bool live, int bits,
+                                                    const uint8_t* __restrict__ dead_mask) {
     const int j = 32 * m + jj;
     float lo = 0.f, hi = 0.f;
 #pragma unroll
@@ -103,7 +104,7 @@ __device__ __forceinline__ GroupParams group_params(const float (&cur)[4], const
     const int64_t gend = (c0 + j + g < d) ? c0 + j + g : d;
     if (live && gend > c0 + bw) {
         for (int64_t c = c0 + bw + l; c < gend; c += 8) {
-            const float v = wrow[c];
+            const float v = (dead_mask != nullptr && dead_mask[c]) ? 0.f : wrow[c];
             lo = fminf(lo, v);
             hi = fmaxf(hi, v);
         }
@@ -150,7 +151,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
                        int64_t d, int64_t ldw, int64_t c0, int bw, int bits, int g,
                        uint8_t* __restrict__ codes, float* __restrict__ scales,
                        int32_t* __restrict__ zeros, float* __restrict__ err_out,
-                       int64_t err_ld, int32_t* status) {
+                       int64_t err_ld, const uint8_t* __restrict__ dead_mask, int32_t* status) {
     extern __shared__ uint8_t smem_raw[];
     float* smem = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -217,6 +218,10 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
+            // columns whose H diagonal is 0 quantize zero weights (in the
+            // permuted form the permutation pass has zeroed them already)
+            if (dead_mask != nullptr && 32 * m + 4 * l + i < bw && dead_mask[c0 + 32 * m + 4 * l + i])
+                v[i] = 0.f;
             if (m == 0) cur[i] = v[i];
             else nxt[4 * (m - 1) + i] = v[i];
         }
@@ -245,7 +250,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
     for (int m = 0; m < 4; ++m) {
         if (32 * m >= bw) break;
         if (!kSmallGroup && ((c0 + 32 * m) % g) == 0) {
-            gp = group_params(cur, nxt, m, 0, l, g, bw, wrow, c0, d, live, bits);
+            gp = group_params(cur, nxt, m, 0, l, g, bw, wrow, c0, d, live, bits, dead_mask);
             if (live && l == 0) {
                 const int64_t grp = (c0 + 32 * m) / g;
                 scales[grp * r + row] = gp.s;
@@ -264,7 +269,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
             const int j = 32 * m + jj;
             if (kFull || j < bw) {
                 if (kSmallGroup && ((c0 + j) % g) == 0) {
-                    gp = group_params(cur, nxt, m, jj, l, g, bw, wrow, c0, d, live, bits);
+                    gp = group_params(cur, nxt, m, jj, l, g, bw, wrow, c0, d, live, bits, dead_mask);
                     if (live && l == 0) {
                         const int64_t grp = (c0 + j) / g;
                         scales[grp * r + row] = gp.s;
@@ -440,8 +445,8 @@ size_t quant_min_workspace_bytes(int64_t d_row, int block) {
 // host checks the schedule and shortens the runs (down to the per-block
 // form) when a group size does not fit it.
 gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw, const float* U,
-                            const int32_t* perm, const uint8_t* dead, int bits, int group,
-                            int block, uint8_t* codes, float* scales, int32_t* zeros,
+                            const int32_t* perm, const uint8_t* dead, int desc_act, int bits,
+                            int group, int block, uint8_t* codes, float* scales, int32_t* zeros,
                             int32_t* status, void* ws, size_t ws_bytes, cudaStream_t stream) {
     if (block != kBlock) return GPTQ_ERR_UNSUPPORTED;
     const int g = (group == -1 || group > d_col) ? static_cast<int>(d_col) : group;
@@ -454,12 +459,19 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
     float* err = static_cast<float*>(ws);
     const int64_t err_ld = static_cast<int64_t>(defer) * kBlock;
 
-    const size_t row_smem = static_cast<size_t>(d_col) * sizeof(float);
-    if (cudaFuncSetAttribute(permute_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(row_smem)) != cudaSuccess)
-        return GPTQ_ERR_CUDA;
-    const int prow_grid = static_cast<int>(d_row < 4 * num_sms() ? d_row : 4 * num_sms());
-    permute_rows_kernel<<<prow_grid, 256, row_smem, stream>>>(W, d_row, d_col, ldw, perm, dead);
+    // With act-order the columns are permuted (and dead ones zeroed) in one
+    // pass; without it the permutation is the identity and the column walk
+    // zeroes dead columns as it loads them.
+    const bool permuted = desc_act != 0;
+    if (permuted) {
+        const size_t row_smem = static_cast<size_t>(d_col) * sizeof(float);
+        if (cudaFuncSetAttribute(permute_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(row_smem)) != cudaSuccess)
+            return GPTQ_ERR_CUDA;
+        const int prow_grid = static_cast<int>(d_row < 4 * num_sms() ? d_row : 4 * num_sms());
+        permute_rows_kernel<<<prow_grid, 256, row_smem, stream>>>(W, d_row, d_col, ldw, perm, dead);
+    }
+    const uint8_t* dead_mask = permuted ? nullptr : dead;
 
     CUtensorMap tU, tUmn, tErr;
     if (!make_tmap_2d(&tU, false, U, d_col, d_col, d_col, kBlock, kBlock, Swz::kNone) ||
@@ -478,16 +490,20 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
     const unsigned qgrid = static_cast<unsigned>((d_row + kRowsPerCta - 1) / kRowsPerCta);
     const int mt = static_cast<int>((d_row + 127) / 128);
     const int sms = num_sms();
-    int64_t launches = 1;
+    int64_t launches = permuted ? 1 : 0;
     int run0 = 0;  // first block of the current run (its errors sit at column 0 of err)
 
     auto quantize_block = [&](int b) -> bool {
         const int64_t c0 = static_cast<int64_t>(b) * kBlock;
         const int bw = static_cast<int>((d_col - c0 < kBlock) ? d_col - c0 : kBlock);
         ++launches;
-        return launch_kernel(true, bw == kBlock ? qfull : qpart, dim3(qgrid), dim3(kWarps * 32),
-                             q_smem, stream, tU, W, d_row, d_col, ldw, c0, bw, bits, g, codes,
-                             scales, zeros, err + static_cast<int64_t>(b - run0) * kBlock, err_ld,
+        // programmatic (early) launch after a kernel of this call only: the
+        // kernel fetches U before waiting, and the work before this call may
+        // still be writing U
+        return launch_kernel(b > 0 || permuted, bw == kBlock ? qfull : qpart, dim3(qgrid),
+                             dim3(kWarps * 32), q_smem, stream, tU, W, d_row, d_col, ldw, c0, bw,
+                             bits, g, codes, scales, zeros,
+                             err + static_cast<int64_t>(b - run0) * kBlock, err_ld, dead_mask,
                              status) == cudaSuccess;
     };
     // W[:, blocks [c, e)) -= Err[:, blocks [a, c)) U[blocks [a, c), blocks [c, e))

@@ -196,15 +196,19 @@ def test_quantize_layer_wide_groups_and_light_damping(d_row, d_col, g, damp, des
     compare_quantization(H.astype(np.float64), W, out, 4, g, desc_act, damp)
 
 
-def test_dead_columns_are_zero_weight():
-    W, X = workloads.small_layer(24, 256, 1024, seed=5)
+@pytest.mark.parametrize("g,desc_act", [(128, True), (128, False), (256, False), (32, False)])
+def test_dead_columns_are_zero_weight(g, desc_act):
+    """Dead input channels quantize to exact zeros, whether the act-order pass
+    zeroes them (desc_act) or the column walk does as it loads its block
+    (including the later columns a group wider than a block reads)."""
+    W, X = workloads.small_layer(24, 512, 2048, seed=5)
     Xf = X.to(torch.float32)
-    Xf[:, [3, 100, 255]] = 0.0
+    Xf[:, [3, 100, 255, 300]] = 0.0
     H = oracle.hessian(Xf.to(torch.bfloat16)).astype(np.float32)
-    out = gpu_quantize(H, W, 4, 128, True)
-    compare_quantization(H.astype(np.float64), W, out, 4, 128, True)
-    pos = np.nonzero(np.isin(out["perm"], [3, 100, 255]))[0]
-    Q = oracle.dequantize(out["codes"], out["scales"], out["zeros"], 128)
+    out = gpu_quantize(H, W, 4, g, desc_act)
+    compare_quantization(H.astype(np.float64), W, out, 4, g, desc_act)
+    pos = np.nonzero(np.isin(out["perm"], [3, 100, 255, 300]))[0]
+    Q = oracle.dequantize(out["codes"], out["scales"], out["zeros"], g)
     assert np.all(Q[:, pos] == 0.0)
 
 
