@@ -71,10 +71,46 @@ __device__ __forceinline__ void rank32_update4(float* D, const float* Ls, const 
     }
 }
 
+// Release store / acquire load of a shared-memory word at CTA scope: the
+// writes before the release are visible to a thread whose acquire load sees
+// the stored value.
+__device__ __forceinline__ void st_release_cta(int* p, int v) {
+    asm volatile("st.release.cta.shared::cta.s32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_cta(const int* p) {
+    int v;
+    asm volatile("ld.acquire.cta.shared::cta.s32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+
 // Barrier among the `count` threads (whole warps) that execute it with this
 // id (ids other than 0, which __syncthreads uses).
 __device__ __forceinline__ void named_barrier_sync(int id, int count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+    asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// 4 x 2 block of  D[i0.., j0..j0+1] -= sum_c Ls[c][i0..] * Ls[c][j0..]  (32 terms).
+__device__ __forceinline__ void rank32_update4x2(float* D, const float* Ls, int i0, int j0) {
+    float acc[4][2] = {};
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) {
+        const float4 li = lds4(Ls + k * LDA + i0);
+        const float2 lj = *reinterpret_cast<const float2*>(Ls + k * LDA + j0);
+        const float a4[4] = {li.x, li.y, li.z, li.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            acc[t][0] = fmaf(a4[t], lj.x, acc[t][0]);
+            acc[t][1] = fmaf(a4[t], lj.y, acc[t][1]);
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        float2* dst = reinterpret_cast<float2*>(D + (i0 + t) * LDA + j0);
+        float2 d2 = *dst;
+        d2.x -= acc[t][0];
+        d2.y -= acc[t][1];
+        *dst = d2;
+    }
 }
 
 // Triangular index u -> (bi, bj), bi >= bj.
@@ -108,8 +144,8 @@ __device__ __forceinline__ void tri_index(int u, int& bi, int& bj) {
 // factor, and those warps also store each finished strip of X.
 //
 // The factor warp keeps its rows in registers and rotates them after every
-// column step, so the pivot column is always register 0: the step loop stays
-// rolled while every register index is a compile-time constant.  Column c of
+// pair of column steps, so the pivot column is always register 0: the step
+// loop stays rolled while every register index is a compile-time constant.  Column c of
 // L below the diagonal is published as a row of Lc (Lc[c][m] = L[o+c+1+m][o+c],
 // zero past the strip), read back with eight broadcast float4 loads.
 __global__ void __launch_bounds__(kDiagThreads, 1)
@@ -172,29 +208,48 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
         }
 #pragma unroll
         for (int r = 0; r < 32; ++r) a[r] = (r <= lane) ? a[r] : 0.f;
+        // two columns per pass: column c+1 is formed in registers from column
+        // c (its pivot row needs only its own value, the other rows one
+        // broadcast), then both are published and applied as one rank-2
+        // update -- the same operations in the same order as two rank-1
+        // passes, with one shared-memory round trip instead of two
 #pragma unroll 1
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < 32; c += 2) {
             float piv = __shfl_sync(0xffffffffu, a[0], c);
             if (!(piv > 0.f)) {  // not positive definite (or NaN): flag, stay finite
                 bad = 1;
                 piv = 1.f;
             }
             const float inv = rsqrtf(piv);
-            const float a0 = (lane > c) ? a[0] * inv : 0.f;
+            const float a0 = (lane > c) ? a[0] * inv : 0.f;           // L[o+lane][o+c]
+            const float t = __shfl_sync(0xffffffffu, a0, c + 1);      // L[o+c+1][o+c]
+            const float n1 = fmaf(-a0, t, a[1]);                       // column c+1 after column c
+            float piv1 = __shfl_sync(0xffffffffu, n1, c + 1);
+            if (!(piv1 > 0.f)) {
+                bad = 1;
+                piv1 = 1.f;
+            }
+            const float inv1 = rsqrtf(piv1);
+            const float a1 = (lane > c + 1) ? n1 * inv1 : 0.f;        // L[o+lane][o+c+1]
             if (lane == c) dinv[o + c] = inv;
+            if (lane == c + 1) dinv[o + c + 1] = inv1;
             // lane i > c holds L[o+i][o+c] -> Lc[c][i-c-1]; lanes <= c fill the tail with 0
             Lc[c * 32 + ((lane - c - 1) & 31)] = a0;
-            __threadfence_block();
-            __syncwarp();
-            if (lane == 0) *reinterpret_cast<volatile int*>(&progress) = 32 * b + c + 1;
+            Lc[(c + 1) * 32 + ((lane - c - 2) & 31)] = a1;
+            __syncwarp();  // orders the warp's writes above before lane 0's release
+            if (lane == 0) st_release_cta(&progress, 32 * b + c + 2);
+            // a[r] <- a[r+2] - a0 L[o+c+2+r][o+c] - a1 L[o+c+2+r][o+c+1]
+            float l0[32], l1[32];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {  // update and rotate
-                const float4 l = lds4(Lc + c * 32 + 4 * q);
-                a[4 * q] = fmaf(-a0, l.x, a[4 * q + 1]);
-                a[4 * q + 1] = fmaf(-a0, l.y, a[4 * q + 2]);
-                a[4 * q + 2] = fmaf(-a0, l.z, a[4 * q + 3]);
-                a[4 * q + 3] = (q < 7) ? fmaf(-a0, l.w, a[4 * q + 4]) : 0.f;
+            for (int q = 0; q < 8; ++q) {
+                const float4 u = lds4(Lc + c * 32 + 4 * q), v = lds4(Lc + (c + 1) * 32 + 4 * q);
+                l0[4 * q] = u.x; l0[4 * q + 1] = u.y; l0[4 * q + 2] = u.z; l0[4 * q + 3] = u.w;
+                l1[4 * q] = v.x; l1[4 * q + 1] = v.y; l1[4 * q + 2] = v.z; l1[4 * q + 3] = v.w;
             }
+#pragma unroll
+            for (int r = 0; r < 30; ++r) a[r] = fmaf(-a1, l1[r], fmaf(-a0, l0[r + 1], a[r + 2]));
+            a[30] = 0.f;
+            a[31] = 0.f;
         }
     };
 
@@ -216,29 +271,34 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
             }
         }
         int spins = 0;
+        // the factor publishes two columns at a time: one wait per pair
 #pragma unroll 1
-        for (int c = 0; c < 32; ++c) {
-            const int need = 32 * b + c + 1;
-            while (*reinterpret_cast<volatile int*>(&progress) < need) {
+        for (int c2 = 0; c2 < 32; c2 += 2) {
+            const int need = 32 * b + c2 + 2;
+            while (ld_acquire_cta(&progress) < need) {
                 if (++spins > kStepSpinLimit) {
                     stalled = 1;
                     break;
                 }
+                __nanosleep(32);  // leave the issue slots to the factor warp (same sub-partition)
             }
-            __threadfence_block();
-            float4 l[8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) l[q] = lds4(Lc + c * 32 + 4 * q);
-            const float xc = x[0] * dinv[o + c];
+            for (int h = 0; h < 2; ++h) {
+                const int c = c2 + h;
+                float4 l[8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                x[4 * q] = fmaf(-l[q].x, xc, x[4 * q + 1]);
-                x[4 * q + 1] = fmaf(-l[q].y, xc, x[4 * q + 2]);
-                x[4 * q + 2] = fmaf(-l[q].z, xc, x[4 * q + 3]);
-                x[4 * q + 3] = (q < 7) ? fmaf(-l[q].w, xc, x[4 * q + 4]) : 0.f;
+                for (int q = 0; q < 8; ++q) l[q] = lds4(Lc + c * 32 + 4 * q);
+                const float xc = x[0] * dinv[o + c];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    x[4 * q] = fmaf(-l[q].x, xc, x[4 * q + 1]);
+                    x[4 * q + 1] = fmaf(-l[q].y, xc, x[4 * q + 2]);
+                    x[4 * q + 2] = fmaf(-l[q].z, xc, x[4 * q + 3]);
+                    x[4 * q + 3] = (q < 7) ? fmaf(-l[q].w, xc, x[4 * q + 4]) : 0.f;
+                }
+                if (rhs) Xs[(o + c) * LDA + t] = xc;
+                else Ls[c * LDA + t] = xc;
             }
-            if (rhs) Xs[(o + c) * LDA + t] = xc;
-            else Ls[c * LDA + t] = xc;
         }
     };
 
@@ -254,10 +314,13 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
         const int nb4 = o1 / 4;             // 4-column blocks of B's live columns
         const int below = (NB - o1 - 32) / 4;  // 4-row blocks below the next strip
         if (part == 0) {
-            for (int u = u0; u < 36; u += stride) {
-                int bi, bj;
-                tri_index(u, bi, bj);
-                rank32_update4(A, Ls, Ls, LDA, o1 + 4 * bi, o1 + 4 * bj);
+            // 72 units of 4 rows x 2 columns: row block i holds 2 i + 2 of them
+            for (int u = u0; u < 72; u += stride) {
+                int i = static_cast<int>((sqrtf(4.f * u + 1.f) - 1.f) * 0.5f);
+                while (i * (i + 1) > u) --i;
+                while ((i + 1) * (i + 2) <= u) ++i;
+                const int j = u - i * (i + 1);
+                rank32_update4x2(A, Ls, o1 + 4 * i, o1 + 2 * j);
             }
         } else if (part == 1) {
             const int n_panel = below * 8, n_b = 8 * nb4;
@@ -311,16 +374,16 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
         }
         __syncthreads();
         if (b < 3) {
-            // what the next strip reads first: warps 0-1 update its diagonal
-            // block (then warp 0 factors it), warps 2-7 its columns below it
+            // what the next strip reads first: warps 0-2 update its diagonal
+            // block (then warp 0 factors it), warps 3-7 its columns below it
             // and its rows of B (then warps 4-7 substitute); each group goes on
             // as soon as its own part is done
-            if (warp < 2) {
-                update(b, 0, tid, 64);
-                named_barrier_sync(1, 64);
+            if (warp < 3) {
+                update(b, 0, tid, 96);
+                named_barrier_sync(1, 96);
             } else {
-                update(b, 1, tid - 64, 192);
-                named_barrier_sync(2, 192);
+                update(b, 1, tid - 96, 160);
+                named_barrier_sync(2, 160);
             }
         }
     }
