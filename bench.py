@@ -6,7 +6,8 @@ tokens, damping / act-order / inverse factor, the column walk with OBQ
 feedback and lazy updates, and code packing.  Inputs are resident in HBM when
 the timed region starts; each step is timed with CUDA events on the launching
 stream, with the working copy of W restored and L2 flushed between steps
-(outside the events).  Multi-GPU runs are independent replicas (one layer per
+(outside the events).  Each stage's launches are captured once in a CUDA graph
+after the warm-up and replayed (--no-graph: launched on the stream).  Multi-GPU runs are independent replicas (one layer per
 rank, no collective on the data path): weak scaling, max over ranks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -49,6 +50,8 @@ def parse():
                    help="override the calibration token count (profiling of a smaller case)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-graph", action="store_true",
+                   help="launch each stage on the stream instead of replaying captured CUDA graphs")
     p.add_argument("--dequant-matmul", type=int, default=0, metavar="TOKENS",
                    help="instead of the quantizer step, time the product of TOKENS tokens with a "
                         "quantized Llama-70B down_proj (gptq_dequant_matmul)")
@@ -267,6 +270,30 @@ def run_ours(args, rank: int, world: int, dist):
     if status != 0:
         raise RuntimeError(f"device status {g.STATUS.get(status, status)} during warm-up")
 
+    # Each stage's launch sequence (hundreds of dependent kernels in prepare_hinv,
+    # with their cross-stream events) is captured once in a CUDA graph and
+    # replayed in the timed steps; the library's side streams join the capture
+    # through its events.  Their one-time set-up ran in the warm-up above.
+    stages = [lambda: g.gptq_hessian_accumulate(X, H, st),
+              lambda: g.gptq_prepare_hinv(H, cfg, U, perm, dead, st, ws),
+              lambda: g.gptq_quantize_layer(W, U, perm, dead, cfg, codes, scales, zeros, st, ws),
+              lambda: g.gptq_pack(codes, wl.bits, packed)]
+    launches_per_step = None
+    if not args.no_graph:
+        between()
+        H.zero_()
+        torch.cuda.synchronize(dev)
+        graphs = []
+        l0 = g.gptq_launch_counter()
+        for fn in stages:
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, capture_error_mode="thread_local"):
+                fn()
+            graphs.append(gr)
+        launches_per_step = g.gptq_launch_counter() - l0  # kernels in the captured graphs
+        torch.cuda.synchronize(dev)
+        stages = [gr.replay for gr in graphs]
+
     K = args.steps
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev_h0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
@@ -283,19 +310,19 @@ def run_ours(args, rank: int, world: int, dist):
         ev_s[k].record(stream)
         H.zero_()
         ev_h0[k].record(stream)
-        g.gptq_hessian_accumulate(X, H, st)
+        stages[0]()
         ev_mid[k][0].record(stream)
-        g.gptq_prepare_hinv(H, cfg, U, perm, dead, st, ws)
+        stages[1]()
         ev_mid[k][1].record(stream)
-        g.gptq_quantize_layer(W, U, perm, dead, cfg, codes, scales, zeros, st, ws)
+        stages[2]()
         ev_mid[k][2].record(stream)
-        g.gptq_pack(codes, wl.bits, packed)
+        stages[3]()
         ev_e[k].record(stream)
     torch.cuda.synchronize(dev)
     if dist is not None:
         dist.barrier()
     clocks.stop()
-    launches = (g.gptq_launch_counter() - launches0) / K
+    launches = (g.gptq_launch_counter() - launches0) / K if launches_per_step is None else launches_per_step
     status = g.gptq_sync_status(st)
     if status != 0:
         raise RuntimeError(f"device status {g.STATUS.get(status, status)} in the timed steps")
@@ -388,6 +415,7 @@ def run_ours(args, rank: int, world: int, dist):
                      "frac": achieved / peak, "traffic": traffic,
                      "algorithmic": f"n*d*(d+1) = {hess_flops:.4e} flop per launch"},
         "gpu_launches": launches,
+        "launch": "stream" if args.no_graph else "CUDA graphs (one per stage, captured once)",
         "clocks": clocks.summary(),
     }
     if e2e is not None:

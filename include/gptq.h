@@ -37,6 +37,11 @@
  *     outputs of that call are not valid.
  *   - Calls on the same stream are ordered; calls that share buffers on
  *     different streams must be ordered by the caller.
+ *   - gptq_hessian_accumulate, gptq_prepare_hinv, gptq_quantize_layer and
+ *     gptq_pack may be captured in a CUDA graph (stream capture on `stream`);
+ *     the library's own streams join the capture through its events.  The
+ *     first gptq_prepare_hinv and gptq_hessian_accumulate_host calls on a
+ *     device create those streams and events, so make them outside capture.
  */
 #ifndef GPTQ_B200_GPTQ_H
 #define GPTQ_B200_GPTQ_H

@@ -251,3 +251,52 @@ def test_pack_is_bit_exact(bits, d):
     g.gptq_pack(cd, bits, packed)
     torch.cuda.synchronize()
     assert np.array_equal(packed.cpu().numpy().view(np.uint32), oracle.pack(c, bits))
+
+
+def test_stages_replay_from_a_cuda_graph_bit_exactly():
+    """The four stages captured once in CUDA graphs (the library's side streams
+    join the capture through its events) and replayed twice give the same bits
+    as the stream-launched calls: U, perm, codes, scales, zeros, packed words."""
+    g = gpu()
+    r, d, n = 96, 640, 2560
+    W, X = workloads.small_layer(r, d, n, seed=31, kind="correlated")
+    cfg = g.GPTQConfig(bits=4, group_size=128, desc_act=True, damp=0.01)
+    dev = torch.device("cuda")
+    Xd, W0 = X.to(dev), W.to(dev).contiguous()
+    bufs = dict(H=torch.zeros(d, d, device=dev), U=torch.empty(d, d, device=dev),
+                perm=torch.empty(d, dtype=torch.int32, device=dev),
+                dead=torch.empty(d, dtype=torch.uint8, device=dev), W=torch.empty_like(W0),
+                codes=torch.empty(r, d, dtype=torch.uint8, device=dev),
+                scales=torch.empty(g.n_groups(d, 128), r, device=dev),
+                zeros=torch.empty(g.n_groups(d, 128), r, dtype=torch.int32, device=dev),
+                packed=torch.empty(r, g.packed_words(d, 4), dtype=torch.int32, device=dev),
+                ws=torch.empty(g.gptq_workspace_size(cfg, r, d), dtype=torch.uint8, device=dev),
+                st=torch.zeros(1, dtype=torch.int32, device=dev))
+    b = bufs
+
+    def stages():
+        return [lambda: (b["H"].zero_(), g.gptq_hessian_accumulate(Xd, b["H"], b["st"])),
+                lambda: g.gptq_prepare_hinv(b["H"], cfg, b["U"], b["perm"], b["dead"], b["st"], b["ws"]),
+                lambda: (b["W"].copy_(W0), g.gptq_quantize_layer(b["W"], b["U"], b["perm"], b["dead"], cfg,
+                                                                  b["codes"], b["scales"], b["zeros"],
+                                                                  b["st"], b["ws"])),
+                lambda: g.gptq_pack(b["codes"], 4, b["packed"])]
+
+    for fn in stages():  # stream launches (also the one-time set-up of the side streams)
+        fn()
+    assert g.gptq_sync_status(b["st"]) == 0
+    ref = {k: b[k].clone() for k in ("U", "perm", "codes", "scales", "zeros", "packed")}
+    graphs = []
+    for fn in stages():
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, capture_error_mode="thread_local"):
+            fn()
+        graphs.append(gr)
+    for _ in range(2):
+        for k in ("U", "codes", "packed"):
+            b[k].zero_()
+        for gr in graphs:
+            gr.replay()
+        assert g.gptq_sync_status(b["st"]) == 0
+        for k, v in ref.items():
+            assert torch.equal(b[k], v), k
