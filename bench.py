@@ -392,9 +392,9 @@ def run_ours(args, rank: int, world: int, dist):
     pk, which = peaks()
     hess_flops = n * d * (d + 1)
     # DRAM traffic of one Hessian launch from ncu (profiles/
-    # hessian_syrk_tcgen05_llama7b_q_proj_65k_tokens.md): 790.2 MB at 65,536 tokens,
+    # hessian_syrk_tcgen05_llama7b_q_proj_65k_tokens.md): 792.0 MB at 65,536 tokens,
     # d = 4,096; X reads and the per-16k-token drains both grow with the tokens.
-    traffic = 790.2e6 * n / 65536 if (d == 4096 and n % 16384 == 0) else None
+    traffic = 792.0e6 * n / 65536 if (d == 4096 and n % 16384 == 0) else None
     h_ms = statistics.mean(hess_ms)
     achieved = hess_flops / (h_ms / 1e3) / 1e12
     peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])

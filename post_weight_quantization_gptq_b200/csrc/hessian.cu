@@ -17,7 +17,9 @@
 //    stage.  All CTAs sweep the tokens in lockstep, so each token slice of X
 //    is fetched from HBM once and served to every CTA from L2.
 //  * Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs,
-//    warps 2..5 drain the accumulators (TMEM -> registers -> H).
+//    warps 2..9 drain the accumulators (TMEM -> registers -> H), two warps
+//    per TMEM lane quarter, each with half of the columns (twice the H loads
+//    in flight while the tensor cores wait for the drain).
 //  * The epilogue stores D[m][n] into H[n][m]: for a fixed n the 32 lanes of
 //    a warp hold 32 consecutive m, so every store is one coalesced 128-byte
 //    line.  Tiles are chosen with n >= m somewhere inside them, so the
@@ -44,7 +46,7 @@ constexpr int kBoxBytes = kBox * BK * 2;        // 8 KB
 constexpr int kABytes = BM * BK * 2;            // 16 KB
 constexpr int kBBytes = BN * BK * 2;            // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;  // 48 KB
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;   // TMA, MMA, 8 epilogue warps (two per TMEM lane quarter)
 constexpr int kTmemCols = 512;
 // Tokens accumulated in TMEM before the partial tile is added into H.  The
 // tensor cores' fp32 accumulation loses about 2^-25 of the running sum per
@@ -106,7 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->empty[s], 1);
         }
         mbar_init(&bars->acc_full, 1);
-        mbar_init(&bars->acc_empty, 128);
+        mbar_init(&bars->acc_empty, 256);
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
         fence_barrier_init();
@@ -220,8 +222,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(&bars->drain, 0, &no_abort)) *abort = 1;
         }
     } else {
-        // ------------------------------------------------ epilogue warps 2..5
+        // ------------------------------------------------ epilogue warps 2..9
         const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2;  // which 128 of each tile's 256 columns it drains
         for (int w = 0; w < waves && !*abort; ++w) {
             if (!mbar_wait(&bars->acc_full, w & 1, abort)) break;
             tc_fence_after();
@@ -233,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int m = mi * BM + q * 32 + lane;
                 const int nb = nj * BN;
 #pragma unroll 1
-                for (int cc = 0; cc < BN / 32; ++cc) {
+                for (int cc = half * (BN / 64); cc < (half + 1) * (BN / 64); ++cc) {
                     float v[32];
                     tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + s * BN + cc * 32, v);
                     if (m < d) {
