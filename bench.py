@@ -55,7 +55,39 @@ def parse():
     p.add_argument("--dequant-matmul", type=int, default=0, metavar="TOKENS",
                    help="instead of the quantizer step, time the product of TOKENS tokens with a "
                         "quantized Llama-70B down_proj (gptq_dequant_matmul)")
+    p.add_argument("--gemm-peaks", action="store_true",
+                   help="instead of the quantizer step, measure the library-GEMM denominators of the "
+                        "fp32 stages: cuBLAS 8192^3 fp32 with TF32 tensor cores and with plain FFMA")
     return p.parse_args()
+
+
+def run_gemm_peaks():
+    """cuBLAS (through torch.matmul) 8192^3 fp32 products, best of 10 after
+    3 warm-up: with TF32 tensor cores allowed (the kind::tf32 roof of the
+    3xTF32 GEMMs, which run three MMAs per product) and without (the FFMA
+    roof of an fp32-exact SIMT product)."""
+    n = 8192
+    a = torch.randn(n, n, device="cuda")
+    b = torch.randn(n, n, device="cuda")
+    c = torch.empty(n, n, device="cuda")
+    out = {}
+    for name, tf32 in (("tf32_tflops", True), ("fp32_ffma_tflops", False)):
+        torch.backends.cuda.matmul.allow_tf32 = tf32
+        for _ in range(3):
+            torch.matmul(a, b, out=c)
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch.matmul(a, b, out=c)
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        out[name] = 2 * n ** 3 / (best * 1e-3) / 1e12
+    torch.backends.cuda.matmul.allow_tf32 = False
+    print(json.dumps({"gemm_peaks": out, "how": "torch.matmul fp32 8192^3, best of 10 (burst)",
+                      "gpu": torch.cuda.get_device_name()}), flush=True)
 
 
 def peaks():
@@ -516,6 +548,9 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = tdist
+    if args.gemm_peaks:
+        run_gemm_peaks()
+        return
     try:
         if args.dequant_matmul > 0:
             run_dequant_matmul(args, rank, world, dist)

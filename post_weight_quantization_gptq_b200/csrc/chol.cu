@@ -402,36 +402,25 @@ __device__ __forceinline__ void tri_coords(int t, int& I, int& J) {
     J = t - i * (i + 1) / 2;
 }
 
-// 32 consecutive floats: dst[j] = sign * v[j], as float4 stores (callers
-// guarantee 16-byte alignment and bounds).
-__device__ __forceinline__ void put32(float* dst, const float (&v)[32], float sign) {
-    float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-        d4[q] = make_float4(sign * v[4 * q], sign * v[4 * q + 1], sign * v[4 * q + 2],
-                            sign * v[4 * q + 3]);
-}
-
 // ---------------------------------------------------------------- schedulers
+// All of them drain directly (one row per lane): the panel chain's GEMMs have
+// one tile per CTA, whose drain is on the critical path, and with the staged
+// drain on the side streams as well the whole inverse measured slower
+// (1.70 and 1.79 ms against 1.66 ms at d = 4096), the faster side kernels
+// competing harder with the chain.
 // Panel solve: L[m0.., kb..kb+kw) = A[m0.., kb..) (L_kk^-1)^T   (in place)
 struct TrsmSched {
     static constexpr bool kRmw = false;
+    static constexpr bool kStaged = false;  // see the note above the schedulers
     float* P;
     int64_t ldp;
     int d, kb, kw;
     __device__ g3::Job job(int t) const { return {kb + kw + NB * t, kb, kb, kb, (kw + 31) / 32}; }
-    __device__ void store(const g3::Job& jb, int row, int col0, const float (&v)[32]) const {
+    __device__ float* dst(const g3::Job& jb, int row) const {
         const int r = jb.m0 + row;
-        if (r >= d) return;
-        float* dst = P + static_cast<int64_t>(r) * ldp + kb + col0;
-        if (col0 + 32 <= kw) {
-            put32(dst, v, 1.f);
-        } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                if (col0 + j < kw) dst[j] = v[j];
-        }
+        return r < d ? P + static_cast<int64_t>(r) * ldp + kb : nullptr;
     }
+    __device__ int ncols(const g3::Job&, int) const { return kw; }
 };
 
 // Trailing update: P[I, J] -= L[I, panel] L[J, panel]^T on lower tiles.
@@ -456,6 +445,7 @@ struct SyrkSched {
         return {s0 + NB * I, s0 + NB * J, kb, kb, (kw + 31) / 32};
     }
     static constexpr bool kRmw = true;
+    static constexpr bool kStaged = false;
     __device__ float* dst(const g3::Job& jb, int row) const {
         const int r = jb.m0 + row;
         return r < d ? P + static_cast<int64_t>(r) * ldp + jb.n0 : nullptr;
@@ -475,14 +465,15 @@ struct SyrkSched {
 // whole B tile before its epilogue overwrites that tile.
 struct XFinSched {
     static constexpr bool kRmw = false;
+    static constexpr bool kStaged = false;
     float* X;
     int64_t ldx;
     int kb, kw;
     __device__ g3::Job job(int t) const { return {kb, NB * t, kb, kb, (kw + 31) / 32}; }
-    __device__ void store(const g3::Job& jb, int row, int col0, const float (&v)[32]) const {
-        if (row >= kw) return;
-        put32(X + static_cast<int64_t>(kb + row) * ldx + jb.n0 + col0, v, 1.f);
+    __device__ float* dst(const g3::Job& jb, int row) const {
+        return row < kw ? X + static_cast<int64_t>(kb + row) * ldx + jb.n0 : nullptr;
     }
+    __device__ int ncols(const g3::Job&, int) const { return g3::BN; }
 };
 
 // Panel k's share of the later block rows of L^-1:
@@ -490,6 +481,7 @@ struct XFinSched {
 // (A = the panel of L, K-major; B = block row k of X, MN-major).
 struct BUpdSched {
     static constexpr bool kRmw = true;
+    static constexpr bool kStaged = false;
     float* X;
     int64_t ldx;
     int d, kb, mt;

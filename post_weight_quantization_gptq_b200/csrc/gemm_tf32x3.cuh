@@ -19,12 +19,19 @@
 //   warp 0      TMA producer
 //   warp 1      TMEM owner and MMA issuer
 //   warps 2..5  write each stage's lo parts
-//   warps 6..9  drain the accumulator (tcgen05.ld, one row per thread, 32
-//               columns at a time) through the scheduler: store() for
-//               plain outputs; for read-modify-write outputs (kRmw, D -= AB^T)
-//               the warp loads its whole destination row segment into
-//               registers before the tile's MMAs finish, so the epilogue
-//               costs one store pass instead of a load round trip per chunk.
+//   warps 6..9  drain the accumulator into sched.dst() rows, sched.ncols()
+//               columns (tcgen05.ld gives one tile row per lane).  Plain
+//               outputs store the product; read-modify-write outputs (kRmw,
+//               D -= AB^T) load the destination values while the tile's MMAs
+//               still run.  Two forms:
+//               staged (default): 32 columns at a time through a padded
+//               shared-memory stage, leaving as 4 rows x 128 contiguous bytes
+//               per warp access (4 cache lines where a row per lane touches
+//               32); it frees the L1 for the split warps and wins when a CTA
+//               has several tiles, its drain hidden behind the next tile;
+//               direct (Sched::kStaged = false): each lane stores its own row
+//               straight from registers, the shorter path for a single tile
+//               whose drain is on the critical path.
 // Every wait is bounded; on expiry GPTQ_ERR_TIMEOUT is recorded and the CTA
 // winds down after its copies and MMAs have landed.
 #pragma once
@@ -44,7 +51,10 @@ constexpr int kStages = 3;
 constexpr int kTileBytes = 128 * BK * 4;      // 16 KB
 constexpr int kStageBytes = 4 * kTileBytes;   // A (as loaded), A lo, B (as loaded), B lo
 constexpr int kThreads = 320;                 // TMA, MMA, 4 split warps, 4 epilogue warps
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+constexpr int kEpiPitch = 36;                 // floats per staged row (16-byte groups of 8
+                                              // consecutive rows fall in distinct banks)
+constexpr int kEpiBytes = 4 * 32 * kEpiPitch * 4;  // one 32 x 32 stage per epilogue warp
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256 + kEpiBytes;
 constexpr uint32_t kTmemCols = 256;           // two 128-column accumulators
 
 // One output tile: rows m0.. of A, rows n0.. of B, K from ka0 (A) / kb0 (B),
@@ -67,6 +77,23 @@ struct Bars {
 // x minus the part of it a kind::tf32 MMA sees (exact: both share x's exponent)
 __device__ __forceinline__ float tf32_rest(float x) {
     return x - __uint_as_float(__float_as_uint(x) & 0xffffe000u);
+}
+
+// 16-byte shared-memory accesses by address (explicitly shared, so the
+// compiler neither routes them through generic addressing nor orders them
+// against the epilogue's global stores).
+__device__ __forceinline__ void sts128(uint32_t addr, float4 v) {
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y),
+                 "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ float4 lds128(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
 }
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -93,6 +120,20 @@ template <bool MN>
 __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk) {
     if (MN) return smem_desc(base + kk * 1024, 4096, 512, 1);
     return smem_desc(base + kk * 32, 16, 1024, 2);
+}
+
+// Epilogue form of a schedule: staged (coalesced) unless it says otherwise.
+template <class S, class = void>
+struct StagedEpi {
+    static constexpr bool value = true;
+};
+template <class S>
+struct StagedEpi<S, decltype(void(S::kStaged))> {
+    static constexpr bool value = S::kStaged;
+};
+template <class S>
+__host__ __device__ constexpr bool staged_epilogue() {
+    return StagedEpi<S>::value;
 }
 
 template <class Sched, bool A_MN, bool B_MN>
@@ -238,66 +279,141 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------------------------------------------- epilogue
-        const int q = warp & 3;  // TMEM lane quarter of this warp
-        const int row = q * 32 + lane;
+        const int q = warp & 3;  // TMEM lane quarter of this warp: tile rows 32 q ..
+        const uint32_t stage = smem_u32(smem + kStages * kStageBytes + 256) + q * 32 * kEpiPitch * 4;
+        const int rsub = lane >> 3;     // row within each group of 4 rows
+        const int c4 = 4 * (lane & 7);  // this lane's first column within a chunk
         int lt = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
             const Job job = sched.job(t);
             if (job.nk <= 0) continue;
             const int slot = lt & 1;
             const uint32_t use = static_cast<uint32_t>(lt >> 1);
-            if constexpr (Sched::kRmw) {
-                // destination row segment: the first nc of its BN columns are updated;
-                // when all BN columns may be read (aligned), the segment is loaded
-                // before the accumulator is ready
-                float* dst = sched.dst(job, row);
-                const int nc = dst != nullptr ? sched.ncols(job, row) : 0;
-                const bool pre = dst != nullptr && sched.nreadable(job) == BN &&
-                                 (reinterpret_cast<uintptr_t>(dst) & 15) == 0;
-                const bool full = pre && nc == BN;
+            if constexpr (!staged_epilogue<Sched>()) {
+                // one tile row per lane, straight from TMEM to its destination
+                const int row = 32 * q + lane;
+                float* d = sched.dst(job, row);
+                const int nc = d != nullptr ? sched.ncols(job, row) : 0;
+                const bool al = d != nullptr && (reinterpret_cast<uintptr_t>(d) & 15) == 0;
+                bool pre = false;
                 float4 old[BN / 4];
-                if (pre) {
+                if constexpr (Sched::kRmw) {
+                    pre = al && sched.nreadable(job) == BN;
+                    if (pre) {
 #pragma unroll
-                    for (int i = 0; i < BN / 4; ++i) old[i] = reinterpret_cast<const float4*>(dst)[i];
-                }
-                if (!mbar_wait(&bars->acc_full[slot], use & 1u, abort)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int c = 0; c < BN / 16; ++c) {  // 16 columns at a time: the
-                    float v[16];                      // prefetched row holds the registers
-                    tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + slot * BN + c * 16, v);
-                    if (full) {
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float4 o = old[4 * c + i];
-                            reinterpret_cast<float4*>(dst)[4 * c + i] =
-                                make_float4(o.x - v[4 * i], o.y - v[4 * i + 1], o.z - v[4 * i + 2],
-                                            o.w - v[4 * i + 3]);
-                        }
-                    } else if (pre) {  // partly written row (a diagonal tile)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float4 o = old[4 * c + i];
-                            const int j = 16 * c + 4 * i;
-                            if (j + 0 < nc) dst[j + 0] = o.x - v[4 * i + 0];
-                            if (j + 1 < nc) dst[j + 1] = o.y - v[4 * i + 1];
-                            if (j + 2 < nc) dst[j + 2] = o.z - v[4 * i + 2];
-                            if (j + 3 < nc) dst[j + 3] = o.w - v[4 * i + 3];
-                        }
-                    } else {  // row at the matrix edge: element-wise
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            if (16 * c + j < nc) dst[16 * c + j] -= v[j];
+                        for (int i = 0; i < BN / 4; ++i) old[i] = reinterpret_cast<const float4*>(d)[i];
                     }
                 }
-            } else {
                 if (!mbar_wait(&bars->acc_full[slot], use & 1u, abort)) break;
                 tc_fence_after();
-#pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
-                    float v[32];
-                    tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + slot * BN + c * 32, v);
-                    sched.store(job, row, c * 32, v);
+#pragma unroll
+                for (int c = 0; c < BN / 16; ++c) {
+                    float v[16];
+                    tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + slot * BN + c * 16, v);
+                    if (nc >= 16 * c + 16 && al && (!Sched::kRmw || pre)) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            float4 out = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                            if constexpr (Sched::kRmw) {
+                                const float4 o = old[4 * c + i];
+                                out = make_float4(o.x - out.x, o.y - out.y, o.z - out.z, o.w - out.w);
+                            }
+                            reinterpret_cast<float4*>(d)[4 * c + i] = out;
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            if (16 * c + j < nc) {
+                                if constexpr (Sched::kRmw) d[16 * c + j] -= v[j];
+                                else d[16 * c + j] = v[j];
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&bars->acc_empty[slot]);
+                ++lt;
+                continue;
+            }
+            // read-modify-write: this lane's destination values (rows
+            // 32 q + 4 i + rsub, columns 32 cc + c4 ..) when the whole row
+            // segment may be read: chunks 0 and 1 are loaded before the
+            // accumulator is ready, chunk cc + 2 once chunk cc is written
+            float4 old[2][8];
+            bool pre = false;
+            auto fetch = [&](int cc, float4 (&o)[8]) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float* d = sched.dst(job, 32 * q + 4 * i + rsub);
+                    const float* p = d != nullptr ? d + 32 * cc + c4 : nullptr;
+                    o[i] = (p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15) == 0)
+                               ? *reinterpret_cast<const float4*>(p)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            };
+            if constexpr (Sched::kRmw) {
+                pre = sched.nreadable(job) == BN;
+                if (pre) {
+                    fetch(0, old[0]);
+                    fetch(1, old[1]);
+                }
+            }
+            if (!mbar_wait(&bars->acc_full[slot], use & 1u, abort)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int cc = 0; cc < BN / 32; ++cc) {
+                // the chunk into the stage, one tile row per lane
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float v[16];
+                    tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + slot * BN + cc * 32 + h * 16,
+                              v);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        sts128(stage + (lane * kEpiPitch + h * 16 + 4 * j) * 4,
+                               make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+                }
+                __syncwarp();
+                // and out, 8 lanes per row: 4 columns each, 4 rows per access
+                float4 st[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) st[i] = lds128(stage + ((4 * i + rsub) * kEpiPitch + c4) * 4);
+                __syncwarp();  // every lane has read the stage: the next chunk may rewrite it
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int row = 32 * q + 4 * i + rsub;
+                    float* d = sched.dst(job, row);
+                    const int col = 32 * cc + c4;
+                    const int n = d != nullptr ? sched.ncols(job, row) - col : 0;
+                    if (n > 0) {
+                        const float4 a = st[i];
+                        float* p = d + col;
+                        const bool vec = n >= 4 && (reinterpret_cast<uintptr_t>(p) & 15) == 0;
+                        float4 out = a;
+                        if constexpr (Sched::kRmw) {
+                            float4 o;
+                            if (pre && vec) {
+                                o = old[cc & 1][i];
+                            } else {
+                                o.x = p[0];
+                                o.y = n > 1 ? p[1] : 0.f;
+                                o.z = n > 2 ? p[2] : 0.f;
+                                o.w = n > 3 ? p[3] : 0.f;
+                            }
+                            out = make_float4(o.x - a.x, o.y - a.y, o.z - a.z, o.w - a.w);
+                        }
+                        if (vec) {
+                            *reinterpret_cast<float4*>(p) = out;
+                        } else {
+                            p[0] = out.x;
+                            if (n > 1) p[1] = out.y;
+                            if (n > 2) p[2] = out.z;
+                            if (n > 3) p[3] = out.w;
+                        }
+                    }
+                }
+                if constexpr (Sched::kRmw) {
+                    if (pre && cc + 2 < BN / 32) fetch(cc + 2, old[cc & 1]);
                 }
             }
             tc_fence_before();
