@@ -37,6 +37,9 @@ import workloads  # noqa: E402
 METRIC = "GPTQ layer quantize: weights/s and ms/layer (4-bit g128); Hessian TFLOP/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# dram__bytes_read.sum + dram__bytes_write.sum of one Hessian launch at 65,536
+# tokens x 4,096 (ncu, current kernel: 32,768-token drains, eight drain warps)
+TRAFFIC_65K = 648.1e6
 
 
 def parse():
@@ -381,7 +384,7 @@ def run_ours(args, rank: int, world: int, dist):
         # X streams from pinned host memory through a two-slot staging buffer
         # (copies overlap the Hessian GEMM); W's copy runs on a second stream
         # beside it and is waited for before the column walk
-        staging = torch.empty(g.gptq_hessian_staging_size(d, 16384), dtype=torch.uint8,
+        staging = torch.empty(g.gptq_hessian_staging_size(d, 32768), dtype=torch.uint8,
                               device=dev)
         wcopy = torch.cuda.Stream(dev)
 
@@ -424,9 +427,10 @@ def run_ours(args, rank: int, world: int, dist):
     pk, which = peaks()
     hess_flops = n * d * (d + 1)
     # DRAM traffic of one Hessian launch from ncu (profiles/
-    # hessian_syrk_tcgen05_llama7b_q_proj_65k_tokens.md): 792.0 MB at 65,536 tokens,
-    # d = 4,096; X reads and the per-16k-token drains both grow with the tokens.
-    traffic = 792.0e6 * n / 65536 if (d == 4096 and n % 16384 == 0) else None
+    # hessian_syrk_tcgen05_llama7b_q_proj_65k_tokens.md) at 65,536 tokens,
+    # d = 4,096; X reads and the per-32k-token drains both grow with the tokens.
+    traffic = (TRAFFIC_65K * n / 65536
+               if (TRAFFIC_65K is not None and d == 4096 and n % 32768 == 0) else None)
     h_ms = statistics.mean(hess_ms)
     achieved = hess_flops / (h_ms / 1e3) / 1e12
     peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])

@@ -129,14 +129,14 @@ gptq_status gptq_hessian_accumulate(const uint16_t *X, int64_t n, int64_t d, int
  *   H, ldh  as gptq_hessian_accumulate (accumulated into; lower triangle).
  *   staging caller-owned DEVICE buffer, 256-byte aligned, of at least
  *           gptq_hessian_staging_size(d, 64) bytes; split into two slots of
- *           `chunk` token rows each (chunk = the largest multiple of 16384
+ *           `chunk` token rows each (chunk = the largest multiple of 32768
  *           tokens that fits, else of 64).  The copy engine fills one slot
  *           while the tensor cores read the other.  Its contents are
  *           scratch.
  *   Copies run on a stream the library owns (one per device) and are ordered
  *   after everything queued on `stream` before the call; every GEMM runs on
  *   `stream`, so work queued on `stream` afterwards sees the finished H.
- *   When chunk is a multiple of 16384 the result is bitwise identical to
+ *   When chunk is a multiple of 32768 the result is bitwise identical to
  *   gptq_hessian_accumulate on the same X in device memory.
  *   Errors: GPTQ_ERR_INVALID_ARG (sizes, NULL X_host / H, ldx < d, ldh < d),
  *   GPTQ_ERR_WORKSPACE (staging NULL, misaligned or too small for 64 tokens).

@@ -24,7 +24,7 @@
 //    a warp hold 32 consecutive m, so every store is one coalesced 128-byte
 //    line.  Tiles are chosen with n >= m somewhere inside them, so the
 //    written entries cover H's lower triangle.
-//  * Tokens are taken in chunks of 16,384: each chunk's partial tile is added
+//  * Tokens are taken in chunks of 32,768: each chunk's partial tile is added
 //    into H by the epilogue (fp32, round to nearest), which bounds the bias of
 //    the tensor cores' long fp32 accumulation.
 //  * No atomics: every H entry has exactly one owner, so the result is
@@ -52,9 +52,11 @@ constexpr int kTmemCols = 512;
 // tensor cores' fp32 accumulation loses about 2^-25 of the running sum per
 // accumulate step, with a consistent sign, so the bias grows with the number
 // of steps (measured ~1.4e-3 relative over 262,144 tokens in one run);
-// draining every 16,384 tokens (1,024 steps) keeps it near 3e-5 and the
-// drains themselves are ordinary round-to-nearest fp32 adds.
-constexpr int kChunkIters = 16384 / BK;
+// draining every 32,768 tokens (512 steps of 64 tokens) keeps it near 6e-5
+// (full-size H rows within 1.8e-4 of a float64 sum; 16,384-token drains gave
+// 8e-5 and cost 3-5 % more time) and the drains themselves are ordinary
+// round-to-nearest fp32 adds.
+constexpr int kChunkIters = 32768 / BK;
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
 constexpr uint32_t kIdesc = instr_desc(/*bf16*/ 1, /*A MN*/ 1, /*B MN*/ 1, BM, BN);
 

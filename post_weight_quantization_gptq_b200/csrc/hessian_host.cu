@@ -22,7 +22,7 @@ namespace gptq {
 namespace {
 
 constexpr int64_t kTokenQuantum = 64;       // tokens per MMA k-step (BK of the GEMM)
-constexpr int64_t kDrainTokens = 16384;     // the GEMM's own accumulation chunk
+constexpr int64_t kDrainTokens = 32768;     // the GEMM's own accumulation chunk
 
 struct CopyPipe {
     cudaStream_t copy = nullptr;

@@ -31,11 +31,11 @@ from . import (GPTQConfig, GPTQError, gptq_hessian_accumulate, gptq_pack, gptq_p
                gptq_quantize_layer, gptq_sync_status, gptq_workspace_size, n_groups,
                packed_words)
 
-# The Hessian kernel adds its fp32 partial sums into H every 16,384 tokens.
+# The Hessian kernel adds its fp32 partial sums into H every 32,768 tokens.
 # Token shards that start on such a boundary keep each rank's partial sums
 # those of the single-process call; only the order of the cross-rank
 # additions differs.
-TOKEN_QUANTUM = 16384
+TOKEN_QUANTUM = 32768
 
 
 def token_range(n_tokens: int, rank: int, world: int, quantum: int = TOKEN_QUANTUM):

@@ -55,13 +55,15 @@ def test_hessian_accumulates_over_token_chunks():
     assert lower_rel_err(three, oracle.hessian(X)) <= 1e-5
 
 
-@pytest.mark.parametrize("n,d,ldx,chunk", [(40000, 256, 256, 16384), (3000, 200, 203, 500),
+@pytest.mark.parametrize("n,d,ldx,chunk", [(70000, 256, 256, 32768), (40000, 256, 256, 16384),
+                                            (3000, 200, 203, 500),
                                             (777, 384, 384, 64), (100, 8, 8, 1 << 20)])
 def test_hessian_from_host_memory(n, d, ldx, chunk):
     """X streamed from pinned host memory through the two-slot staging buffer:
     bitwise equal to the device-resident call when the chunk is a multiple
-    of 16384 tokens (the GEMM's own accumulation chunk), else within fp32
-    summation-order error; ragged last chunk, padded host rows, d not a
+    of 32768 tokens (the GEMM's own accumulation chunk), else within fp32
+    summation-order error plus, past one chunk, the accumulation drift of
+    differently placed drains; ragged last chunk, padded host rows, d not a
     multiple of 8 included."""
     import post_weight_quantization_gptq_b200 as g
     _, X = workloads.small_layer(4, d, n, seed=n + d + 5, kind="student_t")
@@ -79,13 +81,19 @@ def test_hessian_from_host_memory(n, d, ldx, chunk):
     Hh = H.cpu().numpy()
     Hd = gpu_hessian(X)
     L = np.tril(np.ones_like(Hd, dtype=bool))
-    if chunk % 16384 == 0:
+    if chunk % 32768 == 0:
         assert np.array_equal(Hh[L], Hd[L])
-    else:
+    elif n <= 32768:
+        # both sides drain once, at the end of each call: summation order only
         assert np.max(np.abs(Hh - Hd)[L]) <= 1e-5 * np.max(np.abs(Hd))
-    # the tensor cores' fp32 accumulation drifts by ~3e-5 per 16384-token
-    # drain; the H bar of the parity rules is 1e-3
-    assert lower_rel_err(Hh, oracle.hessian(X)) <= 1e-4
+    else:
+        # different drain points: the tensor cores' accumulation drift (up to
+        # ~1.8e-4 per 32768-token drain) differs as well
+        assert np.max(np.abs(Hh - Hd)[L]) <= 2e-4 * np.max(np.abs(Hd))
+    # the tensor cores' fp32 accumulation drifts within each 32768-token
+    # drain (measured 1.4e-4 here, up to 1.8e-4 on full-size rows); the H bar
+    # of the parity rules is 1e-3
+    assert lower_rel_err(Hh, oracle.hessian(X)) <= 3e-4
 
 
 # ------------------------------------------------------------------ stage 2

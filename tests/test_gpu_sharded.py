@@ -61,7 +61,7 @@ def _worker(rank, world, port, case, out):
 
 
 @pytest.mark.parametrize("case", [
-    (3 * 16384 + 1000, 512, 300, 4, 128, False),   # ragged token shard and row slices
+    (3 * 32768 + 1000, 512, 300, 4, 128, False),   # ragged token shard and row slices
     (40000, 384, 257, 4, 32, True),                # act-order, g32
 ])
 def test_two_processes_quantize_one_layer(case):
@@ -77,7 +77,9 @@ def test_two_processes_quantize_one_layer(case):
     o0, o1 = out[0], out[1]
     assert o0["status"] == o1["status"] == 0
     assert np.array_equal(o0["H"], o1["H"])
-    assert lower_rel_err(o0["H"], oracle.hessian(X)) <= 1e-4
+    # per-drain accumulation drift of the tensor cores (32768-token drains);
+    # the H bar of the parity rules is 1e-3
+    assert lower_rel_err(o0["H"], oracle.hessian(X)) <= 3e-4
     for k in ("perm", "dead", "packed_all", "scales_all", "zeros_all"):
         assert np.array_equal(o0[k], o1[k]), k           # both ranks hold the same layer
     codes = np.concatenate([o0["codes"], o1["codes"]])

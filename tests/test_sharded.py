@@ -24,8 +24,8 @@ def _free_port():
 
 
 @pytest.mark.parametrize("n,world,quantum", [(0, 2, 64), (1, 2, 64), (64, 3, 64), (1000, 2, 64),
-                                             (5 * 64 + 7, 4, 64), (262144, 8, 16384),
-                                             (40000, 3, 16384), (100, 5, 64)])
+                                             (5 * 64 + 7, 4, 64), (262144, 8, 32768),
+                                             (40000, 3, 32768), (100, 5, 64)])
 def test_token_shards_cover_the_tokens_on_quantum_boundaries(n, world, quantum):
     spans = [sharded.token_range(n, k, world, quantum) for k in range(world)]
     assert spans[0][0] == 0 and spans[-1][1] == n
