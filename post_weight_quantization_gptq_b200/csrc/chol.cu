@@ -596,11 +596,12 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
     if (la == nullptr) return GPTQ_ERR_CUDA;
     const int sms = num_sms();
     // SMs shared by the two side streams (the panel chain keeps the rest:
-    // its launches are one wave of at most 31 tiles).  Each panel's rest of
-    // the trailing update gets enough of them to finish in about five waves
-    // (it must be done before the column update two launches later on the
-    // chain); the inverse stream, whose work grows as the trailing updates
-    // shrink, gets the others.
+    // at d = 4096 its launches are one wave of at most 31 tiles), split per
+    // panel in proportion to the two streams' tiles (below).  Measured
+    // against a split that gave the rest of the trailing update enough SMs
+    // for five waves and the inverse the others: the same at d = 4096, 2.3x
+    // faster at 8192, 3x at 11008, 3.9x at 28672, where that split starved
+    // the inverse stream.
     const int pool = sms >= 128 ? sms - 32 : (3 * sms) / 4;
     const int pool_min = pool / 8 > 1 ? pool / 8 : 1;
     const int npan = static_cast<int>((d + NB - 1) / NB);
@@ -648,8 +649,14 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
                 return GPTQ_ERR_CUDA;
             ++launches;
         }
+        // the pool is shared in proportion to this panel's tiles on each
+        // stream, so both streams advance one panel in about the same time
+        // (the rest of the trailing update dominates early, the inverse's
+        // block rows late; both carry d^3 / 3 flops in total)
         const int side_tiles = mt * (mt + 1) / 2 - mt;
-        int side_sms = (side_tiles + 4) / 5;
+        const long long inv_tiles = static_cast<long long>(mt) * (k + 1) + k;
+        const long long all_tiles = side_tiles + inv_tiles > 0 ? side_tiles + inv_tiles : 1;
+        int side_sms = static_cast<int>((static_cast<long long>(pool) * side_tiles + all_tiles / 2) / all_tiles);
         side_sms = side_sms < pool_min ? pool_min : (side_sms > pool - pool_min ? pool - pool_min : side_sms);
         const int inv_sms = pool - side_sms;
         if (mt > 1) {
