@@ -403,15 +403,15 @@ __device__ __forceinline__ void tri_coords(int t, int& I, int& J) {
 }
 
 // ---------------------------------------------------------------- schedulers
-// All of them drain directly (one row per lane): the panel chain's GEMMs have
-// one tile per CTA, whose drain is on the critical path, and with the staged
-// drain on the side streams as well the whole inverse measured slower
-// (1.70 and 1.79 ms against 1.66 ms at d = 4096), the faster side kernels
-// competing harder with the chain.
+// Every GEMM of the factorization drains directly (one row per lane): the
+// panel chain's have one tile per CTA, whose drain is on the critical path,
+// and staging the side streams' drains measured slower as well (prepare_hinv
+// 1.70 and 1.79 ms against 1.66 ms at d = 4096, the faster side kernels
+// competing harder with the chain; 8.1 vs 7.5 ms at 8192, 319 vs 292 ms at
+// 28672; 18.5 vs 19.2 ms at 11008).
 // Panel solve: L[m0.., kb..kb+kw) = A[m0.., kb..) (L_kk^-1)^T   (in place)
 struct TrsmSched {
     static constexpr bool kRmw = false;
-    static constexpr bool kStaged = false;  // see the note above the schedulers
     float* P;
     int64_t ldp;
     int d, kb, kw;
@@ -445,7 +445,6 @@ struct SyrkSched {
         return {s0 + NB * I, s0 + NB * J, kb, kb, (kw + 31) / 32};
     }
     static constexpr bool kRmw = true;
-    static constexpr bool kStaged = false;
     __device__ float* dst(const g3::Job& jb, int row) const {
         const int r = jb.m0 + row;
         return r < d ? P + static_cast<int64_t>(r) * ldp + jb.n0 : nullptr;
@@ -465,7 +464,6 @@ struct SyrkSched {
 // whole B tile before its epilogue overwrites that tile.
 struct XFinSched {
     static constexpr bool kRmw = false;
-    static constexpr bool kStaged = false;
     float* X;
     int64_t ldx;
     int kb, kw;
@@ -481,7 +479,6 @@ struct XFinSched {
 // (A = the panel of L, K-major; B = block row k of X, MN-major).
 struct BUpdSched {
     static constexpr bool kRmw = true;
-    static constexpr bool kStaged = false;
     float* X;
     int64_t ldx;
     int d, kb, mt;
@@ -630,7 +627,7 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
         const int mt = static_cast<int>((m + NB - 1) / NB);
         if (m > 0) {
             TrsmSched ts{P, ldp, di, static_cast<int>(kb), kw};
-            if (g3::launch<TrsmSched, false, false>(tP, tX, ts, mt, status, stream, sms, true) !=
+            if (g3::launch<TrsmSched, false, false, false>(tP, tX, ts, mt, status, stream, sms, true) !=
                 cudaSuccess)
                 return GPTQ_ERR_CUDA;
             ++launches;
@@ -645,7 +642,8 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
             if (k > 0 && cudaStreamWaitEvent(stream, la->done[(k - 1) & 3], 0) != cudaSuccess)
                 return GPTQ_ERR_CUDA;
             SyrkSched nx{P, ldp, di, static_cast<int>(kb), kw, static_cast<int>(kb + kw), 1};
-            if (g3::launch<SyrkSched, false, false>(tP, tP, nx, mt, status, stream, sms) != cudaSuccess)
+            if (g3::launch<SyrkSched, false, false, false>(tP, tP, nx, mt, status, stream, sms) !=
+                cudaSuccess)
                 return GPTQ_ERR_CUDA;
             ++launches;
         }
@@ -661,8 +659,9 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
         const int inv_sms = pool - side_sms;
         if (mt > 1) {
             SyrkSched rs{P, ldp, di, static_cast<int>(kb), kw, static_cast<int>(kb + kw), 2};
-            if (g3::launch<SyrkSched, false, false>(tP, tP, rs, mt * (mt + 1) / 2 - mt, status,
-                                                    la->side, side_sms) != cudaSuccess)
+            const int rt = mt * (mt + 1) / 2 - mt;
+            if (g3::launch<SyrkSched, false, false, false>(tP, tP, rs, rt, status, la->side, side_sms) !=
+                cudaSuccess)
                 return GPTQ_ERR_CUDA;
             ++launches;
         }
@@ -670,15 +669,16 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
         // inverse stream: finish row k of L^-1, then pass panel k on to the rows below
         if (k > 0) {
             XFinSched xf{X, ldx, static_cast<int>(kb), kw};
-            if (g3::launch<XFinSched, false, true>(tX, tXmn, xf, k, status, la->inv, inv_sms) !=
+            if (g3::launch<XFinSched, false, true, false>(tX, tXmn, xf, k, status, la->inv, inv_sms) !=
                 cudaSuccess)
                 return GPTQ_ERR_CUDA;
             ++launches;
         }
         if (m > 0) {
             BUpdSched bu{X, ldx, di, static_cast<int>(kb), mt};
-            if (g3::launch<BUpdSched, false, true>(tP, tXmn, bu, mt * (k + 1), status, la->inv,
-                                                   inv_sms, k > 0) != cudaSuccess)
+            const int bt = mt * (k + 1);
+            if (g3::launch<BUpdSched, false, true, false>(tP, tXmn, bu, bt, status, la->inv, inv_sms,
+                                                          k > 0) != cudaSuccess)
                 return GPTQ_ERR_CUDA;
             ++launches;
         }

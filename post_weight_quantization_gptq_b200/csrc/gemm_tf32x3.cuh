@@ -29,7 +29,7 @@
 //               per warp access (4 cache lines where a row per lane touches
 //               32); it frees the L1 for the split warps and wins when a CTA
 //               has several tiles, its drain hidden behind the next tile;
-//               direct (Sched::kStaged = false): each lane stores its own row
+//               direct (Staged = false): each lane stores its own row
 //               straight from registers, the shorter path for a single tile
 //               whose drain is on the critical path.
 // Every wait is bounded; on expiry GPTQ_ERR_TIMEOUT is recorded and the CTA
@@ -122,21 +122,7 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk) {
     return smem_desc(base + kk * 32, 16, 1024, 2);
 }
 
-// Epilogue form of a schedule: staged (coalesced) unless it says otherwise.
-template <class S, class = void>
-struct StagedEpi {
-    static constexpr bool value = true;
-};
-template <class S>
-struct StagedEpi<S, decltype(void(S::kStaged))> {
-    static constexpr bool value = S::kStaged;
-};
-template <class S>
-__host__ __device__ constexpr bool staged_epilogue() {
-    return StagedEpi<S>::value;
-}
-
-template <class Sched, bool A_MN, bool B_MN>
+template <class Sched, bool A_MN, bool B_MN, bool Staged>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
                        const Sched sched, int tiles, int32_t* status) {
@@ -289,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (job.nk <= 0) continue;
             const int slot = lt & 1;
             const uint32_t use = static_cast<uint32_t>(lt >> 1);
-            if constexpr (!staged_epilogue<Sched>()) {
+            if constexpr (!Staged) {
                 // one tile row per lane, straight from TMEM to its destination
                 const int row = 32 * q + lane;
                 float* d = sched.dst(job, row);
@@ -430,11 +416,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // pdl: launched with programmatic serialization (see launch_kernel).
-template <class Sched, bool A_MN, bool B_MN>
+template <class Sched, bool A_MN, bool B_MN, bool Staged>
 inline cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const Sched& sched,
                           int tiles, int32_t* status, cudaStream_t stream, int sms,
                           bool pdl = false) {
-    auto kern = gemm_tf32x3_kernel<Sched, A_MN, B_MN>;
+    auto kern = gemm_tf32x3_kernel<Sched, A_MN, B_MN, Staged>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     if (tiles <= 0) return cudaSuccess;

@@ -515,7 +515,8 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
         LazySched ls{W, ldw, static_cast<int>(d_row), static_cast<int>(cend), static_cast<int>(c1), mt,
                      (a - run0) * kBlock, a * kBlock, (c - a) * (kBlock / 32)};
         ++launches;
-        return g3::launch<LazySched, false, true>(tErr, tUmn, ls, mt * nt, status, stream, sms, true) ==
+        return g3::launch<LazySched, false, true, true>(tErr, tUmn, ls, mt * nt, status, stream, sms,
+                                                        true) ==
                cudaSuccess;
     };
     // blocks [lo, hi) of the current run, complete w.r.t. every block < lo
