@@ -403,12 +403,18 @@ __device__ __forceinline__ void tri_coords(int t, int& I, int& J) {
 }
 
 // ---------------------------------------------------------------- schedulers
-// Every GEMM of the factorization drains directly (one row per lane): the
-// panel chain's have one tile per CTA, whose drain is on the critical path,
-// and staging the side streams' drains measured slower as well (prepare_hinv
-// 1.70 and 1.79 ms against 1.66 ms at d = 4096, the faster side kernels
-// competing harder with the chain; 8.1 vs 7.5 ms at 8192, 319 vs 292 ms at
-// 28672; 18.5 vs 19.2 ms at 11008).
+// Drains (see gemm_tf32x3.cuh).  The read-modify-write updates (the trailing
+// update, on the chain and beside it, and the inverse's block rows) hand
+// -AB^T to TMA tensor reductions into P and X: the read-modify-write happens
+// in L2 and the SMs issue no global loads or stores for it.  prepare_hinv
+// with them against the direct drain: 1.46 vs 1.66 ms at d = 4096, 4.1 vs
+// 7.5 ms at 8192, 8.9 vs 19.2 ms at 11008, 146 vs 292 ms at 28672.  Full
+// tiles are reduced: the upper part of a diagonal tile of P receives values
+// too, which nothing reads (the diagonal factor loads only j <= i, every GEMM
+// operand lies below the diagonal blocks).  (The shared-memory staged drain
+// measured slower than the direct one here: 1.70 and 1.79 ms at 4096.)
+// kChainStore: the plain-store outputs (panel solve, L^-1 block row).
+constexpr int kChainStore = g3::kEpiStore;
 // Panel solve: L[m0.., kb..kb+kw) = A[m0.., kb..) (L_kk^-1)^T   (in place)
 struct TrsmSched {
     static constexpr bool kRmw = false;
@@ -578,10 +584,12 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
                                 int32_t* status, void*, cudaStream_t stream) {
     const int64_t ldp = d;
     const int di = static_cast<int>(d);
-    CUtensorMap tP, tX, tXmn;
+    CUtensorMap tP, tX, tXmn, tPd, tXd;
     if (!make_tmap_2d(&tP, false, P, d, d, ldp, 32, 128, Swz::k128) ||
         !make_tmap_2d(&tX, false, X, d, d, ldx, 32, 128, Swz::k128) ||
-        !make_tmap_2d(&tXmn, false, X, d, d, ldx, 32, 32, Swz::k128Atom32))
+        !make_tmap_2d(&tXmn, false, X, d, d, ldx, 32, 32, Swz::k128Atom32) ||
+        !make_tmap_2d(&tPd, false, P, d, d, ldp, 32, 32, Swz::k128) ||
+        !make_tmap_2d(&tXd, false, X, d, d, ldx, 32, 32, Swz::k128))
         return GPTQ_ERR_INVALID_ARG;
     if (cudaFuncSetAttribute(potrf_inv_128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kDiagSmem) != cudaSuccess)
@@ -627,7 +635,8 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
         const int mt = static_cast<int>((m + NB - 1) / NB);
         if (m > 0) {
             TrsmSched ts{P, ldp, di, static_cast<int>(kb), kw};
-            if (g3::launch<TrsmSched, false, false, false>(tP, tX, ts, mt, status, stream, sms, true) !=
+            if (g3::launch<TrsmSched, false, false, kChainStore>(tP, tX, ts, mt, status, stream, sms, true,
+                                                                 &tPd) !=
                 cudaSuccess)
                 return GPTQ_ERR_CUDA;
             ++launches;
@@ -642,8 +651,8 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
             if (k > 0 && cudaStreamWaitEvent(stream, la->done[(k - 1) & 3], 0) != cudaSuccess)
                 return GPTQ_ERR_CUDA;
             SyrkSched nx{P, ldp, di, static_cast<int>(kb), kw, static_cast<int>(kb + kw), 1};
-            if (g3::launch<SyrkSched, false, false, false>(tP, tP, nx, mt, status, stream, sms) !=
-                cudaSuccess)
+            if (g3::launch<SyrkSched, false, false, g3::kEpiReduce>(tP, tP, nx, mt, status, stream, sms,
+                                                                    false, &tPd) != cudaSuccess)
                 return GPTQ_ERR_CUDA;
             ++launches;
         }
@@ -660,8 +669,8 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
         if (mt > 1) {
             SyrkSched rs{P, ldp, di, static_cast<int>(kb), kw, static_cast<int>(kb + kw), 2};
             const int rt = mt * (mt + 1) / 2 - mt;
-            if (g3::launch<SyrkSched, false, false, false>(tP, tP, rs, rt, status, la->side, side_sms) !=
-                cudaSuccess)
+            if (g3::launch<SyrkSched, false, false, g3::kEpiReduce>(tP, tP, rs, rt, status, la->side,
+                                                                    side_sms, false, &tPd) != cudaSuccess)
                 return GPTQ_ERR_CUDA;
             ++launches;
         }
@@ -669,7 +678,8 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
         // inverse stream: finish row k of L^-1, then pass panel k on to the rows below
         if (k > 0) {
             XFinSched xf{X, ldx, static_cast<int>(kb), kw};
-            if (g3::launch<XFinSched, false, true, false>(tX, tXmn, xf, k, status, la->inv, inv_sms) !=
+            if (g3::launch<XFinSched, false, true, kChainStore>(tX, tXmn, xf, k, status, la->inv, inv_sms,
+                                                                false, &tXd) !=
                 cudaSuccess)
                 return GPTQ_ERR_CUDA;
             ++launches;
@@ -677,8 +687,8 @@ gptq_status launch_chol_inverse(float* P, float* X, int64_t ldx, int64_t d, floa
         if (m > 0) {
             BUpdSched bu{X, ldx, di, static_cast<int>(kb), mt};
             const int bt = mt * (k + 1);
-            if (g3::launch<BUpdSched, false, true, false>(tP, tXmn, bu, bt, status, la->inv, inv_sms,
-                                                          k > 0) != cudaSuccess)
+            if (g3::launch<BUpdSched, false, true, g3::kEpiReduce>(tP, tXmn, bu, bt, status, la->inv,
+                                                                   inv_sms, k > 0, &tXd) != cudaSuccess)
                 return GPTQ_ERR_CUDA;
             ++launches;
         }

@@ -29,9 +29,18 @@
 //               per warp access (4 cache lines where a row per lane touches
 //               32); it frees the L1 for the split warps and wins when a CTA
 //               has several tiles, its drain hidden behind the next tile;
-//               direct (Staged = false): each lane stores its own row
-//               straight from registers, the shorter path for a single tile
-//               whose drain is on the critical path.
+//               direct (kEpiDirect): each lane stores its own row straight
+//               from registers, the shorter path for a single tile whose
+//               drain is on the critical path;
+//               reduce (kEpiReduce, read-modify-write outputs): the warp
+//               writes -AB^T for 32 x 32 elements into a shared-memory buffer
+//               (128-byte swizzle) and one lane hands it to a TMA tensor
+//               reduction (cp.reduce.async.bulk.tensor .add) into D: the
+//               read-modify-write happens in L2, with no global loads or
+//               stores from the SM; two buffers per warp alternate;
+//               store (kEpiStore, plain outputs): the same with AB^T and a
+//               TMA tensor store.  Both write whole boxes, clipped only at
+//               the tensor map's extent.
 // Every wait is bounded; on expiry GPTQ_ERR_TIMEOUT is recorded and the CTA
 // winds down after its copies and MMAs have landed.
 #pragma once
@@ -55,6 +64,15 @@ constexpr int kEpiPitch = 36;                 // floats per staged row (16-byte 
                                               // consecutive rows fall in distinct banks)
 constexpr int kEpiBytes = 4 * 32 * kEpiPitch * 4;  // one 32 x 32 stage per epilogue warp
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256 + kEpiBytes;
+constexpr int kRedBufBytes = 32 * 32 * 4;  // one 32 x 32 fp32 box
+// drain forms (see the header comment)
+constexpr int kEpiDirect = 0, kEpiStaged = 1, kEpiReduce = 2, kEpiStore = 3;
+// dynamic shared memory of a drain form: the reduce buffers (two per warp)
+// start 1024 bytes after the stages, on the 128-byte swizzle's 1024-byte period
+template <int Epi>
+constexpr int smem_bytes() {
+    return Epi >= kEpiReduce ? kStages * kStageBytes + 1024 + 1024 + 8 * kRedBufBytes : kSmemBytes;
+}
 constexpr uint32_t kTmemCols = 256;           // two 128-column accumulators
 
 // One output tile: rows m0.. of A, rows n0.. of B, K from ka0 (A) / kb0 (B),
@@ -122,10 +140,34 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk) {
     return smem_desc(base + kk * 32, 16, 1024, 2);
 }
 
-template <class Sched, bool A_MN, bool B_MN, bool Staged>
+// 32 x 32 fp32 tensor reduction (add) from shared memory into global memory,
+// tracked by the issuing thread's bulk-async group
+__device__ __forceinline__ void tma_reduce_add_2d(const void* tmap, uint32_t src, int32_t c0, int32_t c1) {
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(tmap)),
+        "r"(src), "r"(c0), "r"(c1)
+        : "memory");
+}
+// 32 x 32 fp32 tensor store from shared memory, tracked like the reduction
+__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int32_t c0, int32_t c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// all but the newest group have finished reading their shared-memory source
+__device__ __forceinline__ void bulk_wait_read_but1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+template <class Sched, bool A_MN, bool B_MN, int Epi>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
-                       const Sched sched, int tiles, int32_t* status) {
+                       const __grid_constant__ CUtensorMap tmd, const Sched sched, int tiles,
+                       int32_t* status) {
     constexpr uint32_t kIdesc = instr_desc(/*tf32*/ 2, A_MN ? 1 : 0, B_MN ? 1 : 0, BM, BN);
 
     extern __shared__ uint8_t smem_raw[];
@@ -152,6 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_barrier_init();
         tma_prefetch_desc(&tma);
         tma_prefetch_desc(&tmb);
+        if constexpr (Epi >= kEpiReduce) tma_prefetch_desc(&tmd);
     }
     if (warp == 1) {
         tmem_alloc(&bars->tmem, kTmemCols);
@@ -275,7 +318,47 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (job.nk <= 0) continue;
             const int slot = lt & 1;
             const uint32_t use = static_cast<uint32_t>(lt >> 1);
-            if constexpr (!Staged) {
+            if constexpr (Epi >= kEpiReduce) {
+                static_assert(Sched::kRmw == (Epi == kEpiReduce),
+                              "reduce serves read-modify-write outputs, store plain ones");
+                constexpr float sgn = Epi == kEpiReduce ? -1.f : 1.f;
+                if (!mbar_wait(&bars->acc_full[slot], use & 1u, abort)) break;
+                tc_fence_after();
+                const uint32_t rbase = smem_u32(smem + kStages * kStageBytes + 1024) + q * 2 * kRedBufBytes;
+#pragma unroll
+                for (int cc = 0; cc < BN / 32; ++cc) {
+                    const uint32_t buf = rbase + (cc & 1) * kRedBufBytes;
+                    // the reduction that last read this buffer (two chunks ago) is done reading
+                    if (lane == 0) bulk_wait_read_but1();
+                    __syncwarp();
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        float v[16];
+                        tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + slot * BN + cc * 32 + h * 16,
+                                  v);
+                        // row `lane` of the box, 16-byte chunk 4 h + j at its 128-byte-swizzle slot
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            sts128(buf + lane * 128 + ((((4 * h + j) ^ (lane & 7))) << 4),
+                                   make_float4(sgn * v[4 * j], sgn * v[4 * j + 1], sgn * v[4 * j + 2],
+                                               sgn * v[4 * j + 3]));
+                    }
+                    fence_async_smem();  // the writes above, before the async proxy reads them
+                    __syncwarp();
+                    if (lane == 0) {
+                        if constexpr (Epi == kEpiReduce)
+                            tma_reduce_add_2d(&tmd, buf, job.n0 + 32 * cc, job.m0 + 32 * q);
+                        else
+                            tma_store_2d(&tmd, buf, job.n0 + 32 * cc, job.m0 + 32 * q);
+                        bulk_commit();
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&bars->acc_empty[slot]);
+                ++lt;
+                continue;
+            }
+            if constexpr (Epi == kEpiDirect) {
                 // one tile row per lane, straight from TMEM to its destination
                 const int row = 32 * q + lane;
                 float* d = sched.dst(job, row);
@@ -406,6 +489,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&bars->acc_empty[slot]);
             ++lt;
         }
+        // reductions issued by this warp have completed (reads and writes)
+        if constexpr (Epi >= kEpiReduce) {
+            if (lane == 0) bulk_wait_all();
+        }
     }
 
     tc_fence_before();
@@ -416,17 +503,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // pdl: launched with programmatic serialization (see launch_kernel).
-template <class Sched, bool A_MN, bool B_MN, bool Staged>
+// td: the destination's tensor map (box 32 x 32 fp32, 128-byte swizzle) for
+// the reduce drain; unused by the other forms.
+template <class Sched, bool A_MN, bool B_MN, int Epi>
 inline cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const Sched& sched,
                           int tiles, int32_t* status, cudaStream_t stream, int sms,
-                          bool pdl = false) {
-    auto kern = gemm_tf32x3_kernel<Sched, A_MN, B_MN, Staged>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+                          bool pdl = false, const CUtensorMap* td = nullptr) {
+    auto kern = gemm_tf32x3_kernel<Sched, A_MN, B_MN, Epi>;
+    if (Epi >= kEpiReduce && td == nullptr) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem_bytes<Epi>());
     if (e != cudaSuccess) return e;
     if (tiles <= 0) return cudaSuccess;
     const int grid = tiles < sms ? tiles : sms;
-    return launch_kernel(pdl, kern, dim3(grid), dim3(kThreads), kSmemBytes, stream, ta, tb, sched,
-                         tiles, status);
+    return launch_kernel(pdl, kern, dim3(grid), dim3(kThreads), smem_bytes<Epi>(), stream, ta, tb,
+                         td != nullptr ? *td : tb, sched, tiles, status);
 }
 
 }  // namespace g3

@@ -473,11 +473,16 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
     }
     const uint8_t* dead_mask = permuted ? nullptr : dead;
 
-    CUtensorMap tU, tUmn, tErr;
+    CUtensorMap tU, tUmn, tErr, tW;
     if (!make_tmap_2d(&tU, false, U, d_col, d_col, d_col, kBlock, kBlock, Swz::kNone) ||
         !make_tmap_2d(&tUmn, false, U, d_col, d_col, d_col, 32, 32, Swz::k128Atom32) ||
         !make_tmap_2d(&tErr, false, err, err_ld, d_row, err_ld, 32, 128, Swz::k128))
         return GPTQ_ERR_INVALID_ARG;
+    // the lazy update adds -Err U into W through TMA reductions when W's rows
+    // can be a tensor map (16-byte aligned base and row pitch); else it
+    // drains through shared memory and plain loads and stores
+    const bool w_tma = (reinterpret_cast<uintptr_t>(W) & 15) == 0 && (ldw % 4) == 0 &&
+                       make_tmap_2d(&tW, false, W, d_col, d_row, ldw, 32, 32, Swz::k128);
     const size_t q_smem = (kBlock * kBlock + kBlock) * sizeof(float) + 1024;
     const bool small_group = g < 32;
     auto qfull = small_group ? block_quant_kernel<true, true> : block_quant_kernel<false, true>;
@@ -515,8 +520,10 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
         LazySched ls{W, ldw, static_cast<int>(d_row), static_cast<int>(cend), static_cast<int>(c1), mt,
                      (a - run0) * kBlock, a * kBlock, (c - a) * (kBlock / 32)};
         ++launches;
-        return g3::launch<LazySched, false, true, true>(tErr, tUmn, ls, mt * nt, status, stream, sms,
-                                                        true) ==
+        return (w_tma ? g3::launch<LazySched, false, true, g3::kEpiReduce>(tErr, tUmn, ls, mt * nt, status,
+                                                                          stream, sms, true, &tW)
+                      : g3::launch<LazySched, false, true, g3::kEpiStaged>(tErr, tUmn, ls, mt * nt, status,
+                                                                          stream, sms, true)) ==
                cudaSuccess;
     };
     // blocks [lo, hi) of the current run, complete w.r.t. every block < lo
