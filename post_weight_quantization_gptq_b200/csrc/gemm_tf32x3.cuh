@@ -19,19 +19,15 @@
 //   warp 0      TMA producer
 //   warp 1      TMEM owner and MMA issuer
 //   warps 2..5  write each stage's lo parts
-//   warps 6..9  drain the accumulator into sched.dst() rows, sched.ncols()
-//               columns (tcgen05.ld gives one tile row per lane).  Plain
-//               outputs store the product; read-modify-write outputs (kRmw,
-//               D -= AB^T) load the destination values while the tile's MMAs
-//               still run.  Two forms:
-//               staged (default): 32 columns at a time through a padded
-//               shared-memory stage, leaving as 4 rows x 128 contiguous bytes
-//               per warp access (4 cache lines where a row per lane touches
-//               32); it frees the L1 for the split warps and wins when a CTA
-//               has several tiles, its drain hidden behind the next tile;
-//               direct (kEpiDirect): each lane stores its own row straight
-//               from registers, the shorter path for a single tile whose
-//               drain is on the critical path;
+//   warps 6..9  drain the accumulator (tcgen05.ld gives one tile row per
+//               lane).  Plain outputs receive the product, read-modify-write
+//               outputs (kRmw) D -= AB^T.  Three forms:
+//               staged (kEpiStaged): into sched.dst() rows, sched.ncols()
+//               columns, 32 columns at a time through a padded shared-memory
+//               stage, leaving as 4 rows x 128 contiguous bytes per warp
+//               access (read-modify-write outputs load the destination
+//               values in the same order while the tile's MMAs still run);
+//               the form for destinations that cannot be a tensor map;
 //               reduce (kEpiReduce, read-modify-write outputs): the warp
 //               writes -AB^T for 32 x 32 elements into a shared-memory buffer
 //               (128-byte swizzle) and one lane hands it to a TMA tensor
@@ -66,7 +62,7 @@ constexpr int kEpiBytes = 4 * 32 * kEpiPitch * 4;  // one 32 x 32 stage per epil
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256 + kEpiBytes;
 constexpr int kRedBufBytes = 32 * 32 * 4;  // one 32 x 32 fp32 box
 // drain forms (see the header comment)
-constexpr int kEpiDirect = 0, kEpiStaged = 1, kEpiReduce = 2, kEpiStore = 3;
+constexpr int kEpiStaged = 1, kEpiReduce = 2, kEpiStore = 3;
 // dynamic shared memory of a drain form: the reduce buffers (two per warp)
 // start 1024 bytes after the stages, on the 128-byte swizzle's 1024-byte period
 template <int Epi>
@@ -351,52 +347,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         else
                             tma_store_2d(&tmd, buf, job.n0 + 32 * cc, job.m0 + 32 * q);
                         bulk_commit();
-                    }
-                }
-                tc_fence_before();
-                mbar_arrive(&bars->acc_empty[slot]);
-                ++lt;
-                continue;
-            }
-            if constexpr (Epi == kEpiDirect) {
-                // one tile row per lane, straight from TMEM to its destination
-                const int row = 32 * q + lane;
-                float* d = sched.dst(job, row);
-                const int nc = d != nullptr ? sched.ncols(job, row) : 0;
-                const bool al = d != nullptr && (reinterpret_cast<uintptr_t>(d) & 15) == 0;
-                bool pre = false;
-                float4 old[BN / 4];
-                if constexpr (Sched::kRmw) {
-                    pre = al && sched.nreadable(job) == BN;
-                    if (pre) {
-#pragma unroll
-                        for (int i = 0; i < BN / 4; ++i) old[i] = reinterpret_cast<const float4*>(d)[i];
-                    }
-                }
-                if (!mbar_wait(&bars->acc_full[slot], use & 1u, abort)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int c = 0; c < BN / 16; ++c) {
-                    float v[16];
-                    tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + slot * BN + c * 16, v);
-                    if (nc >= 16 * c + 16 && al && (!Sched::kRmw || pre)) {
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            float4 out = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-                            if constexpr (Sched::kRmw) {
-                                const float4 o = old[4 * c + i];
-                                out = make_float4(o.x - out.x, o.y - out.y, o.z - out.z, o.w - out.w);
-                            }
-                            reinterpret_cast<float4*>(d)[4 * c + i] = out;
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            if (16 * c + j < nc) {
-                                if constexpr (Sched::kRmw) d[16 * c + j] -= v[j];
-                                else d[16 * c + j] = v[j];
-                            }
-                        }
                     }
                 }
                 tc_fence_before();

@@ -199,7 +199,10 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
                         (lane >> 3);
     const bool live = row < r;
     float* wrow = W + (live ? row : 0) * ldw;
-    const bool vec = (ldw & 3) == 0 && bw == kBlock;
+    // float4 access to W needs 16-byte aligned rows (base and pitch); four
+    // codes go out as one 32-bit store when codes' rows are 4-byte aligned
+    const bool vec = (ldw & 3) == 0 && bw == kBlock && (reinterpret_cast<uintptr_t>(W) & 15) == 0;
+    const bool vec_codes = vec && (d & 3) == 0 && (reinterpret_cast<uintptr_t>(codes) & 3) == 0;
 
     // the row's slice of the block (in flight while the U block arrives)
     float cur[4], nxt[12];
@@ -321,7 +324,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
             if (vec) {
                 *reinterpret_cast<float4*>(wrow + c0 + cb) = make_float4(cur[0], cur[1], cur[2], cur[3]);
             }
-            if (vec && (d & 3) == 0) {
+            if (vec_codes) {
                 *reinterpret_cast<uint32_t*>(codes + row * d + c0 + cb) =
                     qv[0] | (qv[1] << 8) | (qv[2] << 16) | (qv[3] << 24);
             }
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
                 const int c = cb + i;
                 if (c < bw) {
                     if (!vec) wrow[c0 + c] = cur[i];
-                    if (!(vec && (d & 3) == 0)) codes[row * d + c0 + c] = static_cast<uint8_t>(qv[i]);
+                    if (!vec_codes) codes[row * d + c0 + c] = static_cast<uint8_t>(qv[i]);
                 }
             }
         }

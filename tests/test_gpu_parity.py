@@ -308,3 +308,40 @@ def test_stages_replay_from_a_cuda_graph_bit_exactly():
         assert g.gptq_sync_status(b["st"]) == 0
         for k, v in ref.items():
             assert torch.equal(b[k], v), k
+
+
+@pytest.mark.parametrize("pad,offset", [(3, 0), (3, 1), (1, 3)])
+def test_quantize_layer_on_strided_and_offset_weights(pad, offset):
+    """W as a view into a wider buffer: a row pitch that is not a multiple of
+    4 floats, or a base that is not 16-byte aligned.  The lazy update cannot
+    address such rows with a tensor map and drains through shared memory, the
+    column walk moves W element by element; the result must be the contiguous
+    call's bit for bit, and the buffer outside the view stays untouched."""
+    g = gpu()
+    d_row, d_col, bits, gs = 96, 512, 4, 128
+    W, X = workloads.small_layer(d_row, d_col, 2048, seed=pad * 10 + offset, kind="student_t")
+    H = oracle.hessian(X).astype(np.float32)
+    ref = gpu_quantize(H, W, bits, gs, False)
+    cfg = g.GPTQConfig(bits=bits, group_size=gs, desc_act=False)
+    Hd = torch.from_numpy(H).cuda()
+    U = torch.empty(d_col, d_col, device="cuda")
+    perm = torch.empty(d_col, dtype=torch.int32, device="cuda")
+    dead = torch.empty(d_col, dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(g.gptq_workspace_size(cfg, d_row, d_col), dtype=torch.uint8, device="cuda")
+    g.gptq_prepare_hinv(Hd, cfg, U, perm, dead, st, ws)
+    buf = torch.full((d_row, offset + d_col + pad), 7.0, device="cuda")
+    Wv = buf[:, offset:offset + d_col]
+    Wv.copy_(W.cuda())
+    ng = g.n_groups(d_col, gs)
+    codes = torch.empty(d_row, d_col, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(ng, d_row, device="cuda")
+    zeros = torch.empty(ng, d_row, dtype=torch.int32, device="cuda")
+    g.gptq_quantize_layer(Wv, U, perm, dead, cfg, codes, scales, zeros, st, ws)
+    assert g.gptq_sync_status(st) == 0
+    assert np.array_equal(codes.cpu().numpy(), ref["codes"])
+    assert np.array_equal(scales.cpu().numpy(), ref["scales"])
+    assert np.array_equal(zeros.cpu().numpy(), ref["zeros"])
+    assert np.array_equal(Wv.cpu().numpy(), ref["w_at_quant"])
+    outside = torch.cat([buf[:, :offset], buf[:, offset + d_col:]], dim=1)
+    assert bool((outside == 7.0).all())
