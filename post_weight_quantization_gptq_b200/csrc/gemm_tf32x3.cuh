@@ -93,26 +93,7 @@ __device__ __forceinline__ float tf32_rest(float x) {
     return x - __uint_as_float(__float_as_uint(x) & 0xffffe000u);
 }
 
-// 16-byte shared-memory accesses by address (explicitly shared, so the
-// compiler neither routes them through generic addressing nor orders them
-// against the epilogue's global stores).
-__device__ __forceinline__ void sts128(uint32_t addr, float4 v) {
-    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y),
-                 "f"(v.z), "f"(v.w)
-                 : "memory");
-}
-__device__ __forceinline__ float4 lds128(uint32_t addr) {
-    float4 v;
-    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
-}
 
-__device__ __forceinline__ void fence_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 template <bool MN>
 __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
@@ -136,28 +117,6 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk) {
     return smem_desc(base + kk * 32, 16, 1024, 2);
 }
 
-// 32 x 32 fp32 tensor reduction (add) from shared memory into global memory,
-// tracked by the issuing thread's bulk-async group
-__device__ __forceinline__ void tma_reduce_add_2d(const void* tmap, uint32_t src, int32_t c0, int32_t c1) {
-    asm volatile(
-        "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-            reinterpret_cast<uint64_t>(tmap)),
-        "r"(src), "r"(c0), "r"(c1)
-        : "memory");
-}
-// 32 x 32 fp32 tensor store from shared memory, tracked like the reduction
-__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int32_t c0, int32_t c1) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                     reinterpret_cast<uint64_t>(tmap)),
-                 "r"(src), "r"(c0), "r"(c1)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// all but the newest group have finished reading their shared-memory source
-__device__ __forceinline__ void bulk_wait_read_but1() {
-    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 template <class Sched, bool A_MN, bool B_MN, int Epi>
 __global__ void __launch_bounds__(kThreads, 1)
