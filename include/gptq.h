@@ -180,7 +180,8 @@ gptq_status gptq_prepare_hinv(float *H, int64_t d, int64_t ldh, const gptq_confi
 /*
  * Stages 3-4 -- the GPTQ column walk with OBQ error feedback.
  *   W       d_row x d_col fp32, leading dimension ldw, in ORIGINAL column
- *           order.  Scratch: on return column k holds the weights of original
+ *           order; any alignment (rows with a 16-byte aligned base and a
+ *           pitch of a multiple of 4 floats take the vector and TMA paths).  Scratch: on return column k holds the weights of original
  *           column perm[k] as they were when quantized (after the feedback of
  *           every earlier column).
  *   U, perm, dead  the outputs of gptq_prepare_hinv for this layer's H (any

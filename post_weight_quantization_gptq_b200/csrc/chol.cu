@@ -407,7 +407,8 @@ __device__ __forceinline__ void tri_coords(int t, int& I, int& J) {
 // update, on the chain and beside it, and the inverse's block rows) hand
 // -AB^T to TMA tensor reductions into P and X: the read-modify-write happens
 // in L2 and the SMs issue no global loads or stores for it.  prepare_hinv
-// with them against the direct drain: 1.46 vs 1.66 ms at d = 4096, 4.1 vs
+// with them against a drain in which each lane loaded, updated and stored its
+// own tile row: 1.46 vs 1.66 ms at d = 4096, 4.1 vs
 // 7.5 ms at 8192, 8.9 vs 19.2 ms at 11008, 146 vs 292 ms at 28672.  Full
 // tiles are reduced: the upper part of a diagonal tile of P receives values
 // too, which nothing reads (the diagonal factor loads only j <= i, every GEMM
