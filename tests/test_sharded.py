@@ -114,3 +114,35 @@ def test_gloo_ranks_reproduce_the_unsharded_layer(world, case):
         assert np.array_equal(o["packed"].view(np.uint32), oracle.pack(ref["codes"], bits))
         assert np.array_equal(o["scales"], ref["scales"])
         assert np.array_equal(o["zeros"], ref["zeros"])
+
+
+def _bad_shape_worker(rank, world, port, out):
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import post_weight_quantization_gptq_b200 as g
+    from post_weight_quantization_gptq_b200 import sharded as sh
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        d_row, d_col = 10, 16
+        r0, r1 = sh.row_range(d_row, rank, world)
+        X = torch.zeros(4, d_col, dtype=torch.bfloat16)
+        W = torch.zeros(r1 - r0 + 1, d_col)  # one row too many: rejected before any device work
+        try:
+            sh.quantize_layer_sharded(X, W, d_row, g.GPTQConfig())
+            out[rank] = "accepted"
+        except ValueError as e:
+            out[rank] = "rows [%d, %d)" % (r0, r1) in str(e)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_a_wrong_row_slice_is_rejected_on_the_host():
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_bad_shape_worker, args=(world, _free_port(), out), nprocs=world,
+                       start_method="spawn", join=True)
+    assert out[0] is True and out[1] is True
