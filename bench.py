@@ -183,16 +183,20 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- oracle timing
 def oracle_sample(wl: workloads.Workload, seed_offset: int = 0, n_tokens: int = 2048,
-                  n_rows: int = 32) -> dict:
+                  n_rows: int = 32, n_cols: int | None = None) -> dict:
     """Time the float64 oracle on a bounded sample of the workload and
     extrapolate to one full layer: H over a token sample (scaled by tokens),
-    the full-size inverse and elimination, the column loop on a row sample
-    (scaled by rows; rows are independent given H^-1)."""
+    the inverse and elimination, the column loop on a row sample (scaled by
+    rows; rows are independent given H^-1).  With n_cols below d_col the
+    sample keeps only the first n_cols input channels and each part is scaled
+    by its order in d: H and the column loop d^2, the inverse and the
+    elimination d^3."""
     import oracle
     n_s = min(wl.n_tokens, n_tokens)
     r_s = min(wl.d_row, n_rows)
-    X = workloads.activations(wl, n_tokens=n_s, seed_offset=seed_offset)
-    W = workloads.gaussian_weights(r_s, wl.d_col, wl.w_std, wl.seed)
+    d_s = wl.d_col if n_cols is None else min(wl.d_col, n_cols)
+    X = workloads.activations(wl, n_tokens=n_s, seed_offset=seed_offset)[:, :d_s].contiguous()
+    W = workloads.gaussian_weights(r_s, d_s, wl.w_std, wl.seed)
     t0 = time.perf_counter()
     H = oracle.hessian(X)
     t_h = time.perf_counter() - t0
@@ -207,14 +211,19 @@ def oracle_sample(wl: workloads.Workload, seed_offset: int = 0, n_tokens: int = 
     oracle.gptq_columns(prep["W0"], Minv, wl.bits, wl.group_size)
     t_c = time.perf_counter() - t0
     rows_part = max(t_c - t_e, 0.0)
-    total = t_h * wl.n_tokens / n_s + t_p + t_e + rows_part * wl.d_row / r_s
+    f = wl.d_col / d_s
+    total = (t_h * wl.n_tokens / n_s * f ** 2 + (t_p + t_e) * f ** 3
+             + rows_part * wl.d_row / r_s * f ** 2)
     spent = t_h + t_p + t_e + t_c
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     return dict(value=wl.d_row * wl.d_col / total, seconds_extrapolated=total, spent=spent,
                 cores=cores,
                 sample=(f"oracle (numpy + C, float64, OpenMP) on {n_s} of {wl.n_tokens} tokens for H "
-                        f"(x{wl.n_tokens / n_s:g}), full {wl.d_col}^2 inverse + elimination, column "
-                        f"loop on {r_s} of {wl.d_row} rows (x{wl.d_row / r_s:g}); "
+                        f"(x{wl.n_tokens / n_s:g}), "
+                        + (f"full {wl.d_col}^2 inverse + elimination, " if d_s == wl.d_col else
+                           f"{d_s} of {wl.d_col} input channels (H and the column loop x{f:g}^2, "
+                           f"the {d_s}^2 inverse + elimination x{f:g}^3), ")
+                        + f"column loop on {r_s} of {wl.d_row} rows (x{wl.d_row / r_s:g}); "
                         f"{spent:.1f} s of CPU work"))
 
 
@@ -223,12 +232,15 @@ def run_reference(args, rank: int, world: int):
     if rank != 0:
         return
     wl = workloads.WORKLOADS[args.workload]
+    # per step a bounded sample: at most 2048 input channels, so that the
+    # default 3 + 20 steps end within a few minutes on the host cores
+    n_cols = min(wl.d_col, 2048)
     for _ in range(args.warmup):
-        oracle_sample(wl)
+        oracle_sample(wl, n_cols=n_cols)
     vals, spent = [], 0.0
     last = None
     for _ in range(args.steps):
-        last = oracle_sample(wl)
+        last = oracle_sample(wl, n_cols=n_cols)
         vals.append(last["value"])
         spent += last["spent"]
     value = statistics.mean(vals)
