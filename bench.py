@@ -455,6 +455,9 @@ def run_ours(args, rank: int, world: int, dist):
         "config": _config(wl, world),
         "ms_per_layer": ms_max,
         "hessian_tflops": achieved,
+        # the same launch counted as a dense d x d product (2 n d^2 flop), for
+        # comparison with GEMM figures; the roofline uses the algorithmic count
+        "hessian_tflops_dense_equivalent": 2.0 * n * d * d / (h_ms / 1e3) / 1e12,
         "stage_ms": {"hessian": h_ms, "prepare_hinv": statistics.mean(prep_ms),
                      "quantize_layer": statistics.mean(quant_ms), "pack": statistics.mean(pack_ms)},
         "quantize_only_weights_per_s": r * d / ((ms - h_ms) / 1e3),
