@@ -38,4 +38,5 @@ from .gptq import (  # noqa: F401
     rtn,
     unpack,
     upper_factor,
+    upper_factor_flip,
 )

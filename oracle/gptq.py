@@ -58,10 +58,10 @@ def _lib():
         lib.orc_quantize.argtypes = [ctypes.c_double, ctypes.c_double, ctypes.c_int32, ctypes.c_int]
         lib.orc_quantize.restype = ctypes.c_int32
         lib.orc_gptq_columns.argtypes = [P, i64, i64, P, ctypes.c_int, i64, P, P, P, P,
-                                         P, P, P, P, ctypes.c_double, P, P]
+                                         P, P, P, P, ctypes.c_double, ctypes.c_double, P, P, P]
         lib.orc_gptq_columns.restype = ctypes.c_int
         lib.orc_gptq_columns_u.argtypes = [P, i64, i64, P, ctypes.c_int, i64, P, P, P,
-                                           P, P, P, P, ctypes.c_double, P, P]
+                                           P, P, P, P, ctypes.c_double, ctypes.c_double, P, P, P]
         lib.orc_gptq_columns_u.restype = ctypes.c_int
         lib.orc_eliminate.argtypes = [P, i64, i64, P]
         lib.orc_eliminate.restype = ctypes.c_int
@@ -167,7 +167,8 @@ def prepare(H, W, damp: float = 0.01, desc_act: bool = False) -> dict:
     Hu = Hf[np.ix_(perm, perm)]
     W0 = np.ascontiguousarray(Wf[:, perm])
     lam = damp_lambda(Hu, damp)
-    Hd = Hu + lam * np.eye(d)
+    Hd = Hu.copy()
+    Hd[np.diag_indices(d)] += lam
     return dict(H_undamped=Hu, H_damped=Hd, W0=W0, perm=perm.astype(np.int64),
                 dead=dead, lam=lam)
 
@@ -262,11 +263,24 @@ class GPTQResult:
     w_at_quant: np.ndarray     # r x d: column i as it was when quantized
     U: np.ndarray | None       # eliminated rows / sqrt(pivot), if requested
     stats: dict                # teacher-forcing statistics (zeros if not forced)
+    first_tie: np.ndarray | None = None  # per row: first forced decision that differs (d: none)
+
+
+# Relative scale deviation the teacher-forced check accepts: the tolerance the
+# method's statement of parity gives for scales (1e-4 relative).
+SCALE_TOL = 1e-4
+
+
+def _stats(stats, max_dev) -> dict:
+    return dict(code_ties=int(stats[0]), code_invalid=int(stats[1]),
+                zero_ties=int(stats[2]), zero_invalid=int(stats[3]),
+                elements=int(stats[4]), groups=int(stats[5]), scale_invalid=int(stats[6]),
+                max_dev=max_dev.value)
 
 
 def gptq_columns(W0, Hinv, bits: int, group_size: int, want_U: bool = False,
                  forced_codes=None, forced_zeros=None, forced_w=None, forced_scales=None,
-                 tau: float = 0.0) -> GPTQResult:
+                 tau: float = 0.0, stol: float = SCALE_TOL) -> GPTQResult:
     """The OBQ/GPTQ loop one column at a time with explicit elimination of
     H^-1 after every column [OBQ].
 
@@ -275,9 +289,14 @@ def gptq_columns(W0, Hinv, bits: int, group_size: int, want_U: bool = False,
     adopted, so one tie decided the other way does not desynchronise the rest
     of its row: a code is valid when it is the oracle's own rounding or a
     neighbouring level whose rounding boundary lies within
-    tau + |forced_w - w| / s + |y - z| |forced_s - s| / s of the oracle's real
-    level y = w / s + z (the other side's own deviation in the decision's
-    inputs)."""
+    tau + |forced_w - w| / s + |y - z| min(|forced_s - s| / s, stol) of the
+    oracle's real level y = w / s + z (the other side's own deviation in the
+    decision's inputs).  A forced scale further than stol (relative) from the
+    oracle's counts as invalid; a zero point that differs from the oracle's
+    rounding is valid when the oracle's real zero point lies within the
+    group's drift of the rounding boundary.  first_tie[row] is the first
+    column where a forced decision differs: before it the forced run IS the
+    free-running loop."""
     W = _f64(W0).copy()
     r, d = W.shape
     g = _g(d, group_size)
@@ -291,17 +310,16 @@ def gptq_columns(W0, Hinv, bits: int, group_size: int, want_U: bool = False,
     fz = None if forced_zeros is None else np.ascontiguousarray(forced_zeros, dtype=np.int32)
     fw = None if forced_w is None else _f64(forced_w)
     fs = None if forced_scales is None else _f64(forced_scales)
-    stats = np.zeros(6, dtype=np.int64)
+    stats = np.zeros(7, dtype=np.int64)
+    first = np.zeros(r, dtype=np.int64)
     max_dev = ctypes.c_double(0.0)
     rc = _lib().orc_gptq_columns(_ptr(W), r, d, _ptr(M), bits, g, _ptr(codes), _ptr(scales),
                                  _ptr(zeros), _ptr(U), _ptr(fc), _ptr(fz), _ptr(fw), _ptr(fs),
-                                 float(tau), _ptr(stats), ctypes.byref(max_dev))
+                                 float(tau), float(stol), _ptr(stats), ctypes.byref(max_dev),
+                                 _ptr(first))
     if rc != 0:
         raise np.linalg.LinAlgError(f"oracle column loop failed ({rc})")
-    st = dict(code_ties=int(stats[0]), code_invalid=int(stats[1]),
-              zero_ties=int(stats[2]), zero_invalid=int(stats[3]),
-              elements=int(stats[4]), groups=int(stats[5]), max_dev=max_dev.value)
-    return GPTQResult(codes, scales, zeros, W, U, st)
+    return GPTQResult(codes, scales, zeros, W, U, _stats(stats, max_dev), first)
 
 
 def upper_factor(Hd) -> np.ndarray:
@@ -312,8 +330,27 @@ def upper_factor(Hd) -> np.ndarray:
     return np.ascontiguousarray(np.linalg.cholesky(inverse(Hd)).T)
 
 
+def upper_factor_flip(Hd) -> np.ndarray:
+    """The same U through library routines that need one factorization:
+    with J the exchange matrix and J Hd J = L L^T, U = J L^-1 J (a library
+    Cholesky and a library triangular inverse, float64, working in one
+    Fortran-ordered copy).  Pinned equal to upper_factor and to the
+    elimination rows; used for the largest d, where an explicit inverse
+    costs three times as much."""
+    from scipy.linalg import lapack
+    F = np.array(np.asarray(Hd, dtype=np.float64)[::-1, ::-1], order="F")  # J Hd J
+    c, info = lapack.dpotrf(F, lower=1, clean=1, overwrite_a=1)
+    if info != 0:
+        raise np.linalg.LinAlgError(f"Cholesky failed ({info})")
+    c, info = lapack.dtrtri(c, lower=1, overwrite_c=1)
+    if info != 0:
+        raise np.linalg.LinAlgError(f"triangular inverse failed ({info})")
+    return np.ascontiguousarray(c[::-1, ::-1])  # J L^-1 J, upper triangular
+
+
 def gptq_columns_u(W0, U, bits: int, group_size: int, forced_codes=None, forced_zeros=None,
-                   forced_w=None, forced_scales=None, tau: float = 0.0) -> GPTQResult:
+                   forced_w=None, forced_scales=None, tau: float = 0.0,
+                   stol: float = SCALE_TOL) -> GPTQResult:
     """The OBQ column loop driven by U's rows: W_F <- W_F - (e / U_ii) U_{i,F}
     [OBQ] with row i of the reduced inverse equal to U_ii U[i, i:].  Same
     teacher-forcing options as gptq_columns."""
@@ -329,17 +366,16 @@ def gptq_columns_u(W0, U, bits: int, group_size: int, forced_codes=None, forced_
     fz = None if forced_zeros is None else np.ascontiguousarray(forced_zeros, dtype=np.int32)
     fw = None if forced_w is None else _f64(forced_w)
     fs = None if forced_scales is None else _f64(forced_scales)
-    stats = np.zeros(6, dtype=np.int64)
+    stats = np.zeros(7, dtype=np.int64)
+    first = np.zeros(r, dtype=np.int64)
     max_dev = ctypes.c_double(0.0)
     rc = _lib().orc_gptq_columns_u(_ptr(W), r, d, _ptr(Uc), bits, g, _ptr(codes), _ptr(scales),
                                    _ptr(zeros), _ptr(fc), _ptr(fz), _ptr(fw), _ptr(fs),
-                                   float(tau), _ptr(stats), ctypes.byref(max_dev))
+                                   float(tau), float(stol), _ptr(stats), ctypes.byref(max_dev),
+                                   _ptr(first))
     if rc != 0:
         raise np.linalg.LinAlgError(f"oracle U-row loop failed ({rc})")
-    st = dict(code_ties=int(stats[0]), code_invalid=int(stats[1]),
-              zero_ties=int(stats[2]), zero_invalid=int(stats[3]),
-              elements=int(stats[4]), groups=int(stats[5]), max_dev=max_dev.value)
-    return GPTQResult(codes, scales, zeros, W, None, st)
+    return GPTQResult(codes, scales, zeros, W, None, _stats(stats, max_dev), first)
 
 
 def gptq_blocked(W0, U, bits: int, group_size: int, block: int):

@@ -105,21 +105,26 @@ static int code_is_valid(int32_t c, int32_t q, double y, double tol, int bits)
  *           legitimate tie decided the other way does not desynchronise the
  *           rest of the row.  The validity window of a code widens by the
  *           other side's own deviation in the decision's inputs:
- *           |w' - w| / s + |y - z| |s' - s| / s levels.
+ *           |w' - w| / s + |y - z| min(|s' - s| / s, stol) levels.
  *   tau     slack (in quantization levels) added to every validity window.
- *   stats   out [6]: code ties taken the other way, invalid codes, zero-point
+ *   stol    largest relative scale deviation accepted (a scale further off
+ *           counts as invalid and widens no window beyond stol).
+ *   stats   out [7]: code ties taken the other way, invalid codes, zero-point
  *           ties taken the other way, invalid zero points, elements compared,
- *           groups compared.
+ *           groups compared, invalid scales.
  *   max_dev out: max |fwpre - w| / s over all elements (0 without fwpre).
+ *   first_tie  optional out [r]: per row, the first column whose code or
+ *           (group-opening) zero point differs from the loop's own decision,
+ *           d if none.  Until that column the forced run is the free run.
  */
 int orc_gptq_columns(double *W, int64_t r, int64_t d, double *M, int bits,
                      int64_t g, uint8_t *codes, double *scales, int32_t *zeros,
                      double *U, const uint8_t *fcodes, const int32_t *fzeros,
-                     const double *fwpre, const double *fscales, double tau, int64_t *stats,
-                     double *max_dev)
+                     const double *fwpre, const double *fscales, double tau, double stol,
+                     int64_t *stats, double *max_dev, int64_t *first_tie)
 {
     int64_t s_code_tie = 0, s_code_bad = 0, s_zero_tie = 0, s_zero_bad = 0;
-    int64_t s_elems = 0, s_groups = 0;
+    int64_t s_elems = 0, s_groups = 0, s_scale_bad = 0;
     double dev = 0.0;
     double *cur_s = (double *)malloc(sizeof(double) * (size_t)r);
     int32_t *cur_z = (int32_t *)malloc(sizeof(int32_t) * (size_t)r);
@@ -128,19 +133,25 @@ int orc_gptq_columns(double *W, int64_t r, int64_t d, double *M, int bits,
      * group, against the drift the other side showed on that group's weights */
     double *zwin = (double *)calloc((size_t)r, sizeof(double));
     double *gdev = (double *)calloc((size_t)r, sizeof(double));
-    if (!cur_s || !cur_z || !coef || !zwin || !gdev) {
-        free(cur_s); free(cur_z); free(coef); free(zwin); free(gdev);
+    double *sdev = (double *)calloc((size_t)r, sizeof(double));
+    if (!cur_s || !cur_z || !coef || !zwin || !gdev || !sdev) {
+        free(cur_s); free(cur_z); free(coef); free(zwin); free(gdev); free(sdev);
         return -1;
     }
+    if (first_tie)
+        for (int64_t row = 0; row < r; ++row) first_tie[row] = d;
 
     for (int64_t i = 0; i < d; ++i) {
         const double piv = M[i * d + i];
-        if (!(piv > 0.0)) { free(cur_s); free(cur_z); free(coef); free(zwin); free(gdev); return -2; }
+        if (!(piv > 0.0)) {
+            free(cur_s); free(cur_z); free(coef); free(zwin); free(gdev); free(sdev);
+            return -2;
+        }
         const int64_t grp = i / g;
         const int new_group = (i % g) == 0;
         const int64_t gend = (grp * g + g < d) ? grp * g + g : d; /* end of i's group */
 
-#pragma omp parallel for reduction(+:s_code_tie,s_code_bad,s_zero_tie,s_zero_bad,s_elems,s_groups) reduction(max:dev) schedule(static)
+#pragma omp parallel for reduction(+:s_code_tie,s_code_bad,s_zero_tie,s_zero_bad,s_elems,s_groups,s_scale_bad) reduction(max:dev) schedule(static)
         for (int64_t row = 0; row < r; ++row) {
             double *w = W + row * d;
             if (new_group) {
@@ -149,12 +160,19 @@ int orc_gptq_columns(double *W, int64_t r, int64_t d, double *M, int bits,
                 double s, zr;
                 int32_t z;
                 orc_quant_params(w + i, gend - i, bits, &s, &zr, &z);
+                if (fscales) {
+                    const double ds = fabs(fscales[grp * r + row] - s) / s;
+                    if (ds > stol) ++s_scale_bad;
+                    sdev[row] = ds < stol ? ds : stol;
+                }
                 if (fzeros) {
                     int32_t zf = fzeros[grp * r + row];
                     /* distance past the rounding window, judged at group end */
                     zwin[row] = (zf != z) ? fabs((double)zf - zr) - 0.5 - tau : -1.0;
-                    if (zf != z && fscales)
-                        zwin[row] -= fabs(zr) * fabs(fscales[grp * r + row] - s) / s;
+                    if (zf != z) {
+                        zwin[row] -= fabs(zr) * sdev[row];
+                        if (first_tie && first_tie[row] > i) first_tie[row] = i;
+                    }
                     gdev[row] = 0.0;
                     z = zf;
                     ++s_groups;
@@ -177,11 +195,12 @@ int orc_gptq_columns(double *W, int64_t r, int64_t d, double *M, int bits,
                     if (dv > gdev[row]) gdev[row] = dv;
                     tol += dv;
                 }
-                if (fscales) tol += fabs(y - (double)z) * fabs(fscales[grp * r + row] - s) / s;
+                tol += fabs(y - (double)z) * sdev[row];
                 int32_t c = (int32_t)fcodes[row * d + i];
                 if (c != q) {
                     if (code_is_valid(c, q, y, tol, bits)) ++s_code_tie;
                     else ++s_code_bad;
+                    if (first_tie && first_tie[row] > i) first_tie[row] = i;
                 }
                 q = c;
                 ++s_elems;
@@ -226,10 +245,10 @@ int orc_gptq_columns(double *W, int64_t r, int64_t d, double *M, int bits,
     if (stats) {
         stats[0] = s_code_tie; stats[1] = s_code_bad;
         stats[2] = s_zero_tie; stats[3] = s_zero_bad;
-        stats[4] = s_elems; stats[5] = s_groups;
+        stats[4] = s_elems; stats[5] = s_groups; stats[6] = s_scale_bad;
     }
     if (max_dev) *max_dev = dev;
-    free(cur_s); free(cur_z); free(coef); free(zwin); free(gdev);
+    free(cur_s); free(cur_z); free(coef); free(zwin); free(gdev); free(sdev);
     return 0;
 }
 
@@ -245,18 +264,21 @@ int orc_gptq_columns(double *W, int64_t r, int64_t d, double *M, int bits,
 int orc_gptq_columns_u(double *W, int64_t r, int64_t d, const double *U, int bits, int64_t g,
                        uint8_t *codes, double *scales, int32_t *zeros,
                        const uint8_t *fcodes, const int32_t *fzeros, const double *fwpre,
-                       const double *fscales, double tau, int64_t *stats, double *max_dev)
+                       const double *fscales, double tau, double stol, int64_t *stats,
+                       double *max_dev, int64_t *first_tie)
 {
     int64_t s_code_tie = 0, s_code_bad = 0, s_zero_tie = 0, s_zero_bad = 0;
-    int64_t s_elems = 0, s_groups = 0;
+    int64_t s_elems = 0, s_groups = 0, s_scale_bad = 0;
     double dev = 0.0;
     int rc = 0;
-#pragma omp parallel for reduction(+:s_code_tie,s_code_bad,s_zero_tie,s_zero_bad,s_elems,s_groups) reduction(max:dev) schedule(dynamic, 1)
+#pragma omp parallel for reduction(+:s_code_tie,s_code_bad,s_zero_tie,s_zero_bad,s_elems,s_groups,s_scale_bad) reduction(max:dev) schedule(dynamic, 1)
     for (int64_t row = 0; row < r; ++row) {
         double *w = W + row * d;
         double s = 1.0;
         int32_t z = 0;
         double zwin = -1.0, gdv = 0.0; /* pending zero-point check, group drift */
+        double sdv = 0.0;              /* the group's scale deviation, capped at stol */
+        if (first_tie) first_tie[row] = d;
         for (int64_t i = 0; i < d; ++i) {
             const double uii = U[i * d + i];
             if (!(uii > 0.0)) { rc = -2; break; }
@@ -264,11 +286,18 @@ int orc_gptq_columns_u(double *W, int64_t r, int64_t d, const double *U, int bit
                 const int64_t gend = (i + g < d) ? i + g : d;
                 double zr;
                 orc_quant_params(w + i, gend - i, bits, &s, &zr, &z);
+                if (fscales) {
+                    const double ds = fabs(fscales[(i / g) * r + row] - s) / s;
+                    if (ds > stol) ++s_scale_bad;
+                    sdv = ds < stol ? ds : stol;
+                }
                 if (fzeros) {
                     int32_t zf = fzeros[(i / g) * r + row];
                     zwin = (zf != z) ? fabs((double)zf - zr) - 0.5 - tau : -1.0;
-                    if (zf != z && fscales)
-                        zwin -= fabs(zr) * fabs(fscales[(i / g) * r + row] - s) / s;
+                    if (zf != z) {
+                        zwin -= fabs(zr) * sdv;
+                        if (first_tie && first_tie[row] > i) first_tie[row] = i;
+                    }
                     gdv = 0.0;
                     z = zf;
                     ++s_groups;
@@ -287,11 +316,12 @@ int orc_gptq_columns_u(double *W, int64_t r, int64_t d, const double *U, int bit
                     if (dv > gdv) gdv = dv;
                     tol += dv;
                 }
-                if (fscales) tol += fabs(y - (double)z) * fabs(fscales[(i / g) * r + row] - s) / s;
+                tol += fabs(y - (double)z) * sdv;
                 int32_t c = (int32_t)fcodes[row * d + i];
                 if (c != q) {
                     if (code_is_valid(c, q, y, tol, bits)) ++s_code_tie;
                     else ++s_code_bad;
+                    if (first_tie && first_tie[row] > i) first_tie[row] = i;
                 }
                 q = c;
                 ++s_elems;
@@ -310,7 +340,7 @@ int orc_gptq_columns_u(double *W, int64_t r, int64_t d, const double *U, int bit
     if (stats) {
         stats[0] = s_code_tie; stats[1] = s_code_bad;
         stats[2] = s_zero_tie; stats[3] = s_zero_bad;
-        stats[4] = s_elems; stats[5] = s_groups;
+        stats[4] = s_elems; stats[5] = s_groups; stats[6] = s_scale_bad;
     }
     if (max_dev) *max_dev = dev;
     return rc;

@@ -3,11 +3,12 @@
 // D[128 x 128] = sum_k A[m][k] B[n][k] with fp32 operands split as
 // x = hi + lo, and three kind::tf32 MMAs accumulate hi*hi + hi*lo + lo*hi
 // into one fp32 TMEM accumulator.  kind::tf32 reads a 32-bit operand and
-// ignores its 13 low mantissa bits (truncation, measured on sm_100a), so hi
-// is the fp32 value as TMA delivered it and only lo = x - trunc13(x) (exact
-// in fp32) is written, into a second buffer.  The tensor core truncates lo in
-// turn; that and the dropped lo*lo term leave an error of about 2^-20 of
-// |a||b| per product, close to fp32 FFMA, at tensor-core speed.
+// ignores its 13 low mantissa bits (truncation, measured on sm_100a).  Two
+// splits (see kSplitTrunc / kSplitRound below): hi as TMA delivered it and
+// lo = x - trunc13(x) (one buffer written per operand, products within about
+// 2^-20 of |a||b|, biased towards zero), or hi and lo both rounded to the
+// nearest tf32 (two buffers written, products within about 3 2^-22 of |a||b|
+// and unbiased), at tensor-core speed either way.
 //
 // Persistent: each CTA walks a static list of output tiles (tile, tile +
 // grid, ...), the stage ring runs on across tiles and two TMEM accumulators
@@ -18,7 +19,7 @@
 // with 32-byte chunks).  Warp roles:
 //   warp 0      TMA producer
 //   warp 1      TMEM owner and MMA issuer
-//   warps 2..5  write each stage's lo parts
+//   warps 2..5  split each stage's operands (write lo, and hi when rounding)
 //   warps 6..9  drain the accumulator (tcgen05.ld gives one tile row per
 //               lane).  Plain outputs receive the product, read-modify-write
 //               outputs (kRmw) D -= AB^T.  Three forms:
@@ -93,6 +94,30 @@ __device__ __forceinline__ float tf32_rest(float x) {
     return x - __uint_as_float(__float_as_uint(x) & 0xffffe000u);
 }
 
+// x rounded to the nearest tf32 value (ties away from zero): adding half of
+// the 13 dropped bits' range to the bit pattern carries into the kept
+// mantissa (and, at the top of a binade, into the exponent) exactly when the
+// dropped part is at least half a tf32 ulp.  Finite inputs only.
+__device__ __forceinline__ float tf32_round(float x) {
+    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xffffe000u);
+}
+__device__ __forceinline__ float4 tf32_round4(float4 v) {
+    return make_float4(tf32_round(v.x), tf32_round(v.y), tf32_round(v.z), tf32_round(v.w));
+}
+__device__ __forceinline__ float4 sub4(float4 a, float4 b) {
+    return make_float4(a.x - b.x, a.y - b.y, a.z - b.z, a.w - b.w);
+}
+
+// Operand splits.  kSplitTrunc: hi is the value as loaded (the MMA truncates
+// it), lo = the truncated-off remainder, which the MMA truncates in turn:
+// only lo is written, but every product loses up to ~2^-20 of |ab|, always
+// towards zero, so long sums drift one way.  kSplitRound: hi = x rounded to
+// the nearest tf32, lo = the (exact) remainder rounded to the nearest tf32,
+// both written: x - hi - lo is within 2^-22 |x| and of either sign, so a
+// product's error (that, the two roundings and the dropped lo lo term) stays
+// within ~3 2^-22 |ab| and long sums do not drift.
+constexpr int kSplitTrunc = 0, kSplitRound = 1;
+
 
 
 template <bool MN>
@@ -118,7 +143,7 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk) {
 }
 
 
-template <class Sched, bool A_MN, bool B_MN, int Epi>
+template <class Sched, bool A_MN, bool B_MN, int Epi, int Split>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
                        const __grid_constant__ CUtensorMap tmd, const Sched sched, int tiles,
@@ -247,15 +272,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                const float4* a = reinterpret_cast<const float4*>(smem + st * kStageBytes);
-                float4* alo = const_cast<float4*>(a) + kTileBytes / 16;
-                const float4* b = a + 2 * (kTileBytes / 16);
-                float4* blo = const_cast<float4*>(a) + 3 * (kTileBytes / 16);
+                float4* a = reinterpret_cast<float4*>(smem + st * kStageBytes);
+                float4* alo = a + kTileBytes / 16;
+                float4* b = a + 2 * (kTileBytes / 16);
+                float4* blo = a + 3 * (kTileBytes / 16);
 #pragma unroll 4
                 for (int i = t0; i < kTileBytes / 16; i += 128) {
                     const float4 x = a[i], y = b[i];
-                    alo[i] = make_float4(tf32_rest(x.x), tf32_rest(x.y), tf32_rest(x.z), tf32_rest(x.w));
-                    blo[i] = make_float4(tf32_rest(y.x), tf32_rest(y.y), tf32_rest(y.z), tf32_rest(y.w));
+                    if constexpr (Split == kSplitRound) {
+                        const float4 xh = tf32_round4(x), yh = tf32_round4(y);
+                        a[i] = xh;
+                        b[i] = yh;
+                        alo[i] = tf32_round4(sub4(x, xh));
+                        blo[i] = tf32_round4(sub4(y, yh));
+                    } else {
+                        alo[i] = make_float4(tf32_rest(x.x), tf32_rest(x.y), tf32_rest(x.z), tf32_rest(x.w));
+                        blo[i] = make_float4(tf32_rest(y.x), tf32_rest(y.y), tf32_rest(y.z), tf32_rest(y.w));
+                    }
                 }
                 fence_async_smem();
                 mbar_arrive(&bars->conv[st]);
@@ -414,11 +447,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 // pdl: launched with programmatic serialization (see launch_kernel).
 // td: the destination's tensor map (box 32 x 32 fp32, 128-byte swizzle) for
 // the reduce drain; unused by the other forms.
-template <class Sched, bool A_MN, bool B_MN, int Epi>
+template <class Sched, bool A_MN, bool B_MN, int Epi, int Split = kSplitRound>
 inline cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const Sched& sched,
                           int tiles, int32_t* status, cudaStream_t stream, int sms,
                           bool pdl = false, const CUtensorMap* td = nullptr) {
-    auto kern = gemm_tf32x3_kernel<Sched, A_MN, B_MN, Epi>;
+    auto kern = gemm_tf32x3_kernel<Sched, A_MN, B_MN, Epi, Split>;
     if (Epi >= kEpiReduce && td == nullptr) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          smem_bytes<Epi>());

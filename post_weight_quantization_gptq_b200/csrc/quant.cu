@@ -523,11 +523,13 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
         LazySched ls{W, ldw, static_cast<int>(d_row), static_cast<int>(cend), static_cast<int>(c1), mt,
                      (a - run0) * kBlock, a * kBlock, (c - a) * (kBlock / 32)};
         ++launches;
-        return (w_tma ? g3::launch<LazySched, false, true, g3::kEpiReduce>(tErr, tUmn, ls, mt * nt, status,
-                                                                          stream, sms, true, &tW)
-                      : g3::launch<LazySched, false, true, g3::kEpiStaged>(tErr, tUmn, ls, mt * nt, status,
-                                                                          stream, sms, true)) ==
-               cudaSuccess;
+        // truncating split: the walk given the same U matches the float64
+        // loop as closely with it as with the rounding split, which costs the
+        // split warps a second store per operand
+        return (w_tma ? g3::launch<LazySched, false, true, g3::kEpiReduce, g3::kSplitTrunc>(
+                            tErr, tUmn, ls, mt * nt, status, stream, sms, true, &tW)
+                      : g3::launch<LazySched, false, true, g3::kEpiStaged, g3::kSplitTrunc>(
+                            tErr, tUmn, ls, mt * nt, status, stream, sms, true)) == cudaSuccess;
     };
     // blocks [lo, hi) of the current run, complete w.r.t. every block < lo
     std::vector<std::tuple<int, int, int>> stack;

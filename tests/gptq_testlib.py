@@ -13,11 +13,23 @@ fp32 arithmetic of the kernels):
   code is therefore checked for validity by the oracle's column loop run in
   teacher-forcing mode: it must be the oracle's own rounding, or the other
   neighbour of a boundary that lies within |w_gpu - w_oracle| / s +
-  |y - z| |s_gpu - s_oracle| / s + tau of the oracle's value y = w / s + z
-  (w_gpu is the GPU's pre-quantization weight, returned in W): a decision is
-  valid when the GPU's own inputs to it justify it.  At most 0.1 % of the codes may take such a tie the other way
-  (>= 99.9 % identical) and none may be invalid.
+  |y - z| min(|s_gpu - s_oracle| / s, 1e-4) + tau of the oracle's value
+  y = w / s + z (w_gpu is the GPU's pre-quantization weight, returned in W):
+  a decision is valid when the GPU's own inputs to it justify it.  At most
+  0.1 % of the codes may take such a tie the other way (>= 99.9 % identical,
+  the rest +-1 level) and none may be invalid.
+* free running: in every row the GPU's codes equal the unforced oracle's up
+  to the row's first such tie (rows without one: entirely).  After a tie the
+  two rows follow different (both valid) trajectories: one flipped code
+  changes the error fed to every later column, and the flip can cascade.
+  The free-running agreement is printed; with strict_free (the small cases)
+  it must also reach 99.9 %.  Inside a cascade a code may end up two levels
+  from the oracle's, and at full size a cascade can reach a fifth of a row,
+  so there the rate is measured and reported, not asserted.
 * scales: relative error <= 1e-4 against the teacher-forced oracle.
+* weight drift |w_gpu - w_oracle| / s <= 1e-2 levels (largest measured:
+  3.2e-3 at d = 11008 with cond(H) ~ 6e5); a typical drift d makes about 2 d
+  of the codes ties, so this keeps the tie budget of 0.1 % far away.
 * proxy loss tr((W - Q) H (W - Q)^T): within 0.5 % of the free-running
   oracle's.
 """
@@ -50,6 +62,17 @@ def gpu_hessian(X_cpu: torch.Tensor, chunks: int = 1, ldx: int | None = None) ->
         g.gptq_hessian_accumulate(Xd[a:b], H, st)
     assert g.gptq_sync_status(st) == 0
     return H.cpu().numpy()
+
+
+def u_rows_rel_err(Ug, Uo: np.ndarray, rows) -> float:
+    """Largest deviation of the GPU's U on the given rows, relative to each
+    row's largest oracle entry (Ug may be a torch tensor on any device)."""
+    worst = 0.0
+    for i in rows:
+        i = int(i)
+        g = Ug[i].double().cpu().numpy() if hasattr(Ug, "double") else np.asarray(Ug[i], np.float64)
+        worst = max(worst, float(np.abs(g - Uo[i]).max() / np.abs(Uo[i]).max()))
+    return worst
 
 
 def lower_rel_err(Hg: np.ndarray, Ho: np.ndarray) -> float:
@@ -87,10 +110,12 @@ def gpu_quantize(H_fp32: np.ndarray, W: torch.Tensor, bits: int, group_size: int
 
 def compare_quantization(H64: np.ndarray, W: torch.Tensor, out: dict, bits: int,
                          group_size: int, desc_act: bool, damp: float = 0.01,
-                         rows=None, H_loss: np.ndarray | None = None) -> dict:
+                         rows=None, H_loss: np.ndarray | None = None,
+                         strict_free: bool = True, U_oracle: np.ndarray | None = None) -> dict:
     """Check one GPU quantization against the oracle run on H64 (the exact H
     the GPU was given, as float64).  `rows` restricts the column loop to a
-    sample of rows.  Returns the measured statistics."""
+    sample of rows.  `U_oracle` (float64) may pass a precomputed inverse
+    factor of the damped H for large d.  Returns the measured statistics."""
     prep = oracle.prepare(H64, W, damp=damp, desc_act=desc_act)
     assert out["status"] == 0, out["status"]
     assert np.array_equal(out["perm"], prep["perm"]), "act-order permutation differs"
@@ -100,24 +125,32 @@ def compare_quantization(H64: np.ndarray, W: torch.Tensor, out: dict, bits: int,
     codes, zeros = out["codes"][sel], out["zeros"][:, sel]
     wq, scales = out["w_at_quant"][sel], out["scales"][:, sel]
     d = W0.shape[1]
-    if d <= 4096:
+    forced_args = dict(forced_codes=codes, forced_zeros=zeros, forced_w=wq,
+                       forced_scales=scales, tau=TAU)
+    if d <= 4096 and U_oracle is None:
         # the definition: explicit per-column elimination of H^-1
         Minv = oracle.inverse(prep["H_damped"])
-        forced = oracle.gptq_columns(W0, Minv, bits, group_size, forced_codes=codes,
-                                     forced_zeros=zeros, forced_w=wq, forced_scales=scales,
-                                     tau=TAU)
+        forced = oracle.gptq_columns(W0, Minv, bits, group_size, **forced_args)
         free = oracle.gptq_columns(W0, Minv, bits, group_size)
     else:
         # too slow to eliminate on the host: the same loop driven by U's rows
-        # (U from a library Cholesky of the library inverse; pinned equal)
-        U = oracle.upper_factor(prep["H_damped"])
-        forced = oracle.gptq_columns_u(W0, U, bits, group_size, forced_codes=codes,
-                                       forced_zeros=zeros, forced_w=wq, forced_scales=scales,
-                                       tau=TAU)
+        # (U from a library Cholesky and triangular inverse; pinned equal)
+        U = oracle.upper_factor_flip(prep["H_damped"]) if U_oracle is None else U_oracle
+        forced = oracle.gptq_columns_u(W0, U, bits, group_size, **forced_args)
         free = oracle.gptq_columns_u(W0, U, bits, group_size)
     st = forced.stats
     free_match = float(np.mean(free.codes == codes))
     free_maxdiff = int(np.abs(free.codes.astype(int) - codes.astype(int)).max())
+    tied_rows = int(np.sum(forced.first_tie < d))
+    # the free-running loop is the forced loop until the row's first tie
+    for r in range(len(sel)):
+        ft = int(forced.first_tie[r])
+        assert np.array_equal(codes[r, :ft], free.codes[r, :ft]), (r, ft)
+    walk_match = None
+    if out.get("U") is not None:
+        # the column walk alone: the oracle given the GPU's own U
+        walk = oracle.gptq_columns_u(W0, out["U"], bits, group_size)
+        walk_match = float(np.mean(walk.codes == codes))
     srel = float(np.max(np.abs(scales - forced.scales) / np.abs(forced.scales)))
     Hl = prep["H_undamped"] if H_loss is None else H_loss
     Qg = oracle.dequantize(codes, scales, zeros, group_size)
@@ -128,17 +161,22 @@ def compare_quantization(H64: np.ndarray, W: torch.Tensor, out: dict, bits: int,
     loss_rtn = oracle.proxy_loss(W0, oracle.dequantize(rc, rs, rz, group_size), Hl)
     res = dict(code_ties=st["code_ties"], code_invalid=st["code_invalid"],
                zero_ties=st["zero_ties"], zero_invalid=st["zero_invalid"],
+               scale_invalid=st["scale_invalid"],
                elements=st["elements"], tie_frac=st["code_ties"] / max(1, st["elements"]),
                max_dev=st["max_dev"], scale_rel=srel, free_match=free_match,
-               free_maxdiff=free_maxdiff, loss_gpu=loss_g, loss_oracle=loss_o,
+               free_maxdiff=free_maxdiff, tied_rows=tied_rows, rows=len(sel),
+               walk_match=walk_match, loss_gpu=loss_g, loss_oracle=loss_o,
                loss_rtn=loss_rtn, loss_rel=abs(loss_g - loss_o) / loss_o)
     print("parity:", {k: (round(v, 8) if isinstance(v, float) else v) for k, v in res.items()})
     assert st["code_invalid"] == 0, res
     assert st["zero_invalid"] == 0, res
+    assert st["scale_invalid"] == 0, res
     assert res["tie_frac"] <= 1e-3, res
     assert srel <= 1e-4, res
-    assert res["max_dev"] <= 0.05, res
+    assert res["max_dev"] <= 1e-2, res
     assert res["loss_rel"] <= 5e-3, res
+    if strict_free:
+        assert free_match >= 0.999, res
     assert codes.max() <= (1 << bits) - 1
     assert np.array_equal(out["packed"][sel], oracle.pack(codes, bits))
     return res

@@ -168,6 +168,10 @@ def test_elimination_rows_are_the_upper_cholesky_factor_of_the_inverse(d):
     J = np.eye(d)[::-1]
     flip = J @ np.linalg.inv(np.linalg.cholesky(J @ H @ J)) @ J
     assert np.abs(U - flip).max() <= 1e-10 * np.abs(U).max()
+    # the oracle's two library routes to U
+    assert np.abs(U - oracle.upper_factor(H)).max() <= 1e-10 * np.abs(U).max()
+    assert np.abs(U - oracle.upper_factor_flip(H)).max() <= 1e-10 * np.abs(U).max()
+    assert np.all(np.tril(oracle.upper_factor_flip(H), -1) == 0.0)
 
 
 # ------------------------------------------------------------- the OBQ step
@@ -317,10 +321,13 @@ def test_teacher_forcing_accepts_itself_and_flags_a_planted_error():
     Minv = oracle.inverse(H)
     ref = oracle.gptq_columns(W0, Minv, 4, 16)
     same = oracle.gptq_columns(W0, Minv, 4, 16, forced_codes=ref.codes,
-                               forced_zeros=ref.zeros, forced_w=ref.w_at_quant)
+                               forced_zeros=ref.zeros, forced_w=ref.w_at_quant,
+                               forced_scales=ref.scales)
     assert same.stats["code_ties"] == 0 and same.stats["code_invalid"] == 0
     assert same.stats["zero_invalid"] == 0 and same.stats["max_dev"] == 0.0
+    assert same.stats["scale_invalid"] == 0
     assert same.stats["elements"] == 10 * d
+    assert np.all(same.first_tie == d)
     bad = ref.codes.copy()
     rows, cols = np.nonzero((ref.codes > 0) & (ref.codes < 15))
     row, col = int(rows[0]), int(cols[0])
@@ -329,6 +336,81 @@ def test_teacher_forcing_accepts_itself_and_flags_a_planted_error():
     bad[row, col] = q - 1 if y >= q else q + 1   # one level away from y's side
     planted = oracle.gptq_columns(W0, Minv, 4, 16, forced_codes=bad, forced_zeros=ref.zeros)
     assert planted.stats["code_invalid"] >= 1
+    assert planted.first_tie[row] == col
+    # a scale off by far more than the 1e-4 tolerance does not open the code
+    # windows: the planted code stays invalid, and the scale itself is flagged
+    wide = ref.scales * 1.5
+    planted = oracle.gptq_columns(W0, Minv, 4, 16, forced_codes=bad, forced_zeros=ref.zeros,
+                                  forced_w=ref.w_at_quant, forced_scales=wide)
+    assert planted.stats["code_invalid"] >= 1
+    assert planted.stats["scale_invalid"] == ref.scales.size
+
+
+@pytest.mark.parametrize("loop", ["eliminated", "u_rows"])
+def test_teacher_forcing_flags_a_planted_scale(loop):
+    """A forced scale within the 1e-4 relative tolerance passes; one group's
+    scale off by 1e-3 is flagged (by both loops)."""
+    rng = np.random.default_rng(21)
+    d = 64
+    H = _spd(d, 4, cond_spread=0.5)
+    W0 = rng.standard_normal((6, d)) * 0.02
+
+    def run(**kw):
+        if loop == "eliminated":
+            return oracle.gptq_columns(W0, oracle.inverse(H), 4, 16, **kw)
+        return oracle.gptq_columns_u(W0, oracle.upper_factor(H), 4, 16, **kw)
+
+    ref = run()
+    close = ref.scales * (1.0 + 1e-5)
+    ok = run(forced_codes=ref.codes, forced_zeros=ref.zeros, forced_w=ref.w_at_quant,
+             forced_scales=close)
+    assert ok.stats["scale_invalid"] == 0 and ok.stats["code_invalid"] == 0
+    off = ref.scales.copy()
+    off[2, 3] *= 1.0 + 1e-3
+    bad = run(forced_codes=ref.codes, forced_zeros=ref.zeros, forced_w=ref.w_at_quant,
+              forced_scales=off)
+    assert bad.stats["scale_invalid"] == 1
+
+
+@pytest.mark.parametrize("loop", ["eliminated", "u_rows"])
+def test_teacher_forcing_judges_a_planted_zero_point(loop):
+    """Zero points: with H diagonal there is no feedback, so one row's group
+    of values -a .. b gives s = (a + b) / 15 and the real zero point
+    15 a / (a + b) exactly as built.  (1) A zero point one level away from a
+    real zero point far from a rounding boundary is invalid.  (2) A real zero
+    point 2e-4 levels past the boundary 7.5 rounds to 8; the forced 7 is
+    invalid when the other side's weights show no drift, and a legitimate
+    tie when they drift by 1e-3 levels (more than the 2e-4 miss)."""
+    d = 16
+    H = np.eye(d) * 3.0
+
+    def run(W0, **kw):
+        if loop == "eliminated":
+            return oracle.gptq_columns(W0, oracle.inverse(H), 4, d, **kw)
+        return oracle.gptq_columns_u(W0, oracle.upper_factor(H), 4, d, **kw)
+
+    # (1) a = 0.2, b = 0.8: the real zero point 3.0 sits half a level from either boundary
+    w = np.linspace(-0.2, 0.8, d)[None, :]
+    ref = run(w)
+    zr = 15 * 0.2 / 1.0
+    assert ref.zeros[0, 0] == round(zr) == 3
+    planted = run(w, forced_codes=ref.codes, forced_zeros=ref.zeros + 1, forced_w=w)
+    assert planted.stats["zero_invalid"] == 1 and planted.stats["zero_ties"] == 0
+    assert planted.first_tie[0] == 0
+    # (2) a real zero point 2e-4 levels past 7.5
+    eps = 2e-4 / 15.0
+    a, b = 0.5 + eps, 0.5 - eps
+    w = np.linspace(-a, b, d)[None, :]
+    ref = run(w)
+    assert ref.zeros[0, 0] == 8
+    s = ref.scales[0, 0]
+    forced = np.clip(np.rint(w / s) + 7, 0, 15).astype(np.uint8)
+    no_drift = run(w, forced_codes=forced, forced_zeros=ref.zeros - 1, forced_w=w)
+    assert no_drift.stats["zero_invalid"] == 1
+    drift = w.copy()
+    drift[0, 5] += 1e-3 * s
+    tie = run(w, forced_codes=forced, forced_zeros=ref.zeros - 1, forced_w=drift)
+    assert tie.stats["zero_invalid"] == 0 and tie.stats["zero_ties"] == 1
 
 
 @pytest.mark.parametrize("d,g", [(64, 16), (200, 32), (256, -1)])

@@ -166,6 +166,23 @@ LLAMA7B_BLOCK = [
 ]
 LLAMA7B_BLOCK_SOURCES = {"attn_in": 4096, "o_in": 4096, "mlp_in": 4096, "down_in": 11008}
 LLAMA7B_BLOCK_QUANT = dict(bits=3, group_size=128, desc_act=False, damp=0.01)
+_BLOCK_SOURCE_SEED = {"attn_in": 3, "o_in": 5, "mlp_in": 6, "down_in": 8}
+
+
+def block_activations(source: str, n_tokens: int = 128 * 2048, device="cpu") -> torch.Tensor:
+    """Calibration input of one Llama-7B block source (Student-t(4), 1 % of
+    the channels x50): attn_in feeds q/k/v, o_in o_proj, mlp_in gate/up,
+    down_in down_proj."""
+    d = LLAMA7B_BLOCK_SOURCES[source]
+    return student_t_activations(n_tokens, d, seed=BASE_SEED + _BLOCK_SOURCE_SEED[source],
+                                 device=device)
+
+
+def block_weights(name: str, device="cpu") -> torch.Tensor:
+    """W of one Llama-7B block weight (LLAMA7B_BLOCK row), N(0, std^2)."""
+    j = [b[0] for b in LLAMA7B_BLOCK].index(name)
+    _, rows, cols, _, std = LLAMA7B_BLOCK[j]
+    return gaussian_weights(rows, cols, std, seed=BASE_SEED + 3 + 101 * j, device=device)
 
 
 def activations(w: Workload, device="cpu", n_tokens: int | None = None,
