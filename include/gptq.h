@@ -89,6 +89,22 @@ int32_t gptq_version(void);
 int64_t gptq_launch_counter(void);
 
 /*
+ * Test hook for the bounded device-side waits (the pages have no counterpart;
+ * it exists so the timeout path can be exercised without a faulty GPU).
+ * Arms the NEXT launch of one kernel kind -- 1: the Hessian GEMM of
+ * gptq_hessian_accumulate; 2: the next fp32-accurate tensor-core GEMM of any
+ * call (gptq_prepare_hinv's first one is its first panel solve) -- so that
+ * its MMA-issuing thread first waits, bounded by limit_ns (1 .. 10^9), on a
+ * barrier that nothing completes.  That wait runs out like any other: the
+ * kernel lets its issued copies and MMAs land (normal limit), frees its
+ * tensor memory, writes GPTQ_ERR_TIMEOUT to the call's dev_status and
+ * returns; the call's outputs are then not valid, later calls are
+ * unaffected.  One launch consumes the arming.  Never needed in normal use.
+ * Errors: GPTQ_ERR_INVALID_ARG for another kernel number or limit.
+ */
+gptq_status gptq_debug_arm_wait_probe(int32_t kernel, int64_t limit_ns);
+
+/*
  * Workspace bytes needed by gptq_hessian_accumulate, gptq_prepare_hinv and
  * gptq_quantize_layer for a layer of d_row x d_col with this config (the
  * maximum over the three, so one workspace serves all of them).
@@ -171,7 +187,9 @@ size_t gptq_hessian_staging_size(int64_t d, int64_t chunk_tokens);
  *         diag(H), ties by lower index).
  *   dead  uint8[d] output: 1 where diag(H) == 0 (that column is treated as
  *         H_ii = 1 and its weights as 0).
- *   Device errors: GPTQ_ERR_NOT_PD if a Cholesky pivot is not positive.
+ *   Device errors: GPTQ_ERR_NOT_PD if a Cholesky pivot is not positive, or
+ *   if a diagonal entry of H is not finite (NaN or infinite; perm is then
+ *   still a permutation, with such columns ranked last under desc_act).
  */
 gptq_status gptq_prepare_hinv(float *H, int64_t d, int64_t ldh, const gptq_config *cfg,
                               float *U, int32_t *perm, uint8_t *dead, int32_t *dev_status,
@@ -186,7 +204,9 @@ gptq_status gptq_prepare_hinv(float *H, int64_t d, int64_t ldh, const gptq_confi
  *           every earlier column).
  *   U, perm, dead  the outputs of gptq_prepare_hinv for this layer's H (any
  *           number of layers sharing one H may reuse them), with the same
- *           desc_act: without act-order perm is the identity and is not read.  d_col must be a
+ *           desc_act: without act-order perm is the identity and is not read.
+ *           A perm entry outside [0, d_col) is reported on the device as
+ *           GPTQ_ERR_INVALID_ARG (and read as the identity).  d_col must be a
  *           multiple of 4 (GPTQ_ERR_UNSUPPORTED otherwise) and at most 57344.
  *   codes   d_row x d_col uint8, contiguous: codes[row][k] is the code of
  *           original column perm[k].
@@ -213,10 +233,19 @@ gptq_status gptq_quantize_layer(float *W, int64_t d_row, int64_t d_col, int64_t 
  *   that loads the library until the process exits; no allocation is made.
  *   Limit: a layer whose gptq_quantize_layer workspace would exceed that
  *   array (currently d_row * 512 bytes, i.e. d_row <= 32768) is rejected with
- *   GPTQ_ERR_WORKSPACE before anything is launched.
+ *   GPTQ_ERR_WORKSPACE before anything is launched.  The lazy update defers
+ *   the errors of up to 8 blocks of 128 columns in the array (d_row * 512
+ *   bytes each); above d_row = 4096 it defers fewer (4 up to 8192, 2 up to
+ *   16384, 1 up to 32768), exactly as gptq_quantize_layer does with a 16 MiB
+ *   workspace: the same sums grouped into more, shorter products.
+ *   Device: the array used is the current device's, so W, U, perm (with
+ *   act-order), dead, codes, scales, zeros and dev_status must be memory of
+ *   the current device (or managed memory); otherwise GPTQ_ERR_INVALID_ARG
+ *   is returned before anything is launched.
  *   Set-up: the first call on each device (with that device current) looks
- *   up the array's device address and caches it; make that first call before
- *   any stream capture on the device.
+ *   up the array's device address and caches it with the device's current
+ *   context (a call in a new context, e.g. after cudaDeviceReset, looks it
+ *   up again); make that first call before any stream capture on the device.
  *   Sharing: every call uses the same array, which keeps the last call's
  *   contents; nothing in it needs to start at zero.  Calls whose work overlaps
  *   on the GPU (e.g. on two unordered streams) race on the array: order them.
@@ -255,7 +284,8 @@ gptq_status gptq_pack(const uint8_t *codes, int64_t d_row, int64_t d_col, int32_
  *   scales, zeros  fp32 / int32 [ceil(d_col / g)][d_row], as
  *           gptq_quantize_layer writes them.
  *   perm    int32[d_col] from gptq_prepare_hinv (quantization position k holds
- *           original column perm[k]); NULL means the identity.
+ *           original column perm[k]); NULL means the identity.  An entry
+ *           outside [0, d_col) is read as k (no access leaves the row).
  *   Y       n_tok x d_row fp32, leading dimension ldy >= d_row (overwritten):
  *           Y[t][n] = sum_k X[t][perm[k]] * scales[k/g][n] * (code[n][k] - zeros[k/g][n]).
  *   Arithmetic: fp32 (per word, the dot of the token values with the codes

@@ -28,7 +28,8 @@ __all__ = [
     "GPTQConfig", "GPTQError", "gptq_hessian_accumulate", "gptq_hessian_accumulate_host",
     "gptq_hessian_staging_size", "gptq_prepare_hinv", "gptq_dequant_matmul", "gptq_dequant_matmul_workspace_size",
     "gptq_quantize_layer", "gptq_quantize_layer_noalloc", "gptq_noalloc_scratch_bytes", "gptq_pack", "gptq_workspace_size", "gptq_sync_status",
-    "gptq_status_string", "gptq_version", "gptq_launch_counter", "library_path", "n_groups", "packed_words",
+    "gptq_status_string", "gptq_version", "gptq_launch_counter", "gptq_debug_arm_wait_probe",
+    "library_path", "n_groups", "packed_words",
     "STATUS",
 ]
 
@@ -89,6 +90,7 @@ def _load():
                                         ctypes.c_int),
         "gptq_noalloc_scratch_bytes": ([], ctypes.c_size_t),
         "gptq_sync_status": ([P, P, ctypes.POINTER(i32)], ctypes.c_int),
+        "gptq_debug_arm_wait_probe": ([i32, i64], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -254,11 +256,18 @@ def gptq_quantize_layer_noalloc(W: torch.Tensor, U: torch.Tensor, perm: torch.Te
     for t, name in ((codes, "codes"), (scales, "scales"), (zeros, "zeros"), (U, "U")):
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
-    _check(_lib.gptq_quantize_layer_noalloc(_ptr(W), d_row, d_col, _row_major(W, "W"), _ptr(U),
-                                            _ptr(perm), _ptr(dead), ctypes.byref(cfg),
-                                            _ptr(codes), _ptr(scales), _ptr(zeros),
-                                            _ptr(dev_status), _stream(stream)),
-           "gptq_quantize_layer_noalloc")
+    # the scratch array used is the current device's: every buffer must be on
+    # W's device, and the call runs with that device current
+    for t, name in ((U, "U"), (perm, "perm"), (dead, "dead"), (codes, "codes"),
+                    (scales, "scales"), (zeros, "zeros"), (dev_status, "dev_status")):
+        if t is not None and (not t.is_cuda or t.device != W.device):
+            raise ValueError(f"{name} must be on {W.device}, like W")
+    with torch.cuda.device(W.device):
+        _check(_lib.gptq_quantize_layer_noalloc(_ptr(W), d_row, d_col, _row_major(W, "W"),
+                                                _ptr(U), _ptr(perm), _ptr(dead),
+                                                ctypes.byref(cfg), _ptr(codes), _ptr(scales),
+                                                _ptr(zeros), _ptr(dev_status), _stream(stream)),
+               "gptq_quantize_layer_noalloc")
 
 
 def gptq_noalloc_scratch_bytes() -> int:
@@ -305,6 +314,14 @@ def gptq_dequant_matmul(X: torch.Tensor, packed: torch.Tensor, scales: torch.Ten
 
 def gptq_dequant_matmul_workspace_size(n_tok: int, d_col: int) -> int:
     return int(_lib.gptq_dequant_matmul_workspace_size(int(n_tok), int(d_col)))
+
+
+def gptq_debug_arm_wait_probe(kernel: int, limit_ns: int) -> None:
+    """Test hook: the next launch of kernel kind 1 (Hessian) or 2 (the next
+    fp32-accurate tensor-core GEMM) waits once, bounded by limit_ns, on a
+    barrier nothing completes, and reports GPTQ_ERR_TIMEOUT."""
+    _check(_lib.gptq_debug_arm_wait_probe(int(kernel), int(limit_ns)),
+           "gptq_debug_arm_wait_probe")
 
 
 def gptq_sync_status(dev_status: torch.Tensor, stream=None) -> int:

@@ -11,9 +11,20 @@ namespace gptq {
 
 namespace {
 std::atomic<int64_t> g_launches{0};
+std::atomic<uint64_t> g_probe[3] = {};
 }
 
 void count_launches(int64_t k) { g_launches.fetch_add(k, std::memory_order_relaxed); }
+
+uint64_t take_wait_probe(int kind) {
+    if (kind < 1 || kind > 2) return 0;
+    if (g_probe[kind].load(std::memory_order_relaxed) == 0) return 0;
+    return g_probe[kind].exchange(0, std::memory_order_acq_rel);
+}
+
+void arm_wait_probe(int kind, uint64_t ns) {
+    if (kind >= 1 && kind <= 2) g_probe[kind].store(ns, std::memory_order_release);
+}
 
 int64_t launches() { return g_launches.load(std::memory_order_relaxed); }
 
@@ -76,6 +87,12 @@ const char* gptq_status_string(int32_t status) {
 }
 
 int32_t gptq_version(void) { return 100; }
+
+gptq_status gptq_debug_arm_wait_probe(int32_t kernel, int64_t limit_ns) {
+    if ((kernel != 1 && kernel != 2) || limit_ns <= 0 || limit_ns > 1000000000) return GPTQ_ERR_INVALID_ARG;
+    gptq::arm_wait_probe(kernel, static_cast<uint64_t>(limit_ns));
+    return GPTQ_OK;
+}
 
 int64_t gptq_launch_counter(void) { return gptq::launches(); }
 
@@ -141,7 +158,7 @@ gptq_status gptq_prepare_hinv(float* H, int64_t d, int64_t ldh, const gptq_confi
         ws_bytes < gptq::chol_workspace_bytes(d))
         return GPTQ_ERR_WORKSPACE;
     gptq_status s =
-        gptq::launch_prep(H, d, ldh, cfg->damp, cfg->desc_act, U, perm, dead, ws, stream);
+        gptq::launch_prep(H, d, ldh, cfg->damp, cfg->desc_act, U, perm, dead, dev_status, ws, stream);
     if (s != GPTQ_OK) return s;
     s = gptq::launch_chol_inverse(U, H, ldh, d, U, dev_status, ws, stream);
     return launch_status(s);

@@ -76,20 +76,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity.  Returns false (and
-// raises *abort) when the limit runs out or another thread already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// raises *abort) when limit_ns runs out or another thread already aborted.
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                             uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 255u) == 0u) {
             if (*abort) return false;
-            if (globaltimer() - t0 > kWaitLimitNs) {
+            if (globaltimer() - t0 > limit_ns) {
                 *abort = 1;
                 return false;
             }
         }
     }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    return mbar_wait_ns(bar, parity, abort, kWaitLimitNs);
+}
+
+// Timeout probe (a test of the expiry path, armed from the host through
+// gptq_debug_arm_wait_probe): when probe_ns > 0 the kernel's MMA-issuing
+// thread first waits, bounded by probe_ns, on a barrier that nothing ever
+// arrives on.  The wait runs out, raises *abort and the kernel winds down
+// exactly as after any expired wait (issued copies and MMAs still land under
+// the normal limit) and reports GPTQ_ERR_TIMEOUT.  Returns false then.
+__device__ __forceinline__ bool wait_probe(uint64_t* never, uint64_t probe_ns, volatile int* abort) {
+    if (probe_ns == 0) return true;
+    return mbar_wait_ns(never, 0, abort, probe_ns);
 }
 
 // ---------------------------------------------------------------- TMA

@@ -44,7 +44,8 @@ __global__ void gather_tokens_kernel(const uint16_t* __restrict__ X, int64_t ldx
     for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
          e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int64_t t = e / K, k = e - t * K;
-        const int64_t col = perm != nullptr ? perm[k] : k;
+        int64_t col = perm != nullptr ? perm[k] : k;
+        if (col < 0 || col >= K) col = k;  // not a permutation entry: stay inside the row
         Xq[e] = bf16_to_f32(X[t * ldx + col]);
     }
 }

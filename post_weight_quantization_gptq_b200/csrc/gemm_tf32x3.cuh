@@ -85,6 +85,7 @@ struct Bars {
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
+    uint64_t never;  // the timeout probe's barrier: nothing arrives on it
     uint32_t tmem;
     int abort;
 };
@@ -147,7 +148,7 @@ template <class Sched, bool A_MN, bool B_MN, int Epi, int Split>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
                        const __grid_constant__ CUtensorMap tmd, const Sched sched, int tiles,
-                       int32_t* status) {
+                       int32_t* status, uint64_t probe_ns) {
     constexpr uint32_t kIdesc = instr_desc(/*tf32*/ 2, A_MN ? 1 : 0, B_MN ? 1 : 0, BM, BN);
 
     extern __shared__ uint8_t smem_raw[];
@@ -170,6 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->acc_empty[s], 128);
         }
         mbar_init(&bars->drain, 1);
+        mbar_init(&bars->never, 1);
         bars->abort = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tma);
@@ -218,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------------------------------------------- MMA issuer
         if (lane == 0) {
             int it = 0, lt = 0;
-            bool ok = true;
+            bool ok = wait_probe(&bars->never, probe_ns, abort);
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
                 const Job job = sched.job(t);
                 if (job.nk <= 0) continue;
@@ -459,7 +461,7 @@ inline cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const Sc
     if (tiles <= 0) return cudaSuccess;
     const int grid = tiles < sms ? tiles : sms;
     return launch_kernel(pdl, kern, dim3(grid), dim3(kThreads), smem_bytes<Epi>(), stream, ta, tb,
-                         td != nullptr ? *td : tb, sched, tiles, status);
+                         td != nullptr ? *td : tb, sched, tiles, status, take_wait_probe(kProbeGemm));
 }
 
 }  // namespace g3

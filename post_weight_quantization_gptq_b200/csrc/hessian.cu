@@ -66,6 +66,7 @@ struct Barriers {
     uint64_t acc_full;
     uint64_t acc_empty;
     uint64_t drain;
+    uint64_t never;  // the timeout probe's barrier: nothing arrives on it
     uint32_t tmem_base;
     int abort;
 };
@@ -86,7 +87,8 @@ __device__ __forceinline__ void tile_coords(int t, int MT, int NT, int& mi, int&
 
 __global__ void __launch_bounds__(kThreads, 1)
     hessian_syrk_tcgen05(const __grid_constant__ CUtensorMap tmap_x, float* __restrict__ H,
-                         int64_t ldh, int d, int n, int num_tiles, int32_t* status) {
+                         int64_t ldh, int d, int n, int num_tiles, int32_t* status,
+                         uint64_t probe_ns) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -112,6 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bars->acc_full, 1);
         mbar_init(&bars->acc_empty, 256);
         mbar_init(&bars->drain, 1);
+        mbar_init(&bars->never, 1);
         bars->abort = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmap_x);
@@ -182,6 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             uint32_t it = 0;
+            wait_probe(&bars->never, probe_ns, abort);
             for (int w = 0; w < waves && !*abort; ++w) {
                 const int tw = w / nchunk;
                 const int k0 = (w % nchunk) * kChunkIters;
@@ -292,7 +296,8 @@ gptq_status launch_hessian(const uint16_t* X, int64_t n, int64_t d, int64_t ldx,
     int grid = (T + 1) / 2;
     if (grid > sms) grid = sms;
     hessian_syrk_tcgen05<<<grid, kThreads, kSmemBytes, stream>>>(
-        tmap, H, ldh, static_cast<int>(d), static_cast<int>(n), T, status);
+        tmap, H, ldh, static_cast<int>(d), static_cast<int>(n), T, status,
+        take_wait_probe(kProbeHessian));
     count_launches(1);
     return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
 }

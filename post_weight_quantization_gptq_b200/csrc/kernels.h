@@ -18,6 +18,11 @@ int num_sms();
 void count_launches(int64_t k);
 int64_t launches();
 
+// Timeout probes armed by gptq_debug_arm_wait_probe: the limit (ns) for the
+// next launch of the kernel kind, 0 when unarmed; taking it disarms it.
+enum ProbeKind { kProbeHessian = 1, kProbeGemm = 2 };
+uint64_t take_wait_probe(int kind);
+
 // Launch with the programmatic-serialization attribute when pdl is set; an
 // ordinary launch otherwise.  Such a kernel calls pdl_wait() before its first
 // global memory access, and reads data an earlier kernel wrote only through
@@ -68,7 +73,8 @@ gptq_status launch_hessian_from_host(const uint16_t* Xh, int64_t n, int64_t d, i
 // ---- stage 2 (prep.cu): dead columns, lambda, act-order, flipped working copy
 size_t prep_workspace_bytes(int64_t d);
 gptq_status launch_prep(const float* H, int64_t d, int64_t ldh, float damp, int desc_act,
-                        float* P, int32_t* perm, uint8_t* dead, void* ws, cudaStream_t stream);
+                        float* P, int32_t* perm, uint8_t* dead, int32_t* status, void* ws,
+                        cudaStream_t stream);
 
 // ---- stage 2 (chol.cu): P = L L^T in place, X = L^-1, U = J X J
 size_t chol_workspace_bytes(int64_t d);

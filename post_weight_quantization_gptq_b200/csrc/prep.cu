@@ -21,20 +21,27 @@ struct PrepScratch {
     float pad[2];
 };
 
-// diag -> keys (dead columns count as 1), dead mask, lambda (fp64 sum).
+// diag -> keys (dead columns count as 1), dead mask, lambda (fp64 sum).  A
+// diagonal that is not finite (NaN or infinite: the calibration data held a
+// non-finite value) makes H unusable: it is reported as not positive
+// definite, and the act-order ranking below still yields a permutation.
 __global__ void __launch_bounds__(1024)
     diag_kernel(const float* __restrict__ H, int64_t d, int64_t ldh, float damp,
-                float* __restrict__ keys, uint8_t* __restrict__ dead, PrepScratch* scratch) {
+                float* __restrict__ keys, uint8_t* __restrict__ dead, PrepScratch* scratch,
+                int32_t* status) {
     __shared__ double part[32];
     double acc = 0.0;
+    bool finite = true;
     for (int64_t i = threadIdx.x; i < d; i += blockDim.x) {
         const float h = H[i * ldh + i];
         const bool is_dead = (h == 0.f);
         const float k = is_dead ? 1.f : h;
+        finite = finite && isfinite(h);
         keys[i] = k;
         dead[i] = is_dead ? 1 : 0;
         acc += static_cast<double>(k);
     }
+    if (!finite) report(status, GPTQ_ERR_NOT_PD);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
@@ -47,22 +54,33 @@ __global__ void __launch_bounds__(1024)
     }
 }
 
+// Sort key of a float as an unsigned integer whose order is the float order
+// (negative values: all bits flipped; others: the sign bit set), with every
+// NaN mapped to 0, below all of them.  Integers compare totally, so the ranks
+// below are a permutation whatever the keys hold; NaN keys rank last, after
+// every number, in index order (as a stable sort of -diag puts them).
+__device__ __forceinline__ uint32_t order_key(float x) {
+    const uint32_t b = __float_as_uint(x);
+    if (isnan(x)) return 0u;
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
 // Stable descending rank of every key: rank_i = #{j : k_j > k_i} +
 // #{j < i : k_j == k_i}; perm[rank_i] = i.  O(d^2) comparisons, exact.
 __global__ void __launch_bounds__(256)
     rank_kernel(const float* __restrict__ keys, int64_t d, int32_t* __restrict__ perm) {
-    __shared__ float tile[1024];
+    __shared__ uint32_t tile[1024];
     const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-    const float ki = (i < d) ? keys[i] : 0.f;
-    int64_t rank = 0;
+    const uint32_t ki = (i < d) ? order_key(keys[i]) : 0u;
+    int rank = 0;  // d < 2^31
     for (int64_t j0 = 0; j0 < d; j0 += 1024) {
         __syncthreads();
         for (int t = threadIdx.x; t < 1024; t += blockDim.x)
-            tile[t] = (j0 + t < d) ? keys[j0 + t] : 0.f;
+            tile[t] = (j0 + t < d) ? order_key(keys[j0 + t]) : 0u;
         __syncthreads();
         const int64_t jn = (d - j0 < 1024) ? d - j0 : 1024;
         for (int t = 0; t < jn; ++t) {
-            const float kj = tile[t];
+            const uint32_t kj = tile[t];
             rank += (kj > ki) || (kj == ki && j0 + t < i);
         }
     }
@@ -122,11 +140,12 @@ size_t prep_workspace_bytes(int64_t d) {
 }
 
 gptq_status launch_prep(const float* H, int64_t d, int64_t ldh, float damp, int desc_act,
-                        float* P, int32_t* perm, uint8_t* dead, void* ws, cudaStream_t stream) {
+                        float* P, int32_t* perm, uint8_t* dead, int32_t* status, void* ws,
+                        cudaStream_t stream) {
     uint8_t* base = static_cast<uint8_t*>(ws);
     PrepScratch* scratch = reinterpret_cast<PrepScratch*>(base);
     float* keys = reinterpret_cast<float*>(base + ((sizeof(PrepScratch) + 255) / 256) * 256);
-    diag_kernel<<<1, 1024, 0, stream>>>(H, d, ldh, damp, keys, dead, scratch);
+    diag_kernel<<<1, 1024, 0, stream>>>(H, d, ldh, damp, keys, dead, scratch, status);
     if (desc_act) {
         rank_kernel<<<static_cast<unsigned>((d + 255) / 256), 256, 0, stream>>>(keys, d, perm);
     } else {

@@ -36,9 +36,12 @@ constexpr int kRowsPerCta = kRowsPerWarp * kWarps;
 static_assert(kWarps * 32 == kBlock, "block_quant_kernel: one thread per column of the U block");
 
 // ------------------------------------------------------------------------
+// A perm entry outside [0, d) (the caller passed something other than
+// gptq_prepare_hinv's output) is reported as GPTQ_ERR_INVALID_ARG and read as
+// the column's own index, so no access leaves the row.
 __global__ void permute_rows_kernel(float* __restrict__ W, int64_t r, int64_t d, int64_t ldw,
                                     const int32_t* __restrict__ perm,
-                                    const uint8_t* __restrict__ dead) {
+                                    const uint8_t* __restrict__ dead, int32_t* status) {
     extern __shared__ float rowbuf[];
     pdl_trigger();
     for (int64_t row = blockIdx.x; row < r; row += gridDim.x) {
@@ -46,7 +49,11 @@ __global__ void permute_rows_kernel(float* __restrict__ W, int64_t r, int64_t d,
         for (int64_t k = threadIdx.x; k < d; k += blockDim.x) rowbuf[k] = w[k];
         __syncthreads();
         for (int64_t k = threadIdx.x; k < d; k += blockDim.x) {
-            const int32_t src = perm[k];
+            int64_t src = perm[k];
+            if (src < 0 || src >= d) {
+                if (row == blockIdx.x) report(status, GPTQ_ERR_INVALID_ARG);
+                src = k;
+            }
             w[k] = dead[src] ? 0.f : rowbuf[src];
         }
         __syncthreads();
@@ -472,7 +479,8 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
                                  static_cast<int>(row_smem)) != cudaSuccess)
             return GPTQ_ERR_CUDA;
         const int prow_grid = static_cast<int>(d_row < 4 * num_sms() ? d_row : 4 * num_sms());
-        permute_rows_kernel<<<prow_grid, 256, row_smem, stream>>>(W, d_row, d_col, ldw, perm, dead);
+        permute_rows_kernel<<<prow_grid, 256, row_smem, stream>>>(W, d_row, d_col, ldw, perm, dead,
+                                                                   status);
     }
     const uint8_t* dead_mask = permuted ? nullptr : dead;
 

@@ -159,3 +159,12 @@ def test_dequant_matmul_validation(pkg):
     assert call(g=12) == 2                                  # a word would span two groups
     assert call(ws=None) == 6 and call(wsb=1023) == 6       # workspace missing / too small
     assert call(ws=ctypes.c_void_p((1 << 20) + 16)) == 6    # workspace misaligned
+
+
+def test_wait_probe_arguments_are_checked_on_the_host(pkg):
+    """The timeout test hook takes kernel kinds 1 and 2 and limits in
+    1 .. 10^9 ns; anything else is refused before any state changes."""
+    for kernel, ns in ((0, 1000), (3, 1000), (1, 0), (2, -5), (1, 2_000_000_000)):
+        with pytest.raises(pkg.GPTQError) as e:
+            pkg.gptq_debug_arm_wait_probe(kernel, ns)
+        assert e.value.status == 1

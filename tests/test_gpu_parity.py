@@ -166,6 +166,56 @@ def test_not_positive_definite_is_reported():
     assert torch.isfinite(U).all()
 
 
+@pytest.mark.parametrize("bad", [float("nan"), float("inf")])
+def test_non_finite_diagonal_is_reported_and_perm_stays_a_permutation(bad):
+    """A non-finite diagonal entry of H (e.g. a NaN in the calibration data)
+    is reported as not positive definite; the act-order permutation is still a
+    permutation (NaN columns ranked last, as a stable sort of -diag does), so
+    nothing downstream indexes outside the matrix."""
+    g = gpu()
+    d = 256
+    _, X = workloads.small_layer(4, d, 4 * d, seed=3, kind="student_t")
+    H = oracle.hessian(X).astype(np.float32)
+    for i in (5, 77, 200):
+        H[i, i] = bad
+    cfg = g.GPTQConfig(bits=4, group_size=128, desc_act=True)
+    ws = torch.empty(g.gptq_workspace_size(cfg, 4, d), dtype=torch.uint8, device="cuda")
+    U = torch.empty(d, d, device="cuda")
+    perm = torch.empty(d, dtype=torch.int32, device="cuda")
+    dead = torch.empty(d, dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g.gptq_prepare_hinv(torch.from_numpy(H).cuda(), cfg, U, perm, dead, st, ws)
+    assert g.gptq_sync_status(st) == 3
+    p = perm.cpu().numpy()
+    assert np.array_equal(np.sort(p), np.arange(d))
+    assert np.array_equal(p, np.argsort(-np.diag(H).astype(np.float64), kind="stable"))
+
+
+def test_out_of_range_permutation_entry_is_reported():
+    """quantize_layer with act-order reads perm; an entry outside [0, d_col)
+    is reported as an invalid argument on the device and no access leaves
+    the row (the entry is read as the identity)."""
+    g = gpu()
+    d, r = 256, 8
+    W, X = workloads.small_layer(r, d, 4 * d, seed=4, kind="student_t")
+    H = oracle.hessian(X).astype(np.float32)
+    cfg = g.GPTQConfig(bits=4, group_size=128, desc_act=True)
+    ws = torch.empty(g.gptq_workspace_size(cfg, r, d), dtype=torch.uint8, device="cuda")
+    U = torch.empty(d, d, device="cuda")
+    perm = torch.empty(d, dtype=torch.int32, device="cuda")
+    dead = torch.empty(d, dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g.gptq_prepare_hinv(torch.from_numpy(H).cuda(), cfg, U, perm, dead, st, ws)
+    assert g.gptq_sync_status(st) == 0
+    perm[10] = d + 1000
+    perm[11] = -7
+    codes = torch.empty(r, d, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(2, r, device="cuda")
+    zeros = torch.empty(2, r, dtype=torch.int32, device="cuda")
+    g.gptq_quantize_layer(W.cuda().contiguous(), U, perm, dead, cfg, codes, scales, zeros, st, ws)
+    assert g.gptq_sync_status(st) == 1
+
+
 # ------------------------------------------------------------ stages 3 + 4
 QUANT_CASES = [
     # d_row, d_col, tokens, kind, bits, group, desc_act
