@@ -53,21 +53,24 @@ def _lib():
         lib = ctypes.CDLL(build_native())
         P = ctypes.c_void_p
         i64 = ctypes.c_int64
-        lib.orc_quant_params.argtypes = [P, i64, ctypes.c_int, P, P, P]
+        lib.orc_quant_params.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, P, P, P]
         lib.orc_quant_params.restype = None
         lib.orc_quantize.argtypes = [ctypes.c_double, ctypes.c_double, ctypes.c_int32, ctypes.c_int]
         lib.orc_quantize.restype = ctypes.c_int32
-        lib.orc_gptq_columns.argtypes = [P, i64, i64, P, ctypes.c_int, i64, P, P, P, P,
-                                         P, P, P, P, ctypes.c_double, ctypes.c_double, P, P, P]
+        lib.orc_gptq_columns.argtypes = [P, i64, i64, P, ctypes.c_int, i64, ctypes.c_int, P, P,
+                                         P, P, P, P, P, P, ctypes.c_double, ctypes.c_double, P, P,
+                                         P]
         lib.orc_gptq_columns.restype = ctypes.c_int
-        lib.orc_gptq_columns_u.argtypes = [P, i64, i64, P, ctypes.c_int, i64, P, P, P,
-                                           P, P, P, P, ctypes.c_double, ctypes.c_double, P, P, P]
+        lib.orc_gptq_columns_u.argtypes = [P, i64, i64, P, ctypes.c_int, i64, ctypes.c_int, P, P,
+                                           P, P, P, P, P, ctypes.c_double, ctypes.c_double, P, P,
+                                           P]
         lib.orc_gptq_columns_u.restype = ctypes.c_int
         lib.orc_eliminate.argtypes = [P, i64, i64, P]
         lib.orc_eliminate.restype = ctypes.c_int
-        lib.orc_gptq_blocked.argtypes = [P, i64, i64, P, ctypes.c_int, i64, i64, P, P, P]
+        lib.orc_gptq_blocked.argtypes = [P, i64, i64, P, ctypes.c_int, i64, ctypes.c_int, i64, P,
+                                         P, P]
         lib.orc_gptq_blocked.restype = ctypes.c_int
-        lib.orc_rtn.argtypes = [P, i64, i64, ctypes.c_int, i64, P, P, P]
+        lib.orc_rtn.argtypes = [P, i64, i64, ctypes.c_int, i64, ctypes.c_int, P, P, P]
         lib.orc_rtn.restype = None
         _lib_handle = lib
     return _lib_handle
@@ -200,17 +203,20 @@ def eliminate(Minv, steps: int | None = None):
 # --------------------------------------------------------------------------
 # The quantizer  [GROUP]
 # --------------------------------------------------------------------------
-def quant_params(x, bits: int):
+def quant_params(x, bits: int, pure: bool = False):
     """(scale, zero_real, zero) of one group: asymmetric min-max over the
-    group's current weights, with 0 always inside the range (so the integer
-    zero point lies in [0, 2^b - 1]) and an all-equal range widened to
-    [-1, 1].  zero = rint(-xmin / scale), round half to even."""
+    group's current weights [GROUP].  Default: 0 always inside the range (so
+    the integer zero point lies in [0, 2^b - 1]) and an all-zero group widened
+    to [-1, 1].  pure: the group's own [min, max] (the zero point may fall
+    outside [0, 2^b - 1]); a constant group, or one whose real zero point lies
+    more than 2^20 levels away, falls back to the widened range.
+    zero = rint(-xmin / scale), round half to even."""
     x = np.ascontiguousarray(x, dtype=np.float64)
     s = ctypes.c_double()
     zr = ctypes.c_double()
     z = ctypes.c_int32()
-    _lib().orc_quant_params(_ptr(x), x.size, bits, ctypes.byref(s), ctypes.byref(zr),
-                            ctypes.byref(z))
+    _lib().orc_quant_params(_ptr(x), x.size, bits, int(bool(pure)), ctypes.byref(s),
+                            ctypes.byref(zr), ctypes.byref(z))
     return s.value, zr.value, z.value
 
 
@@ -230,7 +236,7 @@ def dequantize(codes, scales, zeros, group_size: int) -> np.ndarray:
     return s * (codes.astype(np.float64) - z)
 
 
-def rtn(W0, bits: int, group_size: int):
+def rtn(W0, bits: int, group_size: int, pure: bool = False):
     """Round-to-nearest: the same group quantizer applied to W0 with no error
     feedback (the baseline GPTQ is compared with, "GPTQ" article,
     "Desempenho e Precisao")."""
@@ -241,7 +247,8 @@ def rtn(W0, bits: int, group_size: int):
     codes = np.zeros((r, d), dtype=np.uint8)
     scales = np.zeros((ng, r), dtype=np.float64)
     zeros = np.zeros((ng, r), dtype=np.int32)
-    _lib().orc_rtn(_ptr(W0), r, d, bits, g, _ptr(codes), _ptr(scales), _ptr(zeros))
+    _lib().orc_rtn(_ptr(W0), r, d, bits, g, int(bool(pure)), _ptr(codes), _ptr(scales),
+                   _ptr(zeros))
     return codes, scales, zeros
 
 
@@ -280,7 +287,7 @@ def _stats(stats, max_dev) -> dict:
 
 def gptq_columns(W0, Hinv, bits: int, group_size: int, want_U: bool = False,
                  forced_codes=None, forced_zeros=None, forced_w=None, forced_scales=None,
-                 tau: float = 0.0, stol: float = SCALE_TOL) -> GPTQResult:
+                 tau: float = 0.0, stol: float = SCALE_TOL, pure: bool = False) -> GPTQResult:
     """The OBQ/GPTQ loop one column at a time with explicit elimination of
     H^-1 after every column [OBQ].
 
@@ -313,7 +320,8 @@ def gptq_columns(W0, Hinv, bits: int, group_size: int, want_U: bool = False,
     stats = np.zeros(7, dtype=np.int64)
     first = np.zeros(r, dtype=np.int64)
     max_dev = ctypes.c_double(0.0)
-    rc = _lib().orc_gptq_columns(_ptr(W), r, d, _ptr(M), bits, g, _ptr(codes), _ptr(scales),
+    rc = _lib().orc_gptq_columns(_ptr(W), r, d, _ptr(M), bits, g, int(bool(pure)), _ptr(codes),
+                                 _ptr(scales),
                                  _ptr(zeros), _ptr(U), _ptr(fc), _ptr(fz), _ptr(fw), _ptr(fs),
                                  float(tau), float(stol), _ptr(stats), ctypes.byref(max_dev),
                                  _ptr(first))
@@ -350,7 +358,7 @@ def upper_factor_flip(Hd) -> np.ndarray:
 
 def gptq_columns_u(W0, U, bits: int, group_size: int, forced_codes=None, forced_zeros=None,
                    forced_w=None, forced_scales=None, tau: float = 0.0,
-                   stol: float = SCALE_TOL) -> GPTQResult:
+                   stol: float = SCALE_TOL, pure: bool = False) -> GPTQResult:
     """The OBQ column loop driven by U's rows: W_F <- W_F - (e / U_ii) U_{i,F}
     [OBQ] with row i of the reduced inverse equal to U_ii U[i, i:].  Same
     teacher-forcing options as gptq_columns."""
@@ -369,7 +377,8 @@ def gptq_columns_u(W0, U, bits: int, group_size: int, forced_codes=None, forced_
     stats = np.zeros(7, dtype=np.int64)
     first = np.zeros(r, dtype=np.int64)
     max_dev = ctypes.c_double(0.0)
-    rc = _lib().orc_gptq_columns_u(_ptr(W), r, d, _ptr(Uc), bits, g, _ptr(codes), _ptr(scales),
+    rc = _lib().orc_gptq_columns_u(_ptr(W), r, d, _ptr(Uc), bits, g, int(bool(pure)), _ptr(codes),
+                                   _ptr(scales),
                                    _ptr(zeros), _ptr(fc), _ptr(fz), _ptr(fw), _ptr(fs),
                                    float(tau), float(stol), _ptr(stats), ctypes.byref(max_dev),
                                    _ptr(first))
@@ -378,7 +387,7 @@ def gptq_columns_u(W0, U, bits: int, group_size: int, forced_codes=None, forced_
     return GPTQResult(codes, scales, zeros, W, None, _stats(stats, max_dev), first)
 
 
-def gptq_blocked(W0, U, bits: int, group_size: int, block: int):
+def gptq_blocked(W0, U, bits: int, group_size: int, block: int, pure: bool = False):
     """The pages' batched loop [ALGO] with B = block: in-batch OBQ feedback,
     then one lazy product W[:, i1:] -= Err U[i0:i1, i1:] per batch.  Reading
     of the garbled lazy-update line: Err_j = (w_j - q_j) / U_jj is divided
@@ -391,7 +400,8 @@ def gptq_blocked(W0, U, bits: int, group_size: int, block: int):
     codes = np.zeros((r, d), dtype=np.uint8)
     scales = np.zeros((ng, r), dtype=np.float64)
     zeros = np.zeros((ng, r), dtype=np.int32)
-    rc = _lib().orc_gptq_blocked(_ptr(W), r, d, _ptr(Uc), bits, g, int(block), _ptr(codes),
+    rc = _lib().orc_gptq_blocked(_ptr(W), r, d, _ptr(Uc), bits, g, int(bool(pure)), int(block),
+                                 _ptr(codes),
                                  _ptr(scales), _ptr(zeros))
     if rc != 0:
         raise MemoryError("oracle blocked loop failed")
@@ -446,7 +456,7 @@ def dequant_matmul(X, packed, scales, zeros, perm, bits: int, group_size: int,
 def quantize_layer(H, W, bits: int = 4, group_size: int = 128, desc_act: bool = False,
                    damp: float = 0.01, want_U: bool = False, rows=None,
                    forced_codes=None, forced_zeros=None, forced_w=None, forced_scales=None,
-                   tau: float = 0.0) -> dict:
+                   tau: float = 0.0, pure: bool = False) -> dict:
     """H (d x d, original column order) and W (r x d) -> GPTQ result.
 
     Steps [ALGO]: dead-column fix, act-order permutation, damping, H^-1, then
@@ -458,9 +468,9 @@ def quantize_layer(H, W, bits: int = 4, group_size: int = 128, desc_act: bool = 
     Minv = inverse(prep["H_damped"])
     res = gptq_columns(W0, Minv, bits, group_size, want_U=want_U,
                        forced_codes=forced_codes, forced_zeros=forced_zeros,
-                       forced_w=forced_w, forced_scales=forced_scales, tau=tau)
+                       forced_w=forced_w, forced_scales=forced_scales, tau=tau, pure=pure)
     Q = dequantize(res.codes, res.scales, res.zeros, group_size)
-    rc, rs, rz = rtn(W0, bits, group_size)
+    rc, rs, rz = rtn(W0, bits, group_size, pure=pure)
     Qr = dequantize(rc, rs, rz, group_size)
     return dict(codes=res.codes, scales=res.scales, zeros=res.zeros, perm=prep["perm"],
                 dead=prep["dead"], lam=prep["lam"], W0=W0, Q=Q, w_at_quant=res.w_at_quant,

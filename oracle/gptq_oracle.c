@@ -35,16 +35,36 @@
 #include <string.h>
 
 /* Asymmetric min-max quantizer parameters of one group (AutoGPTQ guide,
- * "Quantizacao group-wise": own scale and zero point per group). */
-void orc_quant_params(const double *x, int64_t n, int bits, double *scale,
+ * "Quantizacao group-wise": own scale and zero point per group).
+ *
+ * Default (pure == 0): the range is widened to contain 0, so the integer zero
+ * point lies in [0, 2^b - 1] and 0 is exactly representable.
+ * pure != 0: the range is the group's own [min, max]; the zero point may lie
+ * outside [0, 2^b - 1] (every code still does).  Two groups fall back to the
+ * widened range: a constant group (its own range is empty) and one whose real
+ * zero point lies more than 2^20 levels away (a range that narrow next to its
+ * offset from zero is below the resolution of fp32 arithmetic on w / s). */
+void orc_quant_params(const double *x, int64_t n, int bits, int pure, double *scale,
                       double *zero_real, int32_t *zero)
 {
-    double xmin = 0.0, xmax = 0.0; /* the range always contains 0 */
+    double maxq = (double)((1 << bits) - 1);
+    double xmin = 0.0, xmax = 0.0; /* widened: the range always contains 0 */
+    if (pure && n > 0) {
+        xmin = x[0];
+        xmax = x[0];
+    }
     for (int64_t k = 0; k < n; ++k) {
         if (x[k] < xmin) xmin = x[k];
         if (x[k] > xmax) xmax = x[k];
     }
-    double maxq = (double)((1 << bits) - 1);
+    if (pure) {
+        int widen = (xmax == xmin);
+        if (!widen) widen = fabs(xmin / ((xmax - xmin) / maxq)) > 1048576.0;
+        if (widen) {
+            if (xmin > 0.0) xmin = 0.0;
+            if (xmax < 0.0) xmax = 0.0;
+        }
+    }
     if (xmax == xmin) {
         /* all-zero group: the range becomes [-1, 1], so s = 2 / (2^b - 1) and
          * -xmin / s = (2^b - 1) / 2 exactly, a tie that rounds half to even
@@ -95,6 +115,7 @@ static int code_is_valid(int32_t c, int32_t q, double y, double tol, int bits)
  *   M       d x d row-major, in: inverse of the damped Hessian (only the upper
  *           triangle, j >= i, is read).  Destroyed.
  *   g       group size (1 <= g; a caller maps "-1" to d).
+ *   pure    the group range rule of orc_quant_params (0: widened to 0).
  *   codes   r x d uint8; scales / zeros  [ceil(d/g)][r].
  *   U       optional d x d row-major (NULL to skip): row i receives the
  *           eliminated row of M scaled by 1/sqrt(M_ii), for columns >= i.
@@ -118,7 +139,7 @@ static int code_is_valid(int32_t c, int32_t q, double y, double tol, int bits)
  *           d if none.  Until that column the forced run is the free run.
  */
 int orc_gptq_columns(double *W, int64_t r, int64_t d, double *M, int bits,
-                     int64_t g, uint8_t *codes, double *scales, int32_t *zeros,
+                     int64_t g, int pure, uint8_t *codes, double *scales, int32_t *zeros,
                      double *U, const uint8_t *fcodes, const int32_t *fzeros,
                      const double *fwpre, const double *fscales, double tau, double stol,
                      int64_t *stats, double *max_dev, int64_t *first_tie)
@@ -159,7 +180,7 @@ int orc_gptq_columns(double *W, int64_t r, int64_t d, double *M, int bits,
                  * [i, i+g) of this row */
                 double s, zr;
                 int32_t z;
-                orc_quant_params(w + i, gend - i, bits, &s, &zr, &z);
+                orc_quant_params(w + i, gend - i, bits, pure, &s, &zr, &z);
                 if (fscales) {
                     const double ds = fabs(fscales[grp * r + row] - s) / s;
                     if (ds > stol) ++s_scale_bad;
@@ -262,7 +283,7 @@ int orc_gptq_columns(double *W, int64_t r, int64_t d, double *M, int bits,
  * orc_gptq_columns, with U (d x d, row-major, upper) in place of M.
  */
 int orc_gptq_columns_u(double *W, int64_t r, int64_t d, const double *U, int bits, int64_t g,
-                       uint8_t *codes, double *scales, int32_t *zeros,
+                       int pure, uint8_t *codes, double *scales, int32_t *zeros,
                        const uint8_t *fcodes, const int32_t *fzeros, const double *fwpre,
                        const double *fscales, double tau, double stol, int64_t *stats,
                        double *max_dev, int64_t *first_tie)
@@ -285,7 +306,7 @@ int orc_gptq_columns_u(double *W, int64_t r, int64_t d, const double *U, int bit
             if (i % g == 0) {
                 const int64_t gend = (i + g < d) ? i + g : d;
                 double zr;
-                orc_quant_params(w + i, gend - i, bits, &s, &zr, &z);
+                orc_quant_params(w + i, gend - i, bits, pure, &s, &zr, &z);
                 if (fscales) {
                     const double ds = fabs(fscales[(i / g) * r + row] - s) / s;
                     if (ds > stol) ++s_scale_bad;
@@ -384,7 +405,7 @@ int orc_eliminate(double *M, int64_t d, int64_t steps, double *U)
  * (e / U_ii) * U_{i,F}; Err holds e_j / U_jj.
  */
 int orc_gptq_blocked(double *W, int64_t r, int64_t d, const double *U, int bits,
-                     int64_t g, int64_t B, uint8_t *codes, double *scales,
+                     int64_t g, int pure, int64_t B, uint8_t *codes, double *scales,
                      int32_t *zeros)
 {
     double *err = (double *)malloc(sizeof(double) * (size_t)(r * B));
@@ -401,7 +422,7 @@ int orc_gptq_blocked(double *W, int64_t r, int64_t d, const double *U, int bits,
                     const int64_t gend = (j + g < d) ? j + g : d;
                     double s, zr;
                     int32_t z;
-                    orc_quant_params(w + j, gend - j, bits, &s, &zr, &z);
+                    orc_quant_params(w + j, gend - j, bits, pure, &s, &zr, &z);
                     cur_s[row] = s;
                     cur_z[row] = z;
                     scales[(j / g) * r + row] = s;
@@ -428,7 +449,7 @@ int orc_gptq_blocked(double *W, int64_t r, int64_t d, const double *U, int bits,
 }
 
 /* Round-to-nearest baseline: the same group quantizer with no error feedback. */
-void orc_rtn(const double *W, int64_t r, int64_t d, int bits, int64_t g,
+void orc_rtn(const double *W, int64_t r, int64_t d, int bits, int64_t g, int pure,
              uint8_t *codes, double *scales, int32_t *zeros)
 {
 #pragma omp parallel for schedule(static)
@@ -440,7 +461,7 @@ void orc_rtn(const double *W, int64_t r, int64_t d, int bits, int64_t g,
             if (j % g == 0) {
                 const int64_t gend = (j + g < d) ? j + g : d;
                 double zr;
-                orc_quant_params(w + j, gend - j, bits, &s, &zr, &z);
+                orc_quant_params(w + j, gend - j, bits, pure, &s, &zr, &z);
                 scales[(j / g) * r + row] = s;
                 zeros[(j / g) * r + row] = z;
             }

@@ -53,6 +53,41 @@ def test_quantizer_worked_examples():
         assert np.allclose(deq, [float(v) for v in what.split()], atol=1e-15), name
 
 
+def test_pure_minmax_quantizer_worked_examples():
+    """The pure min-max range (the group's own [min, max]): hand-computed
+    scale / zero / codes / dequantized values (golden file), zero points
+    outside [0, 2^b - 1] included, and the two fall-backs to the widened
+    range."""
+    path = os.path.join(GOLDEN, "quantizer_pure_minmax_worked_example.txt")
+    for name, bits, ws, s, z, codes, what in _rows(path):
+        bits = int(bits)
+        w = np.array([float(v) for v in ws.split()])
+        scale, _, zero = oracle.quant_params(w, bits, pure=True)
+        assert scale == pytest.approx(float(s), rel=1e-15), name
+        assert zero == int(z), name
+        got = [oracle.quantize_code(x, scale, zero, bits) for x in w]
+        assert got == [int(c) for c in codes.split()], name
+        deq = scale * (np.array(got, dtype=np.float64) - zero)
+        assert np.allclose(deq, [float(v) for v in what.split()], rtol=1e-15, atol=1e-15), name
+
+
+def test_pure_minmax_is_the_default_when_the_range_holds_zero():
+    """A group whose values straddle 0 has the same range either way, so the
+    two rules agree exactly; a one-signed group gets a finer scale."""
+    rng = np.random.default_rng(12)
+    for bits in (2, 3, 4, 8):
+        w = rng.standard_normal(64)
+        w[0], w[1] = -abs(w[0]), abs(w[1])
+        assert oracle.quant_params(w, bits, pure=True) == oracle.quant_params(w, bits)
+        pos = np.abs(w) + 0.5
+        sp, _, zp = oracle.quant_params(pos, bits, pure=True)
+        sd, _, _ = oracle.quant_params(pos, bits)
+        assert sp < sd and zp < 0
+        q = np.array([oracle.quantize_code(x, sp, zp, bits) for x in pos])
+        assert q.min() >= 0 and q.max() <= (1 << bits) - 1
+        assert np.abs(sp * (q - zp) - pos).max() <= 0.5 * sp * (1 + 1e-12)
+
+
 def test_quantizer_roundtrip_bound():
     """|w_hat - w| <= s/2 for every weight inside the group's range."""
     rng = np.random.default_rng(3)
@@ -238,15 +273,16 @@ def test_gptq_loss_is_not_below_the_exhaustive_optimum():
 # ------------------------------------------------------ lazy batch update
 @pytest.mark.parametrize("B,g", [(1, 16), (2, 16), (4, 16), (8, 16), (128, 16),
                                  (8, 8), (16, 64), (32, 96), (128, 192), (7, 192)])
-def test_lazy_block_update_equals_the_unbatched_loop(B, g):
+@pytest.mark.parametrize("pure", [False, True])
+def test_lazy_block_update_equals_the_unbatched_loop(B, g, pure):
     """The pages' batched loop with its lazy update equals the one-column-at-
-    a-time OBQ loop: same codes, same weights to 1e-10."""
+    a-time OBQ loop: same codes, same weights to 1e-10 (either group range)."""
     rng = np.random.default_rng(B * 1000 + g)
     d, r = 192, 24
     H = _spd(d, B + g, cond_spread=0.6)
-    W0 = rng.standard_normal((r, d)) * 0.02
-    res = oracle.gptq_columns(W0, oracle.inverse(H), 4, g, want_U=True)
-    codes, scales, zeros, Wb = oracle.gptq_blocked(W0, res.U, 4, g, B)
+    W0 = rng.standard_normal((r, d)) * 0.02 + (0.01 if pure else 0.0)
+    res = oracle.gptq_columns(W0, oracle.inverse(H), 4, g, want_U=True, pure=pure)
+    codes, scales, zeros, Wb = oracle.gptq_blocked(W0, res.U, 4, g, B, pure=pure)
     assert np.array_equal(codes, res.codes)
     assert np.array_equal(zeros, res.zeros)
     assert np.allclose(scales, res.scales, rtol=1e-12, atol=0)
@@ -255,16 +291,17 @@ def test_lazy_block_update_equals_the_unbatched_loop(B, g):
 
 # --------------------------------------------------- special cases of GPTQ
 @pytest.mark.parametrize("g", [8, 32, -1])
-def test_identity_hessian_gives_round_to_nearest_exactly(g):
+@pytest.mark.parametrize("pure", [False, True])
+def test_identity_hessian_gives_round_to_nearest_exactly(g, pure):
     """H proportional to I: H^-1 has no off-diagonal terms, so there is no
     feedback and GPTQ equals round-to-nearest exactly (also after damping,
-    since H + lambda I is still proportional to I)."""
+    since H + lambda I is still proportional to I), with either group range."""
     rng = np.random.default_rng(abs(g))
     d = 64
-    W = rng.standard_normal((16, d)) * 0.03
+    W = rng.standard_normal((16, d)) * 0.03 + (0.02 if pure else 0.0)
     H = 3.7 * np.eye(d)
-    out = oracle.quantize_layer(H, W, bits=4, group_size=g, damp=0.01)
-    rc, rs, rz = oracle.rtn(out["W0"], 4, g)
+    out = oracle.quantize_layer(H, W, bits=4, group_size=g, damp=0.01, pure=pure)
+    rc, rs, rz = oracle.rtn(out["W0"], 4, g, pure=pure)
     assert np.array_equal(out["codes"], rc)
     assert np.array_equal(out["scales"], rs)
     assert np.array_equal(out["zeros"], rz)
