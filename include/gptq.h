@@ -76,12 +76,20 @@ typedef struct gptq_config {
     int32_t block_size;  /* columns per lazy-update block; must be 128               */
     int32_t desc_act;    /* nonzero: quantize columns by descending diag(H)          */
     float damp;          /* lambda = damp * mean(diag H); the guide's default 0.01   */
+    int32_t pure_minmax; /* 0 (default): each group's range is widened to contain 0,
+                            so zero points lie in [0, 2^bits - 1];  nonzero: the
+                            group's own [min, max] (a one-signed group gets a finer
+                            scale; its zero point may lie outside [0, 2^bits - 1],
+                            its codes never do).  A constant group, or one whose
+                            zero point would lie more than 2^20 levels away, uses
+                            the widened range.                                    */
 } gptq_config;
 
 /* Human-readable text of a status code (static storage, never NULL). */
 const char *gptq_status_string(int32_t status);
 
-/* Library ABI version (major * 10000 + minor * 100 + patch). */
+/* Library ABI version (major * 10000 + minor * 100 + patch); 200 added
+ * gptq_config.pure_minmax. */
 int32_t gptq_version(void);
 
 /* Number of CUDA kernels this library has launched in this process since it

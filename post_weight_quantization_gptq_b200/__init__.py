@@ -43,14 +43,17 @@ STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID_ARG", 2: "GPTQ_ERR_UNSUPPORTED",
 
 class GPTQConfig(ctypes.Structure):
     """Mirror of ``gptq_config``: bits, group_size (-1 = one group per row),
-    block_size (128), desc_act, damp (lambda = damp * mean(diag H))."""
+    block_size (128), desc_act, damp (lambda = damp * mean(diag H)),
+    pure_minmax (each group's own [min, max] instead of the range widened to
+    contain 0)."""
     _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32),
                 ("block_size", ctypes.c_int32), ("desc_act", ctypes.c_int32),
-                ("damp", ctypes.c_float)]
+                ("damp", ctypes.c_float), ("pure_minmax", ctypes.c_int32)]
 
-    def __init__(self, bits=4, group_size=128, desc_act=False, damp=0.01, block_size=128):
+    def __init__(self, bits=4, group_size=128, desc_act=False, damp=0.01, block_size=128,
+                 pure_minmax=False):
         super().__init__(int(bits), int(group_size), int(block_size), int(bool(desc_act)),
-                         float(damp))
+                         float(damp), int(bool(pure_minmax)))
 
 
 class GPTQError(RuntimeError):

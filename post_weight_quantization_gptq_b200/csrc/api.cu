@@ -86,7 +86,7 @@ const char* gptq_status_string(int32_t status) {
     }
 }
 
-int32_t gptq_version(void) { return 100; }
+int32_t gptq_version(void) { return 200; }
 
 gptq_status gptq_debug_arm_wait_probe(int32_t kernel, int64_t limit_ns) {
     if ((kernel != 1 && kernel != 2) || limit_ns <= 0 || limit_ns > 1000000000) return GPTQ_ERR_INVALID_ARG;
@@ -180,7 +180,8 @@ gptq_status gptq_quantize_layer(float* W, int64_t d_row, int64_t d_col, int64_t 
         ws_bytes < gptq::quant_min_workspace_bytes(d_row, cfg->block_size))
         return GPTQ_ERR_WORKSPACE;
     return launch_status(gptq::launch_quantize(W, d_row, d_col, ldw, U, perm, dead, cfg->desc_act, cfg->bits,
-                                               cfg->group_size, cfg->block_size, codes, scales,
+                                               cfg->group_size, cfg->block_size, cfg->pure_minmax,
+                                               codes, scales,
                                                zeros, dev_status, ws, ws_bytes, stream));
 }
 

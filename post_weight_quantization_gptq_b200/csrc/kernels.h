@@ -88,7 +88,7 @@ size_t quant_workspace_bytes(int64_t d_row, int64_t d_col, int block);
 size_t quant_min_workspace_bytes(int64_t d_row, int block);
 gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw, const float* U,
                             const int32_t* perm, const uint8_t* dead, int desc_act, int bits, int group,
-                            int block, uint8_t* codes, float* scales, int32_t* zeros,
+                            int block, int pure_minmax, uint8_t* codes, float* scales, int32_t* zeros,
                             int32_t* status, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 // ---- using the quantized layer (dequant_matmul.cu): Y = X W_hat^T, decode form

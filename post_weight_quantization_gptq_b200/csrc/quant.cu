@@ -9,7 +9,8 @@
 //   e_i = (w_i - q_i) / U_ii,  W_F <- W_F - e_i * U_{i,F}.
 // The quantizer is the AutoGPTQ guide's group-wise asymmetric one
 // ("Quantizacao group-wise"): per row and group, scale and zero point from
-// the group's current min / max (range widened to contain 0).
+// the group's current min / max (range widened to contain 0, or the group's
+// own range with the pure min-max option).
 //
 // Kernels:
 //  permute_rows_kernel  W[:, k] <- W[:, perm[k]] (0 for dead columns), in place
@@ -80,16 +81,19 @@ struct GroupParams {
 // Scale / zero point of the group [c0 + j, c0 + j + g) of this row from its
 // current weights: the group's columns in this block (cur: chunk m, nxt:
 // chunks m+1..3) plus, for groups wider than the block, the later columns in
-// W (which already hold every earlier block's feedback).  Range widened to
-// contain 0; an all-zero group gets the range [-1, 1] (zero point exactly
-// 2^(bits-1)).
+// W (which already hold every earlier block's feedback).  Default: range
+// widened to contain 0.  pure: the group's own [min, max] (the zero point may
+// fall outside [0, maxq]); a constant group, or one whose real zero point
+// lies more than 2^20 levels away (w / s then has an fp32 ulp of 1/16 level
+// or more), takes the widened range.  An all-zero group gets the range
+// [-1, 1] (zero point exactly 2^(bits-1)).
 __device__ __forceinline__ GroupParams group_params(const float (&cur)[4], const float (&nxt)[12],
                                                     int m, int jj, int l, int g, int bw,
                                                     const float* __restrict__ wrow, int64_t c0,
-                                                    int64_t d, bool live, int bits,
+                                                    int64_t d, bool live, int bits, bool pure,
                                                     const uint8_t* __restrict__ dead_mask) {
     const int j = 32 * m + jj;
-    float lo = 0.f, hi = 0.f;
+    float lo = pure ? INFINITY : 0.f, hi = pure ? -INFINITY : 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int c = 32 * m + 4 * l + i;
@@ -122,6 +126,14 @@ __device__ __forceinline__ GroupParams group_params(const float (&cur)[4], const
         hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
     }
     const float maxq = static_cast<float>((1 << bits) - 1);
+    if (pure) {
+        bool widen = !(hi > lo);
+        if (!widen) widen = fabsf(lo / ((hi - lo) / maxq)) > 1048576.f;
+        if (widen) {
+            lo = fminf(lo, 0.f);
+            hi = fmaxf(hi, 0.f);
+        }
+    }
     GroupParams p;
     if (hi == lo) {
         p.s = 2.f / maxq;
@@ -155,7 +167,7 @@ template <bool kSmallGroup,  // group_size < 32: groups start inside a chunk
           bool kFull>        // a full 128-column block (no column guard)
 __global__ void __launch_bounds__(kWarps * 32, 4)
     block_quant_kernel(const __grid_constant__ CUtensorMap tmu, float* __restrict__ W, int64_t r,
-                       int64_t d, int64_t ldw, int64_t c0, int bw, int bits, int g,
+                       int64_t d, int64_t ldw, int64_t c0, int bw, int bits, int g, int pure,
                        uint8_t* __restrict__ codes, float* __restrict__ scales,
                        int32_t* __restrict__ zeros, float* __restrict__ err_out,
                        int64_t err_ld, const uint8_t* __restrict__ dead_mask, int32_t* status) {
@@ -260,7 +272,8 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
     for (int m = 0; m < 4; ++m) {
         if (32 * m >= bw) break;
         if (!kSmallGroup && ((c0 + 32 * m) % g) == 0) {
-            gp = group_params(cur, nxt, m, 0, l, g, bw, wrow, c0, d, live, bits, dead_mask);
+            gp = group_params(cur, nxt, m, 0, l, g, bw, wrow, c0, d, live, bits, pure != 0,
+                              dead_mask);
             if (live && l == 0) {
                 const int64_t grp = (c0 + 32 * m) / g;
                 scales[grp * r + row] = gp.s;
@@ -279,7 +292,8 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
             const int j = 32 * m + jj;
             if (kFull || j < bw) {
                 if (kSmallGroup && ((c0 + j) % g) == 0) {
-                    gp = group_params(cur, nxt, m, jj, l, g, bw, wrow, c0, d, live, bits, dead_mask);
+                    gp = group_params(cur, nxt, m, jj, l, g, bw, wrow, c0, d, live, bits, pure != 0,
+                                      dead_mask);
                     if (live && l == 0) {
                         const int64_t grp = (c0 + j) / g;
                         scales[grp * r + row] = gp.s;
@@ -456,9 +470,11 @@ size_t quant_min_workspace_bytes(int64_t d_row, int block) {
 // form) when a group size does not fit it.
 gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw, const float* U,
                             const int32_t* perm, const uint8_t* dead, int desc_act, int bits,
-                            int group, int block, uint8_t* codes, float* scales, int32_t* zeros,
-                            int32_t* status, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                            int group, int block, int pure_minmax, uint8_t* codes, float* scales,
+                            int32_t* zeros, int32_t* status, void* ws, size_t ws_bytes,
+                            cudaStream_t stream) {
     if (block != kBlock) return GPTQ_ERR_UNSUPPORTED;
+    const int pure = pure_minmax != 0 ? 1 : 0;
     const int g = (group == -1 || group > d_col) ? static_cast<int>(d_col) : group;
     const int nb = static_cast<int>(num_blocks(d_col));
     int defer = nb < kMaxDefer ? nb : kMaxDefer;
@@ -518,7 +534,7 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
         // still be writing U
         return launch_kernel(b > 0 || permuted, bw == kBlock ? qfull : qpart, dim3(qgrid),
                              dim3(kWarps * 32), q_smem, stream, tU, W, d_row, d_col, ldw, c0, bw,
-                             bits, g, codes, scales, zeros,
+                             bits, g, pure, codes, scales, zeros,
                              err + static_cast<int64_t>(b - run0) * kBlock, err_ld, dead_mask,
                              status) == cudaSuccess;
     };

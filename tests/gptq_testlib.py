@@ -81,11 +81,12 @@ def lower_rel_err(Hg: np.ndarray, Ho: np.ndarray) -> float:
 
 
 def gpu_quantize(H_fp32: np.ndarray, W: torch.Tensor, bits: int, group_size: int,
-                 desc_act: bool, damp: float = 0.01) -> dict:
+                 desc_act: bool, damp: float = 0.01, pure: bool = False) -> dict:
     """prepare_hinv + quantize_layer + pack on the GPU from a given H."""
     g = gpu()
     d_row, d_col = W.shape
-    cfg = g.GPTQConfig(bits=bits, group_size=group_size, desc_act=desc_act, damp=damp)
+    cfg = g.GPTQConfig(bits=bits, group_size=group_size, desc_act=desc_act, damp=damp,
+                       pure_minmax=pure)
     ws = torch.empty(g.gptq_workspace_size(cfg, d_row, d_col), dtype=torch.uint8, device="cuda")
     Hd = torch.from_numpy(np.ascontiguousarray(H_fp32, dtype=np.float32)).cuda()
     U = torch.empty(d_col, d_col, dtype=torch.float32, device="cuda")
@@ -111,7 +112,8 @@ def gpu_quantize(H_fp32: np.ndarray, W: torch.Tensor, bits: int, group_size: int
 def compare_quantization(H64: np.ndarray, W: torch.Tensor, out: dict, bits: int,
                          group_size: int, desc_act: bool, damp: float = 0.01,
                          rows=None, H_loss: np.ndarray | None = None,
-                         strict_free: bool = True, U_oracle: np.ndarray | None = None) -> dict:
+                         strict_free: bool = True, U_oracle: np.ndarray | None = None,
+                         pure: bool = False) -> dict:
     """Check one GPU quantization against the oracle run on H64 (the exact H
     the GPU was given, as float64).  `rows` restricts the column loop to a
     sample of rows.  `U_oracle` (float64) may pass a precomputed inverse
@@ -126,18 +128,18 @@ def compare_quantization(H64: np.ndarray, W: torch.Tensor, out: dict, bits: int,
     wq, scales = out["w_at_quant"][sel], out["scales"][:, sel]
     d = W0.shape[1]
     forced_args = dict(forced_codes=codes, forced_zeros=zeros, forced_w=wq,
-                       forced_scales=scales, tau=TAU)
+                       forced_scales=scales, tau=TAU, pure=pure)
     if d <= 4096 and U_oracle is None:
         # the definition: explicit per-column elimination of H^-1
         Minv = oracle.inverse(prep["H_damped"])
         forced = oracle.gptq_columns(W0, Minv, bits, group_size, **forced_args)
-        free = oracle.gptq_columns(W0, Minv, bits, group_size)
+        free = oracle.gptq_columns(W0, Minv, bits, group_size, pure=pure)
     else:
         # too slow to eliminate on the host: the same loop driven by U's rows
         # (U from a library Cholesky and triangular inverse; pinned equal)
         U = oracle.upper_factor_flip(prep["H_damped"]) if U_oracle is None else U_oracle
         forced = oracle.gptq_columns_u(W0, U, bits, group_size, **forced_args)
-        free = oracle.gptq_columns_u(W0, U, bits, group_size)
+        free = oracle.gptq_columns_u(W0, U, bits, group_size, pure=pure)
     st = forced.stats
     free_match = float(np.mean(free.codes == codes))
     free_maxdiff = int(np.abs(free.codes.astype(int) - codes.astype(int)).max())
@@ -149,7 +151,7 @@ def compare_quantization(H64: np.ndarray, W: torch.Tensor, out: dict, bits: int,
     walk_match = None
     if out.get("U") is not None:
         # the column walk alone: the oracle given the GPU's own U
-        walk = oracle.gptq_columns_u(W0, out["U"], bits, group_size)
+        walk = oracle.gptq_columns_u(W0, out["U"], bits, group_size, pure=pure)
         walk_match = float(np.mean(walk.codes == codes))
     srel = float(np.max(np.abs(scales - forced.scales) / np.abs(forced.scales)))
     Hl = prep["H_undamped"] if H_loss is None else H_loss
@@ -157,7 +159,7 @@ def compare_quantization(H64: np.ndarray, W: torch.Tensor, out: dict, bits: int,
     Qo = oracle.dequantize(free.codes, free.scales, free.zeros, group_size)
     loss_g = oracle.proxy_loss(W0, Qg, Hl)
     loss_o = oracle.proxy_loss(W0, Qo, Hl)
-    rc, rs, rz = oracle.rtn(W0, bits, group_size)
+    rc, rs, rz = oracle.rtn(W0, bits, group_size, pure=pure)
     loss_rtn = oracle.proxy_loss(W0, oracle.dequantize(rc, rs, rz, group_size), Hl)
     res = dict(code_ties=st["code_ties"], code_invalid=st["code_invalid"],
                zero_ties=st["zero_ties"], zero_invalid=st["zero_invalid"],
@@ -178,5 +180,7 @@ def compare_quantization(H64: np.ndarray, W: torch.Tensor, out: dict, bits: int,
     if strict_free:
         assert free_match >= 0.999, res
     assert codes.max() <= (1 << bits) - 1
+    if not pure:
+        assert zeros.min() >= 0 and zeros.max() <= (1 << bits) - 1
     assert np.array_equal(out["packed"][sel], oracle.pack(codes, bits))
     return res

@@ -240,6 +240,31 @@ def test_quantize_layer_matches_oracle(d_row, d_col, n, kind, bits, g, desc_act)
     compare_quantization(H.astype(np.float64), W, out, bits, g, desc_act)
 
 
+@pytest.mark.parametrize("d_row,d_col,n,kind,bits,g,desc_act,offset",
+                         [(256, 512, 2048, "correlated", 4, 128, False, 0.0),
+                          (64, 384, 2048, "student_t", 3, 32, True, 0.03),
+                          (40, 256, 1024, "half_normal", 2, 8, True, 0.0),
+                          (33, 512, 2048, "student_t", 4, -1, False, -0.12),
+                          (16, 1024, 4096, "student_t", 8, 256, False, 0.12)])
+def test_pure_minmax_range_matches_oracle(d_row, d_col, n, kind, bits, g, desc_act, offset):
+    """The pure min-max option (each group's own [min, max]): weights
+    shifted off zero so that many groups are one-signed and get zero points
+    outside the code range; small groups (8) make one-signed groups common
+    without a shift."""
+    W, X = workloads.small_layer(d_row, d_col, n, seed=d_row * 5 + d_col, kind=kind)
+    W = W + offset
+    H = oracle.hessian(X).astype(np.float32)
+    out = gpu_quantize(H, W, bits, g, desc_act, pure=True)
+    # at 8 bits a level is 16 times finer than at 4, so the same fp32 drift
+    # puts 16 times more codes on ties: the free-running rate is reported only
+    res = compare_quantization(H.astype(np.float64), W, out, bits, g, desc_act, pure=True,
+                               strict_free=bits < 8)
+    if offset != 0.0:
+        z = out["zeros"]
+        assert z.min() < 0 or z.max() > (1 << bits) - 1  # one-signed groups occurred
+    assert res["loss_gpu"] < res["loss_rtn"]
+
+
 @pytest.mark.parametrize("d_row,d_col,g,damp,desc_act", [(24, 2048, 1024, 0.01, False),
                                                          (24, 2048, 1024, 0.005, True),
                                                          (48, 768, 32, 0.005, True)])
@@ -395,3 +420,32 @@ def test_quantize_layer_on_strided_and_offset_weights(pad, offset):
     assert np.array_equal(Wv.cpu().numpy(), ref["w_at_quant"])
     outside = torch.cat([buf[:, :offset], buf[:, offset + d_col:]], dim=1)
     assert bool((outside == 7.0).all())
+
+
+# ------------------------------------------------ streaming calibration (hook)
+@pytest.mark.parametrize("d,shapes", [(384, [(2, 700), (3, 128), (1, 5000)]),
+                                      (200, [(4, 33), (1, 1), (2, 900)])])
+def test_forward_hook_accumulates_the_layer_inputs(d, shapes):
+    """HessianAccumulator attached to a Linear layer as a forward pre-hook
+    sums H = 2 X^T X over every calibration batch that flows through it, in
+    any leading shape (d = 200: rows copied into a 16-byte pitch); compared
+    with the oracle on all the tokens seen."""
+    from post_weight_quantization_gptq_b200.calibration import HessianAccumulator
+    lin = torch.nn.Linear(d, 48, bias=False, dtype=torch.bfloat16, device="cuda")
+    acc = HessianAccumulator(d).attach(lin)
+    seen = []
+    for i, (b, t) in enumerate(shapes):
+        _, X = workloads.small_layer(1, d, b * t, seed=100 + i, kind="student_t")
+        x = X.reshape(b, t, d).cuda()
+        with torch.no_grad():
+            lin(x)
+        seen.append(X)
+    acc.detach()
+    with torch.no_grad():
+        lin(torch.ones(3, d, dtype=torch.bfloat16, device="cuda"))  # not accumulated
+    acc.check()
+    Xall = torch.cat(seen)
+    assert acc.tokens == Xall.shape[0]
+    # separate calls, each drained into H once (fp32 sums; the tensor cores'
+    # accumulation drifts by ~2^-25 per step within a call): well inside 1e-3
+    assert lower_rel_err(acc.H.cpu().numpy(), oracle.hessian(Xall)) <= 1e-4
