@@ -58,6 +58,9 @@ def parse():
     p.add_argument("--dequant-matmul", type=int, default=0, metavar="TOKENS",
                    help="instead of the quantizer step, time the product of TOKENS tokens with a "
                         "quantized Llama-70B down_proj (gptq_dequant_matmul)")
+    p.add_argument("--dequant-gemm", type=int, default=0, metavar="TOKENS",
+                   help="instead of the quantizer step, time the many-token product of TOKENS "
+                        "tokens with a quantized Llama-70B down_proj (gptq_dequant_gemm, tcgen05)")
     p.add_argument("--gemm-peaks", action="store_true",
                    help="instead of the quantizer step, measure the library-GEMM denominators of the "
                         "fp32 stages: cuBLAS 8192^3 fp32 with TF32 tensor cores and with plain FFMA")
@@ -534,13 +537,17 @@ def stage_rooflines(wl, pk, which, stage_ms, layer_ms):
 
 # ---------------------------------------------------------------- the product
 def run_dequant_matmul(args, rank: int, world: int, dist):
-    """Y = X W_hat^T for a quantized 8192 x 28672 layer (4-bit, g128, act-order),
-    decode form; HBM-bound on the packed words for one token."""
+    """Y = X W_hat^T for a quantized 8192 x 28672 layer (4-bit, g128, act-order):
+    the decode form (HBM-bound on the packed words for one token), or with
+    --dequant-gemm the many-token form on the tensor cores (bf16 dense
+    contraction, 2 tokens x d_row x d_col flop)."""
     import post_weight_quantization_gptq_b200 as g
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
-    n_tok, d_row, d_col, bits, gs = args.dequant_matmul, 8192, 28672, 4, 128
+    gemm = args.dequant_gemm > 0
+    n_tok = args.dequant_gemm if gemm else args.dequant_matmul
+    d_row, d_col, bits, gs = 8192, 28672, 4, 128
     gen = torch.Generator(device=dev)
     gen.manual_seed(4321 + rank)
     ng = d_col // gs
@@ -551,13 +558,22 @@ def run_dequant_matmul(args, rank: int, world: int, dist):
     perm = torch.randperm(d_col, device=dev, generator=gen).to(torch.int32)
     X = torch.randn(n_tok, d_col, device=dev, generator=gen).to(torch.bfloat16)
     Y = torch.empty(n_tok, d_row, dtype=torch.float32, device=dev)
-    ws = torch.empty(g.gptq_dequant_matmul_workspace_size(n_tok, d_col), dtype=torch.uint8,
-                     device=dev)
+    wsz = (g.gptq_dequant_gemm_workspace_size if gemm else g.gptq_dequant_matmul_workspace_size)(
+        n_tok, d_col)
+    ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+
+    def product():
+        if gemm:
+            g.gptq_dequant_gemm(X, packed, scales, zeros, perm, bits, gs, Y, ws, st)
+        else:
+            g.gptq_dequant_matmul(X, packed, scales, zeros, perm, bits, gs, Y, ws)
+
     for _ in range(args.warmup):
         flush.fill_(1)
-        g.gptq_dequant_matmul(X, packed, scales, zeros, perm, bits, gs, Y, ws)
+        product()
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(K)]
@@ -570,7 +586,7 @@ def run_dequant_matmul(args, rank: int, world: int, dist):
     for k in range(K):
         flush.fill_(1)
         ev[k][0].record(stream)
-        g.gptq_dequant_matmul(X, packed, scales, zeros, perm, bits, gs, Y, ws)
+        product()
         ev[k][1].record(stream)
     torch.cuda.synchronize(dev)
     if dist is not None:
@@ -581,24 +597,37 @@ def run_dequant_matmul(args, rank: int, world: int, dist):
     ms_max = max_over_ranks(ms, dist, dev)
     if rank != 0:
         return
+    if g.gptq_sync_status(st) != 0:
+        raise RuntimeError("device status error in the timed products")
     pk, which = peaks()
     nbytes = (d_row * d_col * bits // 8 + 8 * ng * d_row + 2 * n_tok * d_col + 4 * d_col
               + 4 * n_tok * d_row)
     gbs = nbytes / (ms / 1e3) / 1e9
     peak = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    if gemm:
+        flops = 2.0 * n_tok * d_row * d_col
+        tf = flops / (ms / 1e3) / 1e12
+        bpk = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        roof = {"kernel": "dequant_gemm_kernel", "bound": "tensor", "achieved": tf, "peak": bpk,
+                "peak_source": f"{which} bf16 dense (burst)", "unit": "TFLOP/s", "frac": tf / bpk,
+                "traffic": None,
+                "algorithmic": f"2 tokens d_row d_col = {flops:.4e} flop (bf16 operands, fp32 sums)"}
+    else:
+        roof = {"kernel": "dequant_matmul_kernel", "bound": "hbm", "achieved": gbs,
+                "peak": peak, "peak_source": f"{which} HBM copy", "unit": "GB/s",
+                "frac": gbs / peak, "traffic": None,
+                "algorithmic": f"packed codes + scales + zeros + X + perm + Y = {nbytes} bytes"}
     line = {
         "metric": f"dequantized product with a quantized layer ({n_tok} token(s)): weights/s",
         "value": world * d_row * d_col / (ms_max / 1e3), "unit": "weights/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16-in/fp32",
         "data": "synthetic (seeded random codes, scales, zeros, act-order permutation)",
-        "config": {"workload": "llama70b_down_proj_dequant_matmul", "d_row": d_row, "d_col": d_col,
+        "config": {"workload": "llama70b_down_proj_dequant_" + ("gemm" if gemm else "matmul"),
+                   "d_row": d_row, "d_col": d_col,
                    "tokens": n_tok, "bits": bits, "group_size": gs, "desc_act": True,
                    "l2": "flushed between steps (256 MiB write)"},
-        "roofline": {"kernel": "dequant_matmul_kernel", "bound": "hbm", "achieved": gbs,
-                     "peak": peak, "peak_source": f"{which} HBM copy", "unit": "GB/s",
-                     "frac": gbs / peak, "traffic": None,
-                     "algorithmic": f"packed codes + scales + zeros + X + perm + Y = {nbytes} bytes"},
+        "roofline": roof,
         "gpu_launches": launches, "clocks": clocks.summary(),
     }
     print(json.dumps(line), flush=True)
@@ -623,7 +652,7 @@ def main():
         run_gemm_peaks()
         return
     try:
-        if args.dequant_matmul > 0:
+        if args.dequant_matmul > 0 or args.dequant_gemm > 0:
             run_dequant_matmul(args, rank, world, dist)
         else:
             run_ours(args, rank, world, dist)

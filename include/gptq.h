@@ -320,6 +320,38 @@ gptq_status gptq_dequant_matmul(const uint16_t *X, int64_t n_tok, int64_t d_col,
 size_t gptq_dequant_matmul_workspace_size(int64_t n_tok, int64_t d_col);
 
 /*
+ * Using the quantized layer, many-token (prefill) form -- Y = X W_hat^T on the
+ * tensor cores ("GPTQ (GPT Quantization)", "Limitations", items 1-2: weights
+ * dequantized to 16 bits before each product, activations at 16 bits).  Each
+ * stage of 64 codes of a 256-row slice of the packed layer is dequantized
+ * into a bf16 tile in shared memory and multiplied with the bf16 activations
+ * (tcgen05, fp32 accumulation):
+ *   W_hat[n][k] = bf16_rne( fp32 scales[k/g][n] * (code[n][k] - zeros[k/g][n]) )
+ *   Y[t][n]     = sum_k X[t][perm[k]] * W_hat[n][k]
+ * (the products of two bf16 values are exact; the sums are fp32).
+ *   X, packed, scales, zeros, perm, Y, ldx, ldy  as gptq_dequant_matmul; packed
+ *           16-byte aligned.
+ *   dev_status  device int32 (may be NULL) receiving GPTQ_ERR_TIMEOUT if a
+ *           bounded wait runs out.
+ *   ws      caller-owned device workspace, 256-byte aligned, of at least
+ *           gptq_dequant_gemm_workspace_size(n_tok, d_col) bytes, used when
+ *           perm is given or X's rows are not 16-byte aligned (the tokens are
+ *           gathered into quantization order as bf16); may be NULL otherwise.
+ *   Supported: bits 2, 4 or 8; d_col a multiple of 64; group size -1, >= d_col
+ *   or a multiple of 8; n_tok <= 2^24; otherwise GPTQ_ERR_UNSUPPORTED /
+ *   GPTQ_ERR_INVALID_ARG.  n_tok == 0 is a no-op.  Deterministic.
+ */
+gptq_status gptq_dequant_gemm(const uint16_t *X, int64_t n_tok, int64_t d_col, int64_t ldx,
+                              const uint32_t *packed, const float *scales, const int32_t *zeros,
+                              const int32_t *perm, int64_t d_row, int32_t bits,
+                              int32_t group_size, float *Y, int64_t ldy, int32_t *dev_status,
+                              void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Workspace bytes gptq_dequant_gemm needs (n_tok x d_col bf16); 0 for invalid
+ * sizes. */
+size_t gptq_dequant_gemm_workspace_size(int64_t n_tok, int64_t d_col);
+
+/*
  * Waits for `stream`, then copies the device status word to *out.
  * Returns GPTQ_ERR_CUDA if the wait or the copy fails, else GPTQ_OK (the
  * device-side status itself is in *out).

@@ -17,6 +17,7 @@ is "parity unpinned".
 from .gptq import (  # noqa: F401
     GPTQResult,
     act_order,
+    bf16_round,
     damp_lambda,
     dead_columns,
     dequant_matmul,

@@ -438,15 +438,36 @@ def unpack(packed, d: int, bits: int) -> np.ndarray:
 # 1-2): weight-only quantization, the activations stay at 16 bits and the
 # integer weights are dequantized before each product
 # --------------------------------------------------------------------------
+def bf16_round(x) -> np.ndarray:
+    """Round float32 values to the nearest bfloat16 (ties to even), returned
+    as float64: the 16 high bits of the float32 pattern after adding
+    0x7FFF plus the lowest kept bit (finite inputs)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000).astype(np.uint32)
+    return r.view(np.float32).astype(np.float64)
+
+
 def dequant_matmul(X, packed, scales, zeros, perm, bits: int, group_size: int,
-                   d_col: int) -> np.ndarray:
+                   d_col: int, weights_bf16: bool = False) -> np.ndarray:
     """Y = X W_hat^T for a layer quantized by this library: X is tokens x d_col
     in the layer's original column order, the packed codes are in quantization
     order, and W_hat[:, perm[k]] = scale[k // g] * (code[:, k] - zero[k // g]).
-    perm None is the identity.  float64 throughout."""
+    perm None is the identity.  float64 throughout, except with weights_bf16:
+    each weight is then the 16-bit value the "Limitations" passage speaks of,
+    bf16_round(float32(scale) * float32(code - zero)) (one float32 product,
+    rounded to the nearest bf16)."""
     Xf = _f64(X)
     Xq = Xf if perm is None else Xf[:, np.asarray(perm)]
-    Q = dequantize(unpack(packed, d_col, bits), scales, zeros, group_size)
+    if weights_bf16:
+        codes = unpack(packed, d_col, bits)
+        r, d = codes.shape
+        g = _g(d, group_size)
+        gi = np.arange(d) // g
+        s = np.asarray(scales, dtype=np.float32)[gi, :].T
+        z = np.asarray(zeros, dtype=np.float32)[gi, :].T
+        Q = bf16_round(s * (codes.astype(np.float32) - z))
+    else:
+        Q = dequantize(unpack(packed, d_col, bits), scales, zeros, group_size)
     return Xq @ Q.T
 
 

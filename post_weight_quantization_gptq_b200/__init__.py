@@ -16,6 +16,7 @@ Stages (see the header for the exact contracts):
 * ``gptq_quantize_layer``      column walk with OBQ error feedback and lazy updates
 * ``gptq_pack``                codes -> uint32 bit stream (8 codes per word at 4 bits)
 * ``gptq_dequant_matmul``      Y = X W_hat^T from the packed layer (decode form)
+* ``gptq_dequant_gemm``        the same for many tokens on the tensor cores (bf16 W_hat)
 """
 from __future__ import annotations
 
@@ -27,6 +28,7 @@ import torch
 __all__ = [
     "GPTQConfig", "GPTQError", "gptq_hessian_accumulate", "gptq_hessian_accumulate_host",
     "gptq_hessian_staging_size", "gptq_prepare_hinv", "gptq_dequant_matmul", "gptq_dequant_matmul_workspace_size",
+    "gptq_dequant_gemm", "gptq_dequant_gemm_workspace_size",
     "gptq_quantize_layer", "gptq_quantize_layer_noalloc", "gptq_noalloc_scratch_bytes", "gptq_pack", "gptq_workspace_size", "gptq_sync_status",
     "gptq_status_string", "gptq_version", "gptq_launch_counter", "gptq_debug_arm_wait_probe",
     "library_path", "n_groups", "packed_words",
@@ -89,6 +91,9 @@ def _load():
         "gptq_dequant_matmul": ([P, i64, i64, i64, P, P, P, P, i64, i32, i32, P, i64, P,
                                  ctypes.c_size_t, P], ctypes.c_int),
         "gptq_dequant_matmul_workspace_size": ([i64, i64], ctypes.c_size_t),
+        "gptq_dequant_gemm": ([P, i64, i64, i64, P, P, P, P, i64, i32, i32, P, i64, P, P,
+                               ctypes.c_size_t, P], ctypes.c_int),
+        "gptq_dequant_gemm_workspace_size": ([i64, i64], ctypes.c_size_t),
         "gptq_quantize_layer_noalloc": ([P, i64, i64, i64, P, P, P, cfgp, P, P, P, P, P],
                                         ctypes.c_int),
         "gptq_noalloc_scratch_bytes": ([], ctypes.c_size_t),
@@ -317,6 +322,38 @@ def gptq_dequant_matmul(X: torch.Tensor, packed: torch.Tensor, scales: torch.Ten
 
 def gptq_dequant_matmul_workspace_size(n_tok: int, d_col: int) -> int:
     return int(_lib.gptq_dequant_matmul_workspace_size(int(n_tok), int(d_col)))
+
+
+def gptq_dequant_gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+                      zeros: torch.Tensor, perm: torch.Tensor | None, bits: int, group_size: int,
+                      Y: torch.Tensor, ws: torch.Tensor | None = None,
+                      dev_status: torch.Tensor | None = None, stream=None) -> None:
+    """Y = X W_hat^T for a quantized layer, many-token form on the tensor
+    cores (W_hat dequantized to bf16 per stage): X (tokens x d_col bf16,
+    original column order), packed / scales / zeros / perm as the quantizer
+    wrote them, Y (tokens x d_row fp32) overwritten; ws (bytes of
+    gptq_dequant_gemm_workspace_size) is needed with a permutation."""
+    _cuda(X, "X", torch.bfloat16)
+    _cuda(packed, "packed")
+    _cuda(scales, "scales", torch.float32)
+    _cuda(zeros, "zeros", torch.int32)
+    _cuda(Y, "Y", torch.float32)
+    if perm is not None:
+        _cuda(perm, "perm", torch.int32)
+    for t, name in ((packed, "packed"), (scales, "scales"), (zeros, "zeros")):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    n_tok, d_col = X.shape
+    d_row = packed.shape[0]
+    _check(_lib.gptq_dequant_gemm(_ptr(X), n_tok, d_col, _row_major(X, "X"), _ptr(packed),
+                                  _ptr(scales), _ptr(zeros), _ptr(perm), d_row, int(bits),
+                                  int(group_size), _ptr(Y), _row_major(Y, "Y"), _ptr(dev_status),
+                                  _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                  _stream(stream)), "gptq_dequant_gemm")
+
+
+def gptq_dequant_gemm_workspace_size(n_tok: int, d_col: int) -> int:
+    return int(_lib.gptq_dequant_gemm_workspace_size(int(n_tok), int(d_col)))
 
 
 def gptq_debug_arm_wait_probe(kernel: int, limit_ns: int) -> None:

@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libgptq_b200.so")
-SOURCES = ["api.cu", "hessian.cu", "hessian_host.cu", "prep.cu", "chol.cu", "quant.cu", "pack.cu", "dequant_matmul.cu", "noalloc.cu", "tmap.cu"]
+SOURCES = ["api.cu", "hessian.cu", "hessian_host.cu", "prep.cu", "chol.cu", "quant.cu", "pack.cu", "dequant_matmul.cu", "dequant_gemm.cu", "noalloc.cu", "tmap.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--shared",
          "-Xptxas", "-warn-spills"]

@@ -227,6 +227,39 @@ gptq_status gptq_dequant_matmul(const uint16_t* X, int64_t n_tok, int64_t d_col,
                                                      stream));
 }
 
+size_t gptq_dequant_gemm_workspace_size(int64_t n_tok, int64_t d_col) {
+    if (n_tok <= 0 || d_col <= 0 || d_col > kMaxDim) return 0;
+    return gptq::dequant_gemm_workspace_bytes(n_tok, d_col);
+}
+
+gptq_status gptq_dequant_gemm(const uint16_t* X, int64_t n_tok, int64_t d_col, int64_t ldx,
+                              const uint32_t* packed, const float* scales, const int32_t* zeros,
+                              const int32_t* perm, int64_t d_row, int32_t bits, int32_t group_size,
+                              float* Y, int64_t ldy, int32_t* dev_status, void* ws,
+                              size_t ws_bytes, cudaStream_t stream) {
+    if (X == nullptr || packed == nullptr || scales == nullptr || zeros == nullptr || Y == nullptr)
+        return GPTQ_ERR_INVALID_ARG;
+    if (n_tok < 0 || n_tok > (int64_t{1} << 24) || d_col <= 0 || d_row <= 0 || d_col > kMaxDim ||
+        d_row > kMaxDim || ldx < d_col || ldy < d_row)
+        return GPTQ_ERR_INVALID_ARG;
+    if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return GPTQ_ERR_INVALID_ARG;
+    if (group_size == 0 || group_size < -1) return GPTQ_ERR_INVALID_ARG;
+    if (!aligned(packed, 16) || !aligned(scales, 4) || !aligned(zeros, 4) || !aligned(Y, 4) ||
+        !aligned(X, 2))
+        return GPTQ_ERR_INVALID_ARG;
+    // whole 64-code stages, 16-byte packed rows, no 8-code chunk across two groups
+    const int64_t g = (group_size == -1 || group_size > d_col) ? d_col : group_size;
+    if (bits == 3 || d_col % 64 != 0 || (g % 8 != 0 && g != d_col)) return GPTQ_ERR_UNSUPPORTED;
+    if (n_tok == 0) return GPTQ_OK;
+    const bool gather = perm != nullptr || (ldx % 8) != 0 || !aligned(X, 16);
+    if (gather && (ws == nullptr || !aligned(ws, 256) ||
+                   ws_bytes < gptq::dequant_gemm_workspace_bytes(n_tok, d_col)))
+        return GPTQ_ERR_WORKSPACE;
+    return launch_status(gptq::launch_dequant_gemm(X, n_tok, d_col, ldx, packed, scales, zeros, perm,
+                                                   d_row, bits, group_size, Y, ldy, dev_status, ws,
+                                                   stream));
+}
+
 gptq_status gptq_sync_status(cudaStream_t stream, const int32_t* dev_status, int32_t* out) {
     if (dev_status == nullptr || out == nullptr) return GPTQ_ERR_INVALID_ARG;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return GPTQ_ERR_CUDA;

@@ -245,6 +245,11 @@ __device__ __forceinline__ void sts128(uint32_t addr, float4 v) {
                  "f"(v.z), "f"(v.w)
                  : "memory");
 }
+__device__ __forceinline__ void sts128_u(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
 __device__ __forceinline__ float4 lds128(uint32_t addr) {
     float4 v;
     asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"

@@ -1,0 +1,318 @@
+// Using the quantized layer, many-token (prefill) form: Y = X W_hat^T on the
+// 5th-generation tensor cores.
+//
+// "GPTQ (GPT Quantization)", "Limitations" (items 1-2): the quantization is
+// weight-only -- activations stay at 16 bits -- and the integer weights are
+// dequantized to 16 bits before each product.  Here each CTA dequantizes a
+// 256-row slice of the packed layer into bf16 tiles in shared memory, stage by
+// stage, and the tensor cores multiply them with the (act-order gathered) bf16
+// activations:
+//   W_hat[n][k] = bf16( fp32(s[k/g][n]) * (q[n][k] - z[k/g][n]) )   (fp32 product,
+//                 rounded to nearest-even bf16)
+//   Y[t][n]     = sum_k Xq[t][k] W_hat[n][k]     (exact bf16 products, fp32 sums)
+// with Xq[t][k] = X[t][perm[k]] (quantization order; gathered into the
+// workspace when perm is given).
+//
+// CTA tile: 256 tokens x 256 layer outputs, K in stages of 64.  Warp roles:
+//   warp 0      TMA: the stage's activations (256 x 64 bf16, 128-byte swizzle)
+//               and packed words (256 rows x 64 codes)
+//   warp 1      TMEM owner (512 columns: two 128-token accumulators of 256
+//               fp32 columns) and MMA issuer: per stage, 2 x 4 MMAs
+//               kind::f16 M=128 N=256 K=16, both operands K-major
+//   warps 2..9  dequantize: thread n turns row n's 64 codes of the stage into
+//               bf16 and writes them, 16 bytes at a time, in the 128-byte
+//               swizzled K-major layout the MMA reads (two alternating
+//               buffers); after the K loop they drain the accumulators
+// Every wait is bounded (GPTQ_ERR_TIMEOUT, as in the other tensor-core kernels).
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gptq {
+namespace {
+
+constexpr int TM = 256;                       // tokens per CTA tile
+constexpr int TN = 256;                       // layer outputs per CTA tile (MMA N)
+constexpr int BK = 64;                        // k per stage: 128 bytes of bf16
+constexpr int kStages = 3;
+constexpr int kABytes = TM * BK * 2;          // 32 KB
+constexpr int kBBytes = TN * BK * 2;          // 32 KB (one dequantized bf16 tile)
+constexpr int kPackedMax = TN * BK;           // packed words of a stage at 8 bits: 16 KB
+constexpr int kStageBytes = kABytes + kPackedMax;
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kIdesc = instr_desc(/*bf16*/ 1, /*A K-major*/ 0, /*B K-major*/ 0, 128, TN);
+constexpr int kSmemBytes = kStages * kStageBytes + 2 * kBBytes + 1024 + 256;
+
+struct Bars {
+    uint64_t full[kStages];   // TMA: activations + packed words landed
+    uint64_t empty[kStages];  // MMA: stage consumed
+    uint64_t bfull[2];        // dequant warps: bf16 tile written (256 arrivals)
+    uint64_t bempty[2];       // MMA: bf16 tile consumed
+    uint64_t acc_full;        // MMA: every product of the tile done
+    uint64_t drain;
+    uint32_t tmem;
+    int abort;
+};
+
+__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kThreads, 1)
+    dequant_gemm_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmp,
+                        const float* __restrict__ scales, const int32_t* __restrict__ zeros,
+                        float* __restrict__ Y, int64_t ldy, int n_tok, int d_row, int K, int g,
+                        int32_t* status) {
+    constexpr int kCpw = 32 / BITS;               // codes per packed word
+    constexpr int kWords = BK / kCpw;             // words per row per stage
+    constexpr int kRowBytes = kWords * 4;         // packed bytes per row per stage
+    constexpr uint32_t kMask = (1u << BITS) - 1u;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* bbuf = smem + kStages * kStageBytes;  // two bf16 tiles, 1024-aligned
+    Bars* bars = reinterpret_cast<Bars*>(bbuf + 2 * kBBytes);
+    volatile int* abort = &bars->abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * TN, t0 = blockIdx.y * TM;
+    const int nk = K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->bfull[b], 256);
+            mbar_init(&bars->bempty[b], 1);
+        }
+        mbar_init(&bars->acc_full, 1);
+        mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tma);
+        tma_prefetch_desc(&tmp);
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars->tmem, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int it = 0;
+            for (; it < nk && !*abort; ++it) {
+                const int st = it % kStages;
+                const uint32_t ph = (it / kStages) & 1u;
+                if (!mbar_wait(&bars->empty[st], ph ^ 1u, abort)) break;
+                uint8_t* a = smem + st * kStageBytes;
+                mbar_arrive_expect_tx(&bars->full[st], kABytes + TN * kRowBytes);
+                tma_load_2d(a, &tma, &bars->full[st], it * BK, t0);
+                tma_load_2d(a + kABytes, &tmp, &bars->full[st], it * kWords, n0);
+            }
+            // never leave with copies in flight (bounded even when aborting)
+            volatile int no_abort = 0;
+            const int last = it < kStages ? it : kStages;
+            for (int j = 0; j < last; ++j) {
+                const int i2 = it - 1 - j;
+                if (!mbar_wait(&bars->full[i2 % kStages], (i2 / kStages) & 1u, &no_abort)) {
+                    *abort = 1;
+                    break;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            bool ok = true;
+            for (int it = 0; it < nk && ok; ++it) {
+                const int st = it % kStages, b = it & 1;
+                if (!mbar_wait(&bars->full[st], (it / kStages) & 1u, abort) ||
+                    !mbar_wait(&bars->bfull[b], (it >> 1) & 1u, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a = smem_u32(smem + st * kStageBytes);
+                const uint32_t bt = smem_u32(bbuf + b * kBBytes);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_f16_ss(tmem + h * TN, smem_desc(a + h * (kABytes / 2) + kk * 32, 16, 1024, 2),
+                                   smem_desc(bt + kk * 32, 16, 1024, 2), kIdesc,
+                                   (it > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&bars->empty[st]);
+                mma_commit(&bars->bempty[b]);
+            }
+            if (ok) mma_commit(&bars->acc_full);
+            mma_commit(&bars->drain);
+            volatile int no_abort = 0;
+            if (!mbar_wait(&bars->drain, 0, &no_abort)) *abort = 1;
+        }
+    } else {
+        // ------------------------------------------------ dequantize
+        const int n = threadIdx.x - 64;  // row of the tile, 0..255
+        const int ng = n0 + n;
+        const bool live = ng < d_row;
+        int cur_g = -1;
+        float s = 0.f, z = 0.f;
+        bool ok = true;
+        for (int it = 0; it < nk; ++it) {
+            const int st = it % kStages, b = it & 1;
+            if (!mbar_wait(&bars->full[st], (it / kStages) & 1u, abort) ||
+                !mbar_wait(&bars->bempty[b], ((it >> 1) & 1u) ^ 1u, abort)) {
+                ok = false;
+                break;
+            }
+            const uint32_t* words = reinterpret_cast<const uint32_t*>(
+                smem + st * kStageBytes + kABytes + n * kRowBytes);
+            uint32_t w[kWords];
+#pragma unroll
+            for (int q = 0; q < kWords / 4; ++q) {
+                const uint4 v = reinterpret_cast<const uint4*>(words)[q];
+                w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+            }
+            const uint32_t row = smem_u32(bbuf + b * kBBytes) + n * 128;
+            // 8 codes (one 16-byte chunk of bf16) at a time
+#pragma unroll
+            for (int c = 0; c < BK / 8; ++c) {
+                const int k = it * BK + 8 * c;
+                const int gi = k / g;  // g is a multiple of 8: a chunk never spans two groups
+                if (gi != cur_g) {
+                    cur_g = gi;
+                    s = live ? __ldg(scales + static_cast<int64_t>(gi) * d_row + ng) : 0.f;
+                    z = live ? static_cast<float>(__ldg(zeros + static_cast<int64_t>(gi) * d_row + ng)) : 0.f;
+                }
+                float v[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int e = 8 * c + i;  // code index within the stage
+                    const uint32_t q = (w[e / kCpw] >> (BITS * (e % kCpw))) & kMask;
+                    v[i] = (static_cast<float>(q) - z) * s;
+                }
+                sts128_u(row + ((c ^ (n & 7)) << 4), make_uint4(bf16x2(v[0], v[1]), bf16x2(v[2], v[3]),
+                                                                 bf16x2(v[4], v[5]), bf16x2(v[6], v[7])));
+            }
+            fence_async_smem();
+            mbar_arrive(&bars->bfull[b]);
+        }
+        // ------------------------------------------------ drain: TMEM -> Y
+        if (ok && mbar_wait(&bars->acc_full, 0, abort)) {
+            tc_fence_after();
+            const int q = warp & 3;           // TMEM lane quarter of this warp
+            const int h = (warp - 2) >> 2;    // accumulator (token half)
+            const int t = t0 + h * 128 + 32 * q + lane;
+            float* yrow = Y + static_cast<int64_t>(t) * ldy;
+#pragma unroll 1
+            for (int c = 0; c < TN / 32; ++c) {
+                float v[32];
+                tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + h * TN + c * 32, v);
+                const int nb = n0 + 32 * c;
+                if (t < n_tok) {
+                    if (nb + 32 <= d_row && (reinterpret_cast<uintptr_t>(yrow + nb) & 15) == 0) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            *reinterpret_cast<float4*>(yrow + nb + 4 * j) =
+                                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (nb + j < d_row) yrow[nb + j] = v[j];
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+    if (threadIdx.x == 0 && bars->abort) report(status, GPTQ_ERR_TIMEOUT);
+}
+
+// Xq[t][k] = X[t][perm[k]] (bf16, row pitch K); perm entries outside [0, K)
+// are read as k.
+__global__ void gather_bf16_kernel(const uint16_t* __restrict__ X, int64_t ldx, int64_t n_tok,
+                                   int K, const int32_t* __restrict__ perm,
+                                   uint16_t* __restrict__ Xq) {
+    const int64_t total = n_tok * K;
+    for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t t = e / K, k = e - t * K;
+        int64_t col = perm != nullptr ? perm[k] : k;
+        if (col < 0 || col >= K) col = k;
+        Xq[e] = X[t * ldx + col];
+    }
+}
+
+template <int BITS>
+cudaError_t launch_bits(const CUtensorMap& ta, const CUtensorMap& tp, const float* scales,
+                        const int32_t* zeros, float* Y, int64_t ldy, int n_tok, int d_row, int K,
+                        int g, int32_t* status, cudaStream_t stream) {
+    auto kern = dequant_gemm_kernel<BITS>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((d_row + TN - 1) / TN, (n_tok + TM - 1) / TM);
+    kern<<<grid, kThreads, kSmemBytes, stream>>>(ta, tp, scales, zeros, Y, ldy, n_tok, d_row, K, g,
+                                                 status);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t dequant_gemm_workspace_bytes(int64_t n_tok, int64_t d_col) {
+    return ((static_cast<size_t>(n_tok) * d_col * 2 + 255) / 256) * 256;
+}
+
+gptq_status launch_dequant_gemm(const uint16_t* X, int64_t n_tok, int64_t d_col, int64_t ldx,
+                                const uint32_t* packed, const float* scales, const int32_t* zeros,
+                                const int32_t* perm, int64_t d_row, int bits, int group, float* Y,
+                                int64_t ldy, int32_t* status, void* ws, cudaStream_t stream) {
+    const int K = static_cast<int>(d_col);
+    const int g = (group == -1 || group > K) ? K : group;
+    const uint16_t* A = X;
+    int64_t lda = ldx;
+    int64_t launches = 1;
+    if (perm != nullptr || (ldx % 8) != 0 || (reinterpret_cast<uintptr_t>(X) & 15) != 0) {
+        uint16_t* Xq = static_cast<uint16_t*>(ws);
+        const int64_t total = n_tok * d_col;
+        const int64_t blocks = (total + 255) / 256;
+        const int gb = static_cast<int>(blocks < 8 * num_sms() ? blocks : 8 * num_sms());
+        gather_bf16_kernel<<<gb, 256, 0, stream>>>(X, ldx, n_tok, K, perm, Xq);
+        A = Xq;
+        lda = d_col;
+        ++launches;
+    }
+    CUtensorMap ta, tp;
+    const int64_t P = d_col * bits / 32;  // packed words per row
+    // the packed words move as raw 32-bit elements (the map's fp32 type only
+    // sizes them; nothing converts)
+    if (!make_tmap_2d(&ta, true, A, d_col, n_tok, lda, BK, TM, Swz::k128) ||
+        !make_tmap_2d(&tp, false, packed, P, d_row, P, BK * bits / 32, TN, Swz::kNone))
+        return GPTQ_ERR_INVALID_ARG;
+    cudaError_t e;
+    const int nt = static_cast<int>(n_tok), nr = static_cast<int>(d_row);
+    switch (bits) {
+        case 2: e = launch_bits<2>(ta, tp, scales, zeros, Y, ldy, nt, nr, K, g, status, stream); break;
+        case 4: e = launch_bits<4>(ta, tp, scales, zeros, Y, ldy, nt, nr, K, g, status, stream); break;
+        case 8: e = launch_bits<8>(ta, tp, scales, zeros, Y, ldy, nt, nr, K, g, status, stream); break;
+        default: return GPTQ_ERR_UNSUPPORTED;
+    }
+    if (e != cudaSuccess) return GPTQ_ERR_CUDA;
+    count_launches(launches);
+    return GPTQ_OK;
+}
+
+}  // namespace gptq

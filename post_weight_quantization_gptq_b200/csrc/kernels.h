@@ -100,6 +100,14 @@ gptq_status launch_dequant_matmul(const uint16_t* X, int64_t n_tok, int64_t d_co
                                   int bits, int group, float* Y, int64_t ldy, void* ws,
                                   cudaStream_t stream);
 
+// ---- using the quantized layer, many-token form (dequant_gemm.cu): tcgen05
+// bf16 GEMM with the weights dequantized into shared memory per stage
+size_t dequant_gemm_workspace_bytes(int64_t n_tok, int64_t d_col);
+gptq_status launch_dequant_gemm(const uint16_t* X, int64_t n_tok, int64_t d_col, int64_t ldx,
+                                const uint32_t* packed, const float* scales, const int32_t* zeros,
+                                const int32_t* perm, int64_t d_row, int bits, int group, float* Y,
+                                int64_t ldy, int32_t* status, void* ws, cudaStream_t stream);
+
 // ---- stage 5 (pack.cu)
 gptq_status launch_pack(const uint8_t* codes, int64_t d_row, int64_t d_col, int bits,
                         uint32_t* packed, cudaStream_t stream);

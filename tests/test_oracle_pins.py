@@ -500,3 +500,26 @@ def test_dequant_matmul_hand_example():
     # without the permutation the same codes meet the activations unreversed
     Y_id = oracle.dequant_matmul(X, packed, sc, ze, None, bits, gs, len(perm))
     assert Y_id[0, 1] == 1 * 16 + 2 * -14 + 3 * 16 + 4 * -14
+
+
+def test_bf16_dequantized_weights_hand_example():
+    """The many-token product's 16-bit weights ("GPTQ (GPT Quantization)",
+    "Limitations": weights dequantized to 16 bits before the product):
+    bf16 rounding to nearest, ties to even, worked by hand: 0.3 (float32
+    0.300000012) has the bf16 neighbours 0.30078125 (1.203125 x 2^-2) and
+    0.298828125 and rounds up; 1 + 2^-8 lies halfway between 1 and 1 + 2^-7
+    and goes to the even mantissa, 1; 1 + 3 2^-8 lies halfway between
+    1 + 2^-7 and 1 + 2^-6 and goes to 1 + 2^-6.  A one-row layer with scale
+    1 + 2^-8, zero point 0 and codes 1, 1 then gives X W_hat^T = 1 + 2 = 3
+    for X = [1, 2], against 3 + 3 2^-8 with the exact weights."""
+    got = oracle.bf16_round(np.array([0.3, 1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(1 + 2.0 ** -8)],
+                                     dtype=np.float32))
+    assert list(got) == [0.30078125, 1.0, 1.015625, -1.0]
+    codes = np.array([[1, 1, 0, 0, 0, 0, 0, 0]], dtype=np.uint8)
+    packed = oracle.pack(codes, 4)
+    X = np.array([[1.0, 2.0, 0, 0, 0, 0, 0, 0]])
+    sc = np.array([[1 + 2.0 ** -8]], dtype=np.float32)
+    ze = np.zeros((1, 1), dtype=np.int32)
+    assert oracle.dequant_matmul(X, packed, sc, ze, None, 4, 8, 8, weights_bf16=True)[0, 0] == 3.0
+    assert oracle.dequant_matmul(X, packed, sc, ze, None, 4, 8, 8)[0, 0] == 3 + 3 * 2.0 ** -8
+
