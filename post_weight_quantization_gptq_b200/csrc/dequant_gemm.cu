@@ -194,12 +194,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     s = live ? __ldg(scales + static_cast<int64_t>(gi) * d_row + ng) : 0.f;
                     z = live ? static_cast<float>(__ldg(zeros + static_cast<int64_t>(gi) * d_row + ng)) : 0.f;
                 }
+                // code q as the float 2^23 + q (its bits ORed into the
+                // mantissa of 2^23: no int-to-float conversion); subtracting
+                // 2^23 + z leaves q - z exactly, then one rounded product
+                const float off = 8388608.f + z;
                 float v[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int e = 8 * c + i;  // code index within the stage
                     const uint32_t q = (w[e / kCpw] >> (BITS * (e % kCpw))) & kMask;
-                    v[i] = (static_cast<float>(q) - z) * s;
+                    v[i] = (__uint_as_float(q | 0x4B000000u) - off) * s;
                 }
                 sts128_u(row + ((c ^ (n & 7)) << 4), make_uint4(bf16x2(v[0], v[1]), bf16x2(v[2], v[3]),
                                                                  bf16x2(v[4], v[5]), bf16x2(v[6], v[7])));

@@ -21,6 +21,7 @@
 //                       (3xTF32 tcgen05 GEMM, fp32-accurate)
 #include <cmath>
 #include <tuple>
+#include <type_traits>
 #include <vector>
 
 #include "common.cuh"
@@ -268,9 +269,11 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
     float t1 = __shfl_sync(0xffffffffu, cur[1], gbase);
     float t2 = __shfl_sync(0xffffffffu, cur[2], gbase);
 
-#pragma unroll 1
-    for (int m = 0; m < 4; ++m) {
-        if (32 * m >= bw) break;
+    // one 32-column chunk; m is a compile-time constant in each of the four
+    // instantiations, so the feedback into the later chunks (nxt) is exactly
+    // the live part: 3, 2, 1, 0 chunks
+    auto walk_chunk = [&](auto mc) {
+        constexpr int m = decltype(mc)::value;
         if (!kSmallGroup && ((c0 + 32 * m) % g) == 0) {
             gp = group_params(cur, nxt, m, 0, l, g, bw, wrow, c0, d, live, bits, pure != 0,
                               dead_mask);
@@ -287,55 +290,53 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
 #pragma unroll 1
         for (int jq = 0; jq < 8; ++jq) {
 #pragma unroll
-        for (int i4 = 0; i4 < 4; ++i4) {
-            const int jj = 4 * jq + i4;
-            const int j = 32 * m + jj;
-            if (kFull || j < bw) {
-                if (kSmallGroup && ((c0 + j) % g) == 0) {
-                    gp = group_params(cur, nxt, m, jj, l, g, bw, wrow, c0, d, live, bits, pure != 0,
-                                      dead_mask);
-                    if (live && l == 0) {
-                        const int64_t grp = (c0 + j) / g;
-                        scales[grp * r + row] = gp.s;
-                        zeros[grp * r + row] = static_cast<int32_t>(gp.zf);
+            for (int i4 = 0; i4 < 4; ++i4) {
+                const int jj = 4 * jq + i4;
+                const int j = 32 * m + jj;
+                if (kFull || j < bw) {
+                    if (kSmallGroup && ((c0 + j) % g) == 0) {
+                        gp = group_params(cur, nxt, m, jj, l, g, bw, wrow, c0, d, live, bits,
+                                          pure != 0, dead_mask);
+                        if (live && l == 0) {
+                            const int64_t grp = (c0 + j) / g;
+                            scales[grp * r + row] = gp.s;
+                            zeros[grp * r + row] = static_cast<int32_t>(gp.zf);
+                        }
                     }
-                }
-                const float* urow = Us + j * kBlock;
-                const float dj = dinv[j];
-                const float u1 = urow[(j + 1) & (kBlock - 1)];
-                const float u2 = urow[(j + 2) & (kBlock - 1)];
-                // q = clamp(rint(w / s) + z, 0, maxq) = rint(clamp(w / s, -z, maxq - z)) + z
-                // (z and maxq are integers); e = (w - s (q - z)) / U_jj
-                const float cq = round_even(fminf(fmaxf(wcur * gp.inv_s, -gp.zf), gp.hi));
-                const float e = fmaf(-(gp.s * dj), cq, wcur * dj);
-                const bool mine = l == jq;
-                qv[i4] = mine ? static_cast<uint32_t>(cq + gp.zf) : qv[i4];
-                ev[i4] = mine ? e : ev[i4];
-                // columns j+1 and j+2 for every lane: the owners' own updates, replicated
-                wcur = fmaf(-e, u1, t1);
-                t1 = fmaf(-e, u2, t2);
-                // feedback into this block's later columns (U row j is zero
-                // at and left of the diagonal, so earlier columns are untouched)
-                const float4* urow4 = reinterpret_cast<const float4*>(urow);
-                float4 u = urow4[8 * m + l];
-                cur[0] = fmaf(-e, u.x, cur[0]);
-                cur[1] = fmaf(-e, u.y, cur[1]);
-                cur[2] = fmaf(-e, u.z, cur[2]);
-                cur[3] = fmaf(-e, u.w, cur[3]);
+                    const float* urow = Us + j * kBlock;
+                    const float dj = dinv[j];
+                    const float u1 = urow[(j + 1) & (kBlock - 1)];
+                    const float u2 = urow[(j + 2) & (kBlock - 1)];
+                    // q = clamp(rint(w / s) + z, 0, maxq) = rint(clamp(w / s, -z, maxq - z)) + z
+                    // (z and maxq are integers); e = (w - s (q - z)) / U_jj
+                    const float cq = round_even(fminf(fmaxf(wcur * gp.inv_s, -gp.zf), gp.hi));
+                    const float e = fmaf(-(gp.s * dj), cq, wcur * dj);
+                    const bool mine = l == jq;
+                    qv[i4] = mine ? static_cast<uint32_t>(cq + gp.zf) : qv[i4];
+                    ev[i4] = mine ? e : ev[i4];
+                    // columns j+1 and j+2 for every lane: the owners' own updates, replicated
+                    wcur = fmaf(-e, u1, t1);
+                    t1 = fmaf(-e, u2, t2);
+                    // feedback into this block's later columns (U row j is zero
+                    // at and left of the diagonal, so earlier columns are untouched)
+                    const float4* urow4 = reinterpret_cast<const float4*>(urow);
+                    float4 u = urow4[8 * m + l];
+                    cur[0] = fmaf(-e, u.x, cur[0]);
+                    cur[1] = fmaf(-e, u.y, cur[1]);
+                    cur[2] = fmaf(-e, u.z, cur[2]);
+                    cur[3] = fmaf(-e, u.w, cur[3]);
 #pragma unroll
-                for (int s = 0; s < 3; ++s) {
-                    if (m + 1 + s < 4) {
+                    for (int s = 0; s < 3 - m; ++s) {
                         u = urow4[8 * (m + 1 + s) + l];
                         nxt[4 * s + 0] = fmaf(-e, u.x, nxt[4 * s + 0]);
                         nxt[4 * s + 1] = fmaf(-e, u.y, nxt[4 * s + 1]);
                         nxt[4 * s + 2] = fmaf(-e, u.z, nxt[4 * s + 2]);
                         nxt[4 * s + 3] = fmaf(-e, u.w, nxt[4 * s + 3]);
                     }
+                    // column j+3 as of this step (used one step later)
+                    t2 = owner_value(jj + 3, i4, cur, nxt, gbase);
                 }
-                // column j+3 as of this step (used one step later)
-                t2 = owner_value(jj + 3, i4, cur, nxt, gbase);
             }
-        }
         }
         // chunk m done: pre-quantization weights, scaled errors, codes
         if (live) {
@@ -366,7 +367,11 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
             nxt[4 + i] = nxt[8 + i];
             nxt[8 + i] = 0.f;
         }
-    }
+    };
+    walk_chunk(std::integral_constant<int, 0>{});
+    if (kFull || bw > 32) walk_chunk(std::integral_constant<int, 1>{});
+    if (kFull || bw > 64) walk_chunk(std::integral_constant<int, 2>{});
+    if (kFull || bw > 96) walk_chunk(std::integral_constant<int, 3>{});
 }
 
 // ------------------------------------------------------------------------
