@@ -61,6 +61,9 @@ def parse():
     p.add_argument("--dequant-gemm", type=int, default=0, metavar="TOKENS",
                    help="instead of the quantizer step, time the many-token product of TOKENS "
                         "tokens with a quantized Llama-70B down_proj (gptq_dequant_gemm, tcgen05)")
+    p.add_argument("--hessian-only", action="store_true",
+                   help="instead of the whole step, time the Hessian stage alone (X and H only on "
+                        "the device: the profiling case for large d_col)")
     p.add_argument("--gemm-peaks", action="store_true",
                    help="instead of the quantizer step, measure the library-GEMM denominators of the "
                         "fp32 stages: cuBLAS 8192^3 fp32 with TF32 tensor cores and with plain FFMA")
@@ -535,6 +538,61 @@ def stage_rooflines(wl, pk, which, stage_ms, layer_ms):
             "layer_frac_of_summed_bound": total_bound / layer_ms}
 
 
+# ---------------------------------------------------------------- Hessian alone
+def run_hessian_only(args, rank: int, world: int, dist):
+    """H = 2 X^T X of the workload (token count from --tokens), timed alone:
+    only X and H live on the device."""
+    import post_weight_quantization_gptq_b200 as g
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    wl = workloads.WORKLOADS[args.workload]
+    if args.tokens:
+        wl = dataclasses.replace(wl, n_tokens=args.tokens)
+    n, d = wl.n_tokens, wl.d_col
+    X = workloads.activations(wl, device=dev, seed_offset=replica_seed_offset(rank))
+    H = torch.empty(d, d, dtype=torch.float32, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        H.zero_()
+        g.gptq_hessian_accumulate(X, H, st)
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    clocks = ClockSampler(dev.index)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    for k in range(K):
+        flush.fill_(1)
+        H.zero_()
+        ev[k][0].record(stream)
+        g.gptq_hessian_accumulate(X, H, st)
+        ev[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    if g.gptq_sync_status(st) != 0:
+        raise RuntimeError("device status error in the timed Hessians")
+    ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev), dist, dev)
+    if rank != 0:
+        return
+    pk, which = peaks()
+    flops = n * d * (d + 1)
+    tf = flops / (ms / 1e3) / 1e12
+    peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    print(json.dumps({
+        "metric": "Hessian H = 2 X^T X: TFLOP/s (n d (d+1) flop)", "value": world * tf,
+        "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16-in/fp32",
+        "data": "synthetic", "config": {"workload": wl.name + "_hessian", "d_col": d, "tokens": n,
+                                        "x_bytes": 2 * n * d},
+        "roofline": {"kernel": "hessian_syrk_tcgen05", "bound": "tensor", "achieved": tf,
+                     "peak": peak, "peak_source": f"{which} bf16 dense (burst)", "unit": "TFLOP/s",
+                     "frac": tf / peak, "traffic": None},
+        "clocks": clocks.summary()}), flush=True)
+
+
 # ---------------------------------------------------------------- the product
 def run_dequant_matmul(args, rank: int, world: int, dist):
     """Y = X W_hat^T for a quantized 8192 x 28672 layer (4-bit, g128, act-order):
@@ -654,6 +712,8 @@ def main():
     try:
         if args.dequant_matmul > 0 or args.dequant_gemm > 0:
             run_dequant_matmul(args, rank, world, dist)
+        elif args.hessian_only:
+            run_hessian_only(args, rank, world, dist)
         else:
             run_ours(args, rank, world, dist)
     finally:

@@ -71,18 +71,46 @@ struct Barriers {
     int abort;
 };
 
-// Tile t -> (m-block, n-block), n-block major: block nj needs m-blocks
-// 0 .. 2 nj + 1 (those with 128 mi <= 256 nj + 255), clipped to MT.
+// Tile order.  Column block nj (256 wide) needs the row blocks mi (128 tall)
+// with 128 mi <= 256 nj + 255, i.e. mi <= 2 nj + 1, clipped to MT.  The tiles
+// are enumerated in super-blocks of kSuperM row blocks x kSuperN column blocks
+// (column super-blocks outer, row super-blocks inner; inside one, nj outer and
+// mi inner), so that each wave of 2 x grid consecutive tiles touches few
+// columns of X: a wave reads X[:, its columns] for every token, and with
+// compact waves X is read about 11 times in all at d = 28672 (once per wave,
+// 43 times, in an n-block-major order, whose waves span every row block);
+// 2.7 / 4.0 times at d = 8192 / 11008; d <= 4096 is one wave either way.
+// The super-block shape minimised that count over a grid of shapes.
+constexpr int kSuperM = 8;   // 1024 rows of H
+constexpr int kSuperN = 16;  // 4096 columns of H
+
+__device__ __forceinline__ int tiles_in_column(int nj, int mlo, int mhi) {
+    const int top = min(mhi, 2 * nj + 2);
+    return top > mlo ? top - mlo : 0;
+}
+
 __device__ __forceinline__ void tile_coords(int t, int MT, int NT, int& mi, int& nj) {
-    for (nj = 0; nj < NT; ++nj) {
-        const int cnt = min(MT, 2 * nj + 2);
-        if (t < cnt) {
-            mi = t;
-            return;
+    for (int J0 = 0; J0 < NT; J0 += kSuperN) {
+        const int J1 = min(NT, J0 + kSuperN);
+        for (int I0 = 0; I0 < MT && I0 <= 2 * (J1 - 1) + 1; I0 += kSuperM) {
+            const int I1 = min(MT, I0 + kSuperM);
+            int cnt = 0;
+            for (int n = J0; n < J1; ++n) cnt += tiles_in_column(n, I0, I1);
+            if (t < cnt) {
+                for (nj = J0; nj < J1; ++nj) {
+                    const int c = tiles_in_column(nj, I0, I1);
+                    if (t < c) {
+                        mi = I0 + t;
+                        return;
+                    }
+                    t -= c;
+                }
+            }
+            t -= cnt;
         }
-        t -= cnt;
     }
     mi = 0;
+    nj = 0;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
