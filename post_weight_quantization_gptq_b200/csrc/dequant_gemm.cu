@@ -25,7 +25,6 @@
 //               buffers); after the K loop they drain the accumulators
 // Every wait is bounded (GPTQ_ERR_TIMEOUT, as in the other tensor-core kernels).
 #include <cuda.h>
-#include <cuda_bf16.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -57,9 +56,21 @@ struct Bars {
     int abort;
 };
 
+// x rounded to the nearest bf16 (ties to even), as an fp32 whose low 16 bits
+// are zero, on the fp32 pipe (Veltkamp's split with the factor 2^16 + 1:
+// c = x (2^16 + 1), hi = c - (c - x) keeps the 8 leading significant bits of
+// x rounded to nearest-even; explicit round-to-nearest operations so nothing
+// is contracted; |x| < 2^111).  Checked against the integer rounding rule on
+// random values and exact ties.  The conversion instruction runs on the
+// narrow conversion pipe, which the dequantization saturated (ncu: 102 % of
+// its peak); this form does not use it.
+__device__ __forceinline__ uint32_t bf16_bits(float x) {
+    const float c = __fmul_rn(x, 65537.f);
+    return __float_as_uint(__fsub_rn(c, __fsub_rn(c, x)));
+}
+// two values as one bf16x2 word (lo in the low half)
 __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
-    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&v);
+    return __byte_perm(bf16_bits(lo), bf16_bits(hi), 0x7632);
 }
 
 template <int BITS>
@@ -165,7 +176,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = threadIdx.x - 64;  // row of the tile, 0..255
         const int ng = n0 + n;
         const bool live = ng < d_row;
-        int cur_g = -1;
+        // group of the current 8-code chunk, advanced as k crosses a group
+        // start (g is a multiple of 8, so a chunk crosses at most one; no
+        // integer division in the loop: its reciprocal runs on the same
+        // narrow conversion pipe)
+        int cur_g = -1, next_start = 0;
         float s = 0.f, z = 0.f;
         bool ok = true;
         for (int it = 0; it < nk; ++it) {
@@ -188,11 +203,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < BK / 8; ++c) {
                 const int k = it * BK + 8 * c;
-                const int gi = k / g;  // g is a multiple of 8: a chunk never spans two groups
-                if (gi != cur_g) {
-                    cur_g = gi;
-                    s = live ? __ldg(scales + static_cast<int64_t>(gi) * d_row + ng) : 0.f;
-                    z = live ? static_cast<float>(__ldg(zeros + static_cast<int64_t>(gi) * d_row + ng)) : 0.f;
+                if (k >= next_start) {
+                    ++cur_g;
+                    next_start += g;
+                    s = live ? __ldg(scales + static_cast<int64_t>(cur_g) * d_row + ng) : 0.f;
+                    z = live ? static_cast<float>(__ldg(zeros + static_cast<int64_t>(cur_g) * d_row + ng)) : 0.f;
                 }
                 // code q as the float 2^23 + q (its bits ORed into the
                 // mantissa of 2^23: no int-to-float conversion); subtracting
