@@ -205,9 +205,12 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
     //    lane k is broadcast, every lane scales its own a[k] (the symmetric
     //    entry A[o+lane][o+k]) into l = L[o+lane][o+k], then for each later
     //    row r the value L[o+r][o+k] is broadcast from lane r and applied as
-    //    a[r] -= L[o+r][o+k] * l.  The 32 steps are unrolled, so the per-step
-    //    critical path is shuffle -> rsqrt -> multiply -> shuffle -> FMA and
-    //    the remaining broadcasts and FMAs of a step fill the latency.  The
+    //    a[r] -= L[o+r][o+k] * l.  The 32 steps are unrolled; the per-step
+    //    critical path is rsqrt -> multiply -> FMA -> shuffle (the next
+    //    pivot) and the remaining broadcasts and FMAs of a step fill the
+    //    latency.  Measured in a stamped copy: ~3.2 us per strip (about 200
+    //    cycles per step); neither coarser publishing of the step counter nor
+    //    a sub-partition of its own for this warp shortened it.  The
     //    operations (and their operand order) are those of the row-oriented
     //    rank-1 form, so the factor is bitwise the same.  Each lane publishes
     //    its L value of the step (Lc[k][lane-k-1], zero for lanes <= k) and
@@ -219,15 +222,20 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
             const int hi = r > lane ? r : lane, lo = r > lane ? lane : r;
             a[r] = A[(o + hi) * LDA + o + lo];
         }
+        float dn = __shfl_sync(0xffffffffu, a[0], 0);
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
-            float d = __shfl_sync(0xffffffffu, a[k], k);
+            float d = dn;
             if (!(d > 0.f)) {  // not positive definite (or NaN): flag, stay finite
                 bad = 1;
                 d = 1.f;
             }
             const float inv = rsqrtf(d);
             const float l = (lane > k) ? a[k] * inv : 0.f;  // L[o+lane][o+k]
+            // the next pivot straight from its owner's own L value (lane k+1
+            // applies l * l to its diagonal: the FMA the general update below
+            // applies there too), so the step-to-step chain holds one shuffle
+            if (k + 1 < 32) dn = __shfl_sync(0xffffffffu, fmaf(-l, l, a[k + 1]), k + 1);
             Lc[k * 32 + ((lane - k - 1) & 31)] = l;
             if (lane == k) dinv[o + k] = inv;
             if (k & 1) {
