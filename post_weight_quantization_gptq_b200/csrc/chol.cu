@@ -198,52 +198,58 @@ __global__ void __launch_bounds__(kDiagThreads, 1)
     }
     __syncthreads();
 
-    // -- strip factor (warp 0), column-oriented: lane j holds column o + j of
-    //    the strip, register r = row o + r (rows below the diagonal from the
-    //    stored lower triangle, rows above it -- never used as a pivot or an
-    //    L value -- from the symmetric entry).  Step k: the pivot d = a[k] of
-    //    lane k is broadcast, every lane scales its own a[k] (the symmetric
-    //    entry A[o+lane][o+k]) into l = L[o+lane][o+k], then for each later
-    //    row r the value L[o+r][o+k] is broadcast from lane r and applied as
-    //    a[r] -= L[o+r][o+k] * l.  The 32 steps are unrolled; the per-step
-    //    critical path is rsqrt -> multiply -> FMA -> shuffle (the next
-    //    pivot) and the remaining broadcasts and FMAs of a step fill the
-    //    latency.  Measured in a stamped copy: ~3.2 us per strip (about 200
-    //    cycles per step); neither coarser publishing of the step counter nor
-    //    a sub-partition of its own for this warp shortened it.  The
-    //    operations (and their operand order) are those of the row-oriented
-    //    rank-1 form, so the factor is bitwise the same.  Each lane publishes
-    //    its L value of the step (Lc[k][lane-k-1], zero for lanes <= k) and
-    //    every second step the step counter, as the substitution expects.
+    // -- strip factor (warp 0): lane i holds row o + i, register r = column c + r
     auto factor = [&](int o, int b) {
         float a[32];
 #pragma unroll
-        for (int r = 0; r < 32; ++r) {
-            const int hi = r > lane ? r : lane, lo = r > lane ? lane : r;
-            a[r] = A[(o + hi) * LDA + o + lo];
+        for (int q = 0; q < 8; ++q) {
+            const float4 t = lds4(A + (o + lane) * LDA + o + 4 * q);
+            a[4 * q] = t.x; a[4 * q + 1] = t.y; a[4 * q + 2] = t.z; a[4 * q + 3] = t.w;
         }
-        float dn = __shfl_sync(0xffffffffu, a[0], 0);
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            float d = dn;
-            if (!(d > 0.f)) {  // not positive definite (or NaN): flag, stay finite
+        for (int r = 0; r < 32; ++r) a[r] = (r <= lane) ? a[r] : 0.f;
+        // two columns per pass: column c+1 is formed in registers from column
+        // c (its pivot row needs only its own value, the other rows one
+        // broadcast), then both are published and applied as one rank-2
+        // update -- the same operations in the same order as two rank-1
+        // passes, with one shared-memory round trip instead of two
+#pragma unroll 1
+        for (int c = 0; c < 32; c += 2) {
+            float piv = __shfl_sync(0xffffffffu, a[0], c);
+            if (!(piv > 0.f)) {  // not positive definite (or NaN): flag, stay finite
                 bad = 1;
-                d = 1.f;
+                piv = 1.f;
             }
-            const float inv = rsqrtf(d);
-            const float l = (lane > k) ? a[k] * inv : 0.f;  // L[o+lane][o+k]
-            // the next pivot straight from its owner's own L value (lane k+1
-            // applies l * l to its diagonal: the FMA the general update below
-            // applies there too), so the step-to-step chain holds one shuffle
-            if (k + 1 < 32) dn = __shfl_sync(0xffffffffu, fmaf(-l, l, a[k + 1]), k + 1);
-            Lc[k * 32 + ((lane - k - 1) & 31)] = l;
-            if (lane == k) dinv[o + k] = inv;
-            if (k & 1) {
-                __syncwarp();  // orders the warp's writes above before lane 0's release
-                if (lane == 0) st_release_cta(&progress, 32 * b + k + 1);
+            const float inv = rsqrtf(piv);
+            const float a0 = (lane > c) ? a[0] * inv : 0.f;           // L[o+lane][o+c]
+            const float t = __shfl_sync(0xffffffffu, a0, c + 1);      // L[o+c+1][o+c]
+            const float n1 = fmaf(-a0, t, a[1]);                       // column c+1 after column c
+            float piv1 = __shfl_sync(0xffffffffu, n1, c + 1);
+            if (!(piv1 > 0.f)) {
+                bad = 1;
+                piv1 = 1.f;
+            }
+            const float inv1 = rsqrtf(piv1);
+            const float a1 = (lane > c + 1) ? n1 * inv1 : 0.f;        // L[o+lane][o+c+1]
+            if (lane == c) dinv[o + c] = inv;
+            if (lane == c + 1) dinv[o + c + 1] = inv1;
+            // lane i > c holds L[o+i][o+c] -> Lc[c][i-c-1]; lanes <= c fill the tail with 0
+            Lc[c * 32 + ((lane - c - 1) & 31)] = a0;
+            Lc[(c + 1) * 32 + ((lane - c - 2) & 31)] = a1;
+            __syncwarp();  // orders the warp's writes above before lane 0's release
+            if (lane == 0) st_release_cta(&progress, 32 * b + c + 2);
+            // a[r] <- a[r+2] - a0 L[o+c+2+r][o+c] - a1 L[o+c+2+r][o+c+1]
+            float l0[32], l1[32];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 u = lds4(Lc + c * 32 + 4 * q), v = lds4(Lc + (c + 1) * 32 + 4 * q);
+                l0[4 * q] = u.x; l0[4 * q + 1] = u.y; l0[4 * q + 2] = u.z; l0[4 * q + 3] = u.w;
+                l1[4 * q] = v.x; l1[4 * q + 1] = v.y; l1[4 * q + 2] = v.z; l1[4 * q + 3] = v.w;
             }
 #pragma unroll
-            for (int r = k + 1; r < 32; ++r) a[r] = fmaf(-__shfl_sync(0xffffffffu, l, r), l, a[r]);
+            for (int r = 0; r < 30; ++r) a[r] = fmaf(-a1, l1[r], fmaf(-a0, l0[r + 1], a[r + 2]));
+            a[30] = 0.f;
+            a[31] = 0.f;
         }
     };
 
