@@ -32,10 +32,22 @@ namespace gptq {
 namespace {
 
 constexpr int kBlock = 128;       // columns per block (the only supported block size)
-constexpr int kRowsPerWarp = 4;   // 8 lanes per row
 constexpr int kWarps = 4;
-constexpr int kRowsPerCta = kRowsPerWarp * kWarps;
 static_assert(kWarps * 32 == kBlock, "block_quant_kernel: one thread per column of the U block");
+// Lanes per row of the column walk (each owns 32 / kWalkLanes columns of every
+// 32-column chunk).  8 lanes: 4096 rows give ~7 warps per SM.  4 lanes halve
+// the per-column work replicated on every lane of a row (quantizing the
+// current column, the shuffles) for twice the feedback FMAs per lane, but
+// leave one warp per SM sub-partition: measured slower (quantize_layer 1.287
+// against 1.207 ms at 4096 x 4096, 5.31 against 5.08 ms at 4096 x 11008,
+// interleaved A/B, identical codes).
+constexpr int kWalkLanes = 8;
+template <int L>
+struct WalkShape {
+    static constexpr int kCols = 32 / L;            // columns per lane per chunk
+    static constexpr int kRowsPerWarp = 32 / L;
+    static constexpr int kRowsPerCta = kRowsPerWarp * kWarps;
+};
 
 // ------------------------------------------------------------------------
 // A perm entry outside [0, d) (the caller passed something other than
@@ -63,12 +75,13 @@ __global__ void permute_rows_kernel(float* __restrict__ W, int64_t r, int64_t d,
 }
 
 // Register layout: the block's 128 columns form four 32-column chunks; in
-// every chunk lane l of a row's 8-lane group owns columns 4l .. 4l+3, so the
-// 8 lanes of a row read one 128-byte row segment of the U block per vector
-// load without bank conflicts.  A lane keeps the chunk being quantized in
-// cur[4] and the later chunks in nxt[12]; after each chunk the window
-// rotates, so every register index below is a compile-time constant while the
-// chunk loop stays rolled (the code fits the instruction cache).
+// every chunk lane l of a row's L-lane group owns the C = 32 / L columns
+// C l .. C l + C - 1, so the lanes of a row read one 128-byte row segment of
+// the U block per C / 4 vector loads without bank conflicts.  A lane keeps the
+// chunk being quantized in cur[C] and the later chunks in nxt[3 C]; after each
+// chunk the window rotates, so every register index below is a compile-time
+// constant while the chunk loop stays rolled (the code fits the instruction
+// cache).
 //
 // The column being quantized is held by every lane of the group (wcur): a
 // lane derives columns j+1 and j+2 from values shuffled from their owners two
@@ -88,7 +101,8 @@ struct GroupParams {
 // lies more than 2^20 levels away (w / s then has an fp32 ulp of 1/16 level
 // or more), takes the widened range.  An all-zero group gets the range
 // [-1, 1] (zero point exactly 2^(bits-1)).
-__device__ __forceinline__ GroupParams group_params(const float (&cur)[4], const float (&nxt)[12],
+template <int L, int C = 32 / L>
+__device__ __forceinline__ GroupParams group_params(const float (&cur)[C], const float (&nxt)[3 * C],
                                                     int m, int jj, int l, int g, int bw,
                                                     const float* __restrict__ wrow, int64_t c0,
                                                     int64_t d, bool live, int bits, bool pure,
@@ -96,8 +110,8 @@ __device__ __forceinline__ GroupParams group_params(const float (&cur)[4], const
     const int j = 32 * m + jj;
     float lo = pure ? INFINITY : 0.f, hi = pure ? -INFINITY : 0.f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int c = 32 * m + 4 * l + i;
+    for (int i = 0; i < C; ++i) {
+        const int c = 32 * m + C * l + i;
         if (c >= j && c < j + g && c < bw) {
             lo = fminf(lo, cur[i]);
             hi = fmaxf(hi, cur[i]);
@@ -106,23 +120,23 @@ __device__ __forceinline__ GroupParams group_params(const float (&cur)[4], const
 #pragma unroll
     for (int s = 0; s < 3; ++s)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int c = 32 * (m + 1 + s) + 4 * l + i;
+        for (int i = 0; i < C; ++i) {
+            const int c = 32 * (m + 1 + s) + C * l + i;
             if (m + 1 + s < 4 && c < j + g && c < bw) {
-                lo = fminf(lo, nxt[4 * s + i]);
-                hi = fmaxf(hi, nxt[4 * s + i]);
+                lo = fminf(lo, nxt[C * s + i]);
+                hi = fmaxf(hi, nxt[C * s + i]);
             }
         }
     const int64_t gend = (c0 + j + g < d) ? c0 + j + g : d;
     if (live && gend > c0 + bw) {
-        for (int64_t c = c0 + bw + l; c < gend; c += 8) {
+        for (int64_t c = c0 + bw + l; c < gend; c += L) {
             const float v = (dead_mask != nullptr && dead_mask[c]) ? 0.f : wrow[c];
             lo = fminf(lo, v);
             hi = fmaxf(hi, v);
         }
     }
 #pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
+    for (int o = 1; o < L; o <<= 1) {
         lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
         hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
     }
@@ -148,13 +162,14 @@ __device__ __forceinline__ GroupParams group_params(const float (&cur)[4], const
     return p;
 }
 
-// Value of column 32 m + k (3 <= k < 35, k = 4 jq + i4 + 3) of this row, as
-// held by its owner lane: the current chunk for k < 32, the next one after.
-__device__ __forceinline__ float owner_value(int k, int i4, const float (&cur)[4],
-                                             const float (&nxt)[12], int gbase) {
-    // k & 3 == (i4 + 3) & 3 with i4 a compile-time constant
-    const float v = (k < 32) ? cur[(i4 + 3) & 3] : nxt[(i4 + 3) & 3];
-    return __shfl_sync(0xffffffffu, v, gbase + ((k & 31) >> 2));
+// Value of column 32 m + k (3 <= k < 35) of this row, as held by its owner
+// lane: the current chunk for k < 32, the next one after; ii = k mod C is a
+// compile-time register index.
+template <int C>
+__device__ __forceinline__ float owner_value(int k, int ii, const float (&cur)[C],
+                                             const float (&nxt)[3 * C], int gbase) {
+    const float v = (k < 32) ? cur[ii] : nxt[ii];
+    return __shfl_sync(0xffffffffu, v, gbase + ((k & 31) / C));
 }
 
 // Round half to even of |x| <= 2^22 by adding and removing 1.5 * 2^23 (its
@@ -164,14 +179,17 @@ __device__ __forceinline__ float round_even(float x) {
     return __fadd_rn(__fadd_rn(x, 12582912.f), -12582912.f);
 }
 
-template <bool kSmallGroup,  // group_size < 32: groups start inside a chunk
+template <int L,               // lanes per row
+          bool kSmallGroup,  // group_size < 32: groups start inside a chunk
           bool kFull>        // a full 128-column block (no column guard)
-__global__ void __launch_bounds__(kWarps * 32, 4)
+__global__ void __launch_bounds__(kWarps * 32, L >= 8 ? 4 : 2)
     block_quant_kernel(const __grid_constant__ CUtensorMap tmu, float* __restrict__ W, int64_t r,
                        int64_t d, int64_t ldw, int64_t c0, int bw, int bits, int g, int pure,
                        uint8_t* __restrict__ codes, float* __restrict__ scales,
                        int32_t* __restrict__ zeros, float* __restrict__ err_out,
                        int64_t err_ld, const uint8_t* __restrict__ dead_mask, int32_t* status) {
+    constexpr int C = WalkShape<L>::kCols;
+    constexpr int C4 = C / 4;  // float4s per lane per chunk
     extern __shared__ uint8_t smem_raw[];
     float* smem = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -213,40 +231,43 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
     pdl_wait();
 
     const int lane = tid & 31;
-    const int l = lane & 7;
-    const int gbase = lane & ~7;
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + (tid >> 5) * kRowsPerWarp +
-                        (lane >> 3);
+    const int l = lane % L;
+    const int gbase = lane - l;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * WalkShape<L>::kRowsPerCta +
+                        (tid >> 5) * WalkShape<L>::kRowsPerWarp + lane / L;
     const bool live = row < r;
     float* wrow = W + (live ? row : 0) * ldw;
-    // float4 access to W needs 16-byte aligned rows (base and pitch); four
-    // codes go out as one 32-bit store when codes' rows are 4-byte aligned
+    // float4 access to W needs 16-byte aligned rows (base and pitch); a
+    // lane's C codes go out as one C-byte store when codes' rows allow it
     const bool vec = (ldw & 3) == 0 && bw == kBlock && (reinterpret_cast<uintptr_t>(W) & 15) == 0;
-    const bool vec_codes = vec && (d & 3) == 0 && (reinterpret_cast<uintptr_t>(codes) & 3) == 0;
+    const bool vec_codes = vec && (d % C) == 0 && (reinterpret_cast<uintptr_t>(codes) % C) == 0;
 
     // the row's slice of the block (in flight while the U block arrives)
-    float cur[4], nxt[12];
+    float cur[C], nxt[3 * C];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-        float v[4];
+        float v[C];
         if (live && vec) {
-            const float4 t = *reinterpret_cast<const float4*>(wrow + c0 + 32 * m + 4 * l);
-            v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+#pragma unroll
+            for (int q = 0; q < C4; ++q) {
+                const float4 t = *reinterpret_cast<const float4*>(wrow + c0 + 32 * m + C * l + 4 * q);
+                v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
+            }
         } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int c = 32 * m + 4 * l + i;
+            for (int i = 0; i < C; ++i) {
+                const int c = 32 * m + C * l + i;
                 v[i] = (live && c < bw) ? wrow[c0 + c] : 0.f;
             }
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < C; ++i) {
             // columns whose H diagonal is 0 quantize zero weights (in the
             // permuted form the permutation pass has zeroed them already)
-            if (dead_mask != nullptr && 32 * m + 4 * l + i < bw && dead_mask[c0 + 32 * m + 4 * l + i])
+            if (dead_mask != nullptr && 32 * m + C * l + i < bw && dead_mask[c0 + 32 * m + C * l + i])
                 v[i] = 0.f;
             if (m == 0) cur[i] = v[i];
-            else nxt[4 * (m - 1) + i] = v[i];
+            else nxt[C * (m - 1) + i] = v[i];
         }
     }
     GroupParams gp{1.f, 1.f, 0.f, 0.f};
@@ -275,28 +296,33 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
     auto walk_chunk = [&](auto mc) {
         constexpr int m = decltype(mc)::value;
         if (!kSmallGroup && ((c0 + 32 * m) % g) == 0) {
-            gp = group_params(cur, nxt, m, 0, l, g, bw, wrow, c0, d, live, bits, pure != 0,
-                              dead_mask);
+            gp = group_params<L>(cur, nxt, m, 0, l, g, bw, wrow, c0, d, live, bits, pure != 0,
+                                 dead_mask);
             if (live && l == 0) {
                 const int64_t grp = (c0 + 32 * m) / g;
                 scales[grp * r + row] = gp.s;
                 zeros[grp * r + row] = static_cast<int32_t>(gp.zf);
             }
         }
-        float ev[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t qv[4] = {0u, 0u, 0u, 0u};
-        // 8 rolled steps of 4 unrolled columns: register indices stay
-        // compile-time while the loop body stays small
-#pragma unroll 1
-        for (int jq = 0; jq < 8; ++jq) {
+        float ev[C];
+        uint32_t qv[C];
 #pragma unroll
-            for (int i4 = 0; i4 < 4; ++i4) {
-                const int jj = 4 * jq + i4;
+        for (int i = 0; i < C; ++i) {
+            ev[i] = 0.f;
+            qv[i] = 0u;
+        }
+        // L rolled steps (one per owner lane) of C unrolled columns: register
+        // indices stay compile-time while the loop body stays small
+#pragma unroll 1
+        for (int jo = 0; jo < L; ++jo) {
+#pragma unroll
+            for (int ii = 0; ii < C; ++ii) {
+                const int jj = C * jo + ii;
                 const int j = 32 * m + jj;
                 if (kFull || j < bw) {
                     if (kSmallGroup && ((c0 + j) % g) == 0) {
-                        gp = group_params(cur, nxt, m, jj, l, g, bw, wrow, c0, d, live, bits,
-                                          pure != 0, dead_mask);
+                        gp = group_params<L>(cur, nxt, m, jj, l, g, bw, wrow, c0, d, live, bits,
+                                             pure != 0, dead_mask);
                         if (live && l == 0) {
                             const int64_t grp = (c0 + j) / g;
                             scales[grp * r + row] = gp.s;
@@ -311,47 +337,64 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
                     // (z and maxq are integers); e = (w - s (q - z)) / U_jj
                     const float cq = round_even(fminf(fmaxf(wcur * gp.inv_s, -gp.zf), gp.hi));
                     const float e = fmaf(-(gp.s * dj), cq, wcur * dj);
-                    const bool mine = l == jq;
-                    qv[i4] = mine ? static_cast<uint32_t>(cq + gp.zf) : qv[i4];
-                    ev[i4] = mine ? e : ev[i4];
+                    const bool mine = l == jo;
+                    qv[ii] = mine ? static_cast<uint32_t>(cq + gp.zf) : qv[ii];
+                    ev[ii] = mine ? e : ev[ii];
                     // columns j+1 and j+2 for every lane: the owners' own updates, replicated
                     wcur = fmaf(-e, u1, t1);
                     t1 = fmaf(-e, u2, t2);
                     // feedback into this block's later columns (U row j is zero
                     // at and left of the diagonal, so earlier columns are untouched)
                     const float4* urow4 = reinterpret_cast<const float4*>(urow);
-                    float4 u = urow4[8 * m + l];
-                    cur[0] = fmaf(-e, u.x, cur[0]);
-                    cur[1] = fmaf(-e, u.y, cur[1]);
-                    cur[2] = fmaf(-e, u.z, cur[2]);
-                    cur[3] = fmaf(-e, u.w, cur[3]);
 #pragma unroll
-                    for (int s = 0; s < 3 - m; ++s) {
-                        u = urow4[8 * (m + 1 + s) + l];
-                        nxt[4 * s + 0] = fmaf(-e, u.x, nxt[4 * s + 0]);
-                        nxt[4 * s + 1] = fmaf(-e, u.y, nxt[4 * s + 1]);
-                        nxt[4 * s + 2] = fmaf(-e, u.z, nxt[4 * s + 2]);
-                        nxt[4 * s + 3] = fmaf(-e, u.w, nxt[4 * s + 3]);
+                    for (int q = 0; q < C4; ++q) {
+                        const float4 u = urow4[8 * m + C4 * l + q];
+                        cur[4 * q + 0] = fmaf(-e, u.x, cur[4 * q + 0]);
+                        cur[4 * q + 1] = fmaf(-e, u.y, cur[4 * q + 1]);
+                        cur[4 * q + 2] = fmaf(-e, u.z, cur[4 * q + 2]);
+                        cur[4 * q + 3] = fmaf(-e, u.w, cur[4 * q + 3]);
                     }
+#pragma unroll
+                    for (int s = 0; s < 3 - m; ++s)
+#pragma unroll
+                        for (int q = 0; q < C4; ++q) {
+                            const float4 u = urow4[8 * (m + 1 + s) + C4 * l + q];
+                            nxt[C * s + 4 * q + 0] = fmaf(-e, u.x, nxt[C * s + 4 * q + 0]);
+                            nxt[C * s + 4 * q + 1] = fmaf(-e, u.y, nxt[C * s + 4 * q + 1]);
+                            nxt[C * s + 4 * q + 2] = fmaf(-e, u.z, nxt[C * s + 4 * q + 2]);
+                            nxt[C * s + 4 * q + 3] = fmaf(-e, u.w, nxt[C * s + 4 * q + 3]);
+                        }
                     // column j+3 as of this step (used one step later)
-                    t2 = owner_value(jj + 3, i4, cur, nxt, gbase);
+                    t2 = owner_value<C>(jj + 3, (ii + 3) % C, cur, nxt, gbase);
                 }
             }
         }
         // chunk m done: pre-quantization weights, scaled errors, codes
         if (live) {
-            const int cb = 32 * m + 4 * l;
-            *reinterpret_cast<float4*>(err_out + row * err_ld + cb) =
-                make_float4(ev[0], ev[1], ev[2], ev[3]);
+            const int cb = 32 * m + C * l;
+#pragma unroll
+            for (int q = 0; q < C4; ++q)
+                *reinterpret_cast<float4*>(err_out + row * err_ld + cb + 4 * q) =
+                    make_float4(ev[4 * q], ev[4 * q + 1], ev[4 * q + 2], ev[4 * q + 3]);
             if (vec) {
-                *reinterpret_cast<float4*>(wrow + c0 + cb) = make_float4(cur[0], cur[1], cur[2], cur[3]);
+#pragma unroll
+                for (int q = 0; q < C4; ++q)
+                    *reinterpret_cast<float4*>(wrow + c0 + cb + 4 * q) =
+                        make_float4(cur[4 * q], cur[4 * q + 1], cur[4 * q + 2], cur[4 * q + 3]);
             }
             if (vec_codes) {
-                *reinterpret_cast<uint32_t*>(codes + row * d + c0 + cb) =
-                    qv[0] | (qv[1] << 8) | (qv[2] << 16) | (qv[3] << 24);
+                uint32_t word[C4];
+#pragma unroll
+                for (int q = 0; q < C4; ++q)
+                    word[q] = qv[4 * q] | (qv[4 * q + 1] << 8) | (qv[4 * q + 2] << 16) |
+                              (qv[4 * q + 3] << 24);
+                if constexpr (C4 == 2)
+                    *reinterpret_cast<uint2*>(codes + row * d + c0 + cb) = make_uint2(word[0], word[1]);
+                else
+                    *reinterpret_cast<uint32_t*>(codes + row * d + c0 + cb) = word[0];
             }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < C; ++i) {
                 const int c = cb + i;
                 if (c < bw) {
                     if (!vec) wrow[c0 + c] = cur[i];
@@ -361,11 +404,11 @@ __global__ void __launch_bounds__(kWarps * 32, 4)
         }
         // rotate the window
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < C; ++i) {
             cur[i] = nxt[i];
-            nxt[i] = nxt[4 + i];
-            nxt[4 + i] = nxt[8 + i];
-            nxt[8 + i] = 0.f;
+            nxt[i] = nxt[C + i];
+            nxt[C + i] = nxt[2 * C + i];
+            nxt[2 * C + i] = 0.f;
         }
     };
     walk_chunk(std::integral_constant<int, 0>{});
@@ -517,13 +560,15 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
                        make_tmap_2d(&tW, false, W, d_col, d_row, ldw, 32, 32, Swz::k128);
     const size_t q_smem = (kBlock * kBlock + kBlock) * sizeof(float) + 1024;
     const bool small_group = g < 32;
-    auto qfull = small_group ? block_quant_kernel<true, true> : block_quant_kernel<false, true>;
-    auto qpart = small_group ? block_quant_kernel<true, false> : block_quant_kernel<false, false>;
+    constexpr int Lw = kWalkLanes;
+    auto qfull = small_group ? block_quant_kernel<Lw, true, true> : block_quant_kernel<Lw, false, true>;
+    auto qpart = small_group ? block_quant_kernel<Lw, true, false> : block_quant_kernel<Lw, false, false>;
     if (cudaFuncSetAttribute(qfull, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(q_smem)) != cudaSuccess ||
         cudaFuncSetAttribute(qpart, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(q_smem)) != cudaSuccess)
         return GPTQ_ERR_CUDA;
+    constexpr int kRowsPerCta = WalkShape<kWalkLanes>::kRowsPerCta;
     const unsigned qgrid = static_cast<unsigned>((d_row + kRowsPerCta - 1) / kRowsPerCta);
     const int mt = static_cast<int>((d_row + 127) / 128);
     const int sms = num_sms();
