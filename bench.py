@@ -23,7 +23,6 @@ import json
 import os
 import statistics
 import sys
-import threading
 import time
 
 import numpy as np
@@ -134,57 +133,85 @@ def job_weights_per_s(world: int, d_row: int, d_col: int, ms_max: float) -> floa
 
 
 # ---------------------------------------------------------------- clocks
+_SAMPLER_SRC = r"""
+import select, sys, time
+import pynvml
+pynvml.nvmlInit()
+h = pynvml.nvmlDeviceGetHandleByUUID(sys.argv[1].encode())
+period = float(sys.argv[2])
+print("ready", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
+out = []
+while not select.select([sys.stdin], [], [], period)[0]:
+    try:
+        out.append((time.monotonic(), pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                    pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)))
+    except Exception:
+        pass
+for t, mhz, mask in out:
+    print(t, mhz, mask)
+"""
+
+
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML while running."""
+    """SM clock and clock-event reasons through NVML, sampled every few ms by
+    a separate process (a thread of this one would wait for the interpreter
+    lock while the main thread blocks in a device synchronize).  Samples are
+    kept between start() and stop()."""
     REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
                0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
-        self.period = period_s
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        import subprocess
         self.samples = []
         self.reasons = set()
         self.max_mhz = None
-        self._stop = threading.Event()
-        self._thread = None
+        self.error = None
+        self.t0 = self.t1 = None
+        self.proc = None
         try:
-            import pynvml
-            pynvml.nvmlInit()
             uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
-            self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.proc = subprocess.Popen([sys.executable, "-c", _SAMPLER_SRC, uuid, str(period_s)],
+                                         stdin=subprocess.PIPE, stdout=subprocess.PIPE,
+                                         stderr=subprocess.PIPE, text=True)
+            first = self.proc.stdout.readline().split()
+            if len(first) != 2 or first[0] != "ready":
+                raise RuntimeError("clock sampler did not start: "
+                                   + self.proc.stderr.read()[-300:].strip())
+            self.max_mhz = int(first[1])
         except Exception as exc:  # NVML missing: report that, do not guess
-            self.nv = None
             self.error = repr(exc)
-
-    def _run(self):
-        while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for bit, name in self.REASONS.items():
-                    if mask & bit:
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(self.period)
+            if self.proc is not None and self.proc.poll() is None:
+                self.proc.kill()
+            self.proc = None
 
     def start(self):
-        if self.nv is not None:
-            self._thread = threading.Thread(target=self._run, daemon=True)
-            self._thread.start()
+        self.t0 = time.monotonic()
 
     def stop(self):
-        if self._thread is not None:
-            self._stop.set()
-            self._thread.join()
+        self.t1 = time.monotonic()
+        if self.proc is None:
+            return
+        try:
+            out, _ = self.proc.communicate(input="", timeout=30)
+        except Exception as exc:
+            self.proc.kill()
+            self.error = repr(exc)
+            return
+        for ln in out.splitlines():
+            t, mhz, mask = ln.split()
+            if self.t0 <= float(t) <= self.t1:
+                self.samples.append(int(mhz))
+                for bit, name in self.REASONS.items():
+                    if int(mask) & bit:
+                        self.reasons.add(name)
 
     def summary(self):
-        if self.nv is None:
+        if self.proc is None and self.max_mhz is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.error}
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_min_mhz": min(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                "samples": len(self.samples)}
+                "samples": len(self.samples), "period_ms": 5}
 
 
 # ---------------------------------------------------------------- oracle timing
@@ -653,6 +680,19 @@ def run_dequant_matmul(args, rank: int, world: int, dist):
     launches = (g.gptq_launch_counter() - launches0) / K
     ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     ms_max = max_over_ranks(ms, dist, dev)
+    kernel_ms = None
+    if gemm:
+        # the contraction kernel alone (the activations already in
+        # quantization order: no gather launch), for its roofline
+        kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+        for k in range(K):
+            flush.fill_(1)
+            kev[k][0].record(stream)
+            g.gptq_dequant_gemm(X, packed, scales, zeros, None, bits, gs, Y, ws, st)
+            kev[k][1].record(stream)
+        torch.cuda.synchronize(dev)
+        kernel_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in kev), dist, dev)
     if rank != 0:
         return
     if g.gptq_sync_status(st) != 0:
@@ -664,11 +704,11 @@ def run_dequant_matmul(args, rank: int, world: int, dist):
     peak = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     if gemm:
         flops = 2.0 * n_tok * d_row * d_col
-        tf = flops / (ms / 1e3) / 1e12
+        tf = flops / (kernel_ms / 1e3) / 1e12
         bpk = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         roof = {"kernel": "dequant_gemm_kernel", "bound": "tensor", "achieved": tf, "peak": bpk,
                 "peak_source": f"{which} bf16 dense (burst)", "unit": "TFLOP/s", "frac": tf / bpk,
-                "traffic": None,
+                "traffic": None, "kernel_ms": kernel_ms, "gather_ms": ms_max - kernel_ms,
                 "algorithmic": f"2 tokens d_row d_col = {flops:.4e} flop (bf16 operands, fp32 sums)"}
     else:
         roof = {"kernel": "dequant_matmul_kernel", "bound": "hbm", "achieved": gbs,

@@ -263,17 +263,71 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Xq[t][k] = X[t][perm[k]] (bf16, row pitch K); perm entries outside [0, K)
 // are read as k.
-__global__ void gather_bf16_kernel(const uint16_t* __restrict__ X, int64_t ldx, int64_t n_tok,
-                                   int K, const int32_t* __restrict__ perm,
-                                   uint16_t* __restrict__ Xq) {
-    const int64_t total = n_tok * K;
-    for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
-         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t t = e / K, k = e - t * K;
-        int64_t col = perm != nullptr ? perm[k] : k;
-        if (col < 0 || col >= K) col = k;
-        Xq[e] = X[t * ldx + col];
+// Xq[t][k] = X[t][perm[k]] (bf16 bits, quantization order), one token row per
+// CTA at a time.  The row is first copied into shared memory with 16-byte
+// loads when X's rows allow it (kStaged), so that HBM sees it read once and
+// in order whatever the permutation; the permuted row leaves in 16-byte
+// stores of 8 values (K is a multiple of 64 and Xq's rows are contiguous).
+// Rows too wide for shared memory read their values through L1 instead.
+constexpr int kGatherThreads = 256;
+constexpr int kGatherSmemMax = 160 * 1024;
+
+template <bool kStaged, bool kVecLoad>
+__global__ void __launch_bounds__(kGatherThreads)
+gather_bf16_kernel(const uint16_t* __restrict__ X, int64_t ldx, int64_t n_tok, int K,
+                   const int32_t* __restrict__ perm, uint16_t* __restrict__ Xq) {
+    extern __shared__ __align__(16) uint16_t row_s[];
+    const int chunks = K / 8;
+    for (int64_t t = blockIdx.x; t < n_tok; t += gridDim.x) {
+        const uint16_t* xr = X + t * ldx;
+        if constexpr (kStaged) {
+            if constexpr (kVecLoad) {
+                const uint4* src = reinterpret_cast<const uint4*>(xr);
+                for (int c = threadIdx.x; c < chunks; c += kGatherThreads)
+                    reinterpret_cast<uint4*>(row_s)[c] = __ldg(src + c);
+            } else {
+                for (int k = threadIdx.x; k < K; k += kGatherThreads) row_s[k] = xr[k];
+            }
+            __syncthreads();
+        }
+        uint4* dst = reinterpret_cast<uint4*>(Xq + t * static_cast<int64_t>(K));
+        for (int c = threadIdx.x; c < chunks; c += kGatherThreads) {
+            uint32_t v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int k = c * 8 + i;
+                int col = perm != nullptr ? __ldg(perm + k) : k;
+                if (col < 0 || col >= K) col = k;
+                v[i] = kStaged ? row_s[col] : __ldg(xr + col);
+            }
+            dst[c] = make_uint4(v[0] | (v[1] << 16), v[2] | (v[3] << 16), v[4] | (v[5] << 16),
+                                v[6] | (v[7] << 16));
+        }
+        if constexpr (kStaged) __syncthreads();  // the row buffer is refilled next
     }
+}
+
+cudaError_t launch_gather(const uint16_t* X, int64_t ldx, int64_t n_tok, int K,
+                          const int32_t* perm, uint16_t* Xq, cudaStream_t stream) {
+    const size_t smem = static_cast<size_t>(K) * 2;
+    const bool vec = (ldx % 8) == 0 && (reinterpret_cast<uintptr_t>(X) & 15) == 0;
+    if (smem > kGatherSmemMax) {
+        const int grid = static_cast<int>(n_tok < 8 * num_sms() ? n_tok : 8 * num_sms());
+        gather_bf16_kernel<false, false><<<grid, kGatherThreads, 0, stream>>>(X, ldx, n_tok, K,
+                                                                              perm, Xq);
+        return cudaGetLastError();
+    }
+    auto kern = vec ? gather_bf16_kernel<true, true> : gather_bf16_kernel<true, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGatherThreads, smem);
+    if (e != cudaSuccess) return e;
+    const int64_t resident = static_cast<int64_t>(per_sm > 0 ? per_sm : 1) * num_sms();
+    const int grid = static_cast<int>(n_tok < resident ? n_tok : resident);
+    kern<<<grid, kGatherThreads, smem, stream>>>(X, ldx, n_tok, K, perm, Xq);
+    return cudaGetLastError();
 }
 
 template <int BITS>
@@ -306,10 +360,8 @@ gptq_status launch_dequant_gemm(const uint16_t* X, int64_t n_tok, int64_t d_col,
     int64_t launches = 1;
     if (perm != nullptr || (ldx % 8) != 0 || (reinterpret_cast<uintptr_t>(X) & 15) != 0) {
         uint16_t* Xq = static_cast<uint16_t*>(ws);
-        const int64_t total = n_tok * d_col;
-        const int64_t blocks = (total + 255) / 256;
-        const int gb = static_cast<int>(blocks < 8 * num_sms() ? blocks : 8 * num_sms());
-        gather_bf16_kernel<<<gb, 256, 0, stream>>>(X, ldx, n_tok, K, perm, Xq);
+        if (launch_gather(X, ldx, n_tok, K, perm, Xq, stream) != cudaSuccess)
+            return GPTQ_ERR_CUDA;
         A = Xq;
         lda = d_col;
         ++launches;

@@ -7,26 +7,32 @@
 // computed.
 //
 // Design (sm_100a):
-//  * Output tile 128 x 256 of D = X[:, m-block]^T X[:, n-block]; tcgen05.mma
-//    kind::f16 with bf16 operands and an fp32 accumulator in tensor memory.
+//  * Each CTA owns one 256 x 256 block of D = X[:, m-block]^T X[:, n-block]
+//    as two 128 x 256 halves (rows m0..m0+127 and m0+128..m0+255), each a
+//    tcgen05.mma kind::f16 with bf16 operands and an fp32 accumulator in
+//    tensor memory (2 x 256 of the 512 columns).  The two halves share the
+//    n-block's operand B, so a 64-token stage brings 512 channels
+//    (64 KB) for 2 x 128 x 256 x 64 multiply-adds, against 768 channels for
+//    two unrelated 128 x 256 tiles: a third less L2-to-SM operand traffic,
+//    which is what bounds the main loop (the same ~15.6 TB/s of operands at
+//    1.54 and 1.97 GHz SM clocks with unrelated tiles).  On a diagonal block
+//    (m-block = n-block) both halves' A is B itself: only B is loaded.
 //  * Both operands are slices of the row-major X, so both are MN-major in
 //    shared memory: a TMA box of 64 channels (128 bytes) x 64 tokens with the
 //    128-byte swizzle is exactly one column of canonical SW128 MN-major atoms.
-//  * Each CTA owns two tiles (both accumulators live in TMEM: 2 x 256 of the
-//    512 columns) and sweeps all tokens for both, interleaving them stage by
-//    stage.  All CTAs sweep the tokens in lockstep, so each token slice of X
-//    is fetched from HBM once and served to every CTA from L2.
+//  * All CTAs sweep the tokens in lockstep, so each token slice of X is
+//    fetched from HBM once and served to every CTA from L2.
 //  * Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs,
 //    warps 2..9 drain the accumulators (TMEM -> registers -> H), two warps
 //    per TMEM lane quarter, each with half of the columns (twice the H loads
 //    in flight while the tensor cores wait for the drain).
 //  * The epilogue stores D[m][n] into H[n][m]: for a fixed n the 32 lanes of
 //    a warp hold 32 consecutive m, so every store is one coalesced 128-byte
-//    line.  Tiles are chosen with n >= m somewhere inside them, so the
-//    written entries cover H's lower triangle.
-//  * Tokens are taken in chunks of 32,768: each chunk's partial tile is added
-//    into H by the epilogue (fp32, round to nearest), which bounds the bias of
-//    the tensor cores' long fp32 accumulation.
+//    line.  Blocks have m-block <= n-block, so the written entries cover H's
+//    lower triangle.
+//  * Tokens are taken in chunks of 32,768: each chunk's partial block is
+//    added into H by the epilogue (fp32, round to nearest), which bounds the
+//    bias of the tensor cores' long fp32 accumulation.
 //  * No atomics: every H entry has exactly one owner, so the result is
 //    deterministic.  Every wait is bounded (GPTQ_ERR_TIMEOUT).
 #include <cuda.h>
@@ -37,18 +43,18 @@
 namespace gptq {
 namespace {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 128;                         // rows per MMA (one half of a block)
+constexpr int BN = 256;                         // block width (and height: two halves)
 constexpr int BK = 64;
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kBox = 64;                        // channels per TMA box (128 bytes)
 constexpr int kBoxBytes = kBox * BK * 2;        // 8 KB
-constexpr int kABytes = BM * BK * 2;            // 16 KB
+constexpr int kABytes = BM * BK * 2;            // 16 KB per half
 constexpr int kBBytes = BN * BK * 2;            // 32 KB
-constexpr int kStageBytes = kABytes + kBBytes;  // 48 KB
+constexpr int kStageBytes = kBBytes + 2 * kABytes;  // 64 KB: B, then A of both halves
 constexpr int kThreads = 320;   // TMA, MMA, 8 epilogue warps (two per TMEM lane quarter)
 constexpr int kTmemCols = 512;
-// Tokens accumulated in TMEM before the partial tile is added into H.  The
+// Tokens accumulated in TMEM before the partial block is added into H.  The
 // tensor cores' fp32 accumulation loses about 2^-25 of the running sum per
 // accumulate step, with a consistent sign, so the bias grows with the number
 // of steps (measured ~1.4e-3 relative over 262,144 tokens in one run);
@@ -71,36 +77,34 @@ struct Barriers {
     int abort;
 };
 
-// Tile order.  Column block nj (256 wide) needs the row blocks mi (128 tall)
-// with 128 mi <= 256 nj + 255, i.e. mi <= 2 nj + 1, clipped to MT.  The tiles
-// are enumerated in super-blocks of kSuperM row blocks x kSuperN column blocks
-// (column super-blocks outer, row super-blocks inner; inside one, nj outer and
-// mi inner), so that each wave of 2 x grid consecutive tiles touches few
-// columns of X: a wave reads X[:, its columns] for every token, and with
-// compact waves X is read about 11 times in all at d = 28672 (once per wave,
-// 43 times, in an n-block-major order, whose waves span every row block);
-// 2.7 / 4.0 times at d = 8192 / 11008; d <= 4096 is one wave either way.
-// The super-block shape minimised that count over a grid of shapes.
-constexpr int kSuperM = 8;   // 1024 rows of H
+// Block order.  Blocks are (pi, nj) in 256-channel units with pi <= nj.  They
+// are enumerated in super-blocks of kSuperP row blocks x kSuperN column
+// blocks (column super-blocks outer, row super-blocks inner; inside one, nj
+// outer and pi inner), so that each wave of grid consecutive blocks touches
+// few columns of X: a wave reads X[:, its channels] for every token, and
+// compact waves keep the number of passes over X low at large d (about 11
+// at d = 28672, against one per wave, 43, in an n-block-major order whose
+// waves span every row block); d <= 4096 is one wave either way.
+constexpr int kSuperP = 4;   // 1024 rows of H
 constexpr int kSuperN = 16;  // 4096 columns of H
 
-__device__ __forceinline__ int tiles_in_column(int nj, int mlo, int mhi) {
-    const int top = min(mhi, 2 * nj + 2);
-    return top > mlo ? top - mlo : 0;
+__device__ __forceinline__ int blocks_in_column(int nj, int plo, int phi) {
+    const int top = min(phi, nj + 1);
+    return top > plo ? top - plo : 0;
 }
 
-__device__ __forceinline__ void tile_coords(int t, int MT, int NT, int& mi, int& nj) {
+__device__ __forceinline__ void block_coords(int t, int NT, int& pi, int& nj) {
     for (int J0 = 0; J0 < NT; J0 += kSuperN) {
         const int J1 = min(NT, J0 + kSuperN);
-        for (int I0 = 0; I0 < MT && I0 <= 2 * (J1 - 1) + 1; I0 += kSuperM) {
-            const int I1 = min(MT, I0 + kSuperM);
+        for (int P0 = 0; P0 < J1; P0 += kSuperP) {
+            const int P1 = min(NT, P0 + kSuperP);
             int cnt = 0;
-            for (int n = J0; n < J1; ++n) cnt += tiles_in_column(n, I0, I1);
+            for (int n = J0; n < J1; ++n) cnt += blocks_in_column(n, P0, P1);
             if (t < cnt) {
                 for (nj = J0; nj < J1; ++nj) {
-                    const int c = tiles_in_column(nj, I0, I1);
+                    const int c = blocks_in_column(nj, P0, P1);
                     if (t < c) {
-                        mi = I0 + t;
+                        pi = P0 + t;
                         return;
                     }
                     t -= c;
@@ -109,13 +113,13 @@ __device__ __forceinline__ void tile_coords(int t, int MT, int NT, int& mi, int&
             t -= cnt;
         }
     }
-    mi = 0;
+    pi = 0;
     nj = 0;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
     hessian_syrk_tcgen05(const __grid_constant__ CUtensorMap tmap_x, float* __restrict__ H,
-                         int64_t ldh, int d, int n, int num_tiles, int32_t* status,
+                         int64_t ldh, int d, int n, int num_blocks, int32_t* status,
                          uint64_t probe_ns) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -125,14 +129,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int MT = (d + BM - 1) / BM;
     const int NT = (d + BN - 1) / BN;
     const int KB = (n + BK - 1) / BK;
     const int G = gridDim.x;
     const int nchunk = (KB + kChunkIters - 1) / kChunkIters;
-    // a wave = (two tiles, one token chunk); the accumulators are drained
+    // a wave = (one block, one token chunk); the accumulators are drained
     // into H after every wave
-    const int waves = ((num_tiles + 2 * G - 1) / (2 * G)) * nchunk;
+    const int waves = ((num_blocks + G - 1) / G) * nchunk;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -161,40 +164,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             uint32_t it = 0;
             for (int w = 0; w < waves && !*abort; ++w) {
-                const int tw = w / nchunk;
+                const int t = blockIdx.x + (w / nchunk) * G;
+                if (t >= num_blocks) break;
                 const int k0 = (w % nchunk) * kChunkIters;
                 const int k1 = min(KB, k0 + kChunkIters);
-                int tiles[2], ns = 0;
-                for (int s = 0; s < 2; ++s) {
-                    const int t = blockIdx.x + (2 * tw + s) * G;
-                    if (t < num_tiles) tiles[ns++] = t;
-                }
-                int m0[2], n0[2];
-                for (int s = 0; s < ns; ++s) {
-                    int mi, nj;
-                    tile_coords(tiles[s], MT, NT, mi, nj);
-                    m0[s] = mi * BM;
-                    n0[s] = nj * BN;
-                }
+                int pi, nj;
+                block_coords(t, NT, pi, nj);
+                const int m0 = pi * BN, n0 = nj * BN;
+                const bool diag = pi == nj;
+                const int halves = (m0 + BM < d) ? 2 : 1;
+                const uint32_t bytes = kBBytes + (diag ? 0 : halves * kABytes);
                 for (int k = k0; k < k1 && !*abort; ++k) {
-                    for (int s = 0; s < ns; ++s) {
-                        const uint32_t st = it % kStages;
-                        const uint32_t ph = (it / kStages) & 1u;
-                        if (!mbar_wait(&bars->empty[st], ph ^ 1u, abort)) break;
-                        uint8_t* a = smem + st * kStageBytes;
-                        uint8_t* b = a + kABytes;
-                        mbar_arrive_expect_tx(&bars->full[st], kStageBytes);
-                        const int tok = k * BK;
+                    const uint32_t st = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1u;
+                    if (!mbar_wait(&bars->empty[st], ph ^ 1u, abort)) break;
+                    uint8_t* b = smem + st * kStageBytes;
+                    mbar_arrive_expect_tx(&bars->full[st], bytes);
+                    const int tok = k * BK;
 #pragma unroll
-                        for (int c = 0; c < BM / kBox; ++c)
-                            tma_load_2d(a + c * kBoxBytes, &tmap_x, &bars->full[st], m0[s] + c * kBox,
-                                        tok);
+                    for (int c = 0; c < BN / kBox; ++c)
+                        tma_load_2d(b + c * kBoxBytes, &tmap_x, &bars->full[st], n0 + c * kBox, tok);
+                    if (!diag) {
+                        for (int h = 0; h < halves; ++h)
 #pragma unroll
-                        for (int c = 0; c < BN / kBox; ++c)
-                            tma_load_2d(b + c * kBoxBytes, &tmap_x, &bars->full[st], n0[s] + c * kBox,
-                                        tok);
-                        ++it;
+                            for (int c = 0; c < BM / kBox; ++c)
+                                tma_load_2d(b + kBBytes + h * kABytes + c * kBoxBytes, &tmap_x,
+                                            &bars->full[st], m0 + h * BM + c * kBox, tok);
                     }
+                    ++it;
                 }
             }
             // Never leave with copies in flight: wait for the last issued
@@ -215,36 +212,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t it = 0;
             wait_probe(&bars->never, probe_ns, abort);
             for (int w = 0; w < waves && !*abort; ++w) {
-                const int tw = w / nchunk;
+                const int t = blockIdx.x + (w / nchunk) * G;
+                if (t >= num_blocks) break;
                 const int k0 = (w % nchunk) * kChunkIters;
                 const int k1 = min(KB, k0 + kChunkIters);
-                int ns = 0;
-                for (int s = 0; s < 2; ++s)
-                    if (blockIdx.x + (2 * tw + s) * G < num_tiles) ++ns;
+                int pi, nj;
+                block_coords(t, NT, pi, nj);
+                const bool diag = pi == nj;
+                const int halves = (pi * BN + BM < d) ? 2 : 1;
                 if (!mbar_wait(&bars->acc_empty, (w & 1) ^ 1, abort)) break;
                 tc_fence_after();
                 bool ok = true;
-                for (int k = k0; k < k1 && ok; ++k) {
-                    for (int s = 0; s < ns; ++s) {
-                        const uint32_t st = it % kStages;
-                        const uint32_t ph = (it / kStages) & 1u;
-                        if (!mbar_wait(&bars->full[st], ph, abort)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t a = smem_u32(smem + st * kStageBytes);
-                        const uint32_t b = a + kABytes;
+                for (int k = k0; k < k1; ++k) {
+                    const uint32_t st = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1u;
+                    if (!mbar_wait(&bars->full[st], ph, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t b = smem_u32(smem + st * kStageBytes);
+                    for (int h = 0; h < halves; ++h) {
+                        // a diagonal block's rows are its own columns: A is
+                        // half h of B (two of its four boxes)
+                        const uint32_t a = diag ? b + h * 2 * kBoxBytes : b + kBBytes + h * kABytes;
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk) {
                             // 16 tokens = two 8-row swizzle atoms (2 x 1024 B)
                             const uint64_t ad = smem_desc(a + kk * 2048, kBoxBytes, 1024, 2);
                             const uint64_t bd = smem_desc(b + kk * 2048, kBoxBytes, 1024, 2);
-                            mma_f16_ss(tmem + s * BN, ad, bd, kIdesc, (k > k0 || kk > 0) ? 1u : 0u);
+                            mma_f16_ss(tmem + h * BN, ad, bd, kIdesc, (k > k0 || kk > 0) ? 1u : 0u);
                         }
-                        mma_commit(&bars->empty[st]);
-                        ++it;
                     }
+                    mma_commit(&bars->empty[st]);
+                    ++it;
                 }
                 if (!ok) break;
                 mma_commit(&bars->acc_full);
@@ -258,33 +259,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------ epilogue warps 2..9
         const int q = warp & 3;  // TMEM lane quarter this warp may access
-        const int half = (warp - 2) >> 2;  // which 128 of each tile's 256 columns it drains
+        const int half = (warp - 2) >> 2;  // which 128 of each accumulator's 256 columns it drains
         for (int w = 0; w < waves && !*abort; ++w) {
+            const int t = blockIdx.x + (w / nchunk) * G;
+            if (t >= num_blocks) break;
             if (!mbar_wait(&bars->acc_full, w & 1, abort)) break;
             tc_fence_after();
-            for (int s = 0; s < 2; ++s) {
-                const int t = blockIdx.x + (2 * (w / nchunk) + s) * G;
-                if (t >= num_tiles) break;
-                int mi, nj;
-                tile_coords(t, MT, NT, mi, nj);
-                const int m = mi * BM + q * 32 + lane;
+            int pi, nj;
+            block_coords(t, NT, pi, nj);
+            const int halves = (pi * BN + BM < d) ? 2 : 1;
+            for (int h = 0; h < halves; ++h) {
+                const int m = pi * BN + h * BM + q * 32 + lane;
                 const int nb = nj * BN;
 #pragma unroll 1
                 for (int cc = half * (BN / 64); cc < (half + 1) * (BN / 64); ++cc) {
                     float v[32];
-                    tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + s * BN + cc * 32, v);
+                    tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + h * BN + cc * 32, v);
                     if (m < d) {
                         // all 32 loads in flight before any store (the
                         // compiler cannot prove the addresses distinct)
-                        float h[32];
+                        float hv[32];
                         float* base = H + static_cast<int64_t>(nb + cc * 32) * ldh + m;
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
-                            h[j] = (nb + cc * 32 + j < d) ? base[static_cast<int64_t>(j) * ldh] : 0.f;
+                            hv[j] = (nb + cc * 32 + j < d) ? base[static_cast<int64_t>(j) * ldh] : 0.f;
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
                             if (nb + cc * 32 + j < d)
-                                base[static_cast<int64_t>(j) * ldh] = fmaf(2.0f, v[j], h[j]);
+                                base[static_cast<int64_t>(j) * ldh] = fmaf(2.0f, v[j], hv[j]);
                     }
                 }
             }
@@ -303,11 +305,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 int hessian_num_tiles(int64_t d) {
-    const int MT = static_cast<int>((d + BM - 1) / BM);
     const int NT = static_cast<int>((d + BN - 1) / BN);
-    int t = 0;
-    for (int nj = 0; nj < NT; ++nj) t += (MT < 2 * nj + 2) ? MT : 2 * nj + 2;
-    return t;
+    return NT * (NT + 1) / 2;
 }
 
 gptq_status launch_hessian(const uint16_t* X, int64_t n, int64_t d, int64_t ldx, float* H,
@@ -321,8 +320,7 @@ gptq_status launch_hessian(const uint16_t* X, int64_t n, int64_t d, int64_t ldx,
         return GPTQ_ERR_INVALID_ARG;
     const int T = hessian_num_tiles(d);
     const int sms = num_sms();
-    int grid = (T + 1) / 2;
-    if (grid > sms) grid = sms;
+    const int grid = T < sms ? T : sms;
     hessian_syrk_tcgen05<<<grid, kThreads, kSmemBytes, stream>>>(
         tmap, H, ldh, static_cast<int>(d), static_cast<int>(n), T, status,
         take_wait_probe(kProbeHessian));

@@ -64,6 +64,7 @@ def _run(X, packed, scales, zeros, perm, bits, g, d_row, ldy=None, ldx=None):
     (512, 1024, 128, 4, 8, True, None),      # smallest groups (8 codes)
     (77, 512, 96, 4, 32, False, 516),        # X rows not 16-byte aligned: gathered
     (2048, 8192, 1024, 4, 128, True, None),
+    (16, 82048, 128, 4, 128, True, None),    # rows too wide to stage: gathered through L1
 ])
 def test_dequant_gemm_matches_oracle(n_tok, d_col, d_row, bits, g, with_perm, ldx):
     X, packed, scales, zeros, perm = _case(n_tok, d_col, d_row, bits, g, with_perm,

@@ -336,6 +336,23 @@ def test_pack_is_bit_exact(bits, d):
     assert np.array_equal(packed.cpu().numpy().view(np.uint32), oracle.pack(c, bits))
 
 
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_pack_is_bit_exact_from_unaligned_codes(bits):
+    """Codes that do not start on a 16-byte boundary take the word-at-a-time
+    kernel instead of the 16-code chunks; same bits."""
+    g = gpu()
+    d = 256
+    rng = np.random.default_rng(bits + 7)
+    c = rng.integers(0, 1 << bits, size=(50, d), dtype=np.uint8)
+    buf = torch.zeros(50 * d + 16, dtype=torch.uint8, device="cuda")
+    cd = buf[3:3 + 50 * d].view(50, d)
+    cd.copy_(torch.from_numpy(c))
+    packed = torch.empty(50, g.packed_words(d, bits), dtype=torch.int32, device="cuda")
+    g.gptq_pack(cd, bits, packed)
+    torch.cuda.synchronize()
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), oracle.pack(c, bits))
+
+
 def test_stages_replay_from_a_cuda_graph_bit_exactly():
     """The four stages captured once in CUDA graphs (the library's side streams
     join the capture through its events) and replayed twice give the same bits
