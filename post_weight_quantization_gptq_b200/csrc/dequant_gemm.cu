@@ -56,24 +56,77 @@ struct Bars {
     int abort;
 };
 
+// Pairs of fp32 values in one 64-bit register, operated on by the packed
+// f32x2 instructions of sm_100 (one instruction, two IEEE round-to-nearest
+// results: the same values as two scalar operations).
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
 // x rounded to the nearest bf16 (ties to even), as an fp32 whose low 16 bits
-// are zero, on the fp32 pipe (Veltkamp's split with the factor 2^16 + 1:
-// c = x (2^16 + 1), hi = c - (c - x) keeps the 8 leading significant bits of
-// x rounded to nearest-even; explicit round-to-nearest operations so nothing
-// is contracted; |x| < 2^111).  Checked against the integer rounding rule on
-// random values and exact ties.  The conversion instruction runs on the
-// narrow conversion pipe, which the dequantization saturated (ncu: 102 % of
-// its peak); this form does not use it.
+// are zero, on the fp32 pipe: Veltkamp's split with the factor 2^16 + 1,
+// c = x (2^16 + 1), hi = c - (c - x), keeps the 8 leading significant bits of
+// x rounded to nearest-even (|x| < 2^111); checked against the integer
+// rounding rule on random values and exact ties.  It needs each step rounded
+// on its own: the scalar intrinsics below are never fused into an fma,
+// whereas the packed f32x2 form of the same steps was (its product merged
+// into the subtraction after it, which turned the rounding into truncation:
+// a one-ulp bf16 error that the parity test caught).  The conversion
+// instruction runs on the narrow conversion pipe, which the dequantization
+// saturated (ncu: 102 % of its peak); this form does not use it.
 __device__ __forceinline__ uint32_t bf16_bits(float x) {
     const float c = __fmul_rn(x, 65537.f);
     return __float_as_uint(__fsub_rn(c, __fsub_rn(c, x)));
 }
-// two values as one bf16x2 word (lo in the low half)
-__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
+// both values of a pair as one bf16x2 word (the low value in the low half)
+__device__ __forceinline__ uint32_t bf16x2_rne(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
     return __byte_perm(bf16_bits(lo), bf16_bits(hi), 0x7632);
 }
 
+// The eight codes of chunk c (codes 8c .. 8c+7 of the stage's row) as the
+// floats 2^23 + q: each code's bits land in the mantissa of 2^23 (a byte
+// permute against the exponent byte 0x4B where a code fills its own byte;
+// no int-to-float conversion).
 template <int BITS>
+__device__ __forceinline__ void chunk_codes(const uint32_t* w, int c, float (&f)[8]) {
+    constexpr uint32_t kMagic = 0x4B000000u;
+    if constexpr (BITS == 4) {
+        const uint32_t x = w[c];
+        const uint32_t ev = x & 0x0F0F0F0Fu;          // codes 0, 2, 4, 6 in bytes 0..3
+        const uint32_t od = (x >> 4) & 0x0F0F0F0Fu;   // codes 1, 3, 5, 7
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            f[2 * b] = __uint_as_float(__byte_perm(ev, kMagic, 0x7440 + b));
+            f[2 * b + 1] = __uint_as_float(__byte_perm(od, kMagic, 0x7440 + b));
+        }
+    } else if constexpr (BITS == 8) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            f[i] = __uint_as_float(__byte_perm(w[2 * c + (i >> 2)], kMagic, 0x7440 + (i & 3)));
+    } else {
+        const uint32_t h = w[c >> 1] >> (16 * (c & 1));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(((h >> (2 * i)) & 3u) | kMagic);
+    }
+}
+
+// kAligned: the group size is a multiple of the stage's 64 codes, so groups
+// change only between stages.
+template <int BITS, bool kAligned>
 __global__ void __launch_bounds__(kThreads, 1)
     dequant_gemm_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmp,
                         const float* __restrict__ scales, const int32_t* __restrict__ zeros,
@@ -82,7 +135,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kCpw = 32 / BITS;               // codes per packed word
     constexpr int kWords = BK / kCpw;             // words per row per stage
     constexpr int kRowBytes = kWords * 4;         // packed bytes per row per stage
-    constexpr uint32_t kMask = (1u << BITS) - 1u;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -176,12 +228,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = threadIdx.x - 64;  // row of the tile, 0..255
         const int ng = n0 + n;
         const bool live = ng < d_row;
-        // group of the current 8-code chunk, advanced as k crosses a group
-        // start (g is a multiple of 8, so a chunk crosses at most one; no
-        // integer division in the loop: its reciprocal runs on the same
-        // narrow conversion pipe)
+        const int groups = (K + g - 1) / g;
+        // the current group's scale and zero point, and the next group's,
+        // loaded one group ahead so that no chunk waits on global memory;
+        // the group starts are tracked by addition (no integer division in
+        // the loop: its reciprocal runs on the narrow conversion pipe)
         int cur_g = -1, next_start = 0;
-        float s = 0.f, z = 0.f;
+        float s = 0.f, z = 0.f, s_nx = 0.f, z_nx = 0.f;
+        auto fetch = [&](int gi, float& sv, float& zv) {
+            if (live && gi < groups) {
+                sv = __ldg(scales + static_cast<int64_t>(gi) * d_row + ng);
+                zv = static_cast<float>(__ldg(zeros + static_cast<int64_t>(gi) * d_row + ng));
+            }
+        };
+        fetch(0, s_nx, z_nx);
+        uint64_t s2 = 0, off2 = 0;
+        auto advance = [&]() {
+            ++cur_g;
+            next_start += g;
+            s = s_nx;
+            z = z_nx;
+            fetch(cur_g + 1, s_nx, z_nx);
+            s2 = pk2(s, s);
+            // subtracting 2^23 + z from 2^23 + q leaves q - z exactly
+            const float off = 8388608.f + z;
+            off2 = pk2(off, off);
+        };
         bool ok = true;
         for (int it = 0; it < nk; ++it) {
             const int st = it % kStages, b = it & 1;
@@ -199,29 +271,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
             }
             const uint32_t row = smem_u32(bbuf + b * kBBytes) + n * 128;
+            if constexpr (kAligned) {
+                if (it * BK >= next_start) advance();
+            }
             // 8 codes (one 16-byte chunk of bf16) at a time
 #pragma unroll
             for (int c = 0; c < BK / 8; ++c) {
-                const int k = it * BK + 8 * c;
-                if (k >= next_start) {
-                    ++cur_g;
-                    next_start += g;
-                    s = live ? __ldg(scales + static_cast<int64_t>(cur_g) * d_row + ng) : 0.f;
-                    z = live ? static_cast<float>(__ldg(zeros + static_cast<int64_t>(cur_g) * d_row + ng)) : 0.f;
+                if constexpr (!kAligned) {
+                    // g is a multiple of 8: a chunk lies inside one group
+                    if (it * BK + 8 * c >= next_start) advance();
                 }
-                // code q as the float 2^23 + q (its bits ORed into the
-                // mantissa of 2^23: no int-to-float conversion); subtracting
-                // 2^23 + z leaves q - z exactly, then one rounded product
-                const float off = 8388608.f + z;
-                float v[8];
+                float f[8];
+                chunk_codes<BITS>(w, c, f);
+                uint32_t o[4];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int e = 8 * c + i;  // code index within the stage
-                    const uint32_t q = (w[e / kCpw] >> (BITS * (e % kCpw))) & kMask;
-                    v[i] = (__uint_as_float(q | 0x4B000000u) - off) * s;
-                }
-                sts128_u(row + ((c ^ (n & 7)) << 4), make_uint4(bf16x2(v[0], v[1]), bf16x2(v[2], v[3]),
-                                                                 bf16x2(v[4], v[5]), bf16x2(v[6], v[7])));
+                for (int p = 0; p < 4; ++p)
+                    o[p] = bf16x2_rne(mul2(sub2(pk2(f[2 * p], f[2 * p + 1]), off2), s2));
+                sts128_u(row + ((c ^ (n & 7)) << 4), make_uint4(o[0], o[1], o[2], o[3]));
             }
             fence_async_smem();
             mbar_arrive(&bars->bfull[b]);
@@ -334,7 +400,7 @@ template <int BITS>
 cudaError_t launch_bits(const CUtensorMap& ta, const CUtensorMap& tp, const float* scales,
                         const int32_t* zeros, float* Y, int64_t ldy, int n_tok, int d_row, int K,
                         int g, int32_t* status, cudaStream_t stream) {
-    auto kern = dequant_gemm_kernel<BITS>;
+    auto kern = (g % BK == 0) ? dequant_gemm_kernel<BITS, true> : dequant_gemm_kernel<BITS, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     const dim3 grid((d_row + TN - 1) / TN, (n_tok + TM - 1) / TM);
