@@ -21,8 +21,9 @@
 //               kind::f16 M=128 N=256 K=16, both operands K-major
 //   warps 2..9  dequantize: thread n turns row n's 64 codes of the stage into
 //               bf16 and writes them, 16 bytes at a time, in the 128-byte
-//               swizzled K-major layout the MMA reads (two alternating
-//               buffers); after the K loop they drain the accumulators
+//               swizzled K-major layout the MMA reads (three rotating
+//               buffers, two at 8 bits); after the K loop they drain the
+//               accumulators
 // Every wait is bounded (GPTQ_ERR_TIMEOUT, as in the other tensor-core kernels).
 #include <cuda.h>
 
@@ -38,18 +39,28 @@ constexpr int BK = 64;                        // k per stage: 128 bytes of bf16
 constexpr int kStages = 3;
 constexpr int kABytes = TM * BK * 2;          // 32 KB
 constexpr int kBBytes = TN * BK * 2;          // 32 KB (one dequantized bf16 tile)
-constexpr int kPackedMax = TN * BK;           // packed words of a stage at 8 bits: 16 KB
-constexpr int kStageBytes = kABytes + kPackedMax;
+// Per code width: the packed words of a stage (TN rows x 64 codes) and the
+// number of bf16 tiles the dequantization rotates through.  Three tiles let
+// it run two stages ahead of the MMAs (with two, each stage waits for the
+// hand-over of the one before); at 8 bits the larger packed stages leave room
+// for two only.
+template <int BITS>
+struct Geom {
+    static constexpr int kPacked = TN * BK * BITS / 8;
+    static constexpr int kStageBytes = kABytes + kPacked;  // a multiple of 1024
+    static constexpr int kBBufs = BITS == 8 ? 2 : 3;
+    static constexpr int kSmemBytes = kStages * kStageBytes + kBBufs * kBBytes + 1024 + 256;
+};
+constexpr int kMaxBBufs = 3;
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kIdesc = instr_desc(/*bf16*/ 1, /*A K-major*/ 0, /*B K-major*/ 0, 128, TN);
-constexpr int kSmemBytes = kStages * kStageBytes + 2 * kBBytes + 1024 + 256;
 
 struct Bars {
     uint64_t full[kStages];   // TMA: activations + packed words landed
     uint64_t empty[kStages];  // MMA: stage consumed
-    uint64_t bfull[2];        // dequant warps: bf16 tile written (256 arrivals)
-    uint64_t bempty[2];       // MMA: bf16 tile consumed
+    uint64_t bfull[kMaxBBufs];   // dequant warps: bf16 tile written (256 arrivals)
+    uint64_t bempty[kMaxBBufs];  // MMA: bf16 tile consumed
     uint64_t acc_full;        // MMA: every product of the tile done
     uint64_t drain;
     uint32_t tmem;
@@ -124,6 +135,60 @@ __device__ __forceinline__ void chunk_codes(const uint32_t* w, int c, float (&f)
     }
 }
 
+// prmt.b32 in its default mode: each selector nibble picks one of the 8
+// bytes of (a, b); with the nibble's top bit set the picked byte's sign bit
+// fills the result byte (0x00 or 0xFF).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// The 16 dequantized weights a 4-bit row group can take, bf16(s (q - z)) for
+// q = 0..15 with the same arithmetic as the direct path, as byte tables: lo[j]
+// holds the low bytes of entries 4j .. 4j+3, hi[j] their high bytes.
+__device__ __forceinline__ void build_table4(float s, float z, uint32_t (&lo)[4], uint32_t (&hi)[4]) {
+    const uint64_t s2 = pk2(s, s), z2 = pk2(z, z);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint32_t r[4];
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const float q0 = static_cast<float>(4 * j + 2 * p);
+            const uint64_t v = mul2(sub2(pk2(q0, q0 + 1.f), z2), s2);  // q - z exact, one rounding
+            float a, b;
+            asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+            r[2 * p] = bf16_bits(a);        // bf16 in the high half
+            r[2 * p + 1] = bf16_bits(b);
+        }
+        const uint32_t u01 = __byte_perm(r[0], r[1], 0x7362);  // lo0 lo1 hi0 hi1
+        const uint32_t u23 = __byte_perm(r[2], r[3], 0x7362);
+        lo[j] = __byte_perm(u01, u23, 0x5410);
+        hi[j] = __byte_perm(u01, u23, 0x7632);
+    }
+}
+
+// The bf16 weights of the eight 4-bit codes of x (code i in bits 4i..4i+3) as
+// four bf16x2 words, by table look-up: a byte permute selects each code's
+// entry among 8 by its low three bits, in the tables' first and second
+// halves, and its fourth bit picks the half.
+__device__ __forceinline__ void lookup8(uint32_t x, const uint32_t (&lo)[4], const uint32_t (&hi)[4],
+                                        uint32_t (&o)[4]) {
+    const uint32_t xs = x << 4;  // a code's fourth bit at the top of a byte, even codes
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t sel = (x >> (16 * h)) & 0x7777u;
+        // 0xFF in byte i where code 4h + i is 8 or more (odd codes' fourth bit
+        // is already the top of a byte of x)
+        const uint32_t m = prmt(xs, x, h == 0 ? 0xD9C8u : 0xFBEAu);
+        const uint32_t la = prmt(lo[0], lo[1], sel), lb = prmt(lo[2], lo[3], sel);
+        const uint32_t ha = prmt(hi[0], hi[1], sel), hb = prmt(hi[2], hi[3], sel);
+        const uint32_t L = (la & ~m) | (lb & m), H = (ha & ~m) | (hb & m);
+        o[2 * h] = __byte_perm(L, H, 0x5140);      // codes 4h, 4h + 1
+        o[2 * h + 1] = __byte_perm(L, H, 0x7362);  // codes 4h + 2, 4h + 3
+    }
+}
+
 // kAligned: the group size is a multiple of the stage's 64 codes, so groups
 // change only between stages.
 template <int BITS, bool kAligned>
@@ -138,8 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    uint8_t* bbuf = smem + kStages * kStageBytes;  // two bf16 tiles, 1024-aligned
-    Bars* bars = reinterpret_cast<Bars*>(bbuf + 2 * kBBytes);
+    constexpr int kStageBytes = Geom<BITS>::kStageBytes;
+    constexpr int kBBufs = Geom<BITS>::kBBufs;
+    uint8_t* bbuf = smem + kStages * kStageBytes;  // the bf16 tiles, 1024-aligned
+    Bars* bars = reinterpret_cast<Bars*>(bbuf + kBBufs * kBBytes);
     volatile int* abort = &bars->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * TN, t0 = blockIdx.y * TM;
@@ -150,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->full[s], 1);
             mbar_init(&bars->empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kBBufs; ++b) {
             mbar_init(&bars->bfull[b], 256);
             mbar_init(&bars->bempty[b], 1);
         }
@@ -199,9 +266,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             bool ok = true;
             for (int it = 0; it < nk && ok; ++it) {
-                const int st = it % kStages, b = it & 1;
+                const int st = it % kStages, b = it % kBBufs;
                 if (!mbar_wait(&bars->full[st], (it / kStages) & 1u, abort) ||
-                    !mbar_wait(&bars->bfull[b], (it >> 1) & 1u, abort)) {
+                    !mbar_wait(&bars->bfull[b], (it / kBBufs) & 1u, abort)) {
                     ok = false;
                     break;
                 }
@@ -242,23 +309,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         };
         fetch(0, s_nx, z_nx);
+        // 4-bit codes with groups of whole stages: a table of the group's 16
+        // weights, built once per group (about 90 instructions, against about
+        // 8 per code computed directly)
+        constexpr bool kTable = BITS == 4 && kAligned;
         uint64_t s2 = 0, off2 = 0;
+        uint32_t tlo[4] = {0, 0, 0, 0}, thi[4] = {0, 0, 0, 0};
         auto advance = [&]() {
             ++cur_g;
             next_start += g;
             s = s_nx;
             z = z_nx;
             fetch(cur_g + 1, s_nx, z_nx);
-            s2 = pk2(s, s);
-            // subtracting 2^23 + z from 2^23 + q leaves q - z exactly
-            const float off = 8388608.f + z;
-            off2 = pk2(off, off);
+            if constexpr (kTable) {
+                build_table4(s, z, tlo, thi);
+            } else {
+                s2 = pk2(s, s);
+                // subtracting 2^23 + z from 2^23 + q leaves q - z exactly
+                const float off = 8388608.f + z;
+                off2 = pk2(off, off);
+            }
         };
         bool ok = true;
         for (int it = 0; it < nk; ++it) {
-            const int st = it % kStages, b = it & 1;
+            const int st = it % kStages, b = it % kBBufs;
             if (!mbar_wait(&bars->full[st], (it / kStages) & 1u, abort) ||
-                !mbar_wait(&bars->bempty[b], ((it >> 1) & 1u) ^ 1u, abort)) {
+                !mbar_wait(&bars->bempty[b], ((it / kBBufs) & 1u) ^ 1u, abort)) {
                 ok = false;
                 break;
             }
@@ -281,12 +357,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // g is a multiple of 8: a chunk lies inside one group
                     if (it * BK + 8 * c >= next_start) advance();
                 }
-                float f[8];
-                chunk_codes<BITS>(w, c, f);
                 uint32_t o[4];
+                if constexpr (kTable) {
+                    lookup8(w[c], tlo, thi, o);
+                } else {
+                    float f[8];
+                    chunk_codes<BITS>(w, c, f);
 #pragma unroll
-                for (int p = 0; p < 4; ++p)
-                    o[p] = bf16x2_rne(mul2(sub2(pk2(f[2 * p], f[2 * p + 1]), off2), s2));
+                    for (int p = 0; p < 4; ++p)
+                        o[p] = bf16x2_rne(mul2(sub2(pk2(f[2 * p], f[2 * p + 1]), off2), s2));
+                }
                 sts128_u(row + ((c ^ (n & 7)) << 4), make_uint4(o[0], o[1], o[2], o[3]));
             }
             fence_async_smem();
@@ -401,6 +481,8 @@ cudaError_t launch_bits(const CUtensorMap& ta, const CUtensorMap& tp, const floa
                         const int32_t* zeros, float* Y, int64_t ldy, int n_tok, int d_row, int K,
                         int g, int32_t* status, cudaStream_t stream) {
     auto kern = (g % BK == 0) ? dequant_gemm_kernel<BITS, true> : dequant_gemm_kernel<BITS, false>;
+    constexpr int kSmemBytes = Geom<BITS>::kSmemBytes;
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     const dim3 grid((d_row + TN - 1) / TN, (n_tok + TM - 1) / TM);
