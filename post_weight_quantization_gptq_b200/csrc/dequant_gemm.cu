@@ -15,7 +15,8 @@
 //
 // CTA tile: 256 tokens x 256 layer outputs, K in stages of 64.  Warp roles:
 //   warp 0      TMA: the stage's activations (256 x 64 bf16, 128-byte swizzle)
-//               and packed words (256 rows x 64 codes)
+//   warp 10     TMA: the stage's packed words (256 rows x 64 codes), several
+//               stages ahead in a ring of their own
 //   warp 1      TMEM owner (512 columns: two 128-token accumulators of 256
 //               fp32 columns) and MMA issuer: per stage, 2 x 4 MMAs
 //               kind::f16 M=128 N=256 K=16, both operands K-major
@@ -36,29 +37,36 @@ namespace {
 constexpr int TM = 256;                       // tokens per CTA tile
 constexpr int TN = 256;                       // layer outputs per CTA tile (MMA N)
 constexpr int BK = 64;                        // k per stage: 128 bytes of bf16
-constexpr int kStages = 3;
+constexpr int kAStages = 3;                   // activation tiles in flight
 constexpr int kABytes = TM * BK * 2;          // 32 KB
 constexpr int kBBytes = TN * BK * 2;          // 32 KB (one dequantized bf16 tile)
-// Per code width: the packed words of a stage (TN rows x 64 codes) and the
-// number of bf16 tiles the dequantization rotates through.  Three tiles let
-// it run two stages ahead of the MMAs (with two, each stage waits for the
-// hand-over of the one before); at 8 bits the larger packed stages leave room
-// for two only.
+// Per code width: the packed words of a stage (TN rows x 64 codes), how many
+// such stages are in flight (their own ring, released by the dequantization
+// as soon as it has read them, so they arrive well before they are needed:
+// when they shared the activations' stages, released only by the MMAs, a
+// stage's words could not be loaded before the MMAs two stages back had
+// finished) and the number of bf16 tiles the dequantization rotates through
+// (three let it run two stages ahead of the MMAs).  Shared memory: the
+// activation ring, the bf16 tiles, then the packed ring.
 template <int BITS>
 struct Geom {
     static constexpr int kPacked = TN * BK * BITS / 8;
-    static constexpr int kStageBytes = kABytes + kPacked;  // a multiple of 1024
+    static constexpr int kPStages = BITS == 8 ? 3 : BITS == 4 ? 4 : 6;
     static constexpr int kBBufs = BITS == 8 ? 2 : 3;
-    static constexpr int kSmemBytes = kStages * kStageBytes + kBBufs * kBBytes + 1024 + 256;
+    static constexpr int kSmemBytes =
+        kAStages * kABytes + kBBufs * kBBytes + kPStages * kPacked + 1024 + 256;
 };
 constexpr int kMaxBBufs = 3;
-constexpr int kThreads = 320;
+constexpr int kMaxPStages = 6;
+constexpr int kThreads = 352;  // TMA (activations), MMA, 8 dequantization warps, TMA (packed)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kIdesc = instr_desc(/*bf16*/ 1, /*A K-major*/ 0, /*B K-major*/ 0, 128, TN);
 
 struct Bars {
-    uint64_t full[kStages];   // TMA: activations + packed words landed
-    uint64_t empty[kStages];  // MMA: stage consumed
+    uint64_t afull[kAStages];     // TMA: activations landed
+    uint64_t aempty[kAStages];    // MMA: activations consumed
+    uint64_t pfull[kMaxPStages];  // TMA: packed words landed
+    uint64_t pempty[kMaxPStages]; // dequantization: packed words read (256 arrivals)
     uint64_t bfull[kMaxBBufs];   // dequant warps: bf16 tile written (256 arrivals)
     uint64_t bempty[kMaxBBufs];  // MMA: bf16 tile consumed
     uint64_t acc_full;        // MMA: every product of the tile done
@@ -203,19 +211,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    constexpr int kStageBytes = Geom<BITS>::kStageBytes;
     constexpr int kBBufs = Geom<BITS>::kBBufs;
-    uint8_t* bbuf = smem + kStages * kStageBytes;  // the bf16 tiles, 1024-aligned
-    Bars* bars = reinterpret_cast<Bars*>(bbuf + kBBufs * kBBytes);
+    constexpr int kPStages = Geom<BITS>::kPStages;
+    constexpr int kPacked = Geom<BITS>::kPacked;
+    uint8_t* bbuf = smem + kAStages * kABytes;     // the bf16 tiles, 1024-aligned
+    uint8_t* pbuf = bbuf + kBBufs * kBBytes;       // the packed ring
+    Bars* bars = reinterpret_cast<Bars*>(pbuf + kPStages * kPacked);
     volatile int* abort = &bars->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * TN, t0 = blockIdx.y * TM;
     const int nk = K / BK;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&bars->full[s], 1);
-            mbar_init(&bars->empty[s], 1);
+        for (int s = 0; s < kAStages; ++s) {
+            mbar_init(&bars->afull[s], 1);
+            mbar_init(&bars->aempty[s], 1);
+        }
+        for (int s = 0; s < kPStages; ++s) {
+            mbar_init(&bars->pfull[s], 1);
+            mbar_init(&bars->pempty[s], 256);
         }
         for (int b = 0; b < kBBufs; ++b) {
             mbar_init(&bars->bfull[b], 256);
@@ -237,25 +251,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = bars->tmem;
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+    if (warp == 0 || warp == 10) {
+        // ------------------------------------------------ TMA producers: warp 0
+        // the activations (ring released by the MMAs), warp 10 the packed
+        // words (ring released by the dequantization)
         if (lane == 0) {
+            const bool act = warp == 0;
+            const int depth = act ? kAStages : kPStages;
+            uint64_t* fullb = act ? bars->afull : bars->pfull;
+            uint64_t* emptyb = act ? bars->aempty : bars->pempty;
             int it = 0;
             for (; it < nk && !*abort; ++it) {
-                const int st = it % kStages;
-                const uint32_t ph = (it / kStages) & 1u;
-                if (!mbar_wait(&bars->empty[st], ph ^ 1u, abort)) break;
-                uint8_t* a = smem + st * kStageBytes;
-                mbar_arrive_expect_tx(&bars->full[st], kABytes + TN * kRowBytes);
-                tma_load_2d(a, &tma, &bars->full[st], it * BK, t0);
-                tma_load_2d(a + kABytes, &tmp, &bars->full[st], it * kWords, n0);
+                const int st = it % depth;
+                const uint32_t ph = (it / depth) & 1u;
+                if (!mbar_wait(&emptyb[st], ph ^ 1u, abort)) break;
+                if (act) {
+                    mbar_arrive_expect_tx(&fullb[st], kABytes);
+                    tma_load_2d(smem + st * kABytes, &tma, &fullb[st], it * BK, t0);
+                } else {
+                    mbar_arrive_expect_tx(&fullb[st], TN * kRowBytes);
+                    tma_load_2d(pbuf + st * kPacked, &tmp, &fullb[st], it * kWords, n0);
+                }
             }
             // never leave with copies in flight (bounded even when aborting)
             volatile int no_abort = 0;
-            const int last = it < kStages ? it : kStages;
+            const int last = it < depth ? it : depth;
             for (int j = 0; j < last; ++j) {
                 const int i2 = it - 1 - j;
-                if (!mbar_wait(&bars->full[i2 % kStages], (i2 / kStages) & 1u, &no_abort)) {
+                if (!mbar_wait(&fullb[i2 % depth], (i2 / depth) & 1u, &no_abort)) {
                     *abort = 1;
                     break;
                 }
@@ -266,14 +289,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             bool ok = true;
             for (int it = 0; it < nk && ok; ++it) {
-                const int st = it % kStages, b = it % kBBufs;
-                if (!mbar_wait(&bars->full[st], (it / kStages) & 1u, abort) ||
+                const int st = it % kAStages, b = it % kBBufs;
+                if (!mbar_wait(&bars->afull[st], (it / kAStages) & 1u, abort) ||
                     !mbar_wait(&bars->bfull[b], (it / kBBufs) & 1u, abort)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a = smem_u32(smem + st * kStageBytes);
+                const uint32_t a = smem_u32(smem + st * kABytes);
                 const uint32_t bt = smem_u32(bbuf + b * kBBytes);
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
@@ -282,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_f16_ss(tmem + h * TN, smem_desc(a + h * (kABytes / 2) + kk * 32, 16, 1024, 2),
                                    smem_desc(bt + kk * 32, 16, 1024, 2), kIdesc,
                                    (it > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&bars->empty[st]);
+                mma_commit(&bars->aempty[st]);
                 mma_commit(&bars->bempty[b]);
             }
             if (ok) mma_commit(&bars->acc_full);
@@ -332,14 +355,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         bool ok = true;
         for (int it = 0; it < nk; ++it) {
-            const int st = it % kStages, b = it % kBBufs;
-            if (!mbar_wait(&bars->full[st], (it / kStages) & 1u, abort) ||
+            const int ps = it % kPStages, b = it % kBBufs;
+            if (!mbar_wait(&bars->pfull[ps], (it / kPStages) & 1u, abort) ||
                 !mbar_wait(&bars->bempty[b], ((it / kBBufs) & 1u) ^ 1u, abort)) {
                 ok = false;
                 break;
             }
-            const uint32_t* words = reinterpret_cast<const uint32_t*>(
-                smem + st * kStageBytes + kABytes + n * kRowBytes);
+            const uint32_t* words =
+                reinterpret_cast<const uint32_t*>(pbuf + ps * kPacked + n * kRowBytes);
             uint32_t w[kWords];
 #pragma unroll
             for (int q = 0; q < kWords / 4; ++q) {
@@ -371,6 +394,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_async_smem();
             mbar_arrive(&bars->bfull[b]);
+            // every word read from the slot has been used (so its load has
+            // completed) before the slot may be refilled; released right after
+            // the loads were issued, 8-bit rows (four-way bank conflicts, longer
+            // loads) read words of the next refill
+            mbar_arrive(&bars->pempty[ps]);
         }
         // ------------------------------------------------ drain: TMEM -> Y
         if (ok && mbar_wait(&bars->acc_full, 0, abort)) {
