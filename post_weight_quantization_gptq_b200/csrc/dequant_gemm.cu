@@ -481,10 +481,85 @@ gather_bf16_kernel(const uint16_t* __restrict__ X, int64_t ldx, int64_t n_tok, i
     }
 }
 
+// The same gather for aligned rows that fit, pipelined: the permutation is
+// staged once per CTA in shared memory as 16-bit indices, and each CTA copies
+// its next token row into the second of two row buffers (cp.async, 16 bytes
+// per copy, no registers) while it gathers the current one, so HBM streams
+// rows in and out while the shared-memory gathers run.  The first form read
+// perm through L2 for every value, one dependent read after another.
+constexpr int kPipeThreads = 512;
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+                 "l"(gsrc)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_older() {
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kPipeThreads)
+gather_bf16_piped_kernel(const uint16_t* __restrict__ X, int64_t ldx, int64_t n_tok, int K,
+                         const int32_t* __restrict__ perm, uint16_t* __restrict__ Xq) {
+    extern __shared__ __align__(16) uint16_t gs[];
+    uint16_t* idx = gs;            // [K] source column of each position
+    uint16_t* rows = gs + K;       // [2][K] token rows
+    const int chunks = K / 8;
+    for (int k = threadIdx.x; k < K; k += kPipeThreads) {
+        int col = perm != nullptr ? perm[k] : k;
+        if (col < 0 || col >= K) col = k;
+        idx[k] = static_cast<uint16_t>(col);
+    }
+    auto fetch = [&](int64_t t, int buf) {
+        if (t < n_tok) {
+            const uint16_t* xr = X + t * ldx;
+            uint16_t* dst = rows + buf * K;
+            for (int c = threadIdx.x; c < chunks; c += kPipeThreads)
+                cp_async16(dst + 8 * c, xr + 8 * c);
+        }
+        cp_async_commit();  // an empty group past the last row keeps the count
+    };
+    int buf = 0;
+    fetch(blockIdx.x, 0);
+    for (int64_t t = blockIdx.x; t < n_tok; t += gridDim.x) {
+        fetch(t + gridDim.x, buf ^ 1);
+        cp_async_wait_older();  // this thread's copies of row t have landed
+        __syncthreads();        // ... and everyone's (and idx is written)
+        const uint16_t* row = rows + buf * K;
+        uint4* dst = reinterpret_cast<uint4*>(Xq + t * static_cast<int64_t>(K));
+        for (int c = threadIdx.x; c < chunks; c += kPipeThreads) {
+            const uint4 ix = reinterpret_cast<const uint4*>(idx)[c];
+            const uint32_t iw[4] = {ix.x, ix.y, ix.z, ix.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                o[j] = static_cast<uint32_t>(row[iw[j] & 0xFFFFu]) |
+                       (static_cast<uint32_t>(row[iw[j] >> 16]) << 16);
+            dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        __syncthreads();  // row buffer `buf` is refilled two rows later
+        buf ^= 1;
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // no copy outlives the CTA
+}
+
 cudaError_t launch_gather(const uint16_t* X, int64_t ldx, int64_t n_tok, int K,
                           const int32_t* perm, uint16_t* Xq, cudaStream_t stream) {
     const size_t smem = static_cast<size_t>(K) * 2;
     const bool vec = (ldx % 8) == 0 && (reinterpret_cast<uintptr_t>(X) & 15) == 0;
+    const size_t piped = 3 * smem;  // indices and two rows
+    if (vec && piped <= 227 * 1024 && K <= 65536) {
+        auto kern = gather_bf16_piped_kernel;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(piped));
+        if (e != cudaSuccess) return e;
+        const int grid = static_cast<int>(n_tok < num_sms() ? n_tok : num_sms());
+        kern<<<grid, kPipeThreads, piped, stream>>>(X, ldx, n_tok, K, perm, Xq);
+        return cudaGetLastError();
+    }
     if (smem > kGatherSmemMax) {
         const int grid = static_cast<int>(n_tok < 8 * num_sms() ? n_tok : 8 * num_sms());
         gather_bf16_kernel<false, false><<<grid, kGatherThreads, 0, stream>>>(X, ldx, n_tok, K,
