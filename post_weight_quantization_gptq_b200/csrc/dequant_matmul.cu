@@ -17,8 +17,10 @@
 //                        stages the step's token values in shared memory.
 //
 // Arithmetic per code: the code's bits are moved into the mantissa of a float
-// (f = 1 + q / 2^b, exact: one shift and one LOP3) and multiplied into a
-// running dot with the token values; per word the dot d = sum_t x_t f_t and
+// (f = 1 + q / 2^b, exact: one shift and one LOP3, or at 4 bits one byte
+// permute after two shared shifts and masks per word) and multiplied into a
+// running dot with the token values (at 4 bits two running dots, even and
+// odd codes, in one packed f32x2 FMA per pair); per word the dot d = sum_t x_t f_t and
 // the token sum S = sum_t x_t give sum_t x_t q_t = 2^b (d - S), so the word
 // adds s 2^b d - s (2^b + z) S to the output (two FMAs, the group's scale s
 // and zero point z folded in once per group).  d and S carry the same rounding
@@ -62,6 +64,42 @@ __device__ __forceinline__ float code_as_float(uint32_t word, int t) {
     return __uint_as_float((v & mask) | 0x3F800000u);
 }
 
+// Packed f32x2 fused multiply-add (sm_100): d = a * b + c on both halves.
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ float sum2(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return lo + hi;
+}
+
+// d = sum_t x[t] (1 + q_t / 16) over the eight 4-bit codes of a word, with
+// the floats built by byte permutes: each code shifted to bits 3..6 of its
+// own byte with the byte's top bit set, then placed as the third byte of a
+// float whose top byte is 0x3F (exponent 0, mantissa q / 16; the same value
+// as code_as_float).  Two running sums (even and odd codes) as one packed
+// f32x2 FMA per code pair.
+__device__ __forceinline__ float dot4bit(uint32_t word, const float (&xv)[8]) {
+    const uint32_t ev = ((word << 3) & 0x78787878u) | 0x80808080u;  // codes 0, 2, 4, 6
+    const uint32_t od = ((word >> 1) & 0x78787878u) | 0x80808080u;  // codes 1, 3, 5, 7
+    uint64_t d = 0;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float f0 = __uint_as_float(__byte_perm(ev, 0x3F000000u, 0x7044 | (p << 8)));
+        const float f1 = __uint_as_float(__byte_perm(od, 0x3F000000u, 0x7044 | (p << 8)));
+        d = fma2(pk2(xv[2 * p], xv[2 * p + 1]), pk2(f0, f1), d);
+    }
+    return sum2(d);
+}
+
 template <int BITS, int LW>
 struct StepShape {
     static constexpr int CPW = 32 / BITS;                 // codes per word
@@ -74,7 +112,9 @@ struct StepShape {
 };
 
 template <int BITS, int MT, int LW>  // LW: words per lane per step
-__global__ void __launch_bounds__(kThreads)
+// 4-bit: two CTAs per SM (at most 128 registers; the packed dot otherwise
+// takes 140 at two tokens and halves the resident warps)
+__global__ void __launch_bounds__(kThreads, BITS == 4 ? 2 : 1)
     dequant_matmul_kernel(const float* __restrict__ Xq, int M, int K,
                           const uint32_t* __restrict__ packed, int64_t P,
                           const float* __restrict__ scales, const int32_t* __restrict__ zeros,
@@ -177,8 +217,12 @@ __global__ void __launch_bounds__(kThreads)
                 for (int r = 0; r < kRowsPerWarp; ++r) {
                     float d = 0.f;
                     const uint32_t word = wd[r][4 * u + i];
+                    if constexpr (BITS == 4) {
+                        d = dot4bit(word, xv);
+                    } else {
 #pragma unroll
-                    for (int t = 0; t < CPW; ++t) d = fmaf(xv[t], code_as_float<BITS>(word, t), d);
+                        for (int t = 0; t < CPW; ++t) d = fmaf(xv[t], code_as_float<BITS>(word, t), d);
+                    }
                     acc[r][m] = fmaf(ga[r], d, fmaf(gb[r], S, acc[r][m]));
                 }
             }
