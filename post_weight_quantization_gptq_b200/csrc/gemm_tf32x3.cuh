@@ -19,8 +19,10 @@
 // with 32-byte chunks).  Warp roles:
 //   warp 0      TMA producer
 //   warp 1      TMEM owner and MMA issuer
-//   warps 2..5  split each stage's operands (write lo, and hi when rounding)
-//   warps 6..9  drain the accumulator (tcgen05.ld gives one tile row per
+//   warps 2..9  split each stage's operands (write lo, and hi when rounding;
+//               with four warps the split was measurably on the critical path:
+//               the lazy update without it ran 9-13 % faster)
+//   warps 10..13 drain the accumulator (tcgen05.ld gives one tile row per
 //               lane).  Plain outputs receive the product, read-modify-write
 //               outputs (kRmw) D -= AB^T.  Three forms:
 //               staged (kEpiStaged): into sched.dst() rows, sched.ncols()
@@ -56,7 +58,8 @@ constexpr int BK = 32;                        // K per stage: 128 bytes of fp32
 constexpr int kStages = 3;
 constexpr int kTileBytes = 128 * BK * 4;      // 16 KB
 constexpr int kStageBytes = 4 * kTileBytes;   // A (as loaded), A lo, B (as loaded), B lo
-constexpr int kThreads = 320;                 // TMA, MMA, 4 split warps, 4 epilogue warps
+constexpr int kThreads = 448;                 // TMA, MMA, 8 split warps, 4 epilogue warps
+constexpr int kSplitThreads = 256;
 constexpr int kEpiPitch = 36;                 // floats per staged row (16-byte groups of 8
                                               // consecutive rows fall in distinct banks)
 constexpr int kEpiBytes = 4 * 32 * kEpiPitch * 4;  // one 32 x 32 stage per epilogue warp
@@ -163,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&bars->full[s], 1);
-            mbar_init(&bars->conv[s], 128);
+            mbar_init(&bars->conv[s], kSplitThreads);
             mbar_init(&bars->empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -260,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             volatile int no_abort = 0;
             if (!mbar_wait(&bars->drain, 0, &no_abort)) *abort = 1;
         }
-    } else if (warp < 6) {
+    } else if (warp < 10) {
         // ---------------------------------------------------- split into hi / lo
         const int t0 = threadIdx.x - 64;
         int it = 0;
@@ -279,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float4* b = a + 2 * (kTileBytes / 16);
                 float4* blo = a + 3 * (kTileBytes / 16);
 #pragma unroll 4
-                for (int i = t0; i < kTileBytes / 16; i += 128) {
+                for (int i = t0; i < kTileBytes / 16; i += kSplitThreads) {
                     const float4 x = a[i], y = b[i];
                     if constexpr (Split == kSplitRound) {
                         const float4 xh = tf32_round4(x), yh = tf32_round4(y);
