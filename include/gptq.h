@@ -221,6 +221,13 @@ gptq_status gptq_prepare_hinv(float *H, int64_t d, int64_t ldh, const gptq_confi
  *   scales  fp32 [ceil(d_col / g)][d_row] and zeros int32 (same shape),
  *           group-major, groups in quantization order.  Dequantization:
  *           W_hat[row][perm[k]] = scales[k/g][row] * (codes[row][k] - zeros[k/g][row]).
+ *   ws      at least d_row * 512 bytes (GPTQ_ERR_WORKSPACE otherwise).  With
+ *           gptq_workspace_size() bytes the lazy update defers up to 8 blocks
+ *           and reads its operands' low-precision parts, split once, from the
+ *           workspace (d_col^2 * 4 bytes for U's, as much again as the
+ *           deferred errors for theirs); smaller workspaces defer fewer blocks
+ *           and split in the GEMM.  The split values are the same, so for a
+ *           given number of deferred blocks the results are identical.
  */
 gptq_status gptq_quantize_layer(float *W, int64_t d_row, int64_t d_col, int64_t ldw,
                                 const float *U, const int32_t *perm, const uint8_t *dead,

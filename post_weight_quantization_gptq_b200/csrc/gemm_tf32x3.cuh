@@ -8,7 +8,9 @@
 // lo = x - trunc13(x) (one buffer written per operand, products within about
 // 2^-20 of |a||b|, biased towards zero), or hi and lo both rounded to the
 // nearest tf32 (two buffers written, products within about 3 2^-22 of |a||b|
-// and unbiased), at tensor-core speed either way.
+// and unbiased), at tensor-core speed either way.  The truncating split can
+// also be done ahead (kSplitPre): the lo parts then come from memory with the
+// operands.
 //
 // Persistent: each CTA walks a static list of output tiles (tile, tile +
 // grid, ...), the stage ring runs on across tiles and two TMEM accumulators
@@ -120,7 +122,11 @@ __device__ __forceinline__ float4 sub4(float4 a, float4 b) {
 // both written: x - hi - lo is within 2^-22 |x| and of either sign, so a
 // product's error (that, the two roundings and the dropped lo lo term) stays
 // within ~3 2^-22 |ab| and long sums do not drift.
-constexpr int kSplitTrunc = 0, kSplitRound = 1;
+// kSplitPre: the truncating split done ahead of the GEMM: both operands' lo
+// parts sit in memory of their own (the same values kSplitTrunc computes) and
+// arrive by TMA with the operands; no split work between a stage's arrival and
+// its MMAs.
+constexpr int kSplitTrunc = 0, kSplitRound = 1, kSplitPre = 2;
 
 
 
@@ -150,7 +156,8 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk) {
 template <class Sched, bool A_MN, bool B_MN, int Epi, int Split>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
-                       const __grid_constant__ CUtensorMap tmd, const Sched sched, int tiles,
+                       const __grid_constant__ CUtensorMap tmd, const __grid_constant__ CUtensorMap tmal,
+                       const __grid_constant__ CUtensorMap tmbl, const Sched sched, int tiles,
                        int32_t* status, uint64_t probe_ns) {
     constexpr uint32_t kIdesc = instr_desc(/*tf32*/ 2, A_MN ? 1 : 0, B_MN ? 1 : 0, BM, BN);
 
@@ -180,6 +187,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tma);
         tma_prefetch_desc(&tmb);
         if constexpr (Epi >= kEpiReduce) tma_prefetch_desc(&tmd);
+        if constexpr (Split == kSplitPre) {
+            tma_prefetch_desc(&tmal);
+            tma_prefetch_desc(&tmbl);
+        }
     }
     if (warp == 1) {
         tmem_alloc(&bars->tmem, kTmemCols);
@@ -202,10 +213,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t ph = (it / kStages) & 1;
                     if (!mbar_wait(&bars->empty[st], ph ^ 1u, abort)) break;
                     uint8_t* a = smem + st * kStageBytes;
-                    mbar_arrive_expect_tx(&bars->full[st], 2 * kTileBytes);
+                    mbar_arrive_expect_tx(&bars->full[st], (Split == kSplitPre ? 4 : 2) * kTileBytes);
                     load_operand<A_MN>(a, &tma, &bars->full[st], job.m0, job.ka0 + s * BK);
                     load_operand<B_MN>(a + 2 * kTileBytes, &tmb, &bars->full[st], job.n0,
                                        job.kb0 + s * BK);
+                    if constexpr (Split == kSplitPre) {
+                        load_operand<A_MN>(a + kTileBytes, &tmal, &bars->full[st], job.m0,
+                                           job.ka0 + s * BK);
+                        load_operand<B_MN>(a + 3 * kTileBytes, &tmbl, &bars->full[st], job.n0,
+                                           job.kb0 + s * BK);
+                    }
                 }
             }
             // never leave with copies in flight (bounded even when aborting)
@@ -238,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int s = 0; s < job.nk; ++s, ++it) {
                     const int st = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
-                    if (!mbar_wait(&bars->conv[st], ph, abort)) {
+                    if (!mbar_wait(Split == kSplitPre ? &bars->full[st] : &bars->conv[st], ph, abort)) {
                         ok = false;
                         break;
                     }
@@ -265,38 +282,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp < 10) {
         // ---------------------------------------------------- split into hi / lo
-        const int t0 = threadIdx.x - 64;
-        int it = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-            const Job job = sched.job(t);
-            for (int s = 0; s < job.nk; ++s, ++it) {
-                const int st = it % kStages;
-                const uint32_t ph = (it / kStages) & 1;
-                if (!mbar_wait(&bars->full[st], ph, abort)) {
-                    ok = false;
-                    break;
-                }
-                float4* a = reinterpret_cast<float4*>(smem + st * kStageBytes);
-                float4* alo = a + kTileBytes / 16;
-                float4* b = a + 2 * (kTileBytes / 16);
-                float4* blo = a + 3 * (kTileBytes / 16);
-#pragma unroll 4
-                for (int i = t0; i < kTileBytes / 16; i += kSplitThreads) {
-                    const float4 x = a[i], y = b[i];
-                    if constexpr (Split == kSplitRound) {
-                        const float4 xh = tf32_round4(x), yh = tf32_round4(y);
-                        a[i] = xh;
-                        b[i] = yh;
-                        alo[i] = tf32_round4(sub4(x, xh));
-                        blo[i] = tf32_round4(sub4(y, yh));
-                    } else {
-                        alo[i] = make_float4(tf32_rest(x.x), tf32_rest(x.y), tf32_rest(x.z), tf32_rest(x.w));
-                        blo[i] = make_float4(tf32_rest(y.x), tf32_rest(y.y), tf32_rest(y.z), tf32_rest(y.w));
+        if constexpr (Split == kSplitPre) {
+            // the lo parts arrive with the operands: nothing to do
+        } else {
+            const int t0 = threadIdx.x - 64;
+            int it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                const Job job = sched.job(t);
+                for (int s = 0; s < job.nk; ++s, ++it) {
+                    const int st = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1;
+                    if (!mbar_wait(&bars->full[st], ph, abort)) {
+                        ok = false;
+                        break;
                     }
+                    float4* a = reinterpret_cast<float4*>(smem + st * kStageBytes);
+                    float4* alo = a + kTileBytes / 16;
+                    float4* b = a + 2 * (kTileBytes / 16);
+                    float4* blo = a + 3 * (kTileBytes / 16);
+#pragma unroll 4
+                    for (int i = t0; i < kTileBytes / 16; i += kSplitThreads) {
+                        const float4 x = a[i], y = b[i];
+                        if constexpr (Split == kSplitRound) {
+                            const float4 xh = tf32_round4(x), yh = tf32_round4(y);
+                            a[i] = xh;
+                            b[i] = yh;
+                            alo[i] = tf32_round4(sub4(x, xh));
+                            blo[i] = tf32_round4(sub4(y, yh));
+                        } else {
+                            alo[i] = make_float4(tf32_rest(x.x), tf32_rest(x.y), tf32_rest(x.z), tf32_rest(x.w));
+                            blo[i] = make_float4(tf32_rest(y.x), tf32_rest(y.y), tf32_rest(y.z), tf32_rest(y.w));
+                        }
+                    }
+                    fence_async_smem();
+                    mbar_arrive(&bars->conv[st]);
                 }
-                fence_async_smem();
-                mbar_arrive(&bars->conv[st]);
             }
         }
     } else {
@@ -452,19 +473,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 // pdl: launched with programmatic serialization (see launch_kernel).
 // td: the destination's tensor map (box 32 x 32 fp32, 128-byte swizzle) for
 // the reduce drain; unused by the other forms.
+// tal, tbl: the lo parts' tensor maps (same boxes as ta, tb) for kSplitPre;
+// unused by the other splits.
 template <class Sched, bool A_MN, bool B_MN, int Epi, int Split = kSplitRound>
 inline cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const Sched& sched,
                           int tiles, int32_t* status, cudaStream_t stream, int sms,
-                          bool pdl = false, const CUtensorMap* td = nullptr) {
+                          bool pdl = false, const CUtensorMap* td = nullptr,
+                          const CUtensorMap* tal = nullptr, const CUtensorMap* tbl = nullptr) {
     auto kern = gemm_tf32x3_kernel<Sched, A_MN, B_MN, Epi, Split>;
     if (Epi >= kEpiReduce && td == nullptr) return cudaErrorInvalidValue;
+    if (Split == kSplitPre && (tal == nullptr || tbl == nullptr)) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          smem_bytes<Epi>());
     if (e != cudaSuccess) return e;
     if (tiles <= 0) return cudaSuccess;
     const int grid = tiles < sms ? tiles : sms;
     return launch_kernel(pdl, kern, dim3(grid), dim3(kThreads), smem_bytes<Epi>(), stream, ta, tb,
-                         td != nullptr ? *td : tb, sched, tiles, status, take_wait_probe(kProbeGemm));
+                         td != nullptr ? *td : tb, tal != nullptr ? *tal : ta,
+                         tbl != nullptr ? *tbl : tb, sched, tiles, status,
+                         take_wait_probe(kProbeGemm));
 }
 
 }  // namespace g3

@@ -74,6 +74,24 @@ __global__ void permute_rows_kernel(float* __restrict__ W, int64_t r, int64_t d,
     }
 }
 
+// U's lo parts for the lazy update's pre-split operand: U_lo = U - trunc13(U)
+// elementwise, from the diagonal's 4-column group to the end of each row (U is
+// d x d, contiguous; the update reads only rows of U right of their diagonal
+// block, so the rest of U_lo is left unwritten).  Rows along grid y, four
+// columns per thread (d is a multiple of 4).
+__global__ void u_lo_kernel(const float* __restrict__ U, int64_t d, float* __restrict__ U_lo) {
+    for (int64_t i = blockIdx.y; i < d; i += gridDim.y) {
+        const float4* src = reinterpret_cast<const float4*>(U + i * d);
+        float4* dst = reinterpret_cast<float4*>(U_lo + i * d);
+        for (int64_t q = (i >> 2) + blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+             q < d / 4; q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+            const float4 u = src[q];
+            dst[q] = make_float4(g3::tf32_rest(u.x), g3::tf32_rest(u.y), g3::tf32_rest(u.z),
+                                 g3::tf32_rest(u.w));
+        }
+    }
+}
+
 // Register layout: the block's 128 columns form four 32-column chunks; in
 // every chunk lane l of a row's L-lane group owns the C = 32 / L columns
 // C l .. C l + C - 1, so the lanes of a row read one 128-byte row segment of
@@ -187,7 +205,11 @@ __global__ void __launch_bounds__(kWarps * 32, L >= 8 ? 4 : 2)
                        int64_t d, int64_t ldw, int64_t c0, int bw, int bits, int g, int pure,
                        uint8_t* __restrict__ codes, float* __restrict__ scales,
                        int32_t* __restrict__ zeros, float* __restrict__ err_out,
-                       int64_t err_ld, const uint8_t* __restrict__ dead_mask, int32_t* status) {
+                       float* __restrict__ err_lo_out, int64_t err_ld,
+                       const uint8_t* __restrict__ dead_mask, int32_t* status) {
+    // err_lo_out (may be null): each error's part below tf32 precision, the
+    // lo operand of the lazy update's truncating 3xTF32 split, stored beside
+    // the errors so that the update need not split them
     constexpr int C = WalkShape<L>::kCols;
     constexpr int C4 = C / 4;  // float4s per lane per chunk
     extern __shared__ uint8_t smem_raw[];
@@ -376,6 +398,13 @@ __global__ void __launch_bounds__(kWarps * 32, L >= 8 ? 4 : 2)
             for (int q = 0; q < C4; ++q)
                 *reinterpret_cast<float4*>(err_out + row * err_ld + cb + 4 * q) =
                     make_float4(ev[4 * q], ev[4 * q + 1], ev[4 * q + 2], ev[4 * q + 3]);
+            if (err_lo_out != nullptr) {
+#pragma unroll
+                for (int q = 0; q < C4; ++q)
+                    *reinterpret_cast<float4*>(err_lo_out + row * err_ld + cb + 4 * q) =
+                        make_float4(g3::tf32_rest(ev[4 * q]), g3::tf32_rest(ev[4 * q + 1]),
+                                    g3::tf32_rest(ev[4 * q + 2]), g3::tf32_rest(ev[4 * q + 3]));
+            }
             if (vec) {
 #pragma unroll
                 for (int q = 0; q < C4; ++q)
@@ -495,10 +524,31 @@ bool schedule_valid(int nb, int defer, int g_blocks) {
 
 }  // namespace
 
+namespace {
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Workspace layout of the column walk: the deferred errors (d_row x 128 per
+// block of the run), then -- for the pre-split lazy update -- the errors' lo
+// parts in the same layout and U's lo parts (d_col x d_col).
+struct QuantWs {
+    size_t err, err_lo, u_lo, total;
+};
+QuantWs quant_ws(int64_t d_row, int64_t d_col, int defer) {
+    QuantWs w;
+    const size_t e = round256(static_cast<size_t>(d_row) * kBlock * defer * sizeof(float));
+    w.err = 0;
+    w.err_lo = e;
+    w.u_lo = 2 * e;
+    w.total = 2 * e + round256(static_cast<size_t>(d_col) * d_col * sizeof(float));
+    return w;
+}
+}  // namespace
+
 size_t quant_workspace_bytes(int64_t d_row, int64_t d_col, int block) {
+    (void)block;
     const int64_t nb = num_blocks(d_col);
-    const int64_t defer = nb < kMaxDefer ? nb : kMaxDefer;
-    return ((static_cast<size_t>(d_row) * block * defer * sizeof(float) + 255) / 256) * 256;
+    const int defer = static_cast<int>(nb < kMaxDefer ? nb : kMaxDefer);
+    return quant_ws(d_row, d_col, defer).total;
 }
 
 size_t quant_min_workspace_bytes(int64_t d_row, int block) {
@@ -525,12 +575,22 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
     const int pure = pure_minmax != 0 ? 1 : 0;
     const int g = (group == -1 || group > d_col) ? static_cast<int>(d_col) : group;
     const int nb = static_cast<int>(num_blocks(d_col));
-    int defer = nb < kMaxDefer ? nb : kMaxDefer;
-    while (defer > 1 && static_cast<size_t>(d_row) * kBlock * defer * sizeof(float) > ws_bytes)
+    const int defer_max = nb < kMaxDefer ? nb : kMaxDefer;
+    // the lazy update reads pre-split operands when the workspace holds the
+    // full layout (and W's rows can be a tensor map: the fallback drain keeps
+    // the in-kernel split); the lo parts are the values the in-kernel split
+    // would compute, so the results are the same bit for bit either way
+    const QuantWs full = quant_ws(d_row, d_col, defer_max);
+    const bool w_aligned = (reinterpret_cast<uintptr_t>(W) & 15) == 0 && (ldw % 4) == 0;
+    const bool pre = ws_bytes >= full.total && w_aligned;
+    int defer = defer_max;
+    while (!pre && defer > 1 && static_cast<size_t>(d_row) * kBlock * defer * sizeof(float) > ws_bytes)
         defer /= 2;
     const int g_blocks = g > kBlock ? (g + kBlock - 1) / kBlock : 1;
     while (defer > 1 && !schedule_valid(nb, defer, g_blocks)) defer /= 2;
     float* err = static_cast<float*>(ws);
+    float* err_lo = pre ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + full.err_lo) : nullptr;
+    float* u_lo = pre ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + full.u_lo) : nullptr;
     const int64_t err_ld = static_cast<int64_t>(defer) * kBlock;
 
     // With act-order the columns are permuted (and dead ones zeroed) in one
@@ -548,16 +608,19 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
     }
     const uint8_t* dead_mask = permuted ? nullptr : dead;
 
-    CUtensorMap tU, tUmn, tErr, tW;
+    CUtensorMap tU, tUmn, tErr, tW, tUlo, tErrLo;
     if (!make_tmap_2d(&tU, false, U, d_col, d_col, d_col, kBlock, kBlock, Swz::kNone) ||
         !make_tmap_2d(&tUmn, false, U, d_col, d_col, d_col, 32, 32, Swz::k128Atom32) ||
         !make_tmap_2d(&tErr, false, err, err_ld, d_row, err_ld, 32, 128, Swz::k128))
         return GPTQ_ERR_INVALID_ARG;
+    if (pre && (!make_tmap_2d(&tUlo, false, u_lo, d_col, d_col, d_col, 32, 32, Swz::k128Atom32) ||
+                !make_tmap_2d(&tErrLo, false, err_lo, err_ld, d_row, err_ld, 32, 128, Swz::k128)))
+        return GPTQ_ERR_INVALID_ARG;
     // the lazy update adds -Err U into W through TMA reductions when W's rows
     // can be a tensor map (16-byte aligned base and row pitch); else it
     // drains through shared memory and plain loads and stores
-    const bool w_tma = (reinterpret_cast<uintptr_t>(W) & 15) == 0 && (ldw % 4) == 0 &&
-                       make_tmap_2d(&tW, false, W, d_col, d_row, ldw, 32, 32, Swz::k128);
+    const bool w_tma = w_aligned && make_tmap_2d(&tW, false, W, d_col, d_row, ldw, 32, 32, Swz::k128);
+    if (pre && !w_tma) return GPTQ_ERR_INVALID_ARG;
     const size_t q_smem = (kBlock * kBlock + kBlock) * sizeof(float) + 1024;
     const bool small_group = g < 32;
     constexpr int Lw = kWalkLanes;
@@ -573,6 +636,12 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
     const int mt = static_cast<int>((d_row + 127) / 128);
     const int sms = num_sms();
     int64_t launches = permuted ? 1 : 0;
+    if (pre) {
+        const unsigned gx = static_cast<unsigned>((d_col / 4 + 255) / 256 < 8 ? (d_col / 4 + 255) / 256 : 8);
+        const unsigned gy = static_cast<unsigned>(d_col < 65535 ? d_col : 65535);
+        u_lo_kernel<<<dim3(gx, gy), 256, 0, stream>>>(U, d_col, u_lo);
+        ++launches;
+    }
     int run0 = 0;  // first block of the current run (its errors sit at column 0 of err)
 
     auto quantize_block = [&](int b) -> bool {
@@ -582,10 +651,11 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
         // programmatic (early) launch after a kernel of this call only: the
         // kernel fetches U before waiting, and the work before this call may
         // still be writing U
-        return launch_kernel(b > 0 || permuted, bw == kBlock ? qfull : qpart, dim3(qgrid),
+        const int64_t eoff = static_cast<int64_t>(b - run0) * kBlock;
+        return launch_kernel(b > 0 || permuted || pre, bw == kBlock ? qfull : qpart, dim3(qgrid),
                              dim3(kWarps * 32), q_smem, stream, tU, W, d_row, d_col, ldw, c0, bw,
-                             bits, g, pure, codes, scales, zeros,
-                             err + static_cast<int64_t>(b - run0) * kBlock, err_ld, dead_mask,
+                             bits, g, pure, codes, scales, zeros, err + eoff,
+                             pre ? err_lo + eoff : nullptr, err_ld, dead_mask,
                              status) == cudaSuccess;
     };
     // W[:, blocks [c, e)) -= Err[:, blocks [a, c)) U[blocks [a, c), blocks [c, e))
@@ -600,6 +670,11 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
         // truncating split: the walk given the same U matches the float64
         // loop as closely with it as with the rounding split, which costs the
         // split warps a second store per operand
+        // (pre-split: the same truncating split, read from the workspace)
+        if (pre)
+            return g3::launch<LazySched, false, true, g3::kEpiReduce, g3::kSplitPre>(
+                       tErr, tUmn, ls, mt * nt, status, stream, sms, true, &tW, &tErrLo, &tUlo) ==
+                   cudaSuccess;
         return (w_tma ? g3::launch<LazySched, false, true, g3::kEpiReduce, g3::kSplitTrunc>(
                             tErr, tUmn, ls, mt * nt, status, stream, sms, true, &tW)
                       : g3::launch<LazySched, false, true, g3::kEpiStaged, g3::kSplitTrunc>(

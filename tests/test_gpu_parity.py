@@ -402,6 +402,41 @@ def test_stages_replay_from_a_cuda_graph_bit_exactly():
             assert torch.equal(b[k], v), k
 
 
+@pytest.mark.parametrize("d_row,d_col,bits,g,desc_act", [(300, 1536, 4, 128, True),
+                                                     (130, 2048, 3, 32, False)])
+def test_lazy_update_presplit_is_bit_identical(d_row, d_col, bits, g, desc_act):
+    """The full workspace makes the lazy update read its operands' low parts,
+    split once by the column walk (errors) and one pass over U; a workspace
+    that only holds the eight deferred blocks' errors makes it split in the
+    GEMM.  Same schedule, same split values: codes, scales, zeros and the
+    pre-quantization weights agree bit for bit."""
+    g_ = gpu()
+    W, X = workloads.small_layer(d_row, d_col, 4 * d_col, seed=d_row + d_col, kind="student_t")
+    H = torch.from_numpy(oracle.hessian(X).astype(np.float32)).cuda()
+    cfg = g_.GPTQConfig(bits=bits, group_size=g, desc_act=desc_act)
+    full = g_.gptq_workspace_size(cfg, d_row, d_col)
+    errs_only = (d_row * 128 * min(8, -(-d_col // 128)) * 4 + 255) // 256 * 256
+    assert errs_only < full
+    ws = torch.empty(full, dtype=torch.uint8, device="cuda")
+    U = torch.empty(d_col, d_col, device="cuda")
+    perm = torch.empty(d_col, dtype=torch.int32, device="cuda")
+    dead = torch.empty(d_col, dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g_.gptq_prepare_hinv(H, cfg, U, perm, dead, st, ws)
+    outs = []
+    for nbytes in (full, errs_only):
+        Wd = W.cuda().contiguous()
+        ng = g_.n_groups(d_col, g)
+        o = (torch.empty(d_row, d_col, dtype=torch.uint8, device="cuda"),
+             torch.empty(ng, d_row, dtype=torch.float32, device="cuda"),
+             torch.empty(ng, d_row, dtype=torch.int32, device="cuda"))
+        g_.gptq_quantize_layer(Wd, U, perm, dead, cfg, *o, st, ws[:nbytes])
+        assert g_.gptq_sync_status(st) == 0
+        outs.append((*o, Wd))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
 @pytest.mark.parametrize("pad,offset", [(3, 0), (3, 1), (1, 3)])
 def test_quantize_layer_on_strided_and_offset_weights(pad, offset):
     """W as a view into a wider buffer: a row pitch that is not a multiple of
