@@ -252,7 +252,9 @@ gptq_status gptq_quantize_layer(float *W, int64_t d_row, int64_t d_col, int64_t 
  *   the errors of up to 8 blocks of 128 columns in the array (d_row * 512
  *   bytes each); above d_row = 4096 it defers fewer (4 up to 8192, 2 up to
  *   16384, 1 up to 32768), exactly as gptq_quantize_layer does with a 16 MiB
- *   workspace: the same sums grouped into more, shorter products.
+ *   workspace: the same sums grouped into more, shorter products (and, for
+ *   layers whose full workspace fits the array, with the lazy update's
+ *   operands split ahead, as gptq_quantize_layer does then).
  *   Device: the array used is the current device's, so W, U, perm (with
  *   act-order), dead, codes, scales, zeros and dev_status must be memory of
  *   the current device (or managed memory); otherwise GPTQ_ERR_INVALID_ARG
