@@ -581,8 +581,13 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
     // the in-kernel split); the lo parts are the values the in-kernel split
     // would compute, so the results are the same bit for bit either way
     const QuantWs full = quant_ws(d_row, d_col, defer_max);
-    const bool w_aligned = (reinterpret_cast<uintptr_t>(W) & 15) == 0 && (ldw % 4) == 0;
-    const bool pre = ws_bytes >= full.total && w_aligned;
+    // the lazy update adds -Err U into W through TMA reductions when W's rows
+    // can be a tensor map (16-byte aligned base and row pitch); else it
+    // drains through shared memory and plain loads and stores
+    CUtensorMap tW;
+    const bool w_tma = (reinterpret_cast<uintptr_t>(W) & 15) == 0 && (ldw % 4) == 0 &&
+                       make_tmap_2d(&tW, false, W, d_col, d_row, ldw, 32, 32, Swz::k128);
+    const bool pre = ws_bytes >= full.total && w_tma;
     int defer = defer_max;
     while (!pre && defer > 1 && static_cast<size_t>(d_row) * kBlock * defer * sizeof(float) > ws_bytes)
         defer /= 2;
@@ -608,7 +613,7 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
     }
     const uint8_t* dead_mask = permuted ? nullptr : dead;
 
-    CUtensorMap tU, tUmn, tErr, tW, tUlo, tErrLo;
+    CUtensorMap tU, tUmn, tErr, tUlo, tErrLo;
     if (!make_tmap_2d(&tU, false, U, d_col, d_col, d_col, kBlock, kBlock, Swz::kNone) ||
         !make_tmap_2d(&tUmn, false, U, d_col, d_col, d_col, 32, 32, Swz::k128Atom32) ||
         !make_tmap_2d(&tErr, false, err, err_ld, d_row, err_ld, 32, 128, Swz::k128))
@@ -616,11 +621,6 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
     if (pre && (!make_tmap_2d(&tUlo, false, u_lo, d_col, d_col, d_col, 32, 32, Swz::k128Atom32) ||
                 !make_tmap_2d(&tErrLo, false, err_lo, err_ld, d_row, err_ld, 32, 128, Swz::k128)))
         return GPTQ_ERR_INVALID_ARG;
-    // the lazy update adds -Err U into W through TMA reductions when W's rows
-    // can be a tensor map (16-byte aligned base and row pitch); else it
-    // drains through shared memory and plain loads and stores
-    const bool w_tma = w_aligned && make_tmap_2d(&tW, false, W, d_col, d_row, ldw, 32, 32, Swz::k128);
-    if (pre && !w_tma) return GPTQ_ERR_INVALID_ARG;
     const size_t q_smem = (kBlock * kBlock + kBlock) * sizeof(float) + 1024;
     const bool small_group = g < 32;
     constexpr int Lw = kWalkLanes;
