@@ -66,6 +66,13 @@ def test_workspace_size_and_config_validation(pkg):
     cfg = pkg.GPTQConfig(bits=4, group_size=128)
     b = pkg.gptq_workspace_size(cfg, 4096, 4096)
     assert b >= 4096 * 128 * 4 and b % 256 == 0
+    # the full layout of the column walk: eight deferred blocks of errors,
+    # their lo parts, and U's lo parts (d_col^2 floats) for the pre-split update
+    assert b == 2 * 4096 * 128 * 8 * 4 + 4096 * 4096 * 4
+    errs = (300 * 128 * 8 * 4 + 255) // 256 * 256
+    assert pkg.gptq_workspace_size(cfg, 300, 1536) == 2 * errs + 1536 * 1536 * 4
+    # fewer blocks than eight: as many as the layer has
+    assert pkg.gptq_workspace_size(cfg, 64, 256) == 2 * 64 * 128 * 2 * 4 + 256 * 256 * 4
     for bad in (dict(bits=5), dict(group_size=0), dict(group_size=-2), dict(damp=-1.0)):
         kw = dict(bits=4, group_size=128, damp=0.01)
         kw.update(bad)
