@@ -502,6 +502,23 @@ def test_dequant_matmul_hand_example():
     assert Y_id[0, 1] == 1 * 16 + 2 * -14 + 3 * 16 + 4 * -14
 
 
+def test_bf16_rounding_agrees_with_an_independent_conversion():
+    """The oracle's bf16 rounding against torch's float32 -> bfloat16 cast on
+    the CPU (round to nearest, ties to even; an implementation the oracle does
+    not share): random magnitudes over 60 binades of both signs, exact ties
+    (the dropped half exactly 0x8000, even and odd kept parts) and values one
+    ulp either side of them."""
+    import torch
+    rng = np.random.default_rng(42)
+    x = (rng.standard_normal(100000) * 2.0 ** rng.integers(-30, 30, 100000)).astype(np.float32)
+    u = rng.integers(0x00800000, 0x7F000000, 20000, dtype=np.uint64).astype(np.uint32)
+    ties = (u & 0xFFFF0000) | 0x8000
+    near = np.concatenate([ties, ties + 1, ties - 1]).astype(np.uint32).view(np.float32)
+    x = np.concatenate([x, near, -near])
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(oracle.bf16_round(x), ref)
+
+
 def test_bf16_dequantized_weights_hand_example():
     """The many-token product's 16-bit weights ("GPTQ (GPT Quantization)",
     "Limitations": weights dequantized to 16 bits before the product):
