@@ -32,8 +32,13 @@ namespace gptq {
 namespace {
 
 constexpr int kBlock = 128;       // columns per block (the only supported block size)
-constexpr int kWarps = 4;
-static_assert(kWarps * 32 == kBlock, "block_quant_kernel: one thread per column of the U block");
+// Warps per column-walk CTA (kWarpsSmall rows * 4 each at 8 lanes per row).
+// Four (16 rows) while the layer's CTAs fit on the GPU at once (three per SM
+// by shared memory: up to 7104 rows); seven (28 rows) beyond, so that larger
+// layers still walk a block in one wave (measured at 8192 x 8192:
+// quantize_layer 5.25 -> 4.51 ms; at 4096 rows seven warps are 4 % slower
+// than four).
+constexpr int kWarpsSmall = 4, kWarpsLarge = 7;
 // Lanes per row of the column walk (each owns 32 / kWalkLanes columns of every
 // 32-column chunk).  8 lanes: 4096 rows give ~7 warps per SM.  4 lanes halve
 // the per-column work replicated on every lane of a row (quantizing the
@@ -42,11 +47,12 @@ static_assert(kWarps * 32 == kBlock, "block_quant_kernel: one thread per column 
 // against 1.207 ms at 4096 x 4096, 5.31 against 5.08 ms at 4096 x 11008,
 // interleaved A/B, identical codes).
 constexpr int kWalkLanes = 8;
-template <int L>
+template <int L, int NW>
 struct WalkShape {
+    static_assert(NW * 32 >= kBlock, "block_quant_kernel: a thread per column of the U block");
     static constexpr int kCols = 32 / L;            // columns per lane per chunk
     static constexpr int kRowsPerWarp = 32 / L;
-    static constexpr int kRowsPerCta = kRowsPerWarp * kWarps;
+    static constexpr int kRowsPerCta = kRowsPerWarp * NW;
 };
 
 // ------------------------------------------------------------------------
@@ -198,9 +204,10 @@ __device__ __forceinline__ float round_even(float x) {
 }
 
 template <int L,               // lanes per row
+          int NW,              // warps per CTA
           bool kSmallGroup,  // group_size < 32: groups start inside a chunk
           bool kFull>        // a full 128-column block (no column guard)
-__global__ void __launch_bounds__(kWarps * 32, L >= 8 ? 4 : 2)
+__global__ void __launch_bounds__(NW * 32, 1)
     block_quant_kernel(const __grid_constant__ CUtensorMap tmu, float* __restrict__ W, int64_t r,
                        int64_t d, int64_t ldw, int64_t c0, int bw, int bits, int g, int pure,
                        uint8_t* __restrict__ codes, float* __restrict__ scales,
@@ -210,7 +217,7 @@ __global__ void __launch_bounds__(kWarps * 32, L >= 8 ? 4 : 2)
     // err_lo_out (may be null): each error's part below tf32 precision, the
     // lo operand of the lazy update's truncating 3xTF32 split, stored beside
     // the errors so that the update need not split them
-    constexpr int C = WalkShape<L>::kCols;
+    constexpr int C = WalkShape<L, NW>::kCols;
     constexpr int C4 = C / 4;  // float4s per lane per chunk
     extern __shared__ uint8_t smem_raw[];
     float* smem = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -237,9 +244,9 @@ __global__ void __launch_bounds__(kWarps * 32, L >= 8 ? 4 : 2)
     if (!ok) return;
     // 1 / U_jj (thread j), then the block is cleared at and below its
     // diagonal, float4 by float4 spread over all threads
-    const float ujj = Us[tid * kBlock + tid];
+    const float ujj = tid < kBlock ? Us[tid * kBlock + tid] : 1.f;
     __syncthreads();
-    for (int q = tid; q < kBlock * kBlock / 4; q += kWarps * 32) {
+    for (int q = tid; q < kBlock * kBlock / 4; q += NW * 32) {
         const int i = q >> 5, c = (q & 31) * 4;
         if (c > i) continue;
         float* u4 = Us + i * kBlock + c;
@@ -249,14 +256,14 @@ __global__ void __launch_bounds__(kWarps * 32, L >= 8 ? 4 : 2)
             for (int t = 0; c + t <= i; ++t) u4[t] = 0.f;
         }
     }
-    dinv[tid] = (tid < bw) ? 1.f / ujj : 0.f;
+    if (tid < kBlock) dinv[tid] = (tid < bw) ? 1.f / ujj : 0.f;
     pdl_wait();
 
     const int lane = tid & 31;
     const int l = lane % L;
     const int gbase = lane - l;
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * WalkShape<L>::kRowsPerCta +
-                        (tid >> 5) * WalkShape<L>::kRowsPerWarp + lane / L;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * WalkShape<L, NW>::kRowsPerCta +
+                        (tid >> 5) * WalkShape<L, NW>::kRowsPerWarp + lane / L;
     const bool live = row < r;
     float* wrow = W + (live ? row : 0) * ldw;
     // float4 access to W needs 16-byte aligned rows (base and pitch); a
@@ -624,15 +631,32 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
     const size_t q_smem = (kBlock * kBlock + kBlock) * sizeof(float) + 1024;
     const bool small_group = g < 32;
     constexpr int Lw = kWalkLanes;
-    auto qfull = small_group ? block_quant_kernel<Lw, true, true> : block_quant_kernel<Lw, false, true>;
-    auto qpart = small_group ? block_quant_kernel<Lw, true, false> : block_quant_kernel<Lw, false, false>;
-    if (cudaFuncSetAttribute(qfull, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(q_smem)) != cudaSuccess ||
-        cudaFuncSetAttribute(qpart, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(q_smem)) != cudaSuccess)
+    auto set_smem = [&](auto kern) {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(q_smem)) == cudaSuccess;
+    };
+    const auto q4f = small_group ? block_quant_kernel<Lw, kWarpsSmall, true, true>
+                                 : block_quant_kernel<Lw, kWarpsSmall, false, true>;
+    const auto q4p = small_group ? block_quant_kernel<Lw, kWarpsSmall, true, false>
+                                 : block_quant_kernel<Lw, kWarpsSmall, false, false>;
+    const auto q7f = small_group ? block_quant_kernel<Lw, kWarpsLarge, true, true>
+                                 : block_quant_kernel<Lw, kWarpsLarge, false, true>;
+    const auto q7p = small_group ? block_quant_kernel<Lw, kWarpsLarge, true, false>
+                                 : block_quant_kernel<Lw, kWarpsLarge, false, false>;
+    if (!set_smem(q4f) || !set_smem(q4p) || !set_smem(q7f) || !set_smem(q7p)) return GPTQ_ERR_CUDA;
+    // four warps per CTA when all the layer's CTAs are resident at once
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, q4f, kWarpsSmall * 32, q_smem) !=
+        cudaSuccess)
         return GPTQ_ERR_CUDA;
-    constexpr int kRowsPerCta = WalkShape<kWalkLanes>::kRowsPerCta;
-    const unsigned qgrid = static_cast<unsigned>((d_row + kRowsPerCta - 1) / kRowsPerCta);
+    constexpr int kRows4 = WalkShape<Lw, kWarpsSmall>::kRowsPerCta;
+    constexpr int kRows7 = WalkShape<Lw, kWarpsLarge>::kRowsPerCta;
+    const bool four = (d_row + kRows4 - 1) / kRows4 <= static_cast<int64_t>(per_sm) * num_sms();
+    const auto qfull = four ? q4f : q7f;
+    const auto qpart = four ? q4p : q7p;
+    const int qthreads = (four ? kWarpsSmall : kWarpsLarge) * 32;
+    const int qrows = four ? kRows4 : kRows7;
+    const unsigned qgrid = static_cast<unsigned>((d_row + qrows - 1) / qrows);
     const int mt = static_cast<int>((d_row + 127) / 128);
     const int sms = num_sms();
     int64_t launches = permuted ? 1 : 0;
@@ -653,7 +677,7 @@ gptq_status launch_quantize(float* W, int64_t d_row, int64_t d_col, int64_t ldw,
         // still be writing U
         const int64_t eoff = static_cast<int64_t>(b - run0) * kBlock;
         return launch_kernel(b > 0 || permuted || pre, bw == kBlock ? qfull : qpart, dim3(qgrid),
-                             dim3(kWarps * 32), q_smem, stream, tU, W, d_row, d_col, ldw, c0, bw,
+                             dim3(qthreads), q_smem, stream, tU, W, d_row, d_col, ldw, c0, bw,
                              bits, g, pure, codes, scales, zeros, err + eoff,
                              pre ? err_lo + eoff : nullptr, err_ld, dead_mask,
                              status) == cudaSuccess;
