@@ -173,6 +173,9 @@ class ClockSampler:
             self.proc = subprocess.Popen([sys.executable, "-c", _SAMPLER_SRC, uuid, str(period_s)],
                                          stdin=subprocess.PIPE, stdout=subprocess.PIPE,
                                          stderr=subprocess.PIPE, text=True)
+            import select
+            if not select.select([self.proc.stdout], [], [], 30.0)[0]:
+                raise RuntimeError("clock sampler did not report within 30 s")
             first = self.proc.stdout.readline().split()
             if len(first) != 2 or first[0] != "ready":
                 raise RuntimeError("clock sampler did not start: "
