@@ -37,8 +37,10 @@ METRIC = "GPTQ layer quantize: weights/s and ms/layer (4-bit g128); Hessian TFLO
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # dram__bytes_read.sum + dram__bytes_write.sum of one Hessian launch at 65,536
-# tokens x 4,096 (ncu, current kernel: 32,768-token drains, eight drain warps)
-TRAFFIC_65K = 648.1e6
+# tokens x 4,096 (ncu, current kernel: 256 x 256 blocks as two MMA halves
+# sharing B, 32,768-token drains, eight drain warps): 608.4 MB read + 40.1 MB
+# written
+TRAFFIC_65K = 648.5e6
 
 
 def parse():
