@@ -182,7 +182,8 @@ size_t gptq_hessian_staging_size(int64_t d, int64_t chunk_tokens);
  * H_inv = cholesky_inverse(H)).
  *   H     d x d fp32 (lower triangle read), leading dimension ldh.  Consumed:
  *         overwritten with scratch.  d and ldh must be multiples of 4 and H
- *         and U 16-byte aligned (tiles move by the tensor-memory accelerator);
+ *         and U 16-byte aligned (tiles move by the tensor-memory accelerator),
+ *         and d at most 57344 (the column walk's limit: U has no other use);
  *         otherwise GPTQ_ERR_UNSUPPORTED.
  *   U     d x d fp32, contiguous (leading dimension d).  Output: the upper
  *         triangular U with U^T U = (P^T H P + lambda I)^-1 in quantization

@@ -152,6 +152,7 @@ gptq_status gptq_prepare_hinv(float* H, int64_t d, int64_t ldh, const gptq_confi
     if (H == U) return GPTQ_ERR_INVALID_ARG;
     if ((d % 4) != 0 || (ldh % 4) != 0 || !aligned(H, 16) || !aligned(U, 16))
         return GPTQ_ERR_UNSUPPORTED;  // tensor-memory-accelerator tiles need 16-byte rows
+    if (d > kMaxQuantCols) return GPTQ_ERR_UNSUPPORTED;  // U only feeds the column walk
     const gptq_status c = check_config(cfg, d);
     if (c != GPTQ_OK) return c;
     if (ws == nullptr || !aligned(ws, 256) || ws_bytes < gptq::prep_workspace_bytes(d) ||

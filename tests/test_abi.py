@@ -175,3 +175,125 @@ def test_wait_probe_arguments_are_checked_on_the_host(pkg):
         with pytest.raises(pkg.GPTQError) as e:
             pkg.gptq_debug_arm_wait_probe(kernel, ns)
         assert e.value.status == 1
+
+
+def _entry(lib, name, argtypes, restype=ctypes.c_int):
+    f = getattr(lib, name)
+    f.restype = restype
+    f.argtypes = argtypes
+    return f
+
+
+def _caller(f, order, ok):
+    def call(**kw):
+        v = dict(ok)
+        v.update(kw)
+        return f(*(v[k] for k in order))
+    return call
+
+
+def test_prepare_hinv_validation(pkg):
+    """Sizes, pointers, alignment, the column walk's width limit, the config
+    and the workspace are checked before anything is launched."""
+    lib = ctypes.CDLL(pkg.library_path())
+    P, i64 = ctypes.c_void_p, ctypes.c_int64
+    f = _entry(lib, "gptq_prepare_hinv",
+               [P, i64, i64, ctypes.POINTER(pkg.GPTQConfig), P, P, P, P, P, ctypes.c_size_t, P])
+    cfg = pkg.GPTQConfig(bits=4, group_size=128)
+    a, b = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 24)
+    order = ("H", "d", "ldh", "cfg", "U", "perm", "dead", "st", "ws", "wsb", "stream")
+    ok = dict(H=a, d=256, ldh=256, cfg=ctypes.byref(cfg), U=b, perm=a, dead=a, st=None, ws=a,
+              wsb=pkg.gptq_workspace_size(cfg, 1, 256), stream=None)
+    call = _caller(f, order, ok)
+    assert call(d=0) == 1 and call(d=-4) == 1 and call(ldh=252) == 1
+    assert call(H=None) == 1 and call(U=None) == 1 and call(perm=None) == 1
+    assert call(dead=None) == 1
+    assert call(U=a) == 1                                       # H is consumed: U apart from it
+    assert call(d=254) == 2 and call(ldh=258) == 2              # rows of whole 16-byte units
+    assert call(H=ctypes.c_void_p((1 << 20) + 4)) == 2          # tiles need 16-byte aligned bases
+    assert call(U=ctypes.c_void_p((1 << 24) + 8)) == 2
+    assert call(d=57348, ldh=57348) == 2                        # wider than the column walk takes
+    assert call(cfg=None) == 1
+    assert call(cfg=ctypes.byref(pkg.GPTQConfig(bits=5))) == 1
+    assert call(cfg=ctypes.byref(pkg.GPTQConfig(damp=float("nan")))) == 1
+    assert call(cfg=ctypes.byref(pkg.GPTQConfig(group_size=48))) == 2
+    assert call(ws=None) == 6 and call(wsb=16) == 6
+    assert call(ws=ctypes.c_void_p((1 << 20) + 128)) == 6       # workspace 256-byte aligned
+
+
+def test_quantize_layer_validation(pkg):
+    lib = ctypes.CDLL(pkg.library_path())
+    P, i64 = ctypes.c_void_p, ctypes.c_int64
+    f = _entry(lib, "gptq_quantize_layer",
+               [P, i64, i64, i64, P, P, P, ctypes.POINTER(pkg.GPTQConfig), P, P, P, P, P,
+                ctypes.c_size_t, P])
+    cfg = pkg.GPTQConfig(bits=4, group_size=128)
+    a, b = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 24)
+    order = ("W", "r", "d", "ldw", "U", "perm", "dead", "cfg", "codes", "scales", "zeros", "st",
+             "ws", "wsb", "stream")
+    ok = dict(W=a, r=64, d=256, ldw=256, U=b, perm=a, dead=a, cfg=ctypes.byref(cfg), codes=a,
+              scales=a, zeros=a, st=None, ws=a, wsb=pkg.gptq_workspace_size(cfg, 64, 256),
+              stream=None)
+    call = _caller(f, order, ok)
+    assert call(r=0) == 1 and call(d=0) == 1 and call(ldw=255) == 1
+    for name in ("W", "U", "perm", "dead", "codes", "scales", "zeros"):
+        assert call(**{name: None}) == 1, name
+    assert call(d=57348, ldw=57348) == 2                        # a row of W must fit on chip
+    assert call(d=250, ldw=256) == 2                            # d_col a multiple of 4
+    assert call(U=ctypes.c_void_p((1 << 24) + 4)) == 2          # U's blocks move by TMA
+    assert call(cfg=None) == 1
+    assert call(cfg=ctypes.byref(pkg.GPTQConfig(bits=1))) == 1
+    assert call(cfg=ctypes.byref(pkg.GPTQConfig(block_size=64))) == 2
+    # the workspace must hold at least one block of errors: d_row * 128 floats
+    assert call(ws=None) == 6 and call(wsb=64 * 512 - 1) == 6
+    assert call(ws=ctypes.c_void_p((1 << 20) + 64)) == 6
+
+
+def test_quantize_layer_noalloc_validation(pkg):
+    """The checks that precede any CUDA call: config, sizes, and a layer whose
+    errors would not fit the fixed 16 MiB scratch."""
+    lib = ctypes.CDLL(pkg.library_path())
+    P, i64 = ctypes.c_void_p, ctypes.c_int64
+    f = _entry(lib, "gptq_quantize_layer_noalloc",
+               [P, i64, i64, i64, P, P, P, ctypes.POINTER(pkg.GPTQConfig), P, P, P, P, P])
+    assert _entry(lib, "gptq_noalloc_scratch_bytes", [], ctypes.c_size_t)() == 16 << 20
+    cfg = pkg.GPTQConfig(bits=4, group_size=128)
+    a = ctypes.c_void_p(1 << 20)
+    order = ("W", "r", "d", "ldw", "U", "perm", "dead", "cfg", "codes", "scales", "zeros", "st",
+             "stream")
+    ok = dict(W=a, r=64, d=256, ldw=256, U=a, perm=a, dead=a, cfg=ctypes.byref(cfg), codes=a,
+              scales=a, zeros=a, st=None, stream=None)
+    call = _caller(f, order, ok)
+    assert call(cfg=None) == 1 and call(r=0) == 1 and call(d=0) == 1
+    assert call(cfg=ctypes.byref(pkg.GPTQConfig(bits=7))) == 1
+    assert call(cfg=ctypes.byref(pkg.GPTQConfig(group_size=96))) == 2
+    assert call(r=32769, d=128, ldw=128) == 6                   # 32769 * 512 bytes > 16 MiB
+
+
+def test_dequant_gemm_validation(pkg):
+    lib = ctypes.CDLL(pkg.library_path())
+    P, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    f = _entry(lib, "gptq_dequant_gemm",
+               [P, i64, i64, i64, P, P, P, P, i64, i32, i32, P, i64, P, P, ctypes.c_size_t, P])
+    ws_size = _entry(lib, "gptq_dequant_gemm_workspace_size", [i64, i64], ctypes.c_size_t)
+    assert ws_size(3, 256) == (3 * 256 * 2 + 255) // 256 * 256  # the tokens as bf16
+    assert ws_size(0, 256) == 0 and ws_size(4, 0) == 0
+    a = ctypes.c_void_p(1 << 20)
+    order = ("X", "n", "k", "ldx", "pk", "sc", "ze", "perm", "n_out", "bits", "g", "Y", "ldy", "st",
+             "ws", "wsb", "stream")
+    ok = dict(X=a, n=16, k=256, ldx=256, pk=a, sc=a, ze=a, perm=a, n_out=256, bits=4, g=128, Y=a,
+              ldy=256, st=None, ws=a, wsb=ws_size(16, 256), stream=None)
+    call = _caller(f, order, ok)
+    assert call(n=0) == 0                                       # no tokens: nothing to do
+    for name in ("X", "pk", "sc", "ze", "Y"):
+        assert call(**{name: None}) == 1, name
+    assert call(n=-1) == 1 and call(n=(1 << 24) + 1) == 1
+    assert call(k=0) == 1 and call(n_out=0) == 1 and call(ldx=128) == 1 and call(ldy=100) == 1
+    assert call(bits=6) == 1 and call(g=0) == 1 and call(g=-2) == 1
+    assert call(pk=ctypes.c_void_p((1 << 20) + 4)) == 1         # packed rows by 16-byte TMA boxes
+    assert call(bits=3) == 2                                    # 3-bit codes straddle words
+    assert call(k=224, ldx=256) == 2                            # whole 64-code stages
+    assert call(g=12) == 2                                      # an 8-code chunk across groups
+    # the act-order gather needs the workspace
+    assert call(ws=None) == 6 and call(wsb=16 * 256 * 2 - 1) == 6
+    assert call(ws=ctypes.c_void_p((1 << 20) + 32)) == 6
