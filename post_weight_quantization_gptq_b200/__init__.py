@@ -165,6 +165,25 @@ def _row_major(t: torch.Tensor, name: str) -> int:
     return t.stride(0) if t.shape[0] > 1 else max(t.shape[1], t.stride(0))
 
 
+def _same_device(ref: torch.Tensor, ref_name: str, *others) -> None:
+    """Every (tensor, name, dtype) of ``others`` that is given lives on ref's
+    device, and that device is the current one: the library launches on the
+    current device and its kernels dereference every pointer there, so a
+    buffer elsewhere (host memory, another GPU) is refused here instead of
+    being read by a kernel.  dtype None accepts any element type."""
+    for t, name, dtype in others:
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.device != ref.device:
+            where = t.device if isinstance(t, torch.Tensor) else type(t).__name__
+            raise ValueError(f"{name} must be on {ref.device} like {ref_name}, not on {where}")
+        if dtype is not None and t.dtype != dtype:
+            raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ref.device.index != torch.cuda.current_device():
+        raise ValueError(f"{ref_name} is on {ref.device} but cuda:{torch.cuda.current_device()} "
+                         "is current: make its device current (torch.cuda.device(...))")
+
+
 def gptq_workspace_size(cfg: GPTQConfig, d_row: int, d_col: int) -> int:
     out = ctypes.c_size_t(0)
     _check(_lib.gptq_workspace_size(ctypes.byref(cfg), int(d_row), int(d_col), ctypes.byref(out)),
@@ -177,6 +196,8 @@ def gptq_hessian_accumulate(X: torch.Tensor, H: torch.Tensor, dev_status: torch.
     """H += 2 X^T X (X: n x d bf16, H: d x d fp32, both CUDA, row-major)."""
     _cuda(X, "X", torch.bfloat16)
     _cuda(H, "H", torch.float32)
+    _same_device(X, "X", (H, "H", torch.float32), (dev_status, "dev_status", torch.int32),
+                 (ws, "ws", None))
     n, d = X.shape
     ldx = _row_major(X, "X")
     ldh = _row_major(H, "H")
@@ -194,6 +215,7 @@ def gptq_hessian_accumulate_host(X: torch.Tensor, H: torch.Tensor, staging: torc
         raise TypeError("X must be a host bf16 tensor")
     _cuda(H, "H", torch.float32)
     _cuda(staging, "staging")
+    _same_device(H, "H", (staging, "staging", None), (dev_status, "dev_status", torch.int32))
     n, d = X.shape
     ldx = _row_major(X, "X")
     _check(_lib.gptq_hessian_accumulate_host(_ptr(X), n, d, ldx, _ptr(H), _row_major(H, "H"),
@@ -216,6 +238,11 @@ def gptq_prepare_hinv(H: torch.Tensor, cfg: GPTQConfig, U: torch.Tensor, perm: t
     _cuda(U, "U", torch.float32)
     _cuda(perm, "perm", torch.int32)
     _cuda(dead, "dead", torch.uint8)
+    if ws is None:
+        raise ValueError("gptq_prepare_hinv needs a workspace (gptq_workspace_size bytes)")
+    _same_device(H, "H", (U, "U", torch.float32), (perm, "perm", torch.int32),
+                 (dead, "dead", torch.uint8), (dev_status, "dev_status", torch.int32),
+                 (ws, "ws", None))
     d = H.shape[0]
     if not U.is_contiguous() or tuple(U.shape) != (d, d):
         raise ValueError("U must be a contiguous d x d tensor")
@@ -235,6 +262,11 @@ def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, perm: torch.Tensor, de
     _cuda(codes, "codes", torch.uint8)
     _cuda(scales, "scales", torch.float32)
     _cuda(zeros, "zeros", torch.int32)
+    if ws is None:
+        raise ValueError("gptq_quantize_layer needs a workspace (gptq_workspace_size bytes)")
+    _same_device(W, "W", (U, "U", torch.float32), (perm, "perm", torch.int32),
+                 (dead, "dead", torch.uint8), (codes, "codes", None), (scales, "scales", None),
+                 (zeros, "zeros", None), (dev_status, "dev_status", torch.int32), (ws, "ws", None))
     d_row, d_col = W.shape
     for t, name in ((codes, "codes"), (scales, "scales"), (zeros, "zeros"), (U, "U")):
         if not t.is_contiguous():
@@ -270,6 +302,10 @@ def gptq_quantize_layer_noalloc(W: torch.Tensor, U: torch.Tensor, perm: torch.Te
                     (scales, "scales"), (zeros, "zeros"), (dev_status, "dev_status")):
         if t is not None and (not t.is_cuda or t.device != W.device):
             raise ValueError(f"{name} must be on {W.device}, like W")
+    for t, name, dtype in ((U, "U", torch.float32), (perm, "perm", torch.int32),
+                           (dead, "dead", torch.uint8), (dev_status, "dev_status", torch.int32)):
+        if t is not None and t.dtype != dtype:
+            raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     with torch.cuda.device(W.device):
         _check(_lib.gptq_quantize_layer_noalloc(_ptr(W), d_row, d_col, _row_major(W, "W"),
                                                 _ptr(U), _ptr(perm), _ptr(dead),
@@ -286,6 +322,7 @@ def gptq_pack(codes: torch.Tensor, bits: int, packed: torch.Tensor, stream=None)
     """codes (d_row x d_col uint8) -> packed (d_row x ceil(d_col*bits/32) int32 view of uint32)."""
     _cuda(codes, "codes", torch.uint8)
     _cuda(packed, "packed")
+    _same_device(codes, "codes", (packed, "packed", None))
     if not codes.is_contiguous() or not packed.is_contiguous():
         raise ValueError("codes and packed must be contiguous")
     d_row, d_col = codes.shape
@@ -308,6 +345,8 @@ def gptq_dequant_matmul(X: torch.Tensor, packed: torch.Tensor, scales: torch.Ten
     _cuda(ws, "ws")
     if perm is not None:
         _cuda(perm, "perm", torch.int32)
+    _same_device(X, "X", (packed, "packed", None), (scales, "scales", None),
+                 (zeros, "zeros", None), (perm, "perm", None), (Y, "Y", None), (ws, "ws", None))
     for t, name in ((packed, "packed"), (scales, "scales"), (zeros, "zeros")):
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
@@ -340,6 +379,9 @@ def gptq_dequant_gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tenso
     _cuda(Y, "Y", torch.float32)
     if perm is not None:
         _cuda(perm, "perm", torch.int32)
+    _same_device(X, "X", (packed, "packed", None), (scales, "scales", None),
+                 (zeros, "zeros", None), (perm, "perm", None), (Y, "Y", None), (ws, "ws", None),
+                 (dev_status, "dev_status", torch.int32))
     for t, name in ((packed, "packed"), (scales, "scales"), (zeros, "zeros")):
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
