@@ -70,9 +70,9 @@ typedef enum gptq_status {
 typedef struct gptq_config {
     int32_t bits;        /* code width: 2, 3, 4 or 8                                  */
     int32_t group_size;  /* weights per (scale, zero) group along d_col; -1 = one
-                            group per row.  Supported: a divisor of block_size
-                            (e.g. 32, 64, 128), a multiple of block_size (256,
-                            1024, ...), or any value >= d_col.                    */
+                            group per row.  Supported: a divisor of block_size of
+                            at least 8 (8, 16, 32, 64, 128), a multiple of
+                            block_size (256, 1024, ...), or any value >= d_col.   */
     int32_t block_size;  /* columns per lazy-update block; must be 128               */
     int32_t desc_act;    /* nonzero: quantize columns by descending diag(H)          */
     float damp;          /* lambda = damp * mean(diag H); the guide's default 0.01   */

@@ -60,7 +60,10 @@ gptq_status check_config(const gptq_config* cfg, int64_t d_col) {
     if (g == 0 || g < -1) return GPTQ_ERR_INVALID_ARG;
     if (cfg->block_size != 128) return GPTQ_ERR_UNSUPPORTED;
     if (g == -1 || g >= d_col) return GPTQ_OK;
-    if (g < cfg->block_size) return (cfg->block_size % g == 0) ? GPTQ_OK : GPTQ_ERR_UNSUPPORTED;
+    // below a block: a divisor of it, at least 8 columns (groups of 1 to 4
+    // weights would carry a scale per handful of codes, and are not tested)
+    if (g < cfg->block_size)
+        return (g >= 8 && cfg->block_size % g == 0) ? GPTQ_OK : GPTQ_ERR_UNSUPPORTED;
     return (g % cfg->block_size == 0) ? GPTQ_OK : GPTQ_ERR_UNSUPPORTED;
 }
 

@@ -79,15 +79,18 @@ def test_workspace_size_and_config_validation(pkg):
         with pytest.raises(pkg.GPTQError) as e:
             pkg.gptq_workspace_size(pkg.GPTQConfig(**kw), 64, 256)
         assert e.value.status == 1
-    for unsup in (dict(group_size=48), dict(group_size=192), dict(block_size=64)):
+    for unsup in (dict(group_size=48), dict(group_size=192), dict(block_size=64),
+                  dict(group_size=4), dict(group_size=1)):
         kw = dict(bits=4, group_size=128)
         kw.update(unsup)
         with pytest.raises(pkg.GPTQError) as e:
             pkg.gptq_workspace_size(pkg.GPTQConfig(**kw), 64, 1024)
         assert e.value.status == 2
     # group sizes the column walk supports
-    for g in (1, 16, 32, 64, 128, 256, 1024, -1, 5000):
+    for g in (8, 16, 32, 64, 128, 256, 1024, -1, 5000):
         pkg.gptq_workspace_size(pkg.GPTQConfig(bits=4, group_size=g), 8, 4096)
+    # a group as wide as the row is one group per row, whatever its size
+    pkg.gptq_workspace_size(pkg.GPTQConfig(bits=4, group_size=4), 8, 4)
 
 
 def test_invalid_arguments_are_rejected_on_the_host(pkg):
