@@ -58,3 +58,38 @@ def test_job_throughput_counts_every_rank():
     assert eight == pytest.approx(8 * one)
     assert one == pytest.approx(4096 * 4096 / 8e-3)
     assert bench.max_over_ranks(3.5) == 3.5
+
+
+def test_stage_rooflines_use_the_closed_forms():
+    """The bench line's per-stage bounds: the lazy update of a d_col that is a
+    whole number of blocks does r d (d - B) flop (each block updates the
+    columns after it), the Hessian n d (d + 1), the inverse factor 2/3 d^3 and
+    pack r d (1 + b/8) bytes; the layer's bound is their sum plus the column
+    walk's r d B flop on the FFMA pipe."""
+    import bench
+    import workloads
+    wl = workloads.WORKLOADS["llama7b_q_proj"]
+    r, d, n, B, b = wl.d_row, wl.d_col, wl.n_tokens, wl.block_size, wl.bits
+    pk = {"bf16_tflops": 1600.0, "hbm_gbs": 6400.0}
+    ms = {"hessian": 3.0, "prepare_hinv": 1.4, "quantize_layer": 1.1, "pack": 0.01}
+    out = bench.stage_rooflines(wl, pk, "measured", ms, 5.6)
+    st = out["stages"]
+    tf32x3 = 1600.0 * 1.1 / 2.25 / 3
+    assert st["hessian"]["bound_ms"] == pytest.approx(n * d * (d + 1) / 1600e12 * 1e3)
+    assert st["prepare_hinv"]["bound_ms"] == pytest.approx(2 * d ** 3 / 3 / (tf32x3 * 1e12) * 1e3)
+    lazy = r * d * (d - B)
+    walk = r * d * B
+    assert st["quantize_layer"]["bound_ms"] == pytest.approx(
+        (lazy / (tf32x3 * 1e12) + walk / (148 * 128 * 2 * 1.965e9)) * 1e3)
+    assert st["pack"]["bound_ms"] == pytest.approx(r * d * (1 + b / 8) / 6400e9 * 1e3)
+    total = sum(v["bound_ms"] for v in st.values())
+    assert out["sum_bound_ms"] == pytest.approx(total)
+    assert out["layer_frac_of_summed_bound"] == pytest.approx(total / 5.6)
+    for name, v in st.items():
+        assert v["frac"] == pytest.approx(v["bound_ms"] / ms[name])
+    # a ragged layer (d_col = 300): block 0 updates the 172 columns after it,
+    # block 1 the last 44, the partial block 2 nothing
+    import dataclasses
+    rag = dataclasses.replace(wl, d_col=300)
+    out = bench.stage_rooflines(rag, pk, "measured", ms, 5.6)
+    assert f"lazy update {2.0 * r * B * (172 + 44):.3e} flop" in out["stages"]["quantize_layer"]["work"]
