@@ -29,14 +29,19 @@ void arm_wait_probe(int kind, uint64_t ns) {
 int64_t launches() { return g_launches.load(std::memory_order_relaxed); }
 
 int num_sms() {
-    static int cache[64] = {0};
+    // per device, filled on first use; threads that race to fill it store the
+    // same value
+    static std::atomic<int> cache[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
-    if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+    if (dev >= 0 && dev < 64) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
     int v = 0;
     if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
         v = 148;
-    if (dev >= 0 && dev < 64) cache[dev] = v;
+    if (dev >= 0 && dev < 64) cache[dev].store(v, std::memory_order_relaxed);
     return v;
 }
 
