@@ -300,3 +300,47 @@ def test_dequant_gemm_validation(pkg):
     # the act-order gather needs the workspace
     assert call(ws=None) == 6 and call(wsb=16 * 256 * 2 - 1) == 6
     assert call(ws=ctypes.c_void_p((1 << 20) + 32)) == 6
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "gptq.h"
+
+int main(void) {
+    gptq_config cfg;
+    size_t bytes = 0;
+    memset(&cfg, 0, sizeof cfg);
+    cfg.bits = 4; cfg.group_size = 128; cfg.block_size = 128; cfg.damp = 0.01f;
+    if (gptq_workspace_size(&cfg, 4096, 4096, &bytes) != GPTQ_OK) return 1;
+    cfg.bits = 5;
+    if (gptq_workspace_size(&cfg, 4096, 4096, &bytes) != GPTQ_ERR_INVALID_ARG) return 2;
+    /* host-side rejection before any launch: a NULL H */
+    if (gptq_hessian_accumulate((const uint16_t *)0x100000, 16, 16, 16, NULL, 16, NULL, NULL, 0,
+                                (cudaStream_t)0) != GPTQ_ERR_INVALID_ARG) return 3;
+    printf("%d %zu %s\n", gptq_version(), bytes, gptq_status_string(GPTQ_ERR_NOT_PD));
+    return 0;
+}
+"""
+
+
+def test_a_plain_c_program_compiles_links_and_calls_the_library(pkg, tmp_path):
+    """The header is C (not only C++): a C99 program includes it, links
+    against the shared library and calls the entry points that need no GPU."""
+    import shutil
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc unavailable")
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(pkg.library_path())
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    "-I", cuda_inc, str(src), "-L", libdir, "-lgptq_b200",
+                    f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, (out.returncode, out.stderr)
+    ver, nbytes, text = out.stdout.split(" ", 2)
+    assert int(ver) == pkg.gptq_version()
+    assert int(nbytes) == pkg.gptq_workspace_size(pkg.GPTQConfig(bits=4, group_size=128), 4096, 4096)
+    assert "positive definite" in text
